@@ -1,0 +1,269 @@
+"""fp64 CPU oracle for fused RoPE + attention and the DynamicNTK sin/cos table.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` are the only callers.  The product library never
+imports this package and this package never loads the product library.
+
+The arithmetic lives in ``rfa_oracle.c`` (plain loops, fp64, pthreads); this
+module only compiles it with gcc and marshals numpy arrays.  What each call
+computes, with the passage it follows:
+
+* ``inv_freq``     invFreq_j = base^(-2j/D) -- page "RoPE fused into attention
+  on Ascend", section 1.2 (the freqs line of the RoPE snippet).
+* ``ntk_base``     base' = base*((f*S/L)-(f-1))^(D/(D-2)) when S > L, else base --
+  page "DynamicNTKOperation", function description (no interpolation up to the
+  training length, an enlarged base beyond it).  The closed form itself is not
+  printed on that page (its InvFreqs formula was lost); this is the dynamic-NTK
+  form named for the long-context workload.
+* ``rope_sincos``  freq = outer(positionIds_b, invFreq_b); emb = cat(freq, freq);
+  sin/cos of emb -- page "DynamicNTKOperation", computation process.
+* ``rope_rotate``  rotate-half: x' = x*cos + rotate_half(x)*sin.
+* ``attention_rows`` / ``attention_probs``  softmax(Q'K'^T * scale) V with the
+  full score row, two passes -- page "FlashAttention in ops-transformer", the
+  attention formula; GQA grouping from page "RoPE, RMSNorm, GQA/MQA", sec. 12.
+
+Pinned by tests/test_oracle_*.py against closed forms, mpmath, numpy's complex
+exponential, torch's CPU scaled_dot_product_attention and brute force.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rfa_oracle.c")
+_LIB = os.path.join(_HERE, "librfa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BF16, FP16 = 0, 1
+BNSD, TND = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (only if missing or stale)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread", _SRC, "-lm", "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [
+        ("layout", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("B", ctypes.c_int32),
+        ("Hq", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32),
+        ("S", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
+        ("scale", ctypes.c_double),
+        ("nthreads", ctypes.c_int32),
+    ]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            lib.oracle_inv_freq.argtypes = [ctypes.c_double, ctypes.c_int32, P]
+            lib.oracle_inv_freq.restype = None
+            lib.oracle_ntk_base.argtypes = [ctypes.c_double, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                            ctypes.c_double]
+            lib.oracle_ntk_base.restype = ctypes.c_double
+            lib.oracle_rope_sincos.argtypes = [P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P]
+            lib.oracle_rope_sincos.restype = ctypes.c_int
+            lib.oracle_rope_rotate.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, P]
+            lib.oracle_rope_rotate.restype = None
+            lib.oracle_attention_rows.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P, P, ctypes.c_int64, P]
+            lib.oracle_attention_rows.restype = ctypes.c_int
+            lib.oracle_attention_probs.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, ctypes.c_int32,
+                                                   ctypes.c_int32, ctypes.c_int32, P]
+            lib.oracle_attention_probs.restype = ctypes.c_int
+            lib.oracle_widen16.argtypes = [ctypes.c_uint16, ctypes.c_int]
+            lib.oracle_widen16.restype = ctypes.c_double
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def widen16(bits: int, dtype: int = BF16) -> float:
+    return _load().oracle_widen16(int(bits), int(dtype))
+
+
+def inv_freq(base: float, D: int) -> np.ndarray:
+    out = np.empty(D // 2, np.float64)
+    _load().oracle_inv_freq(float(base), int(D), _ptr(out))
+    return out
+
+
+def ntk_base(base: float, D: int, S: int, L: int, factor: float) -> float:
+    return float(_load().oracle_ntk_base(float(base), int(D), int(S), int(L), float(factor)))
+
+
+def rope_sincos(position_ids, inv_freq_rows, seq_lens, head_size: int):
+    """sin, cos [ntokens, head_size] in fp64.  inv_freq_rows [batch, head_size/2]
+    (fp32 inputs are widened exactly).  Raises ValueError on bad lengths."""
+    pos = _c(position_ids, np.int32)
+    inv = _c(inv_freq_rows, np.float64)
+    sl = _c(seq_lens, np.int32)
+    batch, T = sl.shape[0], pos.shape[0]
+    assert inv.shape == (batch, head_size // 2)
+    s = np.empty((T, head_size), np.float64)
+    c = np.empty((T, head_size), np.float64)
+    rc = _load().oracle_rope_sincos(_ptr(pos), _ptr(inv), _ptr(sl), batch, T, head_size, _ptr(s), _ptr(c))
+    if rc != 0:
+        raise ValueError("seqLens must be positive and sum to ntokens")
+    return s, c
+
+
+def rope_rotate(x, pos, inv_freq_row):
+    """Rotate-half RoPE of rows x [n, D] (fp64) at positions pos [n]."""
+    x = _c(x, np.float64)
+    n, D = x.shape
+    p = _c(pos, np.int32)
+    inv = _c(inv_freq_row, np.float64)
+    assert p.shape == (n,) and inv.shape == (D // 2,)
+    out = np.empty_like(x)
+    _load().oracle_rope_rotate(_ptr(x), n, D, _ptr(p), _ptr(inv), _ptr(out))
+    return out
+
+
+def _bits16(t) -> np.ndarray:
+    """Raw 16-bit patterns of a bf16/fp16 torch tensor or a uint16 numpy array."""
+    if isinstance(t, np.ndarray):
+        assert t.dtype == np.uint16
+        return np.ascontiguousarray(t)
+    import torch
+
+    assert t.dtype in (torch.bfloat16, torch.float16)
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if isinstance(t, np.ndarray):
+        raise TypeError("pass torch tensors so the 16-bit format is known")
+    return BF16 if t.dtype == torch.bfloat16 else FP16
+
+
+def _desc(layout, dtype, B, Hq, Hkv, S, D, causal, scale, nthreads):
+    return _Desc(layout, dtype, B, Hq, Hkv, S, D, int(bool(causal)), float(scale),
+                 int(nthreads or default_threads()))
+
+
+def attention_rows(q, k, v, position, inv_freq_rows, rows, *, layout=BNSD, seq_lens=None, causal=True,
+                   scale=None, nthreads=None) -> np.ndarray:
+    """fp64 attention output for the given (b, h, i) rows -> [nrows, D].
+
+    BNSD: q [B,Hq,S,D], k/v [B,Hkv,S,D], position [B,S].
+    TND : q [T,Hq,D],   k/v [T,Hkv,D],   position [T], seq_lens [B].
+    inv_freq_rows: [B, D/2] per sequence (float values; fp32 widened exactly).
+    """
+    dt = _dtype_code(q)
+    if layout == BNSD:
+        B, Hq, S, D = q.shape
+        Hkv = k.shape[1]
+        sl = np.zeros(1, np.int32)
+    else:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        sl = _c(seq_lens, np.int32)
+        B, S = sl.shape[0], 0
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    d = _desc(layout, dt, B, Hq, Hkv, S, D, causal, scale, nthreads)
+    qb, kb, vb = _bits16(q), _bits16(k), _bits16(v)
+    pos = _c(np.asarray(position), np.int32).reshape(-1)
+    inv = _c(inv_freq_rows, np.float64).reshape(B, D // 2)
+    r = _c(rows, np.int32).reshape(-1, 3)
+    out = np.zeros((r.shape[0], D), np.float64)
+    rc = _load().oracle_attention_rows(ctypes.byref(d), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(pos), _ptr(sl), _ptr(inv),
+                                       _ptr(r), r.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("invalid attention rows or descriptor")
+    return out
+
+
+def attention_probs(q, k, position, inv_freq_rows, b, h, i, *, layout=BNSD, seq_lens=None, causal=True,
+                    scale=None) -> np.ndarray:
+    """One full softmax row P[b,h,i,:] in fp64."""
+    dt = _dtype_code(q)
+    if layout == BNSD:
+        B, Hq, S, D = q.shape
+        Hkv = k.shape[1]
+        sl = np.zeros(1, np.int32)
+        L = S
+    else:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        sl = _c(seq_lens, np.int32)
+        B, S = sl.shape[0], 0
+        L = int(sl[b])
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    d = _desc(layout, dt, B, Hq, Hkv, S, D, causal, scale, 1)
+    qb, kb = _bits16(q), _bits16(k)
+    pos = _c(np.asarray(position), np.int32).reshape(-1)
+    inv = _c(inv_freq_rows, np.float64).reshape(B, D // 2)
+    p = np.zeros(L, np.float64)
+    rc = _load().oracle_attention_probs(ctypes.byref(d), _ptr(qb), _ptr(kb), _ptr(pos), _ptr(sl), _ptr(inv), b, h, i,
+                                        _ptr(p))
+    if rc != 0:
+        raise ValueError("invalid row")
+    return p
+
+
+def all_rows(B: int, Hq: int, lens) -> np.ndarray:
+    """Every (b, h, i) row of a problem with per-sequence lengths lens."""
+    out = []
+    for b in range(B):
+        L = int(lens[b])
+        i = np.arange(L, dtype=np.int32)
+        for h in range(Hq):
+            out.append(np.stack([np.full(L, b, np.int32), np.full(L, h, np.int32), i], axis=1))
+    return np.concatenate(out, axis=0) if out else np.zeros((0, 3), np.int32)
+
+
+def attention_full(q, k, v, position, inv_freq_rows, *, layout=BNSD, seq_lens=None, causal=True, scale=None,
+                   nthreads=None) -> np.ndarray:
+    """Full fp64 output in the layout of q."""
+    if layout == BNSD:
+        B, Hq, S, D = q.shape
+        rows = all_rows(B, Hq, [S] * B)
+        out = attention_rows(q, k, v, position, inv_freq_rows, rows, layout=layout, causal=causal, scale=scale,
+                             nthreads=nthreads)
+        return out.reshape(B, Hq, S, D)
+    T, Hq, D = q.shape
+    sl = np.asarray(seq_lens, np.int64)
+    rows = all_rows(len(sl), Hq, sl)
+    out = attention_rows(q, k, v, position, inv_freq_rows, rows, layout=layout, seq_lens=seq_lens, causal=causal,
+                         scale=scale, nthreads=nthreads)
+    full = np.zeros((T, Hq, D), np.float64)
+    t0 = np.concatenate([[0], np.cumsum(sl)])
+    tok = t0[rows[:, 0]] + rows[:, 2]
+    full[tok, rows[:, 1]] = out
+    return full
