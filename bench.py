@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Benchmark: fused RoPE + attention forward on B200 (TFLOP/s, % of bf16 peak),
+plus the DynamicNTK sin/cos table (GB/s).
+
+One step = the whole hot path over one batch of the workload: the cos/sin
+table kernel followed by the fused RoPE + attention kernel, inputs resident in
+HBM.  Inputs (q, k, v) are larger than L2, so no flush is needed between
+steps.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload KEY] [--impl rfa|reference]
+
+--impl reference times the fp64 CPU oracle on the host cores on bounded row
+samples of the same workload (the comparison program for this method).
+Multi-GPU (torchrun): the path shards into independent problems with no data
+exchange, so every rank runs its own replica of the workload (weak scaling);
+ranks only meet for the barrier and the max-over-ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "fused RoPE+attention fwd TFLOP/s"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["rope_flashattention_b200/csrc/fused_rope_attn.cuh", "rope_flashattention_b200/csrc/sm100_ptx.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qwen7b", choices=sorted(workloads.BY_KEY))
+    ap.add_argument("--impl", default="rfa", choices=["rfa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-context", action="store_true", help="skip the unfused torch context line")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-oracle sample time")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha1()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(workload_key: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kh = kernel_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == workload_key and parts[1] == kh:
+                return float(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+                power.append(float(p[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s, pw in zip(sm, power) if pw > 250.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "rfa":
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ workload helpers
+def workload_kwargs(w):
+    kw = dict(layout=w.layout, causal=w.causal, rope_base=w.rope_base)
+    if w.ntk_train_len:
+        kw.update(ntk_train_len=w.ntk_train_len, ntk_factor=w.ntk_factor)
+    if w.layout == "TND":
+        kw["seq_lens"] = workloads.seq_lengths(w)
+    return kw
+
+
+def workload_flops(w) -> float:
+    import rope_flashattention_b200 as rfa
+
+    return rfa.attention_flops(workloads.seq_lengths(w), w.Hq, w.D, w.causal)
+
+
+def config_of(w, extra=None):
+    c = {"workload": w.name, "layout": w.layout, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+         "S": w.S if w.layout == "BNSD" else None, "D": w.D, "causal": w.causal, "rope_base": w.rope_base,
+         "ntokens": workloads.ntokens(w), "l2": "inputs larger than L2 (126 MB); no flush between steps"}
+    if w.ntk_train_len:
+        c["ntk"] = {"train_len": w.ntk_train_len, "factor": w.ntk_factor}
+    if w.layout == "TND":
+        c["seq_lens"] = workloads.seq_lengths(w)
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_rows_sample(w, n_rows: int, seed: int):
+    lens = workloads.seq_lengths(w)
+    rng = np.random.default_rng(seed)
+    b = rng.integers(0, w.B, n_rows)
+    h = rng.integers(0, w.Hq, n_rows)
+    i = np.array([rng.integers(0, lens[x]) for x in b])
+    return np.stack([b, h, i], axis=1).astype(np.int32)
+
+
+def rows_flops(w, rows) -> float:
+    lens = workloads.seq_lengths(w)
+    keys = [(int(i) + 1 if w.causal else lens[int(b)]) for b, _, i in rows]
+    return 4.0 * w.D * float(sum(keys))
+
+
+class OracleRunner:
+    """Times the fp64 oracle as it stands on bounded row samples."""
+
+    def __init__(self, w):
+        import oracle
+
+        self.oracle = oracle
+        self.w = w
+        self.q, self.k, self.v = workloads.make_qkv(w)
+        self.pos = workloads.positions(w).numpy()
+        inv = workloads.random_inv_freq(w)
+        lens = workloads.seq_lengths(w)
+        if inv is not None:
+            self.inv = inv.double().numpy()
+        else:
+            rows = []
+            for L in lens:
+                base = w.rope_base
+                if w.ntk_train_len:
+                    base = oracle.ntk_base(w.rope_base, w.D, L, w.ntk_train_len, w.ntk_factor)
+                rows.append(oracle.inv_freq(base, w.D))
+            self.inv = np.stack(rows)
+        self.threads = oracle.default_threads()
+
+    def run(self, rows):
+        w = self.w
+        kw = dict(causal=w.causal, nthreads=self.threads)
+        if w.layout == "TND":
+            kw.update(layout=self.oracle.TND, seq_lens=workloads.seq_lengths(w))
+        t0 = time.perf_counter()
+        self.oracle.attention_rows(self.q, self.k, self.v, self.pos, self.inv, rows, **kw)
+        return time.perf_counter() - t0
+
+    def calibrated_rows(self, seconds: float, seed: int = 0):
+        n = 64
+        dt = self.run(oracle_rows_sample(self.w, n, seed))
+        n = int(min(200000, max(64, n * seconds / max(dt, 1e-3))))
+        return oracle_rows_sample(self.w, n, seed + 1)
+
+
+def cpu_baseline(w, seconds: float):
+    r = OracleRunner(w)
+    rows = r.calibrated_rows(seconds)
+    dt = r.run(rows)
+    fl = rows_flops(w, rows)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": r.threads, "kind": "oracle",
+            "sample": f"{len(rows)} random query rows of the workload (all their causal keys), fp64, "
+                      f"{dt:.1f} s on {r.threads} threads; value = algorithmic FLOPs of those rows / time"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = workloads.BY_KEY[args.workload]
+    r = OracleRunner(w)
+    per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows = r.calibrated_rows(per_step)
+    for i in range(args.warmup):
+        r.run(oracle_rows_sample(w, len(rows), 100 + i))
+    times, flops = [], 0.0
+    for i in range(args.steps):
+        rs = oracle_rows_sample(w, len(rows), 1000 + i)
+        times.append(r.run(rs))
+        flops += rows_flops(w, rs)
+    tot = sum(times)
+    value = flops / tot / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": config_of(w, {"impl_note": "fp64 CPU oracle (plain loops, pthreads), each step a bounded "
+                                             "random row sample of the workload"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": r.threads, "kind": "oracle",
+                         "sample": f"{len(rows)} random query rows per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def sincos_bench(rfa, dev):
+    """rope_sincos at the operator's ceiling shape (T=256000, D=128, fp16):
+    GB/s of algorithmic bytes, L2 flushed (256 MB write) before each launch."""
+    pos, inv, lens = workloads.sincos_problem(256000, 128, 16, seed=7)
+    pos, inv, lens = pos.to(dev), inv.to(dev), lens.to(dev)
+    s = torch.empty((256000, 128), dtype=torch.float16, device=dev)
+    c = torch.empty_like(s)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        rfa.rope_sincos(pos, inv, lens, 128, torch.float16, s, c)
+    times = []
+    for _ in range(20):
+        flush.fill_(1)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        rfa.rope_sincos(pos, inv, lens, 128, torch.float16, s, c)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    assert rfa.get_device_status() == 0
+    byts = 256000 * 4 + 2 * 256000 * 128 * 2 + 16 * 64 * 4 + 16 * 4
+    t = statistics.median(times)
+    return {"shape": "T=256000 (16 x 16000), headSize 128, fp16", "bytes": byts, "us": t * 1e6,
+            "GB/s": byts / t / 1e9}
+
+
+def unfused_context(w, q, k, v, pos, dev, iters=20):
+    """Unfused GPU context: rope with torch ops (rotated q/k written to HBM)
+    then torch scaled_dot_product_attention."""
+    if w.layout != "BNSD":
+        return None
+    import torch.nn.functional as F
+
+    inv = 1.0 / (w.rope_base ** (torch.arange(0, w.D, 2, device=dev, dtype=torch.float64) / w.D))
+    if w.ntk_train_len and w.S > w.ntk_train_len:
+        base = w.rope_base * ((w.ntk_factor * w.S / w.ntk_train_len) - (w.ntk_factor - 1)) ** (w.D / (w.D - 2))
+        inv = 1.0 / (base ** (torch.arange(0, w.D, 2, device=dev, dtype=torch.float64) / w.D))
+    ang = pos.to(torch.float32)[:, None, :, None] * inv.float()[None, None, None, :]
+    cos = torch.cat([ang.cos(), ang.cos()], -1).to(q.dtype)
+    sin = torch.cat([ang.sin(), ang.sin()], -1).to(q.dtype)
+
+    def rot(x):
+        x1, x2 = x[..., : w.D // 2], x[..., w.D // 2:]
+        return x * cos + torch.cat([-x2, x1], -1) * sin
+
+    def step():
+        return F.scaled_dot_product_attention(rot(q), rot(k), v, is_causal=w.causal, enable_gqa=w.Hq != w.Hkv)
+
+    for _ in range(3):
+        step()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(iters):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / iters * 1e-3
+    return {"what": "torch rope ops + F.scaled_dot_product_attention (unfused, library attention)",
+            "TFLOP/s": workload_flops(w) / t / 1e12, "ms": t * 1e3}
+
+
+def run_gpu(args, world, rank, local):
+    import rope_flashattention_b200 as rfa
+
+    rfa.load_library()
+    dev = torch.device("cuda", local)
+    w = workloads.BY_KEY[args.workload]
+    peaks, peak_src = load_peaks()
+    kw = workload_kwargs(w)
+    q_h, k_h, v_h = workloads.make_qkv(w)
+    pos_h = workloads.positions(w)
+    inv_h = workloads.random_inv_freq(w)
+    q, k, v, pos = q_h.to(dev), k_h.to(dev), v_h.to(dev), pos_h.to(dev)
+    inv = inv_h.to(dev) if inv_h is not None else None
+    out = torch.empty_like(q)
+    table = rfa.rope_attention_table(q, k, pos, inv_freq=inv, **kw)
+    flops = workload_flops(w)
+
+    def step(ev=None):
+        rfa.rope_attention_table(q, k, pos, inv_freq=inv, workspace=table, **kw)
+        if ev is not None:
+            ev[0].record()
+        rfa.fused_rope_attention_with_table(q, k, v, table, out=out, **kw)
+        if ev is not None:
+            ev[1].record()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    st = rfa.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {rfa.status_string(st)}")
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    e_start.record()
+    for i in range(K):
+        step(evs[i])
+    e_end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    st = rfa.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {rfa.status_string(st)}")
+    ms_local = e_start.elapsed_time(e_end) / K
+    attn_ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms = max_over_ranks(ms_local, world)
+    attn_ms = max_over_ranks(attn_ms_local, world)
+    value = flops * world / (ms * 1e-3) / 1e12
+
+    # ---------------- end to end: host buffers through the C ABI
+    qp, kp, vp, posp = (x.pin_memory() for x in (q_h, k_h, v_h, pos_h))
+    outp = torch.empty(q_h.shape, dtype=q_h.dtype).pin_memory()
+    ws = torch.empty_like(table)
+    K2 = max(3, min(K, 30))
+
+    def e2e_step():
+        qd, kd, vd, pd = (x.to(dev, non_blocking=True) for x in (qp, kp, vp, posp))
+        o = rfa.fused_rope_attention(qd, kd, vd, pd, inv_freq=inv, workspace=ws, **kw)
+        outp.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K2):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K2, world)
+    h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp, posp))
+    d2h = outp.numel() * outp.element_size()
+
+    extra = {}
+    if rank == 0 and world == 1:
+        extra["sincos"] = sincos_bench(rfa, dev)
+        extra["sincos"]["frac_hbm"] = extra["sincos"]["GB/s"] / peaks["hbm_gbs"]
+        if not args.no_context:
+            try:
+                extra["context_unfused"] = unfused_context(w, q, k, v, pos, dev)
+            except Exception as e:  # context only; never fails the bench
+                extra["context_unfused"] = {"error": str(e)[:200]}
+
+    timed_s = ms * K * 1e-3
+    sustained = timed_s >= 1.0
+    peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    traffic = profiled_traffic(args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "impl": "rfa",
+        "config": config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                                "step": "cos/sin table kernel + fused RoPE/attention kernel"}),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                     "traffic": traffic,
+                     "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
+                     "kernel": "fused_rope_attn_fwd_kernel", "kernel_ms": attn_ms, "kernel_source": kernel_hash()},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": K2, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+        "tok_per_s": workloads.ntokens(w) * world / (ms * 1e-3),
+    }
+    line.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_gpu(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

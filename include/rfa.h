@@ -1,0 +1,177 @@
+/*
+ * rfa.h -- C ABI of librfa.so: rotary position embedding (RoPE) fused into a
+ * FlashAttention-style forward pass, and the DynamicNTK sin/cos table, for
+ * one NVIDIA B200 (sm_100a).
+ *
+ * Conventions for every entry point
+ *   - Plain pointers and sizes only.  "dev" pointers are CUDA device memory on
+ *     the current device, "host" pointers are ordinary host memory.
+ *   - The caller owns every buffer.  The library allocates nothing; scratch
+ *     memory is the caller's workspace.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream).  Host-side validation happens
+ *     synchronously before anything is enqueued: on an error nothing runs.
+ *   - Tensors are dense and row-major in the stated layout; there are no
+ *     stride arguments and no silent fallback to another code path.
+ *   - No C++ exception crosses this boundary.
+ *   - Errors found on the device (a wait that timed out, lengths that do not
+ *     add up) are recorded in a per-device status word that
+ *     rfa_get_device_status() reads and clears.
+ */
+#ifndef RFA_H_
+#define RFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RFA_API __attribute__((visibility("default")))
+#else
+#define RFA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RFA_OK = 0,
+    RFA_ERR_INVALID_ARG = 1, /* null pointer, bad size, inconsistent lengths */
+    RFA_ERR_UNSUPPORTED = 2, /* valid request outside what the kernels cover */
+    RFA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+    RFA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+    RFA_ERR_TIMEOUT = 5      /* a device-side wait gave up (status word only) */
+} rfa_status;
+
+/* Output / IO element types.  UNDEFINED is the default of the DynamicNTK
+ * parameter and is rejected, as on that operator's page (parameter list:
+ * "this default type is not usable").  FP32 is an extension for the sin/cos
+ * table only. */
+typedef enum { RFA_DT_UNDEFINED = 0, RFA_DT_FP16 = 1, RFA_DT_BF16 = 2, RFA_DT_FP32 = 3 } rfa_dtype;
+
+/* BNSD: q [B, Hq, S, D], k/v [B, Hkv, S, D]  (page "RoPE fused into attention
+ *       on Ascend", section 3, input_layout="BNSD").
+ * TND : packed sequences, q [T, Hq, D], k/v [T, Hkv, D], T = sum of lengths
+ *       (the token-major packing of page "DynamicNTKOperation", inputs). */
+typedef enum { RFA_LAYOUT_BNSD = 0, RFA_LAYOUT_TND = 1 } rfa_layout;
+
+/*
+ * rfa_rope_sincos -- the DynamicNTK sin/cos table.
+ * Page "DynamicNTKOperation", sections computation process, inputs, outputs
+ * and constraints: for each batch b (its tokens found through the prefix sums
+ * of seqLens), freq = outer(positionIds_b, invFreq_b), emb = cat(freq, freq),
+ * sin = sin(emb), cos = cos(emb).
+ *
+ *   positionIds  dev  int32 [ntokens]            any int32 value
+ *   invFreq      dev  fp32  [batch, headSize/2]  documented range [0,1), not enforced
+ *   seqLens      dev  int32 [batch]              each > 0, sum == ntokens
+ *   batch        1..16
+ *   ntokens      1..256000
+ *   headSize     multiple of 32, <= 2048
+ *   outType      RFA_DT_FP16 | RFA_DT_BF16 | RFA_DT_FP32 (UNDEFINED rejected)
+ *   sinOut,cosOut dev [ntokens, headSize] of outType, written in full;
+ *                columns j and j+headSize/2 are bit-identical.
+ *
+ * The angle is the fp32 product position*invFreq (as in the page's einsum on
+ * fp32 tensors); sin/cos are evaluated in fp32 and rounded to nearest even.
+ * Returns RFA_ERR_INVALID_ARG / RFA_ERR_UNSUPPORTED on host-checkable errors.
+ * seqLens lives on the device, so its sum is checked by the kernel: if it is
+ * not ntokens (or a length is <= 0) nothing is written and the status word
+ * becomes RFA_ERR_INVALID_ARG.
+ */
+RFA_API rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, const int32_t* seqLens,
+                           int32_t batch, int32_t ntokens, int32_t headSize, rfa_dtype outType,
+                           void* sinOut, void* cosOut, void* stream);
+
+/* Parameters of rfa_fused_rope_attention (plain old data). */
+typedef struct {
+    int32_t B;             /* BNSD: batch size; TND: number of packed sequences (1..16) */
+    int32_t Hq;            /* query heads (head_num) */
+    int32_t Hkv;           /* key/value heads; Hq % Hkv == 0, group G = Hq/Hkv,
+                              query head h reads kv head h / G */
+    int32_t S;             /* BNSD: sequence length (>= 1); TND: ignored */
+    int32_t D;             /* head dim: 64 or 128 */
+    int32_t layout;        /* rfa_layout */
+    int32_t causal;        /* 1: key index > query index (within a sequence) masked */
+    int32_t io_dtype;      /* RFA_DT_BF16 or RFA_DT_FP16 for q, k, v and out */
+    float scale;           /* softmax scale; 0 -> 1/sqrt(D) */
+    double rope_base;      /* invFreq_j = base^(-2j/D) (page "RoPE fused into
+                              attention on Ascend", section 1.2), e.g. 10000 */
+    int32_t ntk_enable;    /* dynamic NTK (page "DynamicNTKOperation", function
+                              description): for a sequence of length S_b > L the
+                              base becomes base*((f*S_b/L)-(f-1))^(D/(D-2)) */
+    int32_t ntk_train_len; /* L */
+    double ntk_factor;     /* f (rope_scaling_factor) */
+} rfa_attn_params;
+
+/* Bytes of device workspace rfa_fused_rope_attention needs for `ntokens`
+ * tokens (BNSD: B*S; TND: sum of lengths).  Returns 0 for invalid params. */
+RFA_API size_t rfa_fused_rope_attention_workspace(const rfa_attn_params* p, int64_t ntokens);
+
+/*
+ * rfa_fused_rope_attention -- out = softmax(Q'K'^T * scale) V with Q' and K'
+ * the rotate-half RoPE rotations of q and k (x' = x*cos + rotate_half(x)*sin
+ * with cos/sin of cat(freq, freq)), causal or not, GQA.
+ * Pages: "RoPE fused into attention on Ascend" (sections 3 and 5: the fused
+ * operator; rotated Q/K stay on chip), "FlashAttention in ops-transformer"
+ * (tiling, online softmax), "DynamicNTKOperation" (the sin/cos definition and
+ * the NTK rule), "RoPE, RMSNorm, GQA/MQA" (section 12, grouped heads).
+ *
+ *   p          host  parameters (see rfa_attn_params)
+ *   q, k, v    dev   io_dtype, layout per p->layout (see rfa_layout)
+ *   position   dev   int32, BNSD [B, S] / TND [T]: the position of each token
+ *                    (any int32; it only sets the rotation angle)
+ *   seqLens_host host int32 [B], TND only (each > 0); NULL for BNSD
+ *   invFreq    dev   fp32 [B, D/2] per-sequence inverse frequencies, or NULL
+ *                    to derive them from rope_base (+ NTK) in fp64 on the host,
+ *                    rounded once to fp32
+ *   out        dev   io_dtype, same shape and layout as q
+ *   workspace  dev   >= rfa_fused_rope_attention_workspace(p, T) bytes,
+ *                    256-byte aligned; holds the cos/sin table of this call
+ *                    (a table, never rotated Q/K)
+ * Rotated Q and K exist only in shared memory.  The call enqueues two
+ * kernels: the cos/sin table and the fused attention.
+ */
+RFA_API rfa_status rfa_fused_rope_attention(const rfa_attn_params* p, const void* q, const void* k, const void* v,
+                                    const int32_t* position, const int32_t* seqLens_host,
+                                    const float* invFreq, void* out, void* workspace, size_t ws_bytes,
+                                    void* stream);
+
+/*
+ * The same operation in two steps, for callers that keep the cos/sin table
+ * of a batch of positions and reuse it across calls (page "RoPE fused into
+ * attention on Ascend", section 6.2: precompute the lookup table once and
+ * register it, rather than regenerating the frequencies on every call).
+ *
+ * rfa_rope_attention_table: writes the cos/sin table of p's tokens into
+ *   workspace (same size and alignment rule as above).  Arguments as for
+ *   rfa_fused_rope_attention.
+ * rfa_fused_rope_attention_with_table: the attention kernel alone, reading a
+ *   table that rfa_rope_attention_table wrote for the same p, positions and
+ *   seqLens_host.  The workspace is only read.
+ * rfa_fused_rope_attention == rfa_rope_attention_table followed by
+ * rfa_fused_rope_attention_with_table on the same stream.
+ */
+RFA_API rfa_status rfa_rope_attention_table(const rfa_attn_params* p, const int32_t* position,
+                                            const int32_t* seqLens_host, const float* invFreq, void* workspace,
+                                            size_t ws_bytes, void* stream);
+RFA_API rfa_status rfa_fused_rope_attention_with_table(const rfa_attn_params* p, const void* q, const void* k,
+                                                       const void* v, const int32_t* seqLens_host, void* out,
+                                                       const void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word (RFA_OK if no kernel recorded an error).  RFA_ERR_CUDA if the
+ * synchronisation itself failed. */
+RFA_API rfa_status rfa_get_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+RFA_API const char* rfa_status_string(rfa_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+RFA_API int32_t rfa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RFA_H_ */

@@ -1,0 +1,297 @@
+"""B200-native rotary position embedding fused into FlashAttention forward.
+
+Thin ctypes binding over librfa.so (C ABI in include/rfa.h).  This module only
+marshals arguments: it checks tensor devices, dtypes and contiguity, passes
+raw pointers and torch's current CUDA stream, and turns status codes into
+exceptions.  Every step of the computation runs in the library's CUDA
+kernels.  There is no CPU fallback: if librfa.so is missing the import fails.
+
+Entry points (C name without the ``rfa_`` prefix):
+    rope_sincos(position_ids, inv_freq, seq_lens, head_size, out_dtype)
+    fused_rope_attention(q, k, v, position, ...)
+    fused_rope_attention_workspace(...)
+    get_device_status()
+    status_string(code)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "RfaError", "LIB_PATH", "EXPORTS", "load_library", "rope_sincos", "fused_rope_attention",
+    "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
+    "get_device_status", "status_string", "AttnParams",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa.so")
+
+# Every symbol include/rfa.h declares.
+EXPORTS = (
+    "rfa_rope_sincos",
+    "rfa_fused_rope_attention_workspace",
+    "rfa_fused_rope_attention",
+    "rfa_rope_attention_table",
+    "rfa_fused_rope_attention_with_table",
+    "rfa_get_device_status",
+    "rfa_status_string",
+    "rfa_version",
+)
+
+RFA_OK, RFA_ERR_INVALID_ARG, RFA_ERR_UNSUPPORTED, RFA_ERR_WORKSPACE, RFA_ERR_CUDA, RFA_ERR_TIMEOUT = range(6)
+DT_UNDEFINED, DT_FP16, DT_BF16, DT_FP32 = range(4)
+LAYOUT_BNSD, LAYOUT_TND = 0, 1
+_TORCH_DT = {torch.float16: DT_FP16, torch.bfloat16: DT_BF16, torch.float32: DT_FP32}
+
+
+class RfaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+class AttnParams(ctypes.Structure):
+    """Mirror of rfa_attn_params."""
+    _fields_ = [
+        ("B", ctypes.c_int32),
+        ("Hq", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32),
+        ("S", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("layout", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
+        ("io_dtype", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("rope_base", ctypes.c_double),
+        ("ntk_enable", ctypes.c_int32),
+        ("ntk_train_len", ctypes.c_int32),
+        ("ntk_factor", ctypes.c_double),
+    ]
+
+
+_lib = None
+
+
+def load_library():
+    """Load librfa.so (built in-tree by __graft_entry__.build())."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"librfa.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.rfa_rope_sincos.argtypes = [P, P, P, I32, I32, I32, ctypes.c_int, P, P, P]
+    lib.rfa_rope_sincos.restype = ctypes.c_int
+    lib.rfa_fused_rope_attention_workspace.argtypes = [ctypes.POINTER(AttnParams), I64]
+    lib.rfa_fused_rope_attention_workspace.restype = SZ
+    lib.rfa_fused_rope_attention.argtypes = [ctypes.POINTER(AttnParams), P, P, P, P, P, P, P, P, SZ, P]
+    lib.rfa_fused_rope_attention.restype = ctypes.c_int
+    lib.rfa_rope_attention_table.argtypes = [ctypes.POINTER(AttnParams), P, P, P, P, SZ, P]
+    lib.rfa_rope_attention_table.restype = ctypes.c_int
+    lib.rfa_fused_rope_attention_with_table.argtypes = [ctypes.POINTER(AttnParams), P, P, P, P, P, P, SZ, P]
+    lib.rfa_fused_rope_attention_with_table.restype = ctypes.c_int
+    lib.rfa_get_device_status.argtypes = [P]
+    lib.rfa_get_device_status.restype = ctypes.c_int
+    lib.rfa_status_string.argtypes = [ctypes.c_int]
+    lib.rfa_status_string.restype = ctypes.c_char_p
+    lib.rfa_version.argtypes = []
+    lib.rfa_version.restype = I32
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().rfa_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != RFA_OK:
+        raise RfaError(code, where)
+
+
+def _stream_ptr(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> ctypes.c_void_p:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def rope_sincos(position_ids: torch.Tensor, inv_freq: torch.Tensor, seq_lens: torch.Tensor, head_size: int,
+                out_dtype=torch.float16, sin_out: Optional[torch.Tensor] = None,
+                cos_out: Optional[torch.Tensor] = None, stream=None):
+    """sin, cos [ntokens, head_size] of cat(outer(pos_b, invFreq_b), same).
+
+    position_ids int32 [ntokens], inv_freq fp32 [batch, head_size/2] and
+    seq_lens int32 [batch] live on the GPU (as on the DynamicNTK operator).
+    """
+    T = position_ids.numel()
+    batch = seq_lens.numel()
+    dev = position_ids.device
+    if sin_out is None:
+        sin_out = torch.empty((T, head_size), dtype=out_dtype, device=dev)
+    if cos_out is None:
+        cos_out = torch.empty((T, head_size), dtype=out_dtype, device=dev)
+    code = load_library().rfa_rope_sincos(
+        _dev(position_ids, "position_ids", torch.int32), _dev(inv_freq, "inv_freq", torch.float32),
+        _dev(seq_lens, "seq_lens", torch.int32), batch, T, int(head_size), _TORCH_DT.get(sin_out.dtype, DT_UNDEFINED),
+        _dev(sin_out, "sin_out"), _dev(cos_out, "cos_out"), _stream_ptr(stream))
+    _check(code, "rfa_rope_sincos")
+    return sin_out, cos_out
+
+
+def _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor) -> AttnParams:
+    if layout == "BNSD":
+        B, Hq, S, D = q.shape
+        Hkv = k.shape[1]
+        lay = LAYOUT_BNSD
+    elif layout == "TND":
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B, S, lay = len(seq_lens), 0, LAYOUT_TND
+    else:
+        raise ValueError("layout must be 'BNSD' or 'TND'")
+    p = AttnParams()
+    p.B, p.Hq, p.Hkv, p.S, p.D, p.layout = B, Hq, Hkv, S, D, lay
+    p.causal = 1 if causal else 0
+    p.io_dtype = _TORCH_DT.get(q.dtype, DT_UNDEFINED)
+    p.scale = 0.0 if scale is None else float(scale)
+    p.rope_base = float(rope_base)
+    p.ntk_enable = 1 if ntk_train_len else 0
+    p.ntk_train_len = int(ntk_train_len or 0)
+    p.ntk_factor = float(ntk_factor)
+    return p
+
+
+def fused_rope_attention_workspace(q, k, *, layout="BNSD", seq_lens=None, causal=True, scale=None,
+                                   rope_base=10000.0, ntk_train_len=0, ntk_factor=1.0) -> int:
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    T = p.B * p.S if layout == "BNSD" else int(sum(int(x) for x in seq_lens))
+    return int(load_library().rfa_fused_rope_attention_workspace(ctypes.byref(p), T))
+
+
+def _lens_arg(layout, seq_lens, p):
+    if layout != "TND":
+        return None, p.B * p.S
+    arr = (ctypes.c_int32 * p.B)(*[int(x) for x in seq_lens])
+    return arr, sum(int(x) for x in seq_lens)
+
+
+def _need(p, T) -> int:
+    need = int(load_library().rfa_fused_rope_attention_workspace(ctypes.byref(p), T))
+    if need == 0:
+        _check(RFA_ERR_INVALID_ARG if p.io_dtype == DT_UNDEFINED else RFA_ERR_UNSUPPORTED,
+               "rfa_fused_rope_attention_workspace")
+    return need
+
+
+def _ptr_or_null(arr):
+    return None if arr is None else ctypes.cast(arr, ctypes.c_void_p)
+
+
+def rope_attention_table(q, k, position: torch.Tensor, *, layout: str = "BNSD", seq_lens=None, causal=True,
+                         scale=None, rope_base: float = 10000.0, ntk_train_len: int = 0, ntk_factor: float = 1.0,
+                         inv_freq: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Build the cos/sin table of this batch's positions into a workspace
+    tensor (returned), for reuse by fused_rope_attention_with_table."""
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    lens, T = _lens_arg(layout, seq_lens, p)
+    need = _need(p, T)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    code = load_library().rfa_rope_attention_table(
+        ctypes.byref(p), _dev(position, "position", torch.int32), _ptr_or_null(lens),
+        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(code, "rfa_rope_attention_table")
+    return workspace
+
+
+def fused_rope_attention_with_table(q, k, v, table: torch.Tensor, *, layout: str = "BNSD", seq_lens=None,
+                                    causal=True, scale=None, rope_base: float = 10000.0, ntk_train_len: int = 0,
+                                    ntk_factor: float = 1.0, out: Optional[torch.Tensor] = None,
+                                    stream=None) -> torch.Tensor:
+    """The attention kernel alone, reading a table from rope_attention_table."""
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    lens, T = _lens_arg(layout, seq_lens, p)
+    if out is None:
+        out = torch.empty_like(q)
+    io = (torch.bfloat16, torch.float16)
+    code = load_library().rfa_fused_rope_attention_with_table(
+        ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _ptr_or_null(lens),
+        _dev(out, "out", q.dtype), _dev(table, "table"), table.numel() * table.element_size(), _stream_ptr(stream))
+    _check(code, "rfa_fused_rope_attention_with_table")
+    return out
+
+
+def fused_rope_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position: torch.Tensor, *,
+                         layout: str = "BNSD", seq_lens: Optional[Sequence[int]] = None, causal: bool = True,
+                         scale: Optional[float] = None, rope_base: float = 10000.0, ntk_train_len: int = 0,
+                         ntk_factor: float = 1.0, inv_freq: Optional[torch.Tensor] = None,
+                         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """softmax(rope(q) rope(k)^T * scale) v, rotated q/k kept on chip.
+
+    BNSD: q [B,Hq,S,D], k/v [B,Hkv,S,D], position int32 [B,S].
+    TND : q [T,Hq,D], k/v [T,Hkv,D], position int32 [T], seq_lens (host ints).
+    ntk_train_len > 0 enables dynamic NTK with factor ntk_factor.
+    inv_freq: optional fp32 [B, D/2] on the GPU.
+    """
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    lens, T = _lens_arg(layout, seq_lens, p)
+    need = _need(p, T)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    io = (torch.bfloat16, torch.float16)
+    code = load_library().rfa_fused_rope_attention(
+        ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+        _dev(position, "position", torch.int32), _ptr_or_null(lens),
+        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32),
+        _dev(out, "out", q.dtype), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream))
+    _check(code, "rfa_fused_rope_attention")
+    return out
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream and return/clear the device status word."""
+    return int(load_library().rfa_get_device_status(_stream_ptr(stream)))
+
+
+# C names, for callers that prefer them.
+rfa_rope_sincos = rope_sincos
+rfa_fused_rope_attention = fused_rope_attention
+rfa_fused_rope_attention_workspace = fused_rope_attention_workspace
+rfa_rope_attention_table = rope_attention_table
+rfa_fused_rope_attention_with_table = fused_rope_attention_with_table
+rfa_get_device_status = get_device_status
+rfa_status_string = status_string
+
+
+def attention_flops(lens, Hq: int, D: int, causal: bool = True) -> float:
+    """Algorithmic FLOPs of the two attention GEMMs: 4*D*Hq*sum(S_b(S_b+1)/2)
+    causal (masked work not counted), 4*D*Hq*sum(S_b^2) otherwise."""
+    tot = 0
+    for s in lens:
+        s = int(s)
+        tot += s * (s + 1) // 2 if causal else s * s
+    return 4.0 * D * Hq * tot
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,354 @@
+// rfa_api.cu -- the C ABI of librfa.so (declared in include/rfa.h): host-side
+// validation, inverse frequencies (fp64 on the host, rounded once to fp32),
+// work decomposition, TMA tensor maps and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "fused_rope_attn.cuh"
+#include "rfa.h"
+#include "rope_sincos.cuh"
+
+namespace {
+
+constexpr int32_t kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16/fp16 tensor map, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, bool fp16, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t st1,
+              uint64_t st2, uint32_t b0, uint32_t b1, uint32_t b2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {st1, st2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename K>
+rfa_status ensure_smem_attr(K kernel, int bytes) {
+    static bool done[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RFA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return RFA_ERR_CUDA;
+        done[dev] = true;
+    }
+    return RFA_OK;
+}
+
+int grid_for(int64_t work, int threads) {
+    int64_t blocks = (work + threads - 1) / threads;
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, 148LL * 64)));
+}
+
+// invFreq_j = base^(-2j/D) in fp64, rounded once to fp32.
+void inv_freq_row(double base, int D, float* out) {
+    for (int j = 0; j < D / 2; ++j) out[j] = static_cast<float>(std::pow(base, -2.0 * j / static_cast<double>(D)));
+}
+
+double ntk_base(const rfa_attn_params* p, int64_t S_b) {
+    if (!p->ntk_enable || S_b <= p->ntk_train_len) return p->rope_base;
+    const double f = p->ntk_factor;
+    return p->rope_base * std::pow(f * static_cast<double>(S_b) / p->ntk_train_len - (f - 1.0),
+                                   static_cast<double>(p->D) / (p->D - 2));
+}
+
+rfa_status validate_attn(const rfa_attn_params* p) {
+    if (!p) return RFA_ERR_INVALID_ARG;
+    if (p->layout != RFA_LAYOUT_BNSD && p->layout != RFA_LAYOUT_TND) return RFA_ERR_INVALID_ARG;
+    if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->D < 1) return RFA_ERR_INVALID_ARG;
+    if (p->Hq % p->Hkv != 0) return RFA_ERR_INVALID_ARG;
+    if (p->layout == RFA_LAYOUT_BNSD && p->S < 1) return RFA_ERR_INVALID_ARG;
+    if (p->layout == RFA_LAYOUT_TND && p->B > rfa::kMaxSeqs) return RFA_ERR_INVALID_ARG;
+    if (p->io_dtype != RFA_DT_BF16 && p->io_dtype != RFA_DT_FP16) {
+        return p->io_dtype == RFA_DT_UNDEFINED ? RFA_ERR_INVALID_ARG : RFA_ERR_UNSUPPORTED;
+    }
+    if (!(p->scale >= 0.0f) || !std::isfinite(p->scale)) return RFA_ERR_INVALID_ARG;
+    if (!(p->rope_base > 0.0) || !std::isfinite(p->rope_base)) return RFA_ERR_INVALID_ARG;
+    if (p->ntk_enable && (p->ntk_train_len < 1 || !(p->ntk_factor >= 1.0) || !std::isfinite(p->ntk_factor)))
+        return RFA_ERR_INVALID_ARG;
+    if ((p->D & 1) != 0) return RFA_ERR_INVALID_ARG;
+    if (p->D != 64 && p->D != 128) return RFA_ERR_UNSUPPORTED;
+    return RFA_OK;
+}
+
+int64_t total_tokens(const rfa_attn_params* p, const int32_t* lens) {
+    if (p->layout == RFA_LAYOUT_BNSD) return static_cast<int64_t>(p->B) * p->S;
+    int64_t t = 0;
+    for (int b = 0; b < p->B; ++b) t += lens[b];
+    return t;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * D * sizeof(float), 256); }
+
+template <int D, bool kFP16>
+rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const rfa::AttnArgs& args,
+                       cudaStream_t st) {
+    auto kern = rfa::fused_rope_attn_fwd_kernel<D, kFP16>;
+    constexpr int smem = rfa::AttnCfg<D>::kSmemBytes;
+    if (ensure_smem_attr(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
+    kern<<<args.n_items, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, args);
+    return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t rfa_version(void) { return kVersion; }
+
+const char* rfa_status_string(rfa_status s) {
+    switch (s) {
+        case RFA_OK: return "RFA_OK";
+        case RFA_ERR_INVALID_ARG: return "RFA_ERR_INVALID_ARG";
+        case RFA_ERR_UNSUPPORTED: return "RFA_ERR_UNSUPPORTED";
+        case RFA_ERR_WORKSPACE: return "RFA_ERR_WORKSPACE";
+        case RFA_ERR_CUDA: return "RFA_ERR_CUDA";
+        case RFA_ERR_TIMEOUT: return "RFA_ERR_TIMEOUT";
+    }
+    return "RFA_ERR_UNKNOWN";
+}
+
+rfa_status rfa_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return RFA_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpyFromSymbol(&v, rfa::g_status, sizeof v) != cudaSuccess) return RFA_ERR_CUDA;
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(rfa::g_status, &zero, sizeof zero) != cudaSuccess) return RFA_ERR_CUDA;
+    return static_cast<rfa_status>(v);
+}
+
+rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, const int32_t* seqLens, int32_t batch,
+                           int32_t ntokens, int32_t headSize, rfa_dtype outType, void* sinOut, void* cosOut,
+                           void* stream) {
+    if (!positionIds || !invFreq || !seqLens || !sinOut || !cosOut) return RFA_ERR_INVALID_ARG;
+    if (outType == RFA_DT_UNDEFINED) return RFA_ERR_INVALID_ARG;
+    if (outType != RFA_DT_FP16 && outType != RFA_DT_BF16 && outType != RFA_DT_FP32) return RFA_ERR_INVALID_ARG;
+    if (batch < 1 || batch > rfa::kMaxSeqs) return RFA_ERR_INVALID_ARG;
+    if (ntokens < 1 || ntokens > 256000) return RFA_ERR_INVALID_ARG;
+    if (headSize < 32 || headSize > 2048 || headSize % 32 != 0) return RFA_ERR_INVALID_ARG;
+    if (!aligned(invFreq, 16) || !aligned(sinOut, 16) || !aligned(cosOut, 16)) return RFA_ERR_INVALID_ARG;
+    const int64_t work = static_cast<int64_t>(ntokens) * (headSize / 16);
+    const int grid = grid_for(work, 256);
+    cudaStream_t st = as_stream(stream);
+    switch (outType) {
+        case RFA_DT_FP16:
+            rfa::rope_sincos_kernel<__half><<<grid, 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
+                                                                   headSize, static_cast<__half*>(sinOut),
+                                                                   static_cast<__half*>(cosOut));
+            break;
+        case RFA_DT_BF16:
+            rfa::rope_sincos_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+                positionIds, invFreq, seqLens, batch, ntokens, headSize, static_cast<__nv_bfloat16*>(sinOut),
+                static_cast<__nv_bfloat16*>(cosOut));
+            break;
+        default:
+            rfa::rope_sincos_kernel<float><<<grid, 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
+                                                                  headSize, static_cast<float*>(sinOut),
+                                                                  static_cast<float*>(cosOut));
+            break;
+    }
+    return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+}
+
+size_t rfa_fused_rope_attention_workspace(const rfa_attn_params* p, int64_t ntokens) {
+    if (validate_attn(p) != RFA_OK || ntokens < 1) return 0;
+    return table_bytes(ntokens, p->D);
+}
+
+}  // extern "C"
+
+namespace {
+
+rfa_status check_common(const rfa_attn_params* p, const int32_t* seqLens_host, int64_t* T_out) {
+    rfa_status vs = validate_attn(p);
+    if (vs != RFA_OK) return vs;
+    if (p->layout == RFA_LAYOUT_TND) {
+        if (!seqLens_host) return RFA_ERR_INVALID_ARG;
+        for (int b = 0; b < p->B; ++b)
+            if (seqLens_host[b] <= 0) return RFA_ERR_INVALID_ARG;
+    }
+    const int64_t T = total_tokens(p, seqLens_host);
+    if (T < 1 || T > (int64_t{1} << 31) / 4 - 1) return RFA_ERR_INVALID_ARG;
+    *T_out = T;
+    return RFA_OK;
+}
+
+rfa_status enqueue_table(const rfa_attn_params* p, int64_t T, const int32_t* position, const int32_t* seqLens_host,
+                         const float* invFreq, void* workspace, cudaStream_t st) {
+    const bool tnd = p->layout == RFA_LAYOUT_TND;
+    const int D = p->D;
+    const int half = D / 2;
+    rfa::TableArgs ta;
+    std::memset(&ta, 0, sizeof ta);
+    ta.pos = position;
+    ta.inv_dev = invFreq;
+    ta.table = static_cast<float*>(workspace);
+    ta.ntokens = static_cast<int32_t>(T);
+    ta.half = half;
+    ta.nseg = p->B;
+    ta.uniform_len = tnd ? 0 : p->S;
+    if (tnd) {
+        int64_t acc = 0;
+        for (int b = 0; b < p->B; ++b) {
+            ta.cum[b] = static_cast<int32_t>(acc);
+            acc += seqLens_host[b];
+        }
+        ta.cum[p->B] = static_cast<int32_t>(acc);
+    }
+    if (!invFreq) {
+        if (!tnd || !p->ntk_enable) {
+            ta.inv_host_rows = 1;
+            inv_freq_row(ntk_base(p, tnd ? 0 : p->S), D, ta.inv_host);
+        } else {
+            ta.inv_host_rows = p->B;
+            for (int b = 0; b < p->B; ++b) inv_freq_row(ntk_base(p, seqLens_host[b]), D, ta.inv_host + b * half);
+        }
+    }
+    rfa::rope_table_kernel<<<grid_for(T * (half / 8), 256), 256, 0, st>>>(ta);
+    return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+}
+
+rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q, const void* k, const void* v,
+                             const int32_t* seqLens_host, void* out, const void* table, cudaStream_t st) {
+    const bool tnd = p->layout == RFA_LAYOUT_TND;
+    const int D = p->D;
+    rfa::AttnArgs aa;
+    std::memset(&aa, 0, sizeof aa);
+    aa.out = out;
+    aa.table = static_cast<const float*>(table);
+    aa.layout = tnd ? 1 : 0;
+    aa.B = p->B;
+    aa.Hq = p->Hq;
+    aa.Hkv = p->Hkv;
+    aa.G = p->Hq / p->Hkv;
+    aa.S = tnd ? 0 : p->S;
+    aa.causal = p->causal ? 1 : 0;
+    const float scale = p->scale > 0.0f ? p->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    aa.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    const bool fp16 = p->io_dtype == RFA_DT_FP16;
+    const uint64_t esz = 2;
+    CUtensorMap mq, mk, mv;
+    bool ok;
+    if (!tnd) {
+        const int64_t nqt = (p->S + rfa::kBlockM - 1) / rfa::kBlockM;
+        const int64_t items = nqt * p->B * p->Hq;
+        if (items > 0x7fffffff) return RFA_ERR_UNSUPPORTED;
+        aa.n_items = static_cast<int32_t>(items);
+        ok = make_map(&mq, q, fp16, D, p->S, static_cast<uint64_t>(p->B) * p->Hq, D * esz, p->S * D * esz, 64,
+                      rfa::kBlockM, 1) &&
+             make_map(&mk, k, fp16, D, p->S, static_cast<uint64_t>(p->B) * p->Hkv, D * esz, p->S * D * esz, 64,
+                      rfa::kBlockN, 1) &&
+             make_map(&mv, v, fp16, D, p->S, static_cast<uint64_t>(p->B) * p->Hkv, D * esz, p->S * D * esz, 64,
+                      rfa::kBlockN, 1);
+    } else {
+        // sequences sorted by query-tile count, descending (longest first)
+        int order[rfa::kMaxSeqs];
+        int starts[rfa::kMaxSeqs];
+        int64_t acc = 0;
+        for (int b = 0; b < p->B; ++b) {
+            order[b] = b;
+            starts[b] = static_cast<int>(acc);
+            acc += seqLens_host[b];
+        }
+        std::stable_sort(order, order + p->B, [&](int x, int y) { return seqLens_host[x] > seqLens_host[y]; });
+        aa.nseg = p->B;
+        int64_t items = 0;
+        for (int i = 0; i < p->B; ++i) {
+            const int b = order[i];
+            aa.seg_start[i] = starts[b];
+            aa.seg_len[i] = seqLens_host[b];
+            aa.seg_tiles[i] = (seqLens_host[b] + rfa::kBlockM - 1) / rfa::kBlockM;
+            items += static_cast<int64_t>(aa.seg_tiles[i]) * p->Hq;
+        }
+        if (items > 0x7fffffff) return RFA_ERR_UNSUPPORTED;
+        aa.n_items = static_cast<int32_t>(items);
+        ok = make_map(&mq, q, fp16, D, p->Hq, T, D * esz, static_cast<uint64_t>(p->Hq) * D * esz, 64, 1,
+                      rfa::kBlockM) &&
+             make_map(&mk, k, fp16, D, p->Hkv, T, D * esz, static_cast<uint64_t>(p->Hkv) * D * esz, 64, 1,
+                      rfa::kBlockN) &&
+             make_map(&mv, v, fp16, D, p->Hkv, T, D * esz, static_cast<uint64_t>(p->Hkv) * D * esz, 64, 1,
+                      rfa::kBlockN);
+    }
+    if (!ok) return RFA_ERR_CUDA;
+    if (D == 128) return fp16 ? launch_attn<128, true>(mq, mk, mv, aa, st) : launch_attn<128, false>(mq, mk, mv, aa, st);
+    return fp16 ? launch_attn<64, true>(mq, mk, mv, aa, st) : launch_attn<64, false>(mq, mk, mv, aa, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+rfa_status rfa_rope_attention_table(const rfa_attn_params* p, const int32_t* position, const int32_t* seqLens_host,
+                                    const float* invFreq, void* workspace, size_t ws_bytes, void* stream) {
+    int64_t T = 0;
+    rfa_status vs = check_common(p, seqLens_host, &T);
+    if (vs != RFA_OK) return vs;
+    if (!position) return RFA_ERR_INVALID_ARG;
+    if (invFreq && !aligned(invFreq, 16)) return RFA_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < table_bytes(T, p->D) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
+    return enqueue_table(p, T, position, seqLens_host, invFreq, workspace, as_stream(stream));
+}
+
+rfa_status rfa_fused_rope_attention_with_table(const rfa_attn_params* p, const void* q, const void* k, const void* v,
+                                               const int32_t* seqLens_host, void* out, const void* workspace,
+                                               size_t ws_bytes, void* stream) {
+    int64_t T = 0;
+    rfa_status vs = check_common(p, seqLens_host, &T);
+    if (vs != RFA_OK) return vs;
+    if (!q || !k || !v || !out) return RFA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return RFA_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < table_bytes(T, p->D) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
+    return enqueue_attention(p, T, q, k, v, seqLens_host, out, workspace, as_stream(stream));
+}
+
+rfa_status rfa_fused_rope_attention(const rfa_attn_params* p, const void* q, const void* k, const void* v,
+                                    const int32_t* position, const int32_t* seqLens_host, const float* invFreq,
+                                    void* out, void* workspace, size_t ws_bytes, void* stream) {
+    int64_t T = 0;
+    rfa_status vs = check_common(p, seqLens_host, &T);
+    if (vs != RFA_OK) return vs;
+    if (!q || !k || !v || !position || !out) return RFA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return RFA_ERR_INVALID_ARG;
+    if (invFreq && !aligned(invFreq, 16)) return RFA_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < table_bytes(T, p->D) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    rfa_status r = enqueue_table(p, T, position, seqLens_host, invFreq, workspace, st);
+    if (r != RFA_OK) return r;
+    return enqueue_attention(p, T, q, k, v, seqLens_host, out, workspace, st);
+}
+
+}  // extern "C"

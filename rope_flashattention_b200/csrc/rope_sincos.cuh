@@ -1,0 +1,147 @@
+// rope_sincos.cuh -- the DynamicNTK sin/cos table (page "DynamicNTKOperation",
+// computation process: freq = outer(positionIds_b, invFreq_b),
+// emb = cat(freq, freq), sin/cos of emb) and the compact cos/sin table that the
+// fused attention kernel reads for its on-chip rotation.
+//
+// Both are HBM-write bound: one fp32 sincos per (token, frequency), each
+// thread handles one token and 8 consecutive frequencies and writes 16-byte
+// vectors.  The duplicated half of the public table reuses the same values, so
+// columns j and j + D/2 are bit-identical by construction.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace rfa {
+
+constexpr int kMaxSeqs = 16;     // page "DynamicNTKOperation", constraints: batch <= 16
+constexpr int kMaxHalfHost = 64; // host-derived invFreq rows carried in kernel params (D <= 128)
+
+template <typename T>
+struct Pack8;  // 8 values -> the vector(s) stored for one chunk
+template <>
+struct Pack8<__half> {
+    static __device__ __forceinline__ void store(__half* dst, const float (&v)[8]) {
+        __half2 h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) h[k] = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(h);
+    }
+};
+template <>
+struct Pack8<__nv_bfloat16> {
+    static __device__ __forceinline__ void store(__nv_bfloat16* dst, const float (&v)[8]) {
+        __nv_bfloat162 h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) h[k] = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(h);
+    }
+};
+template <>
+struct Pack8<float> {
+    static __device__ __forceinline__ void store(float* dst, const float (&v)[8]) {
+        reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+};
+
+// sin/cos of the fp32 angles position * invFreq[j], j = j0 .. j0+7.
+__device__ __forceinline__ void sincos8(float position, const float* inv, float (&s)[8], float (&c)[8]) {
+    // Generic loads: `inv` points either to global memory or into the
+    // kernel's parameter block (host-derived frequencies).
+    const float4 i0 = reinterpret_cast<const float4*>(inv)[0];
+    const float4 i1 = reinterpret_cast<const float4*>(inv)[1];
+    const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sincosf(position * iv[k], &s[k], &c[k]);
+}
+
+// Public table: sin/cos [ntokens, headSize] from device positions, invFreq
+// [batch, headSize/2] and device seqLens [batch].
+template <typename OutT>
+__global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restrict__ pos,
+                                                          const float* __restrict__ inv,
+                                                          const int32_t* __restrict__ seqLens, int32_t batch,
+                                                          int32_t ntokens, int32_t headSize, OutT* __restrict__ sinOut,
+                                                          OutT* __restrict__ cosOut) {
+    __shared__ int32_t s_cum[kMaxSeqs + 1];
+    __shared__ int32_t s_ok;
+    if (threadIdx.x == 0) {
+        int64_t acc = 0;
+        int32_t ok = 1;
+        for (int32_t b = 0; b < batch; ++b) {
+            const int32_t L = seqLens[b];
+            if (L <= 0) ok = 0;
+            s_cum[b] = static_cast<int32_t>(acc);
+            acc += L;
+        }
+        s_cum[batch] = static_cast<int32_t>(acc);
+        if (acc != ntokens) ok = 0;
+        s_ok = ok;
+        if (!ok && blockIdx.x == 0) record_status(1 /* RFA_ERR_INVALID_ARG */);
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    const int32_t half = headSize >> 1;
+    const int32_t chunks = half >> 3;
+    const int64_t work = static_cast<int64_t>(ntokens) * chunks;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < work;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int32_t t = static_cast<int32_t>(w / chunks);
+        const int32_t c = static_cast<int32_t>(w - static_cast<int64_t>(t) * chunks);
+        int32_t b = 0;
+        while (b + 1 < batch && t >= s_cum[b + 1]) ++b;
+        float s[8], co[8];
+        sincos8(static_cast<float>(__ldg(pos + t)), inv + static_cast<int64_t>(b) * half + 8 * c, s, co);
+        const int64_t o = static_cast<int64_t>(t) * headSize + 8 * c;
+        Pack8<OutT>::store(sinOut + o, s);
+        Pack8<OutT>::store(sinOut + o + half, s);
+        Pack8<OutT>::store(cosOut + o, co);
+        Pack8<OutT>::store(cosOut + o + half, co);
+    }
+}
+
+// Compact table for the fused kernel: table[t][0][j] = cos, table[t][1][j] = sin,
+// j < half, fp32.  Segments: uniform_len > 0 -> segment t / uniform_len,
+// otherwise the host-known prefix sums cum[].
+struct TableArgs {
+    const int32_t* pos;
+    const float* inv_dev;  // [nseg, half] or nullptr -> inv_host
+    float* table;
+    int32_t ntokens;
+    int32_t half;
+    int32_t nseg;
+    int32_t uniform_len;
+    int32_t inv_host_rows;  // 1: one row shared by all segments; else one per segment
+    int32_t cum[kMaxSeqs + 1];
+    alignas(16) float inv_host[kMaxSeqs * kMaxHalfHost];
+};
+
+__global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__ TableArgs a) {
+    const int32_t chunks = a.half >> 3;
+    const int64_t work = static_cast<int64_t>(a.ntokens) * chunks;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < work;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int32_t t = static_cast<int32_t>(w / chunks);
+        const int32_t c = static_cast<int32_t>(w - static_cast<int64_t>(t) * chunks);
+        int32_t b;
+        if (a.uniform_len > 0) {
+            b = t / a.uniform_len;
+        } else {
+            b = 0;
+            while (b + 1 < a.nseg && t >= a.cum[b + 1]) ++b;
+        }
+        const float* inv = a.inv_dev ? a.inv_dev + static_cast<int64_t>(b) * a.half
+                                     : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
+        float s[8], co[8];
+        sincos8(static_cast<float>(__ldg(a.pos + t)), inv + 8 * c, s, co);
+        float* row = a.table + static_cast<int64_t>(t) * 2 * a.half + 8 * c;
+        Pack8<float>::store(row, co);
+        Pack8<float>::store(row + a.half, s);
+    }
+}
+
+}  // namespace rfa

@@ -1,0 +1,150 @@
+"""The C-ABI library loads on a CPU-only box, exports every symbol that
+include/rfa.h declares, and rejects invalid arguments on the host before any
+CUDA call (no GPU needed for these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rope_flashattention_b200 as rfa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rope_flashattention_b200 import build
+
+    build.build_library()
+    return rfa.load_library()
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "rfa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rfa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    syms = header_symbols()
+    assert syms == sorted(rfa.EXPORTS)
+    for name in ("rfa_rope_sincos", "rfa_fused_rope_attention"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_only_the_boundary_is_exported(lib):
+    out = os.popen(f"nm -D --defined-only {rfa.LIB_PATH}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert {s for s in exported if s.startswith("rfa_")} == set(header_symbols())
+
+
+def test_status_strings_and_version(lib):
+    assert rfa.status_string(0) == "RFA_OK"
+    assert rfa.status_string(5) == "RFA_ERR_TIMEOUT"
+    assert rfa.status_string(99) == "RFA_ERR_UNKNOWN"
+    assert lib.rfa_version() >= 100
+
+
+def _p(**kw):
+    p = rfa.AttnParams()
+    p.B, p.Hq, p.Hkv, p.S, p.D, p.layout, p.causal = 1, 2, 2, 128, 64, 0, 1
+    p.io_dtype, p.scale, p.rope_base = rfa.DT_BF16, 0.0, 10000.0
+    p.ntk_enable, p.ntk_train_len, p.ntk_factor = 0, 0, 1.0
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_params_struct_matches_c_layout():
+    assert ctypes.sizeof(rfa.AttnParams) == 64
+    assert rfa.AttnParams.rope_base.offset == 40
+    assert rfa.AttnParams.ntk_factor.offset == 56
+
+
+def test_workspace_size(lib):
+    f = lib.rfa_fused_rope_attention_workspace
+    assert f(ctypes.byref(_p()), 128) == 128 * 64 * 4
+    assert f(ctypes.byref(_p(D=128)), 1000) == (1000 * 128 * 4 + 255) // 256 * 256
+    assert f(ctypes.byref(_p(D=96)), 128) == 0          # unsupported head dim
+    assert f(ctypes.byref(_p(Hq=3, Hkv=2)), 128) == 0    # Hq % Hkv != 0
+    assert f(ctypes.byref(_p(io_dtype=0)), 128) == 0     # UNDEFINED dtype
+    assert f(ctypes.byref(_p()), 0) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(io_dtype=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(io_dtype=rfa.DT_FP32), rfa.RFA_ERR_UNSUPPORTED),
+    (dict(D=96), rfa.RFA_ERR_UNSUPPORTED),
+    (dict(D=63), rfa.RFA_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), rfa.RFA_ERR_INVALID_ARG),
+    (dict(Hkv=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(S=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(layout=7), rfa.RFA_ERR_INVALID_ARG),
+    (dict(layout=1, B=17), rfa.RFA_ERR_INVALID_ARG),
+    (dict(rope_base=-1.0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(scale=-0.5), rfa.RFA_ERR_INVALID_ARG),
+    (dict(ntk_enable=1, ntk_train_len=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(ntk_enable=1, ntk_train_len=8, ntk_factor=0.5), rfa.RFA_ERR_INVALID_ARG),
+])
+def test_attention_rejects_invalid_params(lib, kw, code):
+    rc = lib.rfa_fused_rope_attention(ctypes.byref(_p(**kw)), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
+                                      1 << 30, None)
+    assert rc == code
+
+
+def test_attention_rejects_null_and_workspace(lib):
+    p = _p()
+    f = lib.rfa_fused_rope_attention
+    assert f(ctypes.byref(p), None, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 30, None) == rfa.RFA_ERR_INVALID_ARG
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, None, FAKE, FAKE, 1 << 30, None) == rfa.RFA_ERR_INVALID_ARG
+    assert f(None, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 30, None) == rfa.RFA_ERR_INVALID_ARG
+    # misaligned q
+    assert f(ctypes.byref(p), ctypes.c_void_p((1 << 20) + 2), FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 30,
+             None) == rfa.RFA_ERR_INVALID_ARG
+    # workspace too small or missing
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 100, None) == rfa.RFA_ERR_WORKSPACE
+    assert f(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, 1 << 30, None) == rfa.RFA_ERR_WORKSPACE
+    # packed layout: host lengths required and positive
+    pt = _p(layout=1, B=2)
+    assert f(ctypes.byref(pt), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1 << 30, None) == rfa.RFA_ERR_INVALID_ARG
+    lens = (ctypes.c_int32 * 2)(5, 0)
+    assert f(ctypes.byref(pt), FAKE, FAKE, FAKE, FAKE, ctypes.cast(lens, ctypes.c_void_p), None, FAKE, FAKE, 1 << 30,
+             None) == rfa.RFA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("batch,ntok,hs,dt,code", [
+    (1, 128, 64, rfa.DT_UNDEFINED, rfa.RFA_ERR_INVALID_ARG),   # UNDEFINED is not usable
+    (1, 128, 48, rfa.DT_FP16, rfa.RFA_ERR_INVALID_ARG),        # headSize % 32
+    (1, 128, 4096, rfa.DT_FP16, rfa.RFA_ERR_INVALID_ARG),      # headSize <= 2048
+    (17, 128, 64, rfa.DT_FP16, rfa.RFA_ERR_INVALID_ARG),       # batch <= 16
+    (0, 128, 64, rfa.DT_FP16, rfa.RFA_ERR_INVALID_ARG),
+    (1, 256001, 64, rfa.DT_FP16, rfa.RFA_ERR_INVALID_ARG),     # ntokens <= 256000
+    (1, 0, 64, rfa.DT_FP16, rfa.RFA_ERR_INVALID_ARG),
+    (1, 128, 64, 9, rfa.RFA_ERR_INVALID_ARG),
+])
+def test_sincos_rejects_invalid_args(lib, batch, ntok, hs, dt, code):
+    rc = lib.rfa_rope_sincos(FAKE, FAKE, FAKE, batch, ntok, hs, dt, FAKE, FAKE, None)
+    assert rc == code
+
+
+def test_sincos_rejects_null(lib):
+    assert lib.rfa_rope_sincos(None, FAKE, FAKE, 1, 8, 64, rfa.DT_FP16, FAKE, FAKE, None) == rfa.RFA_ERR_INVALID_ARG
+    assert lib.rfa_rope_sincos(FAKE, FAKE, FAKE, 1, 8, 64, rfa.DT_FP16, None, FAKE, None) == rfa.RFA_ERR_INVALID_ARG
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "rope_flashattention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.lower().replace("the oracle", ""), f

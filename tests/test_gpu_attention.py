@@ -1,0 +1,202 @@
+"""GPU parity of rfa_fused_rope_attention against the fp64 oracle.
+
+Each case runs the CUDA path through the C ABI on seeded inputs and compares
+it element by element with the oracle: in full at sizes that span several
+128-row tiles and a ragged tail, and on seeded row samples at the full
+workload sizes.  Bar (fp16/bf16 I/O): max abs error <= 2e-2 and relative
+Frobenius error <= 5e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+MAX_ABS = 2e-2
+REL_FRO = 5e-3
+
+
+@pytest.fixture(scope="module")
+def rfa():
+    import rope_flashattention_b200 as m
+
+    m.load_library()
+    return m
+
+
+def _inv_rows(B, D, base, lens=None, ntk=None):
+    rows = []
+    for b in range(B):
+        bb = base
+        if ntk is not None:
+            L, f = ntk
+            bb = oracle.ntk_base(base, D, int(lens[b]), L, f)
+        rows.append(oracle.inv_freq(bb, D))
+    return np.stack(rows)
+
+
+def _compare(got, ref):
+    got = np.asarray(got, np.float64)
+    assert np.all(np.isfinite(got))
+    err = np.abs(got - ref)
+    fro = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err.max() <= MAX_ABS, f"max abs {err.max():.3e}"
+    assert fro <= REL_FRO, f"rel fro {fro:.3e}"
+    return err.max(), fro
+
+
+def run_bnsd(rfa, B, Hq, Hkv, S, D, *, seed=0, base=10000.0, causal=True, dtype=torch.bfloat16, ntk=None,
+             pos=None, inv=None, scale=None):
+    q = workloads.randn16((B, Hq, S, D), seed, dtype)
+    k = workloads.randn16((B, Hkv, S, D), seed + 1, dtype)
+    v = workloads.randn16((B, Hkv, S, D), seed + 2, dtype)
+    if pos is None:
+        pos = torch.arange(S, dtype=torch.int32).repeat(B, 1).contiguous()
+    kw = dict(layout="BNSD", causal=causal, rope_base=base, scale=scale)
+    if ntk is not None:
+        kw.update(ntk_train_len=ntk[0], ntk_factor=ntk[1])
+    if inv is not None:
+        kw["inv_freq"] = inv.cuda()
+    out = rfa.fused_rope_attention(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), **kw)
+    assert rfa.get_device_status() == 0
+    inv_rows = inv.double().numpy() if inv is not None else _inv_rows(B, D, base, [S] * B, ntk)
+    return q, k, v, pos, inv_rows, out.float().cpu().numpy()
+
+
+def full_bnsd(rfa, B, Hq, Hkv, S, D, **kw):
+    q, k, v, pos, inv, got = run_bnsd(rfa, B, Hq, Hkv, S, D, **kw)
+    ref = oracle.attention_full(q, k, v, pos.numpy(), inv, causal=kw.get("causal", True), scale=kw.get("scale"))
+    return _compare(got, ref)
+
+
+def test_tiny_workload(rfa):
+    w = workloads.TINY
+    full_bnsd(rfa, w.B, w.Hq, w.Hkv, w.S, w.D, seed=w.seed, base=w.rope_base)
+
+
+@pytest.mark.parametrize("S", [1, 5, 127, 128, 129, 300, 640])
+def test_ragged_lengths_d128_gqa(rfa, S):
+    full_bnsd(rfa, 2, 4, 2, S, 128, seed=S)
+
+
+@pytest.mark.parametrize("S", [1, 77, 256, 383])
+def test_ragged_lengths_d64(rfa, S):
+    full_bnsd(rfa, 1, 6, 3, S, 64, seed=100 + S)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_non_causal(rfa, D):
+    full_bnsd(rfa, 2, 2, 1, 333, D, seed=7, causal=False)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp16_io(rfa, D):
+    full_bnsd(rfa, 1, 4, 4, 260, D, seed=9, dtype=torch.float16)
+
+
+def test_mqa_and_scale(rfa):
+    full_bnsd(rfa, 1, 8, 1, 200, 128, seed=13, scale=0.05)
+
+
+def test_ntk_scaling_beyond_train_len(rfa):
+    full_bnsd(rfa, 1, 2, 1, 600, 128, seed=15, ntk=(256, 2.0))
+
+
+def test_explicit_inv_freq_and_arbitrary_positions(rfa):
+    B, S, D = 2, 290, 128
+    g = workloads.gen(21)
+    pos = torch.randint(-100000, 200000, (B, S), generator=g, dtype=torch.int32)
+    inv = torch.rand(B, D // 2, generator=g, dtype=torch.float32)
+    full_bnsd(rfa, B, 4, 2, S, D, seed=22, pos=pos, inv=inv)
+
+
+def test_position_shift_invariance(rfa):
+    """Rotated scores depend only on position differences: shifting every
+    position by a constant leaves the output unchanged (within tolerance)."""
+    B, Hq, Hkv, S, D = 1, 2, 1, 256, 128
+    outs = []
+    for c in (0, 1000):
+        pos = (torch.arange(S, dtype=torch.int32) + c).repeat(B, 1).contiguous()
+        outs.append(run_bnsd(rfa, B, Hq, Hkv, S, D, seed=31, pos=pos)[-1])
+    d = np.abs(outs[0] - outs[1])
+    assert d.max() <= MAX_ABS
+
+
+def _packed(rfa, lens, Hq, Hkv, D, *, seed, base=10000.0, random_inv=False, ntk=None, rows=None, dtype=torch.bfloat16):
+    T = int(sum(lens))
+    q = workloads.randn16((T, Hq, D), seed, dtype)
+    k = workloads.randn16((T, Hkv, D), seed + 1, dtype)
+    v = workloads.randn16((T, Hkv, D), seed + 2, dtype)
+    pos = torch.cat([torch.arange(int(n), dtype=torch.int32) for n in lens])
+    kw = dict(layout="TND", seq_lens=[int(x) for x in lens], rope_base=base)
+    inv_t = None
+    if random_inv:
+        inv_t = torch.rand(len(lens), D // 2, generator=workloads.gen(seed + 3), dtype=torch.float32)
+        kw["inv_freq"] = inv_t.cuda()
+    if ntk is not None:
+        kw.update(ntk_train_len=ntk[0], ntk_factor=ntk[1])
+    out = rfa.fused_rope_attention(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), **kw)
+    assert rfa.get_device_status() == 0
+    got = out.float().cpu().numpy()
+    inv = inv_t.double().numpy() if random_inv else _inv_rows(len(lens), D, base, lens, ntk)
+    if rows is None:
+        ref = oracle.attention_full(q, k, v, pos.numpy(), inv, layout=oracle.TND, seq_lens=lens)
+        return _compare(got, ref)
+    ref = oracle.attention_rows(q, k, v, pos.numpy(), inv, rows, layout=oracle.TND, seq_lens=lens)
+    t0 = np.concatenate([[0], np.cumsum(lens)])
+    return _compare(got[t0[rows[:, 0]] + rows[:, 2], rows[:, 1]], ref)
+
+
+def test_packed_ragged_sequences(rfa):
+    _packed(rfa, [1, 127, 128, 129, 300, 5], 4, 2, 128, seed=40)
+
+
+def test_packed_d64_random_inv(rfa):
+    _packed(rfa, [64, 1, 200], 2, 2, 64, seed=50, random_inv=True)
+
+
+def test_packed_per_sequence_ntk(rfa):
+    _packed(rfa, [100, 700, 300], 4, 1, 128, seed=60, ntk=(256, 2.0))
+
+
+# ---------------------------------------------------------------- full workload sizes, sampled rows
+def _sample_rows(B, Hq, lens, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for _ in range(n):
+        b = int(rng.integers(B))
+        rows.append((b, int(rng.integers(Hq)), int(rng.integers(lens[b]))))
+    for b in range(B):  # first/last rows of each sequence and of its last tile
+        L = int(lens[b])
+        for i in {0, L - 1, max(0, (L - 1) // 128 * 128), min(L - 1, 127)}:
+            rows.append((b, int(rng.integers(Hq)), i))
+    return np.array(rows, np.int32)
+
+
+@pytest.mark.parametrize("key", ["qwen7b", "gqa8k", "ntk16k"])
+def test_full_size_bnsd_sampled(rfa, key):
+    w = workloads.BY_KEY[key]
+    q, k, v = workloads.make_qkv(w)
+    pos = workloads.positions(w)
+    kw = dict(layout="BNSD", rope_base=w.rope_base)
+    ntk = None
+    if w.ntk_train_len:
+        kw.update(ntk_train_len=w.ntk_train_len, ntk_factor=w.ntk_factor)
+        ntk = (w.ntk_train_len, w.ntk_factor)
+    out = rfa.fused_rope_attention(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), **kw)
+    assert rfa.get_device_status() == 0
+    got = out.float().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    rows = _sample_rows(w.B, w.Hq, [w.S] * w.B, 96, seed=w.seed)
+    inv = _inv_rows(w.B, w.D, w.rope_base, [w.S] * w.B, ntk)
+    ref = oracle.attention_rows(q, k, v, pos.numpy(), inv, rows)
+    _compare(got[rows[:, 0], rows[:, 1], rows[:, 2]], ref)
+
+
+def test_full_size_packed_sampled(rfa):
+    w = workloads.PACKED
+    lens = workloads.seq_lengths(w)
+    rows = _sample_rows(w.B, w.Hq, lens, 96, seed=w.seed)
+    _packed(rfa, lens, w.Hq, w.Hkv, w.D, seed=w.seed, random_inv=True, rows=rows)
