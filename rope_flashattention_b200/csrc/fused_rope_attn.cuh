@@ -12,21 +12,23 @@
 //
 // One CTA = one work item (sequence, query head, 128-row query tile).  Warp roles:
 //   warps 0-3  softmax warpgroup: thread t owns query row t of the tile (TMEM
-//              lane t).  Reads S from TMEM, masks, keeps the running max and
-//              sum, rescales O in TMEM only when the max grows by > 2^8,
-//              writes P (bf16/fp16) to shared memory, and at the end
-//              normalises O and stores the output row.
+//              lane t).  Loads S from TMEM, masks, keeps the running max and
+//              sum, writes P (bf16/fp16) back into the same TMEM columns,
+//              rescales O in TMEM only when its max grows by > 2^8, and at the
+//              end normalises O and stores the output row.
 //   warps 4-7  RoPE warpgroup: rotates the Q tile once and every K tile in
-//              place in the 128B-swizzled shared-memory layout.  Element i and
+//              place in the 128B-swizzled shared-memory layout, reading the
+//              cos/sin rows that TMA staged next to the tile.  Element i and
 //              its rotate-half partner i + D/2 sit at the same offset of two
 //              swizzle atoms (D = 128) or in chunks c and c ^ 4 of one atom
 //              (D = 64), so each thread rotates 8 pairs per 2 x 16 B.
-//   warp 8     TMA producer: Q once, K/V tiles through a kStages ring.
-//   warp 9     tcgen05 issuer (one thread): S = Q'K'^T into one of two TMEM S
-//              buffers, O += P V into TMEM; completion signalled by
-//              tcgen05.commit onto mbarriers.  Also allocates TMEM.
-// The issue order QK(j), PV(j-1) lets the tensor core compute the next score
-// tile while the softmax warpgroup works on the current one.
+//   warp 8     TMA producer: Q (+ its cos/sin rows) once, then K (+ cos/sin)
+//              and V tiles through a kStages ring.
+//   warp 9     tcgen05 issuer (one thread) and TMEM owner.  S_j = Q'K_j'^T goes
+//              to TMEM buffer j % 3; O += P_j V_j reads P_j from that buffer
+//              (A operand in TMEM) and V_j from shared memory.  QK runs two
+//              tiles ahead of PV so the softmax never waits for its scores.
+// Completion of every async step is tracked by mbarriers; each wait is bounded.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,37 +46,39 @@ constexpr int kAttnThreads = 320;
 constexpr int kRopeWarp0 = 4;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kSBufs = 3;                  // S/P buffers in TMEM
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
 struct AttnArgs {
     void* out;
-    const float* table;  // [T][2][D/2]: cos then sin, fp32
-    int32_t layout;      // 0 BNSD, 1 TND
+    int32_t layout;  // 0 BNSD, 1 TND
     int32_t B, Hq, Hkv, G;
-    int32_t S;           // BNSD sequence length
+    int32_t S;       // BNSD sequence length
     int32_t causal;
-    float scale_log2;    // softmax scale * log2(e)
+    float scale_log2;  // softmax scale * log2(e)
     int32_t n_items;
-    // TND: sequences sorted by query-tile count, descending
+    // TND: sequences sorted by length, descending; seg_item0[k] = first work item of sequence k
     int32_t nseg;
     int32_t seg_start[16];
     int32_t seg_len[16];
     int32_t seg_tiles[16];
+    int32_t seg_item0[17];
 };
 
 template <int D>
 struct AttnCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
-    static constexpr int kAtoms = D / 64;                    // 128-byte swizzle atoms across a row
-    static constexpr int kAtomBytes = kBlockM * 128;         // one atom column of a 128-row tile
-    static constexpr int kTileBytes = kBlockM * D * 2;       // Q, K or V tile
+    static constexpr int kAtoms = D / 64;                 // 128-byte swizzle atoms across a row
+    static constexpr int kAtomBytes = kBlockM * 128;      // one atom column of a 128-row tile
+    static constexpr int kTileBytes = kBlockM * D * 2;    // Q, K or V tile
+    static constexpr int kTabBytes = kBlockM * D * 2;     // cos/sin rows of a tile: D/2 fp16 pairs per row
+    static constexpr int kTabBoxes = D / 64;              // 128-byte boxes of 32 (cos, sin) pairs
     static constexpr int kStages = (D == 64) ? 4 : 2;
-    static constexpr int kPBytes = kBlockM * kBlockN * 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kTileBytes;
-    static constexpr int kOffP = kOffV + kStages * kTileBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
+    static constexpr int kOffT = kOffV + kStages * kTileBytes;
+    static constexpr int kOffBar = kOffT + kStages * kTabBytes;
     // barrier indices
     static constexpr int kBarQFull = 0, kBarQReady = 1;
     static constexpr int kBarKFull = 2;
@@ -82,64 +86,52 @@ struct AttnCfg {
     static constexpr int kBarKReady = kBarVFull + kStages;
     static constexpr int kBarKEmpty = kBarKReady + kStages;
     static constexpr int kBarVEmpty = kBarKEmpty + kStages;
-    static constexpr int kBarSFull = kBarVEmpty + kStages;   // 2
-    static constexpr int kBarSEmpty = kBarSFull + 2;         // 2
-    static constexpr int kBarPFull = kBarSEmpty + 2;
-    static constexpr int kBarPVDone = kBarPFull + 1;
-    static constexpr int kBarMmaFin = kBarPVDone + 1;
+    static constexpr int kBarSFull = kBarVEmpty + kStages;  // kSBufs
+    static constexpr int kBarPFull = kBarSFull + kSBufs;    // kSBufs
+    static constexpr int kBarBufFree = kBarPFull + kSBufs;  // kSBufs: PV of that buffer done
+    static constexpr int kBarMmaFin = kBarBufFree + kSBufs;
     static constexpr int kNumBars = kBarMmaFin + 1;
     static constexpr int kOffAbort = kOffBar + 8 * kNumBars;
     static constexpr int kOffTmemSlot = kOffAbort + 16;
     static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack for 1024-byte alignment
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS = 0;    // S buffers at columns 0 and 128
-    static constexpr uint32_t kColO = 256;  // O at columns 256 .. 256+D
+    static constexpr uint32_t kColO = kSBufs * kBlockN;  // S/P buffers at 0, 128, 256; O at 384
+    static_assert(kColO + D <= kTmemCols, "TMEM budget");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct WorkItem {
     int32_t tok0;  // first token of the sequence (BNSD: seq * S)
-    int32_t seq;   // BNSD batch index (unused for TND addressing)
+    int32_t seq;   // BNSD batch index
     int32_t L;     // sequence length
     int32_t h;     // query head
     int32_t qt;    // query tile index within the sequence
 };
 
-// Longest-first order: all items of the highest query-tile index come first.
+// Head-major order (all query tiles of one head are neighbours, so the CTAs
+// resident at one time share K/V tiles through L2), largest tile first within
+// a head; packed sequences longest first.
 __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     WorkItem w;
     if (a.layout == 0) {
         const int32_t nqt = (a.S + kBlockM - 1) / kBlockM;
-        const int32_t per = a.B * a.Hq;
-        const int32_t t = x / per;
-        const int32_t r = x - t * per;
-        w.qt = nqt - 1 - t;
-        w.seq = r / a.Hq;
-        w.h = r - w.seq * a.Hq;
+        const int32_t bh = x / nqt;
+        w.qt = nqt - 1 - (x - bh * nqt);
+        w.seq = bh / a.Hq;
+        w.h = bh - w.seq * a.Hq;
         w.tok0 = w.seq * a.S;
         w.L = a.S;
         return w;
     }
-    int32_t rem = x;
-    for (int32_t k = 0; k < a.nseg; ++k) {
-        const int32_t nk = a.seg_tiles[k];
-        const int32_t nk1 = (k + 1 < a.nseg) ? a.seg_tiles[k + 1] : 0;
-        const int32_t width = (k + 1) * a.Hq;  // items per query-tile index in this band
-        const int32_t cnt = (nk - nk1) * width;
-        if (rem < cnt) {
-            const int32_t tt = rem / width;
-            const int32_t r = rem - tt * width;
-            const int32_t s = r / a.Hq;
-            w.qt = nk - 1 - tt;
-            w.h = r - s * a.Hq;
-            w.seq = s;
-            w.tok0 = a.seg_start[s];
-            w.L = a.seg_len[s];
-            return w;
-        }
-        rem -= cnt;
-    }
-    w.qt = -1;  // unreachable for x < n_items
-    w.seq = w.h = w.tok0 = w.L = 0;
+    int32_t s = 0;
+    while (s + 1 < a.nseg && x >= a.seg_item0[s + 1]) ++s;
+    const int32_t r = x - a.seg_item0[s];
+    const int32_t nt = a.seg_tiles[s];
+    w.h = r / nt;
+    w.qt = nt - 1 - (r - w.h * nt);
+    w.seq = s;
+    w.tok0 = a.seg_start[s];
+    w.L = a.seg_len[s];
     return w;
 }
 
@@ -168,55 +160,57 @@ struct IoT<true> {
     static constexpr uint32_t kFmt = 0;
 };
 
+__device__ __forceinline__ float2 h2f2(uint32_t u) { return __half22float2(*reinterpret_cast<const __half2*>(&u)); }
+
 // Rotate 8 rotate-half pairs held in two 16-byte chunks (x1: dims i..i+7,
-// x2: dims i+D/2..i+D/2+7), angles from cos[0..7], sin[0..7].
+// x2: dims i+D/2..i+D/2+7).  t0/t1 hold the 8 (cos, sin) fp16 pairs.
 template <bool kFP16>
-__device__ __forceinline__ void rotate8(uint4& x1, uint4& x2, const float* cs, const float* sn) {
+__device__ __forceinline__ void rotate8(uint4& x1, uint4& x2, const uint4& t0, const uint4& t1) {
     uint32_t* a = reinterpret_cast<uint32_t*>(&x1);
     uint32_t* b = reinterpret_cast<uint32_t*>(&x2);
+    const uint32_t cs[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const float2 u = IoT<kFP16>::unpack(a[k]);
         const float2 v = IoT<kFP16>::unpack(b[k]);
-        const float c0 = cs[2 * k], c1 = cs[2 * k + 1], s0 = sn[2 * k], s1 = sn[2 * k + 1];
-        const float y10 = u.x * c0 - v.x * s0, y11 = u.y * c1 - v.y * s1;
-        const float y20 = v.x * c0 + u.x * s0, y21 = v.y * c1 + u.y * s1;
+        const float2 e0 = h2f2(cs[2 * k]);      // (cos, sin) of dim 2k
+        const float2 e1 = h2f2(cs[2 * k + 1]);  // (cos, sin) of dim 2k+1
+        const float y10 = u.x * e0.x - v.x * e0.y, y11 = u.y * e1.x - v.y * e1.y;
+        const float y20 = v.x * e0.x + u.x * e0.y, y21 = v.y * e1.x + u.y * e1.y;
         a[k] = IoT<kFP16>::pack(y10, y11);
         b[k] = IoT<kFP16>::pack(y20, y21);
     }
 }
 
-// Rotate the first `rows` rows of a 128-row tile in shared memory (128B
-// swizzle: 16-byte chunk c of row r sits at r*128 + ((c ^ (r&7)) << 4) within
-// its atom).  table_row0 points at the cos/sin row of the tile's first token.
+// Rotate the first `rows` rows of a 128-row tile in shared memory with the
+// cos/sin rows staged at `tab`.  128B swizzle: 16-byte chunk c of row r sits at
+// r*128 + ((c ^ (r&7)) << 4) within its 128-row atom.  The table's atoms hold
+// 32 (cos, sin) pairs per row, 4 pairs per chunk.
 template <int D, bool kFP16>
-__device__ __forceinline__ void rope_tile(uint32_t tile, int32_t rows, const float* __restrict__ table_row0,
-                                          int32_t rt) {
-    constexpr int kHalf = D / 2;
-    constexpr int kPairsPerRow = kHalf / 8;             // 16-byte chunk pairs per row
+__device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t rows, int32_t rt) {
+    constexpr int kPairsPerRow = D / 16;  // 16-byte chunk pairs per row
     constexpr int kIters = kBlockM * kPairsPerRow / 128;
-#pragma unroll 2
+#pragma unroll 4
     for (int it = 0; it < kIters; ++it) {
         const int task = rt + 128 * it;
         const int r = task / kPairsPerRow;
         const int cp = task % kPairsPerRow;
         if (r >= rows) continue;
-        const float* row = table_row0 + static_cast<int64_t>(r) * D;  // [cos(half) | sin(half)]
-        const float4* c4 = reinterpret_cast<const float4*>(row + 8 * cp);
-        const float4* s4 = reinterpret_cast<const float4*>(row + kHalf + 8 * cp);
-        const float4 ca = __ldg(c4), cb = __ldg(c4 + 1), sa = __ldg(s4), sb = __ldg(s4 + 1);
-        const float cs[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-        const float sn[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+        const uint32_t sw = static_cast<uint32_t>(r & 7);
         uint32_t o1, o2;
         if constexpr (D == 128) {
-            o1 = tile + r * 128 + ((cp ^ (r & 7)) << 4);
+            o1 = tile + r * 128 + ((cp ^ sw) << 4);
             o2 = o1 + AttnCfg<D>::kAtomBytes;
         } else {
-            o1 = tile + r * 128 + ((cp ^ (r & 7)) << 4);
-            o2 = tile + r * 128 + (((cp + 4) ^ (r & 7)) << 4);
+            o1 = tile + r * 128 + ((cp ^ sw) << 4);
+            o2 = tile + r * 128 + (((cp + 4) ^ sw) << 4);
         }
+        const uint32_t tb = tab + (cp >> 2) * AttnCfg<D>::kAtomBytes + r * 128;
+        const uint32_t tc = static_cast<uint32_t>((cp & 3) * 2);
+        const uint4 t0 = lds128(tb + ((tc ^ sw) << 4));
+        const uint4 t1 = lds128(tb + (((tc + 1) ^ sw) << 4));
         uint4 x1 = lds128(o1), x2 = lds128(o2);
-        rotate8<kFP16>(x1, x2, cs, sn);
+        rotate8<kFP16>(x1, x2, t0, t1);
         sts128(o1, x1);
         sts128(o2, x2);
     }
@@ -234,10 +228,22 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
     }
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, A = P in TMEM.
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 template <int D, bool kFP16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     fused_rope_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+                               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmT,
+                               const __grid_constant__ AttnArgs a) {
     using C = AttnCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -263,12 +269,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(bar(C::kBarKEmpty + s), 1);
             mbar_init(bar(C::kBarVEmpty + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kSBufs; ++b) {
             mbar_init(bar(C::kBarSFull + b), 1);
-            mbar_init(bar(C::kBarSEmpty + b), 4);
+            mbar_init(bar(C::kBarPFull + b), 4);
+            mbar_init(bar(C::kBarBufFree + b), 1);
         }
-        mbar_init(bar(C::kBarPFull), 4);
-        mbar_init(bar(C::kBarPVDone), 1);
         mbar_init(bar(C::kBarMmaFin), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -288,41 +293,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmT);
             const bool bnsd = (a.layout == 0);
             const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h) : w.h;
             const int32_t kvplane = bnsd ? (w.seq * a.Hkv + kvh) : kvh;
-            mbar_expect_tx(bar(C::kBarQFull), C::kTileBytes);
-            for (int at = 0; at < C::kAtoms; ++at) {
-                if (bnsd)
-                    tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64,
-                                w.qt * kBlockM, qplane);
-                else
-                    tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64, qplane,
-                                w.tok0 + w.qt * kBlockM);
-            }
+            auto load_tile = [&](const CUtensorMap* m, uint32_t dst, uint32_t b, int32_t plane, int32_t row0) {
+                for (int at = 0; at < C::kAtoms; ++at) {
+                    if (bnsd)
+                        tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, row0, plane);
+                    else
+                        tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, plane, w.tok0 + row0);
+                }
+            };
+            auto load_tab = [&](uint32_t dst, uint32_t b, int32_t row0) {
+                for (int bx = 0; bx < C::kTabBoxes; ++bx)
+                    tma_load_3d(dst + bx * C::kAtomBytes, &tmT, b, bx * 32, w.tok0 + row0, 0);
+            };
+            // Q and its cos/sin rows; the rows go to table stage 1, free until K tile 1.
+            mbar_expect_tx(bar(C::kBarQFull), C::kTileBytes + C::kTabBytes);
+            load_tile(&tmQ, sbase + C::kOffQ, bar(C::kBarQFull), qplane, w.qt * kBlockM);
+            load_tab(sbase + C::kOffT + 1 * C::kTabBytes, bar(C::kBarQFull), w.qt * kBlockM);
             int32_t issued_k = 0, issued_v = 0;
             for (int32_t j = 0; j < n_kv; ++j) {
                 const int s = j % C::kStages;
                 const uint32_t u = static_cast<uint32_t>(j / C::kStages);
+                if (j == 1 && !mbar_wait(bar(C::kBarQReady), 0, abort_flag)) break;  // Q's rows consumed
                 if (u > 0 && !mbar_wait(bar(C::kBarKEmpty + s), (u - 1) & 1u, abort_flag)) break;
-                mbar_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
-                for (int at = 0; at < C::kAtoms; ++at) {
-                    const uint32_t dst = sbase + C::kOffK + s * C::kTileBytes + at * C::kAtomBytes;
-                    if (bnsd)
-                        tma_load_3d(dst, &tmK, bar(C::kBarKFull + s), at * 64, j * kBlockN, kvplane);
-                    else
-                        tma_load_3d(dst, &tmK, bar(C::kBarKFull + s), at * 64, kvplane, w.tok0 + j * kBlockN);
-                }
+                mbar_expect_tx(bar(C::kBarKFull + s), C::kTileBytes + C::kTabBytes);
+                load_tile(&tmK, sbase + C::kOffK + s * C::kTileBytes, bar(C::kBarKFull + s), kvplane, j * kBlockN);
+                load_tab(sbase + C::kOffT + s * C::kTabBytes, bar(C::kBarKFull + s), j * kBlockN);
                 issued_k = j + 1;
                 if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) break;
                 mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-                for (int at = 0; at < C::kAtoms; ++at) {
-                    const uint32_t dst = sbase + C::kOffV + s * C::kTileBytes + at * C::kAtomBytes;
-                    if (bnsd)
-                        tma_load_3d(dst, &tmV, bar(C::kBarVFull + s), at * 64, j * kBlockN, kvplane);
-                    else
-                        tma_load_3d(dst, &tmV, bar(C::kBarVFull + s), at * 64, kvplane, w.tok0 + j * kBlockN);
-                }
+                load_tile(&tmV, sbase + C::kOffV + s * C::kTileBytes, bar(C::kBarVFull + s), kvplane, j * kBlockN);
                 issued_v = j + 1;
             }
             // Drain: every issued copy must have landed before the CTA exits.
@@ -337,48 +340,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_f16(IoT<kFP16>::kFmt, 0, 0, kBlockM, kBlockN);
             constexpr uint32_t kIdescPV = idesc_f16(IoT<kFP16>::kFmt, 0, 1, kBlockM, D);
-            bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag);
+            auto issue_qk = [&](int32_t j) -> bool {
+                const int s = j % C::kStages;
+                const int b = j % kSBufs;
+                if (!mbar_wait(bar(C::kBarKReady + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag))
+                    return false;
+                // the buffer held P_{j-3}: PV_{j-3} must have read it
+                if (j >= kSBufs && !mbar_wait(bar(C::kBarBufFree + b), static_cast<uint32_t>(j / kSBufs - 1) & 1u,
+                                              abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t kbase = sbase + C::kOffK + s * C::kTileBytes;
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t koff = (k >> 2) * C::kAtomBytes + (k & 3) * 32;
+                    const uint64_t ad = smem_desc_sw128(sbase + C::kOffQ + koff, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(kbase + koff, 16, 1024);
+                    umma_ss(tmem + b * kBlockN, ad, bd, kIdescQK, k > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(C::kBarSFull + b));
+                tc_commit(bar(C::kBarKEmpty + s));
+                return true;
+            };
             auto issue_pv = [&](int32_t i) -> bool {
                 const int s = i % C::kStages;
-                const uint32_t u = static_cast<uint32_t>(i / C::kStages);
-                if (!mbar_wait(bar(C::kBarPFull), static_cast<uint32_t>(i) & 1u, abort_flag)) return false;
-                if (!mbar_wait(bar(C::kBarVFull + s), u & 1u, abort_flag)) return false;
+                const int b = i % kSBufs;
+                if (!mbar_wait(bar(C::kBarPFull + b), static_cast<uint32_t>(i / kSBufs) & 1u, abort_flag))
+                    return false;
+                if (!mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(i / C::kStages) & 1u, abort_flag))
+                    return false;
                 tc_fence_after();
                 const uint32_t vbase = sbase + C::kOffV + s * C::kTileBytes;
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k) {
-                    const uint64_t ad = smem_desc_sw128(sbase + C::kOffP + (k >> 2) * C::kAtomBytes + (k & 3) * 32,
-                                                        16, 1024);
+                    // P_i: 128 x 128 fp16/bf16 packed two per 32-bit column -> 8 columns per K=16 step
                     const uint64_t bd = smem_desc_sw128(vbase + k * 16 * 128, C::kAtomBytes, 1024);
-                    umma_ss(tmem + C::kColO, ad, bd, kIdescPV, (i > 0 || k > 0) ? 1u : 0u);
+                    umma_ts(tmem + C::kColO, tmem + b * kBlockN + k * 8, bd, kIdescPV, (i > 0 || k > 0) ? 1u : 0u);
                 }
-                tc_commit(bar(C::kBarPVDone));
+                tc_commit(bar(C::kBarBufFree + b));
                 tc_commit(bar(C::kBarVEmpty + s));
                 return true;
             };
+            bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
+                ok = issue_qk(0);
+                if (ok && n_kv > 1) ok = issue_qk(1);
                 for (int32_t j = 0; j < n_kv && ok; ++j) {
-                    const int s = j % C::kStages;
-                    const uint32_t u = static_cast<uint32_t>(j / C::kStages);
-                    const int b = j & 1;
-                    if (!mbar_wait(bar(C::kBarKReady + s), u & 1u, abort_flag)) { ok = false; break; }
-                    if (j >= 2 && !mbar_wait(bar(C::kBarSEmpty + b), static_cast<uint32_t>((j >> 1) - 1) & 1u,
-                                             abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t kbase = sbase + C::kOffK + s * C::kTileBytes;
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t koff = (k >> 2) * C::kAtomBytes + (k & 3) * 32;
-                        const uint64_t ad = smem_desc_sw128(sbase + C::kOffQ + koff, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(kbase + koff, 16, 1024);
-                        umma_ss(tmem + C::kColS + b * kBlockN, ad, bd, kIdescQK, k > 0 ? 1u : 0u);
-                    }
-                    tc_commit(bar(C::kBarSFull + b));
-                    tc_commit(bar(C::kBarKEmpty + s));
-                    if (j >= 1) ok = issue_pv(j - 1);
+                    ok = issue_pv(j);
+                    if (ok && j + 2 < n_kv) ok = issue_qk(j + 2);
                 }
-                if (ok) issue_pv(n_kv - 1);
             }
             tc_commit(bar(C::kBarMmaFin));
             mbar_wait_drain(bar(C::kBarMmaFin), 0);
@@ -386,11 +397,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (warp >= kRopeWarp0) {
         // ------------------------------------------------------------ RoPE warpgroup
         const int32_t rt = threadIdx.x - kRopeWarp0 * 32;
-        const float* table = a.table;
         if (mbar_wait(bar(C::kBarQFull), 0, abort_flag)) {
             const int32_t q0 = w.qt * kBlockM;
-            rope_tile<D, kFP16>(sbase + C::kOffQ, min(kBlockM, w.L - q0),
-                                table + static_cast<int64_t>(w.tok0 + q0) * D, rt);
+            rope_tile<D, kFP16>(sbase + C::kOffQ, sbase + C::kOffT + 1 * C::kTabBytes, min(kBlockM, w.L - q0), rt);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::kBarQReady));
@@ -399,8 +408,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint32_t u = static_cast<uint32_t>(j / C::kStages);
                 if (!mbar_wait(bar(C::kBarKFull + s), u & 1u, abort_flag)) break;
                 const int32_t k0 = j * kBlockN;
-                rope_tile<D, kFP16>(sbase + C::kOffK + s * C::kTileBytes, min(kBlockN, w.L - k0),
-                                    table + static_cast<int64_t>(w.tok0 + k0) * D, rt);
+                rope_tile<D, kFP16>(sbase + C::kOffK + s * C::kTileBytes, sbase + C::kOffT + s * C::kTabBytes,
+                                    min(kBlockN, w.L - k0), rt);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::kBarKReady + s));
@@ -417,18 +426,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool ok = true;
         uint32_t sr[4][32];
         for (int32_t j = 0; j < n_kv; ++j) {
-            const int b = j & 1;
+            const int b = j % kSBufs;
             // tcgen05.ld/st are warp-collective: every decision below is warp-uniform.
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + b), static_cast<uint32_t>(j >> 1) & 1u,
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + b), static_cast<uint32_t>(j / kSBufs) & 1u,
                                                    abort_flag))) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sc = tmem + lane_off + C::kColS + b * kBlockN;
+            const uint32_t sc = tmem + lane_off + b * kBlockN;
 #pragma unroll
             for (int q = 0; q < 4; ++q) tmem_ld32(sc + q * 32, sr[q]);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarSEmpty + b));
 
             // mask: keys [kv0, kv0 + lim) are visible to this row
             const int32_t kv0 = j * kBlockN;
@@ -451,12 +457,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             const float m_new = fmaxf(m, mx * sl2);
             if (j > 0) {
-                // PV(j-1) must be done: it reads the P buffer and writes O.
-                if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(j - 1) & 1u,
-                                                       abort_flag))) { ok = false; break; }
-                tc_fence_after();
                 const bool need = m_new > m + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, need)) {
+                    // O holds the sum up to tile j-1 only once PV_{j-1} is done.
+                    const int pb = (j - 1) % kSBufs;
+                    if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarBufFree + pb),
+                                                           static_cast<uint32_t>((j - 1) / kSBufs) & 1u,
+                                                           abort_flag))) { ok = false; break; }
+                    tc_fence_after();
                     const float alpha = need ? ex2(m - m_new) : 1.0f;
                     l *= alpha;
 #pragma unroll 1
@@ -468,42 +476,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
                         tmem_st32(tmem + lane_off + C::kColO + q * 32, o);
                     }
-                    tmem_wait_st();
                     if (need) m = m_new;
                 }
             } else {
                 m = m_new;
             }
             const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-            const uint32_t prow = sbase + C::kOffP + row * 128;
+            // P_j overwrites the first 64 columns of S_j (already in registers).
 #pragma unroll
-            for (int cc = 0; cc < kBlockN / 8; ++cc) {
-                float p[8];
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pw[32];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    p[e] = ex2(fmaf(__uint_as_float(sr[cc >> 2][(cc & 3) * 8 + e]), sl2, neg_m));
-                    l += p[e];
+                for (int c2 = 0; c2 < 32; ++c2) {
+                    const int col = half * 64 + 2 * c2;
+                    const float p0 = ex2(fmaf(__uint_as_float(sr[col >> 5][col & 31]), sl2, neg_m));
+                    const float p1 = ex2(fmaf(__uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]), sl2, neg_m));
+                    l += p0 + p1;
+                    pw[c2] = IoT<kFP16>::pack(p0, p1);
                 }
-                uint4 v;
-                v.x = IoT<kFP16>::pack(p[0], p[1]);
-                v.y = IoT<kFP16>::pack(p[2], p[3]);
-                v.z = IoT<kFP16>::pack(p[4], p[5]);
-                v.w = IoT<kFP16>::pack(p[6], p[7]);
-                sts128(prow + (cc >> 3) * C::kAtomBytes + (((cc & 7) ^ (row & 7)) << 4), v);
+                tmem_st32(sc + half * 32, pw);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarPFull));
+            if (lane == 0) mbar_arrive(bar(C::kBarPFull + b));
         }
-        // epilogue: out = O / l
-        const bool fin = ok && mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(n_kv - 1) & 1u, abort_flag);
+        // epilogue: out = O / l, after the last PV
+        const int lb = (n_kv - 1) % kSBufs;
+        const bool fin = ok && mbar_wait(bar(C::kBarBufFree + lb), static_cast<uint32_t>((n_kv - 1) / kSBufs) & 1u,
+                                         abort_flag);
         if (__all_sync(0xffffffffu, fin)) {
             tc_fence_after();
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
             const bool valid = qi < w.L;
-            using OutT = uint16_t;
-            OutT* outp = reinterpret_cast<OutT*>(a.out);
+            uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
             int64_t o_off;
             if (a.layout == 0)
                 o_off = ((static_cast<int64_t>(w.seq) * a.Hq + w.h) * a.S + qi) * D;

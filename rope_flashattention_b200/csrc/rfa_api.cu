@@ -52,7 +52,24 @@ bool make_map(CUtensorMap* m, const void* base, bool fp16, uint64_t d0, uint64_t
     return r == CUDA_SUCCESS;
 }
 
-template <typename K>
+// Opt-in to large dynamic shared memory, once per (kernel, device).  The
+// template tag keeps one flag set per kernel instantiation.
+// The cos/sin table as a 3-D map of 32-bit (cos, sin) pairs: [1][T][D/2],
+// boxes of 32 pairs (128 B) x 128 tokens, 128-byte swizzle.
+bool make_table_map(CUtensorMap* m, const void* base, uint64_t T, int D) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D / 2), T, 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D / 2) * 4, T * (D / 2) * 4};
+    cuuint32_t box[3] = {32, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int kTag, typename K>
 rfa_status ensure_smem_attr(K kernel, int bytes) {
     static bool done[kMaxDevices] = {};
     static std::mutex mu;
@@ -112,15 +129,16 @@ int64_t total_tokens(const rfa_attn_params* p, const int32_t* lens) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * D * sizeof(float), 256); }
+// cos/sin table: D/2 fp16 (cos, sin) pairs per token.
+size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * D * 2, 256); }
 
 template <int D, bool kFP16>
-rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const rfa::AttnArgs& args,
-                       cudaStream_t st) {
+rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mt,
+                       const rfa::AttnArgs& args, cudaStream_t st) {
     auto kern = rfa::fused_rope_attn_fwd_kernel<D, kFP16>;
     constexpr int smem = rfa::AttnCfg<D>::kSmemBytes;
-    if (ensure_smem_attr(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
-    kern<<<args.n_items, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, args);
+    if (ensure_smem_attr<D * 2 + (kFP16 ? 1 : 0)>(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
+    kern<<<args.n_items, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, mt, args);
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
@@ -216,7 +234,7 @@ rfa_status enqueue_table(const rfa_attn_params* p, int64_t T, const int32_t* pos
     std::memset(&ta, 0, sizeof ta);
     ta.pos = position;
     ta.inv_dev = invFreq;
-    ta.table = static_cast<float*>(workspace);
+    ta.table = static_cast<uint32_t*>(workspace);
     ta.ntokens = static_cast<int32_t>(T);
     ta.half = half;
     ta.nseg = p->B;
@@ -249,7 +267,6 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
     rfa::AttnArgs aa;
     std::memset(&aa, 0, sizeof aa);
     aa.out = out;
-    aa.table = static_cast<const float*>(table);
     aa.layout = tnd ? 1 : 0;
     aa.B = p->B;
     aa.Hq = p->Hq;
@@ -292,8 +309,10 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
             aa.seg_start[i] = starts[b];
             aa.seg_len[i] = seqLens_host[b];
             aa.seg_tiles[i] = (seqLens_host[b] + rfa::kBlockM - 1) / rfa::kBlockM;
+            aa.seg_item0[i] = static_cast<int32_t>(std::min<int64_t>(items, 0x7fffffff));
             items += static_cast<int64_t>(aa.seg_tiles[i]) * p->Hq;
         }
+        aa.seg_item0[p->B] = static_cast<int32_t>(std::min<int64_t>(items, 0x7fffffff));
         if (items > 0x7fffffff) return RFA_ERR_UNSUPPORTED;
         aa.n_items = static_cast<int32_t>(items);
         ok = make_map(&mq, q, fp16, D, p->Hq, T, D * esz, static_cast<uint64_t>(p->Hq) * D * esz, 64, 1,
@@ -303,9 +322,12 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
              make_map(&mv, v, fp16, D, p->Hkv, T, D * esz, static_cast<uint64_t>(p->Hkv) * D * esz, 64, 1,
                       rfa::kBlockN);
     }
+    CUtensorMap mt;
+    ok = ok && make_table_map(&mt, table, static_cast<uint64_t>(T), D);
     if (!ok) return RFA_ERR_CUDA;
-    if (D == 128) return fp16 ? launch_attn<128, true>(mq, mk, mv, aa, st) : launch_attn<128, false>(mq, mk, mv, aa, st);
-    return fp16 ? launch_attn<64, true>(mq, mk, mv, aa, st) : launch_attn<64, false>(mq, mk, mv, aa, st);
+    if (D == 128)
+        return fp16 ? launch_attn<128, true>(mq, mk, mv, mt, aa, st) : launch_attn<128, false>(mq, mk, mv, mt, aa, st);
+    return fp16 ? launch_attn<64, true>(mq, mk, mv, mt, aa, st) : launch_attn<64, false>(mq, mk, mv, mt, aa, st);
 }
 
 }  // namespace

@@ -104,13 +104,14 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
     }
 }
 
-// Compact table for the fused kernel: table[t][0][j] = cos, table[t][1][j] = sin,
-// j < half, fp32.  Segments: uniform_len > 0 -> segment t / uniform_len,
-// otherwise the host-known prefix sums cum[].
+// Compact table for the fused kernel: table[t][j] = (cos, sin) of the angle
+// of token t and frequency j < half, as one fp16 pair (cos in the low half).
+// Segments: uniform_len > 0 -> segment t / uniform_len, otherwise the
+// host-known prefix sums cum[].
 struct TableArgs {
     const int32_t* pos;
     const float* inv_dev;  // [nseg, half] or nullptr -> inv_host
-    float* table;
+    uint32_t* table;       // [ntokens][half] fp16 (cos, sin) pairs
     int32_t ntokens;
     int32_t half;
     int32_t nseg;
@@ -138,9 +139,15 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
                                      : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
         float s[8], co[8];
         sincos8(static_cast<float>(__ldg(a.pos + t)), inv + 8 * c, s, co);
-        float* row = a.table + static_cast<int64_t>(t) * 2 * a.half + 8 * c;
-        Pack8<float>::store(row, co);
-        Pack8<float>::store(row + a.half, s);
+        uint32_t pr[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            __half2 h = __floats2half2_rn(co[k], s[k]);
+            pr[k] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        uint4* row = reinterpret_cast<uint4*>(a.table + static_cast<int64_t>(t) * a.half + 8 * c);
+        row[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+        row[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
     }
 }
 
