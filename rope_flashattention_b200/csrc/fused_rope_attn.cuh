@@ -11,20 +11,25 @@
 // back to global memory.
 //
 // One CTA = one work item (sequence, query head, 128-row query tile).  Warp roles:
-//   warps 0-3  softmax warpgroup: thread t owns query row t of the tile (TMEM
-//              lane t).  Loads S from TMEM, masks, keeps the running max and
-//              sum, writes P (bf16/fp16) back into the same TMEM columns,
-//              rescales O in TMEM only when its max grows by > 2^8, and at the
-//              end normalises O and stores the output row.
-//   warps 4-7  RoPE warpgroup: rotates the Q tile once and every K tile in
+//   warps 0-7  two softmax warpgroups; warpgroup g takes key columns
+//              [64g, 64g + 64) of every score tile, thread t of it owns query
+//              row t (TMEM lane t).  Per tile: load its half of S from TMEM,
+//              mask, exchange the half-row maxima through shared memory, keep
+//              the running max (identical in both) and a partial sum, write P
+//              (bf16/fp16) back into TMEM, rescale its half of O only when the
+//              max grows by > 2^8.  At the end the partial sums are combined
+//              and each warpgroup normalises and stores half of the columns.
+//   warps 8-11 RoPE warpgroup: rotates the Q tile once and every K tile in
 //              place in the 128B-swizzled shared-memory layout, reading the
 //              cos/sin rows that TMA staged next to the tile.  Element i and
 //              its rotate-half partner i + D/2 sit at the same offset of two
 //              swizzle atoms (D = 128) or in chunks c and c ^ 4 of one atom
 //              (D = 64), so each thread rotates 8 pairs per 2 x 16 B.
-//   warp 8     TMA producer: Q (+ its cos/sin rows) once, then K (+ cos/sin)
-//              and V tiles through a kStages ring.
-//   warp 9     tcgen05 issuer (one thread) and TMEM owner.  S_j = Q'K_j'^T goes
+//   warp 12    TMA producer: Q (+ its cos/sin rows) once, then K (+ cos/sin)
+//              tiles through a kStages ring.
+//   warp 14    TMA producer for the V ring (V slots free up later than K
+//              slots, so one producer for both would hold back K prefetch).
+//   warp 13    tcgen05 issuer (one thread) and TMEM owner.  S_j = Q'K_j'^T goes
 //              to TMEM buffer j % 3; O += P_j V_j reads P_j from that buffer
 //              (A operand in TMEM) and V_j from shared memory.  QK runs two
 //              tiles ahead of PV so the softmax never waits for its scores.
@@ -42,10 +47,12 @@ namespace rfa {
 
 constexpr int kBlockM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per tile
-constexpr int kAttnThreads = 320;
-constexpr int kRopeWarp0 = 4;
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kAttnThreads = 512;
+constexpr int kRopeWarp0 = 8;
+constexpr int kTmaWarp = 12;   // Q, K (+ cos/sin rows)
+constexpr int kMmaWarp = 13;
+constexpr int kTmaVWarp = 14;  // V: its own producer, so K prefetch never waits on a V slot
+// warp 15 only takes part in the block-wide barriers
 constexpr int kSBufs = 3;                  // S/P buffers in TMEM
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
@@ -90,10 +97,14 @@ struct AttnCfg {
     static constexpr int kBarPFull = kBarSFull + kSBufs;    // kSBufs
     static constexpr int kBarBufFree = kBarPFull + kSBufs;  // kSBufs: PV of that buffer done
     static constexpr int kBarMmaFin = kBarBufFree + kSBufs;
-    static constexpr int kNumBars = kBarMmaFin + 1;
+    static constexpr int kBarXchg = kBarMmaFin + 1;  // 2: half-row maxima exchanged (256 arrivals)
+    static constexpr int kNumBars = kBarXchg + 2;
     static constexpr int kOffAbort = kOffBar + 8 * kNumBars;
     static constexpr int kOffTmemSlot = kOffAbort + 16;
-    static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;  // + slack for 1024-byte alignment
+    static constexpr int kOffXchg = kOffTmemSlot + 16;  // float [2 slots][2 halves][128 rows]
+    // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (the
+    // kernel checks it), so no alignment slack is requested.
+    static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBlockM * 4;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColO = kSBufs * kBlockN;  // S/P buffers at 0, 128, 256; O at 384
     static_assert(kColO + D <= kTmemCols, "TMEM budget");
@@ -142,6 +153,9 @@ struct IoT<false> {
     static __device__ __forceinline__ float2 unpack(uint32_t u) {
         return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
     }
+    static __device__ __forceinline__ uint64_t unpack2(uint32_t u) {  // exact: bf16 -> fp32 is a shift
+        return f2pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    }
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
         __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
         return *reinterpret_cast<uint32_t*>(&h);
@@ -153,6 +167,10 @@ struct IoT<true> {
     static __device__ __forceinline__ float2 unpack(uint32_t u) {
         return __half22float2(*reinterpret_cast<const __half2*>(&u));
     }
+    static __device__ __forceinline__ uint64_t unpack2(uint32_t u) {
+        const float2 f = unpack(u);
+        return f2pack(f.x, f.y);
+    }
     static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
         __half2 h = __floats2half2_rn(lo, hi);
         return *reinterpret_cast<uint32_t*>(&h);
@@ -160,10 +178,21 @@ struct IoT<true> {
     static constexpr uint32_t kFmt = 0;
 };
 
-__device__ __forceinline__ float2 h2f2(uint32_t u) { return __half22float2(*reinterpret_cast<const __half2*>(&u)); }
+template <bool kFP16>
+__device__ __forceinline__ uint32_t pack2(uint64_t v) {
+    const float2 f = f2unpack(v);
+    return IoT<kFP16>::pack(f.x, f.y);
+}
+
+__device__ __forceinline__ uint64_t h2f2x2(uint32_t u) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
+    return f2pack(f.x, f.y);
+}
 
 // Rotate 8 rotate-half pairs held in two 16-byte chunks (x1: dims i..i+7,
-// x2: dims i+D/2..i+D/2+7).  t0/t1 hold the 8 (cos, sin) fp16 pairs.
+// x2: dims i+D/2..i+D/2+7), two dimensions per packed fp32x2 operation.
+// t0/t1 hold, per two dimensions, a word of fp16 cosines then a word of fp16
+// sines:  x1' = x1 cos - x2 sin,  x2' = x2 cos + x1 sin.
 template <bool kFP16>
 __device__ __forceinline__ void rotate8(uint4& x1, uint4& x2, const uint4& t0, const uint4& t1) {
     uint32_t* a = reinterpret_cast<uint32_t*>(&x1);
@@ -171,14 +200,13 @@ __device__ __forceinline__ void rotate8(uint4& x1, uint4& x2, const uint4& t0, c
     const uint32_t cs[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float2 u = IoT<kFP16>::unpack(a[k]);
-        const float2 v = IoT<kFP16>::unpack(b[k]);
-        const float2 e0 = h2f2(cs[2 * k]);      // (cos, sin) of dim 2k
-        const float2 e1 = h2f2(cs[2 * k + 1]);  // (cos, sin) of dim 2k+1
-        const float y10 = u.x * e0.x - v.x * e0.y, y11 = u.y * e1.x - v.y * e1.y;
-        const float y20 = v.x * e0.x + u.x * e0.y, y21 = v.y * e1.x + u.y * e1.y;
-        a[k] = IoT<kFP16>::pack(y10, y11);
-        b[k] = IoT<kFP16>::pack(y20, y21);
+        const uint64_t X1 = IoT<kFP16>::unpack2(a[k]);
+        const uint64_t X2 = IoT<kFP16>::unpack2(b[k]);
+        const uint64_t C = h2f2x2(cs[2 * k]);
+        const uint64_t S = h2f2x2(cs[2 * k + 1]);
+        const uint64_t NS = h2f2x2(cs[2 * k + 1] ^ 0x80008000u);  // -sin, exact
+        a[k] = pack2<kFP16>(ffma2(X1, C, fmul2(X2, NS)));
+        b[k] = pack2<kFP16>(ffma2(X2, C, fmul2(X1, S)));
     }
 }
 
@@ -205,10 +233,20 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t r
             o1 = tile + r * 128 + ((cp ^ sw) << 4);
             o2 = tile + r * 128 + (((cp + 4) ^ sw) << 4);
         }
-        const uint32_t tb = tab + (cp >> 2) * AttnCfg<D>::kAtomBytes + r * 128;
-        const uint32_t tc = static_cast<uint32_t>((cp & 3) * 2);
-        const uint4 t0 = lds128(tb + ((tc ^ sw) << 4));
-        const uint4 t1 = lds128(tb + (((tc + 1) ^ sw) << 4));
+        uint4 t0, t1;
+        if constexpr (D == 128) {
+            // row layout of the table: chunk cp of atom 0 = pairs 8cp..8cp+3,
+            // chunk cp of atom 1 = pairs 8cp+4..8cp+7 (conflict-free for the 8
+            // lanes of a quarter-warp, which share a row)
+            const uint32_t tb = tab + r * 128 + ((cp ^ sw) << 4);
+            t0 = lds128(tb);
+            t1 = lds128(tb + AttnCfg<D>::kAtomBytes);
+        } else {
+            const uint32_t tb = tab + r * 128;
+            const uint32_t tc = static_cast<uint32_t>(cp * 2);
+            t0 = lds128(tb + ((tc ^ sw) << 4));
+            t1 = lds128(tb + (((tc + 1) ^ sw) << 4));
+        }
         uint4 x1 = lds128(o1), x2 = lds128(o2);
         rotate8<kFP16>(x1, x2, t0, t1);
         sts128(o1, x1);
@@ -245,10 +283,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmT,
                                const __grid_constant__ AttnArgs a) {
     using C = AttnCfg<D>;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t sbase = (raw + 1023u) & ~1023u;
-    uint8_t* smem = smem_raw + (sbase - raw);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    if ((sbase & 1023u) != 0u) {  // 128B-swizzled TMA/UMMA tiles need 1024-byte alignment
+        if (threadIdx.x == 0) record_status(2 /* RFA_ERR_UNSUPPORTED */);
+        return;
+    }
+    uint8_t* smem = smem_raw;
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + C::kOffAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmemSlot);
     auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * static_cast<uint32_t>(i); };
@@ -271,10 +312,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         for (int b = 0; b < kSBufs; ++b) {
             mbar_init(bar(C::kBarSFull + b), 1);
-            mbar_init(bar(C::kBarPFull + b), 4);
+            mbar_init(bar(C::kBarPFull + b), 8);
             mbar_init(bar(C::kBarBufFree + b), 1);
         }
         mbar_init(bar(C::kBarMmaFin), 1);
+        mbar_init(bar(C::kBarXchg + 0), 256);
+        mbar_init(bar(C::kBarXchg + 1), 256);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -313,7 +356,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_expect_tx(bar(C::kBarQFull), C::kTileBytes + C::kTabBytes);
             load_tile(&tmQ, sbase + C::kOffQ, bar(C::kBarQFull), qplane, w.qt * kBlockM);
             load_tab(sbase + C::kOffT + 1 * C::kTabBytes, bar(C::kBarQFull), w.qt * kBlockM);
-            int32_t issued_k = 0, issued_v = 0;
+            int32_t issued_k = 0;
             for (int32_t j = 0; j < n_kv; ++j) {
                 const int s = j % C::kStages;
                 const uint32_t u = static_cast<uint32_t>(j / C::kStages);
@@ -323,15 +366,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 load_tile(&tmK, sbase + C::kOffK + s * C::kTileBytes, bar(C::kBarKFull + s), kvplane, j * kBlockN);
                 load_tab(sbase + C::kOffT + s * C::kTabBytes, bar(C::kBarKFull + s), j * kBlockN);
                 issued_k = j + 1;
-                if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) break;
-                mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-                load_tile(&tmV, sbase + C::kOffV + s * C::kTileBytes, bar(C::kBarVFull + s), kvplane, j * kBlockN);
-                issued_v = j + 1;
             }
             // Drain: every issued copy must have landed before the CTA exits.
             mbar_wait_drain(bar(C::kBarQFull), 0);
             for (int32_t j = (issued_k > C::kStages ? issued_k - C::kStages : 0); j < issued_k; ++j)
                 mbar_wait_drain(bar(C::kBarKFull + j % C::kStages), static_cast<uint32_t>(j / C::kStages) & 1u);
+        }
+    } else if (warp == kTmaVWarp) {
+        // ------------------------------------------------------------ V producer
+        if (lane == 0) {
+            const bool bnsd = (a.layout == 0);
+            const int32_t kvplane = bnsd ? (w.seq * a.Hkv + kvh) : kvh;
+            int32_t issued_v = 0;
+            for (int32_t j = 0; j < n_kv; ++j) {
+                const int s = j % C::kStages;
+                const uint32_t u = static_cast<uint32_t>(j / C::kStages);
+                if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) break;
+                mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+                const uint32_t dst = sbase + C::kOffV + s * C::kTileBytes;
+                for (int at = 0; at < C::kAtoms; ++at) {
+                    if (bnsd)
+                        tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, j * kBlockN, kvplane);
+                    else
+                        tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, kvplane,
+                                    w.tok0 + j * kBlockN);
+                }
+                issued_v = j + 1;
+            }
             for (int32_t j = (issued_v > C::kStages ? issued_v - C::kStages : 0); j < issued_v; ++j)
                 mbar_wait_drain(bar(C::kBarVFull + j % C::kStages), static_cast<uint32_t>(j / C::kStages) & 1u);
         }
@@ -394,7 +455,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_commit(bar(C::kBarMmaFin));
             mbar_wait_drain(bar(C::kBarMmaFin), 0);
         }
-    } else if (warp >= kRopeWarp0) {
+    } else if (warp >= kRopeWarp0 && warp < kRopeWarp0 + 4) {
         // ------------------------------------------------------------ RoPE warpgroup
         const int32_t rt = threadIdx.x - kRopeWarp0 * 32;
         if (mbar_wait(bar(C::kBarQFull), 0, abort_flag)) {
@@ -415,46 +476,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (lane == 0) mbar_arrive(bar(C::kBarKReady + s));
             }
         }
-    } else {
-        // ------------------------------------------------------------ softmax warpgroup
-        const int row = threadIdx.x;  // 0..127 == TMEM lane
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int hf = warp >> 2;            // key-column half of every score tile
+        const int row = threadIdx.x & 127;   // 0..127 == TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        float* xmax = reinterpret_cast<float*>(smem + C::kOffXchg);  // [slot][half][row]
         const int32_t qi = w.qt * kBlockM + row;
         const float sl2 = a.scale_log2;
-        float m = -INFINITY;  // running max of score * scale * log2(e)
-        float l = 0.0f;       // running sum of exp2(score * scale_log2 - m)
+        constexpr int kOHalf = D / 2;        // O columns rescaled / stored by this warpgroup
+        float m = -INFINITY;  // running max of score * scale * log2(e) (same in both warpgroups)
+        float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
         bool ok = true;
-        uint32_t sr[4][32];
         for (int32_t j = 0; j < n_kv; ++j) {
             const int b = j % kSBufs;
             // tcgen05.ld/st are warp-collective: every decision below is warp-uniform.
             if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + b), static_cast<uint32_t>(j / kSBufs) & 1u,
                                                    abort_flag))) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sc = tmem + lane_off + b * kBlockN;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) tmem_ld32(sc + q * 32, sr[q]);
+            uint32_t sr[2][32];
+            const uint32_t sc = tmem + lane_off + b * kBlockN + hf * 64;
+            tmem_ld32(sc, sr[0]);
+            tmem_ld32(sc + 32, sr[1]);
             tmem_wait_ld();
 
-            // mask: keys [kv0, kv0 + lim) are visible to this row
-            const int32_t kv0 = j * kBlockN;
+            // mask: keys [kv0, kv0 + lim) of this half are visible to this row
+            const int32_t kv0 = j * kBlockN + hf * 64;
             const int32_t lim = (a.causal ? min(qi + 1, w.L) : w.L) - kv0;
-            float mx = -INFINITY;
-            if (lim >= kBlockN) {
+            if (lim < 64) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[q][c]));
-            } else {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        float v = (q * 32 + c < lim) ? __uint_as_float(sr[q][c]) : -INFINITY;
-                        sr[q][c] = __float_as_uint(v);
-                        mx = fmaxf(mx, v);
-                    }
+                for (int c = 0; c < 64; ++c)
+                    if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 64; c += 2)
+                mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c >> 5][c & 31]),
+                                          __uint_as_float(sr[c >> 5][(c + 1) & 31]));
+            const float mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+            // exchange half-row maxima with the other warpgroup
+            const int slot = j & 1;
+            xmax[(slot * 2 + hf) * kBlockM + row] = mxh;
+            mbar_arrive(bar(C::kBarXchg + slot));
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarXchg + slot), static_cast<uint32_t>(j >> 1) & 1u,
+                                                   abort_flag))) { ok = false; break; }
+            const float mx = fmaxf(mxh, xmax[(slot * 2 + (hf ^ 1)) * kBlockM + row]);
             const float m_new = fmaxf(m, mx * sl2);
             if (j > 0) {
                 const bool need = m_new > m + kRescaleThreshold;
@@ -468,13 +534,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const float alpha = need ? ex2(m - m_new) : 1.0f;
                     l *= alpha;
 #pragma unroll 1
-                    for (int q = 0; q < D / 32; ++q) {
+                    for (int q = 0; q < kOHalf / 32; ++q) {
                         uint32_t o[32];
-                        tmem_ld32(tmem + lane_off + C::kColO + q * 32, o);
+                        const uint32_t oc = tmem + lane_off + C::kColO + hf * kOHalf + q * 32;
+                        tmem_ld32(oc, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                        tmem_st32(tmem + lane_off + C::kColO + q * 32, o);
+                        tmem_st32(oc, o);
                     }
                     if (need) m = m_new;
                 }
@@ -482,29 +549,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 m = m_new;
             }
             const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-            // P_j overwrites the first 64 columns of S_j (already in registers).
+            // P_j (this half: 32 packed columns) overwrites S_j columns that both
+            // warpgroups have already loaded (the exchange above orders it).
+            uint32_t pw[32];
+            const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
+            uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pw[32];
-#pragma unroll
-                for (int c2 = 0; c2 < 32; ++c2) {
-                    const int col = half * 64 + 2 * c2;
-                    const float p0 = ex2(fmaf(__uint_as_float(sr[col >> 5][col & 31]), sl2, neg_m));
-                    const float p1 = ex2(fmaf(__uint_as_float(sr[(col + 1) >> 5][(col + 1) & 31]), sl2, neg_m));
-                    l += p0 + p1;
-                    pw[c2] = IoT<kFP16>::pack(p0, p1);
-                }
-                tmem_st32(sc + half * 32, pw);
+            for (int c2 = 0; c2 < 32; ++c2) {
+                const int c = 2 * c2;
+                const uint64_t sv = f2pack(__uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[c >> 5][(c + 1) & 31]));
+                const float2 x = f2unpack(ffma2(sv, sl2x2, negm2));
+                const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
+                l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
+                pw[c2] = pack2<kFP16>(pp);
             }
+            const float2 la = f2unpack(fadd2(l2[0], l2[1]));
+            l += la.x + la.y;
+            tmem_st32(tmem + lane_off + b * kBlockN + hf * 32, pw);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::kBarPFull + b));
         }
-        // epilogue: out = O / l, after the last PV
+        // epilogue: combine the partial sums, out = O / l after the last PV
+        bool fin = ok;
+        if (fin) {
+            const int slot = n_kv & 1;  // last read at tile n_kv-2, free for both warpgroups now
+            xmax[(slot * 2 + hf) * kBlockM + row] = l;
+            mbar_arrive(bar(C::kBarXchg + slot));
+            fin = mbar_wait(bar(C::kBarXchg + slot), static_cast<uint32_t>(n_kv >> 1) & 1u, abort_flag);
+            if (fin) l += xmax[(slot * 2 + (hf ^ 1)) * kBlockM + row];
+        }
         const int lb = (n_kv - 1) % kSBufs;
-        const bool fin = ok && mbar_wait(bar(C::kBarBufFree + lb), static_cast<uint32_t>((n_kv - 1) / kSBufs) & 1u,
-                                         abort_flag);
+        fin = fin && mbar_wait(bar(C::kBarBufFree + lb), static_cast<uint32_t>((n_kv - 1) / kSBufs) & 1u, abort_flag);
         if (__all_sync(0xffffffffu, fin)) {
             tc_fence_after();
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
@@ -515,10 +592,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 o_off = ((static_cast<int64_t>(w.seq) * a.Hq + w.h) * a.S + qi) * D;
             else
                 o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + w.h) * D;
+            o_off += hf * kOHalf;
 #pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
+            for (int q = 0; q < kOHalf / 32; ++q) {
                 uint32_t o[32];
-                tmem_ld32(tmem + lane_off + C::kColO + q * 32, o);
+                tmem_ld32(tmem + lane_off + C::kColO + hf * kOHalf + q * 32, o);
                 tmem_wait_ld();
                 if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);

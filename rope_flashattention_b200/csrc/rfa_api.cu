@@ -129,8 +129,9 @@ int64_t total_tokens(const rfa_attn_params* p, const int32_t* lens) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// cos/sin table: D/2 fp16 (cos, sin) pairs per token.
+// cos/sin table: D/2 fp16 cos values and D/2 fp16 sin values per token.
 size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * D * 2, 256); }
+size_t workspace_bytes(int64_t T, int D, int /*nseg*/) { return table_bytes(T, D); }
 
 template <int D, bool kFP16>
 rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mt,
@@ -204,7 +205,7 @@ rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, con
 
 size_t rfa_fused_rope_attention_workspace(const rfa_attn_params* p, int64_t ntokens) {
     if (validate_attn(p) != RFA_OK || ntokens < 1) return 0;
-    return table_bytes(ntokens, p->D);
+    return workspace_bytes(ntokens, p->D, p->B);
 }
 
 }  // extern "C"
@@ -341,7 +342,7 @@ rfa_status rfa_rope_attention_table(const rfa_attn_params* p, const int32_t* pos
     if (vs != RFA_OK) return vs;
     if (!position) return RFA_ERR_INVALID_ARG;
     if (invFreq && !aligned(invFreq, 16)) return RFA_ERR_INVALID_ARG;
-    if (!workspace || ws_bytes < table_bytes(T, p->D) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < workspace_bytes(T, p->D, p->B) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
     return enqueue_table(p, T, position, seqLens_host, invFreq, workspace, as_stream(stream));
 }
 
@@ -353,7 +354,7 @@ rfa_status rfa_fused_rope_attention_with_table(const rfa_attn_params* p, const v
     if (vs != RFA_OK) return vs;
     if (!q || !k || !v || !out) return RFA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return RFA_ERR_INVALID_ARG;
-    if (!workspace || ws_bytes < table_bytes(T, p->D) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < workspace_bytes(T, p->D, p->B) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
     return enqueue_attention(p, T, q, k, v, seqLens_host, out, workspace, as_stream(stream));
 }
 
@@ -366,7 +367,7 @@ rfa_status rfa_fused_rope_attention(const rfa_attn_params* p, const void* q, con
     if (!q || !k || !v || !position || !out) return RFA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return RFA_ERR_INVALID_ARG;
     if (invFreq && !aligned(invFreq, 16)) return RFA_ERR_INVALID_ARG;
-    if (!workspace || ws_bytes < table_bytes(T, p->D) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < workspace_bytes(T, p->D, p->B) || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
     cudaStream_t st = as_stream(stream);
     rfa_status r = enqueue_table(p, T, position, seqLens_host, invFreq, workspace, st);
     if (r != RFA_OK) return r;

@@ -104,14 +104,19 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
     }
 }
 
-// Compact table for the fused kernel: table[t][j] = (cos, sin) of the angle
-// of token t and frequency j < half, as one fp16 pair (cos in the low half).
-// Segments: uniform_len > 0 -> segment t / uniform_len, otherwise the
-// host-known prefix sums cum[].
+// Compact table for the fused kernel.  Per token, 16-byte chunks cover 4
+// frequencies j0..j0+3 as four 32-bit words of fp16 pairs:
+//   (cos j0, cos j0+1), (sin j0, sin j0+1), (cos j0+2, cos j0+3), (sin j0+2, sin j0+3)
+// so that one conversion yields the packed fp32 operands of two dimensions.
+// Chunk order within a row: for half == 64 the chunk of frequency group
+// g = j0/4 is stored at position (g % 2) * 8 + g / 2, so the fused kernel's 8
+// lanes that share a row read distinct shared-memory banks; for other sizes
+// the order is natural.  Segments: uniform_len > 0 -> segment t / uniform_len,
+// otherwise the host-known prefix sums cum[].
 struct TableArgs {
     const int32_t* pos;
     const float* inv_dev;  // [nseg, half] or nullptr -> inv_host
-    uint32_t* table;       // [ntokens][half] fp16 (cos, sin) pairs
+    uint32_t* table;       // [ntokens][half] 32-bit words of fp16 cos/sin pairs
     int32_t ntokens;
     int32_t half;
     int32_t nseg;
@@ -141,13 +146,18 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
         sincos8(static_cast<float>(__ldg(a.pos + t)), inv + 8 * c, s, co);
         uint32_t pr[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            __half2 h = __floats2half2_rn(co[k], s[k]);
-            pr[k] = *reinterpret_cast<uint32_t*>(&h);
+        for (int k = 0; k < 4; ++k) {
+            __half2 hc = __floats2half2_rn(co[2 * k], co[2 * k + 1]);
+            __half2 hs = __floats2half2_rn(s[2 * k], s[2 * k + 1]);
+            pr[2 * k] = *reinterpret_cast<uint32_t*>(&hc);
+            pr[2 * k + 1] = *reinterpret_cast<uint32_t*>(&hs);
         }
-        uint4* row = reinterpret_cast<uint4*>(a.table + static_cast<int64_t>(t) * a.half + 8 * c);
-        row[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
-        row[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
+        uint4* row = reinterpret_cast<uint4*>(a.table + static_cast<int64_t>(t) * a.half);
+        // groups 2c and 2c+1 of 4 pairs each
+        const int g0 = (a.half == 64) ? c : 2 * c;
+        const int g1 = (a.half == 64) ? 8 + c : 2 * c + 1;
+        row[g0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+        row[g1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
     }
 }
 

@@ -67,10 +67,15 @@ def test_params_struct_matches_c_layout():
     assert rfa.AttnParams.ntk_factor.offset == 56
 
 
+def _ru(x, a=256):
+    return (x + a - 1) // a * a
+
+
 def test_workspace_size(lib):
     f = lib.rfa_fused_rope_attention_workspace
-    assert f(ctypes.byref(_p()), 128) == 128 * 64 * 4
-    assert f(ctypes.byref(_p(D=128)), 1000) == (1000 * 128 * 4 + 255) // 256 * 256
+    # cos/sin table: D/2 fp16 cos and D/2 fp16 sin values per token
+    assert f(ctypes.byref(_p()), 128) == _ru(128 * 64 * 2)
+    assert f(ctypes.byref(_p(D=128, B=3)), 1000) == _ru(1000 * 128 * 2)
     assert f(ctypes.byref(_p(D=96)), 128) == 0          # unsupported head dim
     assert f(ctypes.byref(_p(Hq=3, Hkv=2)), 128) == 0    # Hq % Hkv != 0
     assert f(ctypes.byref(_p(io_dtype=0)), 128) == 0     # UNDEFINED dtype
