@@ -129,7 +129,8 @@ RFA_API size_t rfa_fused_rope_attention_workspace(const rfa_attn_params* p, int6
  *   workspace  dev   >= rfa_fused_rope_attention_workspace(p, T) bytes,
  *                    256-byte aligned; holds the cos/sin table of this call
  *                    (T*D*2 bytes: D/2 fp16 cos and D/2 fp16 sin values per
- *                    token) -- a table, never rotated Q/K
+ *                    token) and per-sequence angle-recurrence seeds (9232
+ *                    bytes each) -- tables, never rotated Q/K
  * Rotated Q and K exist only in shared memory.  The call enqueues two
  * kernels: the cos/sin table and the fused attention.
  */

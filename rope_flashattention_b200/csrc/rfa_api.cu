@@ -129,9 +129,11 @@ int64_t total_tokens(const rfa_attn_params* p, const int32_t* lens) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// cos/sin table: D/2 fp16 cos values and D/2 fp16 sin values per token.
+// cos/sin table (D/2 fp16 cos and D/2 fp16 sin values per token), then one
+// recurrence seed block per sequence.
 size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * D * 2, 256); }
-size_t workspace_bytes(int64_t T, int D, int /*nseg*/) { return table_bytes(T, D); }
+size_t seeds_bytes(int nseg) { return round_up(static_cast<size_t>(nseg) * sizeof(rfa::RopeSeed), 256); }
+size_t workspace_bytes(int64_t T, int D, int nseg) { return table_bytes(T, D) + seeds_bytes(nseg); }
 
 template <int D, bool kFP16>
 rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mt,
@@ -236,6 +238,7 @@ rfa_status enqueue_table(const rfa_attn_params* p, int64_t T, const int32_t* pos
     ta.pos = position;
     ta.inv_dev = invFreq;
     ta.table = static_cast<uint32_t*>(workspace);
+    ta.seeds = reinterpret_cast<rfa::RopeSeed*>(static_cast<char*>(workspace) + table_bytes(T, D));
     ta.ntokens = static_cast<int32_t>(T);
     ta.half = half;
     ta.nseg = p->B;
@@ -258,6 +261,8 @@ rfa_status enqueue_table(const rfa_attn_params* p, int64_t T, const int32_t* pos
         }
     }
     rfa::rope_table_kernel<<<grid_for(T * (half / 8), 256), 256, 0, st>>>(ta);
+    if (cudaGetLastError() != cudaSuccess) return RFA_ERR_CUDA;
+    rfa::rope_seed_kernel<<<p->B, 256, 0, st>>>(ta);
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
@@ -268,6 +273,7 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
     rfa::AttnArgs aa;
     std::memset(&aa, 0, sizeof aa);
     aa.out = out;
+    aa.seeds = reinterpret_cast<const rfa::RopeSeed*>(static_cast<const char*>(table) + table_bytes(T, D));
     aa.layout = tnd ? 1 : 0;
     aa.B = p->B;
     aa.Hq = p->Hq;
@@ -308,6 +314,7 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
         for (int i = 0; i < p->B; ++i) {
             const int b = order[i];
             aa.seg_start[i] = starts[b];
+            aa.seg_orig[i] = b;
             aa.seg_len[i] = seqLens_host[b];
             aa.seg_tiles[i] = (seqLens_host[b] + rfa::kBlockM - 1) / rfa::kBlockM;
             aa.seg_item0[i] = static_cast<int32_t>(std::min<int64_t>(items, 0x7fffffff));

@@ -113,10 +113,26 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
 // lanes that share a row read distinct shared-memory banks; for other sizes
 // the order is natural.  Segments: uniform_len > 0 -> segment t / uniform_len,
 // otherwise the host-known prefix sums cum[].
+// Per-sequence seeds of the fused kernel's angle-addition recurrence, used
+// when a sequence's positions are consecutive (pos[tok0 + i] == pos[tok0] + i):
+// with w = invFreq_j, row r of key tile k has angle (P + 128k + r) w, and its
+// (cos, sin) = z0[r % 16] * w16^(r / 16) * w128^k as complex products.
+// Seeds are evaluated in fp64 and rounded once to fp32.
+constexpr int kSeedRows = 16;
+struct RopeSeed {
+    int32_t consecutive;  // 1: the recurrence applies to this sequence
+    int32_t pos0;
+    int32_t pad[2];
+    float2 w16[kMaxHalfHost];            // (cos, sin) of 16 w_j
+    float2 w128[kMaxHalfHost];           // (cos, sin) of 128 w_j
+    float2 z0[kSeedRows][kMaxHalfHost];  // (cos, sin) of (P + r) w_j, r < 16
+};
+
 struct TableArgs {
     const int32_t* pos;
     const float* inv_dev;  // [nseg, half] or nullptr -> inv_host
     uint32_t* table;       // [ntokens][half] 32-bit words of fp16 cos/sin pairs
+    RopeSeed* seeds;       // [nseg]
     int32_t ntokens;
     int32_t half;
     int32_t nseg;
@@ -158,6 +174,46 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
         const int g1 = (a.half == 64) ? 8 + c : 2 * c + 1;
         row[g0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
         row[g1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
+    }
+}
+
+// One block per sequence: consecutive-positions flag and recurrence seeds.
+__global__ void __launch_bounds__(256) rope_seed_kernel(const __grid_constant__ TableArgs a) {
+    const int32_t b = blockIdx.x;
+    int32_t tok0, len;
+    if (a.uniform_len > 0) {
+        tok0 = b * a.uniform_len;
+        len = a.uniform_len;
+    } else {
+        tok0 = a.cum[b];
+        len = a.cum[b + 1] - a.cum[b];
+    }
+    const int32_t p0 = __ldg(a.pos + tok0);
+    int ok = 1;
+    for (int32_t i = threadIdx.x; i < len; i += blockDim.x)
+        if (__ldg(a.pos + tok0 + i) != p0 + i) ok = 0;
+    ok = __syncthreads_and(ok);
+    RopeSeed* sd = a.seeds + b;
+    const float* inv = a.inv_dev ? a.inv_dev + static_cast<int64_t>(b) * a.half
+                                 : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
+    if (threadIdx.x == 0) {
+        sd->consecutive = ok;
+        sd->pos0 = p0;
+    }
+    for (int32_t i = threadIdx.x; i < a.half * (kSeedRows + 2); i += blockDim.x) {
+        const int32_t j = i % a.half;
+        const int32_t k = i / a.half;
+        const double w = static_cast<double>(inv[j]);
+        const double ang = (k < kSeedRows) ? (static_cast<double>(p0) + k) * w : (k == kSeedRows ? 16.0 : 128.0) * w;
+        double sn, cs;
+        sincos(ang, &sn, &cs);
+        const float2 v = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+        if (k < kSeedRows)
+            sd->z0[k][j] = v;
+        else if (k == kSeedRows)
+            sd->w16[j] = v;
+        else
+            sd->w128[j] = v;
     }
 }
 
