@@ -14,7 +14,8 @@
 //   warps 0-7  two softmax warpgroups; warpgroup g takes key columns
 //              [64g, 64g + 64) of every score tile, thread t of it owns query
 //              row t (TMEM lane t).  Per tile: load its half of S from TMEM,
-//              mask, exchange the half-row maxima through shared memory, keep
+//              mask, exchange the half-row maxima through shared memory (named
+//              barrier 1 over the 256 softmax threads), keep
 //              the running max (identical in both) and a partial sum, write P
 //              (bf16/fp16) into TMEM, rescale its half of O only when the max
 //              grows by > 2^8.  At the end the partial sums are combined and
@@ -101,8 +102,7 @@ struct AttnCfg {
     static constexpr int kBarPFull = kBarSEmpty + 2;        // P_j written (8 warp arrivals)
     static constexpr int kBarPVDone = kBarPFull + 1;        // PV_j done: O updated, P free
     static constexpr int kBarMmaFin = kBarPVDone + 1;
-    static constexpr int kBarXchg = kBarMmaFin + 1;         // 2: half-row maxima exchanged (8 warp arrivals)
-    static constexpr int kBarQRot = kBarXchg + 2;           // Q' rotated in shared memory (4 warp arrivals)
+    static constexpr int kBarQRot = kBarMmaFin + 1;         // Q' rotated in shared memory (4 warp arrivals)
     static constexpr int kNumBars = kBarQRot + 1;
     static constexpr int kOffAbort = kOffBar + 8 * kNumBars;
     static constexpr int kOffTmemSlot = kOffAbort + 16;
@@ -408,7 +408,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(C::kBarSFull + b), 1);
             mbar_init(bar(C::kBarSEmpty + b), 8);  // one arrival per softmax warp
-            mbar_init(bar(C::kBarXchg + b), 8);
         }
         mbar_init(bar(C::kBarPFull), 8);
         mbar_init(bar(C::kBarPVDone), 1);
@@ -613,6 +612,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax warpgroups
+        // The two warpgroups meet at named barrier 1 exactly n_kv + 1 times: a
+        // failed (timed-out) wait only turns the remaining work into no-ops,
+        // it never skips a barrier, so the barrier cannot deadlock.
         const int hf = warp >> 2;            // key-column half of every score tile
         const int row = threadIdx.x & 127;   // 0..127 == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -622,49 +624,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         constexpr int kOHalf = D / 2;        // O columns rescaled / stored by this warpgroup
         float m = -INFINITY;  // running max of score * scale * log2(e) (same in both warpgroups)
         float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
-        bool ok = true;
+        bool ok = true;       // warp-uniform
         for (int32_t j = 0; j < n_kv; ++j) {
             const int b = j & 1;
-            // tcgen05.ld/st are warp-collective: every decision below is warp-uniform.
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + b), static_cast<uint32_t>(j >> 1) & 1u,
-                                                   abort_flag))) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[2][32];
-            const uint32_t sc = tmem + lane_off + C::kColS + b * kBlockN + hf * 64;
-            tmem_ld32(sc, sr[0]);
-            tmem_ld32(sc + 32, sr[1]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarSEmpty + b));  // S_j consumed: the buffer may take S_{j+2}
-
-            // mask: keys [kv0, kv0 + lim) of this half are visible to this row
-            const int32_t kv0 = j * kBlockN + hf * 64;
-            const int32_t lim = (a.causal ? min(qi + 1, w.L) : w.L) - kv0;
-            if (lim < 64) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-            }
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int c = 0; c < 64; c += 2)
-                mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c >> 5][c & 31]),
-                                          __uint_as_float(sr[c >> 5][(c + 1) & 31]));
-            const float mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
-            // exchange half-row maxima with the other warpgroup
             const int slot = j & 1;
+            // tcgen05.ld/st are warp-collective: every decision below is warp-uniform.
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + b), static_cast<uint32_t>(j >> 1) & 1u,
+                                                         abort_flag));
+            uint32_t sr[2][32];
+            float mxh = -INFINITY;
+            if (ok) {
+                tc_fence_after();
+                const uint32_t sc = tmem + lane_off + C::kColS + b * kBlockN + hf * 64;
+                tmem_ld32(sc, sr[0]);
+                tmem_ld32(sc + 32, sr[1]);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::kBarSEmpty + b));  // S_j consumed: the buffer may take S_{j+2}
+
+                // mask: keys [kv0, kv0 + lim) of this half are visible to this row
+                const int32_t kv0 = j * kBlockN + hf * 64;
+                const int32_t lim = (a.causal ? min(qi + 1, w.L) : w.L) - kv0;
+                if (lim < 64) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                }
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < 64; c += 2)
+                    mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c >> 5][c & 31]),
+                                              __uint_as_float(sr[c >> 5][(c + 1) & 31]));
+                mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+            }
+            // exchange half-row maxima with the other warpgroup
             xmax[(slot * 2 + hf) * kBlockM + row] = mxh;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarXchg + slot));
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarXchg + slot), static_cast<uint32_t>(j >> 1) & 1u,
-                                                   abort_flag))) { ok = false; break; }
+            named_bar_sync(1, 256);
+            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
+            if (!ok) continue;
             const float mx = fmaxf(mxh, xmax[(slot * 2 + (hf ^ 1)) * kBlockM + row]);
             const float m_new = fmaxf(m, mx * sl2);
             // PV_{j-1} must be done before P_j overwrites P_{j-1} (and before O is rescaled)
             if (j > 0) {
-                if (!__all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(j - 1) & 1u,
-                                                       abort_flag))) { ok = false; break; }
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(j - 1) & 1u, abort_flag));
+                if (!ok) continue;
                 tc_fence_after();
                 const bool need = m_new > m + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, need)) {
@@ -711,18 +715,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::kBarPFull));
         }
-        // epilogue: combine the partial sums, out = O / l after the last PV
-        bool fin = ok;
-        if (fin) {
+        // epilogue: combine the partial sums (one more named barrier), out = O / l after the last PV
+        {
             const int slot = n_kv & 1;  // last read at tile n_kv-2, free for both warpgroups now
             xmax[(slot * 2 + hf) * kBlockM + row] = l;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarXchg + slot));
-            fin = mbar_wait(bar(C::kBarXchg + slot), static_cast<uint32_t>(n_kv >> 1) & 1u, abort_flag);
-            if (fin) l += xmax[(slot * 2 + (hf ^ 1)) * kBlockM + row];
+            named_bar_sync(1, 256);
+            l += xmax[(slot * 2 + (hf ^ 1)) * kBlockM + row];
         }
-        fin = fin && mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(n_kv - 1) & 1u, abort_flag);
-        if (__all_sync(0xffffffffu, fin)) {
+        const bool fin = __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
+                         __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(n_kv - 1) & 1u,
+                                                           abort_flag));
+        if (fin) {
             tc_fence_after();
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
             const bool valid = qi < w.L;

@@ -71,6 +71,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Hardware named barrier over `count` threads (a multiple of 32).  Callers
+// must guarantee every participating thread reaches it the same number of
+// times (no early exit between them), because it cannot time out.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---------------------------------------------------------------- proxies
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, UMMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
