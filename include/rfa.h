@@ -161,6 +161,32 @@ RFA_API rfa_status rfa_fused_rope_attention_with_table(const rfa_attn_params* p,
                                                        const void* v, const int32_t* seqLens_host, void* out,
                                                        const void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * rfa_fused_rope_attention_noalloc -- rfa_fused_rope_attention without a
+ * caller-provided workspace, for callers that cannot allocate device memory
+ * where they call this library: code running while a stream is captured into
+ * a CUDA graph, plugins whose host framework owns every device buffer and
+ * passes a kernel only its inputs and outputs, real-time callers that may not
+ * block on an allocator.  (The pages have no counterpart; this is a service
+ * of this library.)
+ *
+ * Arguments and results are those of rfa_fused_rope_attention minus
+ * workspace/ws_bytes.  The scratch (cos/sin table and recurrence seeds) is a
+ * fixed area of about 16.1 MB inside the library's module, held by every
+ * device that loads the library until the process exits.  Limits: at most
+ * 65536 tokens (BNSD: B*S), at most 16 sequences (BNSD: batches), D <= 128;
+ * larger problems return RFA_ERR_WORKSPACE before anything is enqueued.
+ * This entry point allocates nothing.  Its first call on a device looks up the
+ * scratch's device address (make that first call before any stream capture).
+ * All calls share the one scratch area, which keeps the last call's contents:
+ * calls whose work overlaps on the GPU (e.g. on different streams without
+ * ordering) race and must be serialised by the caller.
+ */
+RFA_API rfa_status rfa_fused_rope_attention_noalloc(const rfa_attn_params* p, const void* q, const void* k,
+                                                    const void* v, const int32_t* position,
+                                                    const int32_t* seqLens_host, const float* invFreq, void* out,
+                                                    void* stream);
+
 /* Synchronises `stream`, then returns and clears the current device's status
  * word (RFA_OK if no kernel recorded an error).  RFA_ERR_CUDA if the
  * synchronisation itself failed. */

@@ -25,6 +25,7 @@ import torch
 __all__ = [
     "RfaError", "LIB_PATH", "EXPORTS", "load_library", "rope_sincos", "fused_rope_attention",
     "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
+    "fused_rope_attention_noalloc",
     "get_device_status", "status_string", "AttnParams",
 ]
 
@@ -37,6 +38,7 @@ EXPORTS = (
     "rfa_fused_rope_attention",
     "rfa_rope_attention_table",
     "rfa_fused_rope_attention_with_table",
+    "rfa_fused_rope_attention_noalloc",
     "rfa_get_device_status",
     "rfa_status_string",
     "rfa_version",
@@ -95,6 +97,8 @@ def load_library():
     lib.rfa_rope_attention_table.restype = ctypes.c_int
     lib.rfa_fused_rope_attention_with_table.argtypes = [ctypes.POINTER(AttnParams), P, P, P, P, P, P, SZ, P]
     lib.rfa_fused_rope_attention_with_table.restype = ctypes.c_int
+    lib.rfa_fused_rope_attention_noalloc.argtypes = [ctypes.POINTER(AttnParams), P, P, P, P, P, P, P, P]
+    lib.rfa_fused_rope_attention_noalloc.restype = ctypes.c_int
     lib.rfa_get_device_status.argtypes = [P]
     lib.rfa_get_device_status.restype = ctypes.c_int
     lib.rfa_status_string.argtypes = [ctypes.c_int]
@@ -268,6 +272,29 @@ def fused_rope_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, posi
     return out
 
 
+def fused_rope_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, position: torch.Tensor, *,
+                                 layout: str = "BNSD", seq_lens: Optional[Sequence[int]] = None, causal: bool = True,
+                                 scale: Optional[float] = None, rope_base: float = 10000.0, ntk_train_len: int = 0,
+                                 ntk_factor: float = 1.0, inv_freq: Optional[torch.Tensor] = None,
+                                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fused_rope_attention with the library's fixed internal scratch instead of
+    a caller workspace (for callers that cannot allocate device memory; see
+    rfa_fused_rope_attention_noalloc in include/rfa.h for limits and the
+    one-scratch-per-device rule)."""
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    lens, _ = _lens_arg(layout, seq_lens, p)
+    if out is None:
+        out = torch.empty_like(q)
+    io = (torch.bfloat16, torch.float16)
+    code = load_library().rfa_fused_rope_attention_noalloc(
+        ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+        _dev(position, "position", torch.int32), _ptr_or_null(lens),
+        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(out, "out", q.dtype),
+        _stream_ptr(stream))
+    _check(code, "rfa_fused_rope_attention_noalloc")
+    return out
+
+
 def get_device_status(stream=None) -> int:
     """Synchronise the stream and return/clear the device status word."""
     return int(load_library().rfa_get_device_status(_stream_ptr(stream)))
@@ -279,6 +306,7 @@ rfa_fused_rope_attention = fused_rope_attention
 rfa_fused_rope_attention_workspace = fused_rope_attention_workspace
 rfa_rope_attention_table = rope_attention_table
 rfa_fused_rope_attention_with_table = fused_rope_attention_with_table
+rfa_fused_rope_attention_noalloc = fused_rope_attention_noalloc
 rfa_get_device_status = get_device_status
 rfa_status_string = status_string
 

@@ -382,3 +382,74 @@ rfa_status rfa_fused_rope_attention(const rfa_attn_params* p, const void* q, con
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- workspace-free variant
+// Some callers cannot allocate device memory on the path that calls us: code
+// running while a stream is being captured into a CUDA graph, plugins whose
+// host framework owns every device buffer and only hands a kernel its inputs
+// and outputs, and real-time callers that may not block on an allocator.
+// rfa_fused_rope_attention_noalloc serves them with a fixed scratch area that
+// lives in this library's module for as long as the library is loaded.
+namespace {
+
+constexpr int64_t kNoAllocMaxTokens = 65536;  // T limit of the fixed scratch
+constexpr int kNoAllocMaxSeqs = 16;           // sequences (BNSD: batches) limit
+constexpr size_t kNoAllocTableBytes = static_cast<size_t>(kNoAllocMaxTokens) * 128 * 2;  // D <= 128
+constexpr size_t kNoAllocSeedBytes = (kNoAllocMaxSeqs * sizeof(rfa::RopeSeed) + 255) / 256 * 256;
+constexpr size_t kNoAllocBytes = kNoAllocTableBytes + kNoAllocSeedBytes;
+
+}  // namespace
+
+// The scratch itself: one copy per device that loads the module (~16.1 MB).
+// Host code must not pass this symbol to a kernel (on the host it is only a
+// stand-in); its device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (the first call on a device does it; make that call before any
+// stream capture begins).
+rfa_status noalloc_scratch(void** out) {
+    static std::mutex mu;
+    static void* ptrs[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RFA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RFA_ERR_CUDA;
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return RFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rfa_status rfa_fused_rope_attention_noalloc(const rfa_attn_params* p, const void* q, const void* k, const void* v,
+                                            const int32_t* position, const int32_t* seqLens_host,
+                                            const float* invFreq, void* out, void* stream) {
+    int64_t T = 0;
+    rfa_status vs = check_common(p, seqLens_host, &T);
+    if (vs != RFA_OK) return vs;
+    if (!q || !k || !v || !position || !out) return RFA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return RFA_ERR_INVALID_ARG;
+    if (invFreq && !aligned(invFreq, 16)) return RFA_ERR_INVALID_ARG;
+    // The fixed scratch bounds the problem: reject what does not fit.
+    if (T > kNoAllocMaxTokens || p->B > kNoAllocMaxSeqs || workspace_bytes(T, p->D, p->B) > kNoAllocBytes)
+        return RFA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    rfa_status r = noalloc_scratch(&scratch);
+    if (r != RFA_OK) return r;
+    // Nothing in the scratch needs to start at zero: the table and seed
+    // kernels write every byte the attention kernel reads.
+    cudaStream_t st = as_stream(stream);
+    r = enqueue_table(p, T, position, seqLens_host, invFreq, scratch, st);
+    if (r != RFA_OK) return r;
+    return enqueue_attention(p, T, q, k, v, seqLens_host, out, scratch, st);
+}
+
+}  // extern "C"
