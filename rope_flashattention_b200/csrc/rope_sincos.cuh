@@ -177,7 +177,11 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
     }
 }
 
-// One block per sequence: consecutive-positions flag and recurrence seeds.
+// Consecutive-positions flag and recurrence seeds.  Grid (sequences, kSeedSplit):
+// block (b, 0) also checks the sequence's positions; every block computes a
+// share of the seed angles.  Each angle is formed and reduced modulo 2 pi in
+// fp64, then evaluated with fp32 sincos of the reduced angle (|error| ~1e-7).
+constexpr int kSeedSplit = 4;
 __global__ void __launch_bounds__(256) rope_seed_kernel(const __grid_constant__ TableArgs a) {
     const int32_t b = blockIdx.x;
     int32_t tok0, len;
@@ -189,25 +193,30 @@ __global__ void __launch_bounds__(256) rope_seed_kernel(const __grid_constant__ 
         len = a.cum[b + 1] - a.cum[b];
     }
     const int32_t p0 = __ldg(a.pos + tok0);
-    int ok = 1;
-    for (int32_t i = threadIdx.x; i < len; i += blockDim.x)
-        if (__ldg(a.pos + tok0 + i) != p0 + i) ok = 0;
-    ok = __syncthreads_and(ok);
     RopeSeed* sd = a.seeds + b;
+    if (blockIdx.y == 0) {
+        int ok = 1;
+        for (int32_t i = threadIdx.x; i < len; i += blockDim.x)
+            if (__ldg(a.pos + tok0 + i) != p0 + i) ok = 0;
+        ok = __syncthreads_and(ok);
+        if (threadIdx.x == 0) {
+            sd->consecutive = ok;
+            sd->pos0 = p0;
+        }
+    }
     const float* inv = a.inv_dev ? a.inv_dev + static_cast<int64_t>(b) * a.half
                                  : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
-    if (threadIdx.x == 0) {
-        sd->consecutive = ok;
-        sd->pos0 = p0;
-    }
-    for (int32_t i = threadIdx.x; i < a.half * (kSeedRows + 2); i += blockDim.x) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const int32_t nval = a.half * (kSeedRows + 2);
+    for (int32_t i = blockIdx.y * blockDim.x + threadIdx.x; i < nval; i += gridDim.y * blockDim.x) {
         const int32_t j = i % a.half;
         const int32_t k = i / a.half;
         const double w = static_cast<double>(inv[j]);
-        const double ang = (k < kSeedRows) ? (static_cast<double>(p0) + k) * w : (k == kSeedRows ? 16.0 : 128.0) * w;
-        double sn, cs;
-        sincos(ang, &sn, &cs);
-        const float2 v = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+        double ang = (k < kSeedRows) ? (static_cast<double>(p0) + k) * w : (k == kSeedRows ? 16.0 : 128.0) * w;
+        ang -= two_pi * rint(ang / two_pi);
+        float sn, cs;
+        sincosf(static_cast<float>(ang), &sn, &cs);
+        const float2 v = make_float2(cs, sn);
         if (k < kSeedRows)
             sd->z0[k][j] = v;
         else if (k == kSeedRows)
