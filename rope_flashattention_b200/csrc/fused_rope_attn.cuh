@@ -230,7 +230,7 @@ template <int D, bool kFP16>
 __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t rows, int32_t rt) {
     constexpr int kPairsPerRow = D / 16;  // 16-byte chunk pairs per row
     constexpr int kIters = kBlockM * kPairsPerRow / 128;
-#pragma unroll 2
+#pragma unroll 1
     for (int it = 0; it < kIters; ++it) {
         const int task = rt + 128 * it;
         const int r = task / kPairsPerRow;
@@ -331,7 +331,7 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
 template <int D>
 __device__ __forceinline__ void tile_row_to_tmem(uint32_t tile, uint32_t taddr, int32_t r) {
     const uint32_t sw = static_cast<uint32_t>(r & 7);
-#pragma unroll
+#pragma unroll 1
     for (int h = 0; h < D / 32; ++h) {  // 16 columns = 32 elements = 4 chunks per store
         uint32_t v[16];
 #pragma unroll

@@ -54,9 +54,10 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Bounded wait for the phase of `bar` with parity `parity` to complete.
 // Returns false (and raises *abort) if the wait timed out or another role of
-// this CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int32_t* abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+// this CTA already aborted.  The first poll is inlined at every call site; the
+// spin loop is one shared out-of-line copy, so warps waiting at different
+// places do not each keep their own copy of it in the instruction cache.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int32_t* abort) {
     uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -69,6 +70,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             }
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int32_t* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort);
 }
 
 // Hardware named barrier over `count` threads (a multiple of 32).  Callers
