@@ -165,13 +165,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's figure: every multi-GPU time is the max over ranks."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job rate: every rank runs its own replica (weak scaling), so the
+    units of all ranks are divided by the slowest rank's time per step."""
+    return units_per_rank * world / (ms * 1e-3)
 
 
 # ------------------------------------------------------------------ workload helpers
@@ -423,7 +431,7 @@ def run_gpu(args, world, rank, local):
     attn_ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
     ms = max_over_ranks(ms_local, world)
     attn_ms = max_over_ranks(attn_ms_local, world)
-    value = flops * world / (ms * 1e-3) / 1e12
+    value = job_throughput(flops, world, ms) / 1e12
 
     # ---------------- end to end: host buffers through the C ABI
     qp, kp, vp, posp = (x.pin_memory() for x in (q_h, k_h, v_h, pos_h))
@@ -479,11 +487,11 @@ def run_gpu(args, world, rank, local):
                      "traffic": traffic,
                      "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
                      "kernel": "fused_rope_attn_fwd_kernel", "kernel_ms": attn_ms, "kernel_source": kernel_hash()},
-        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(flops, world, e2e_ms) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * K,
         "clocks": clk,
-        "tok_per_s": workloads.ntokens(w) * world / (ms * 1e-3),
+        "tok_per_s": job_throughput(workloads.ntokens(w), world, ms),
     }
     line.update(extra)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
