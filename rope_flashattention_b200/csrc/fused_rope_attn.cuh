@@ -10,31 +10,36 @@
 // The rotated tiles exist only in shared memory; nothing rotated is written
 // back to global memory.
 //
-// One CTA = one work item (sequence, query head, 128-row query tile).  Warp roles:
-//   warps 0-7  two softmax warpgroups; warpgroup g takes key columns
-//              [64g, 64g + 64) of every score tile, thread t of it owns query
-//              row t (TMEM lane t).  Per tile: load its half of S from TMEM,
-//              mask, exchange the half-row maxima through shared memory (named
-//              barrier 1 over the 256 softmax threads), keep
-//              the running max (identical in both) and a partial sum, write P
-//              (bf16/fp16) into TMEM, rescale its half of O only when the max
-//              grows by > 2^8.  At the end the partial sums are combined and
-//              each warpgroup normalises and stores half of the columns.
-//   warps 8-11 RoPE warpgroup: rotates the Q tile once (then moves Q' into
-//              TMEM, where the QK MMAs read it) and every K tile in place in
-//              the 128B-swizzled shared-memory layout.  Element i and its
-//              rotate-half partner i + D/2 sit at the same offset of two swizzle
-//              atoms (D = 128) or in chunks c and c ^ 4 of one atom (D = 64).
-//              K angles come from a complex recurrence in registers when the
-//              sequence's positions are consecutive, else from cos/sin rows
-//              that TMA staged next to the tile.
-//   warp 12    TMA producer: Q (+ its cos/sin rows) once, then K tiles (+ rows
-//              when needed) through a kStages ring.
-//   warp 13    tcgen05 issuer (one thread) and TMEM owner: S_j = Q'K_j'^T into
-//              TMEM buffer j % 2 (A = Q' from TMEM), O += P_j V_j (A = P from
-//              TMEM, B = V from shared memory); S_{j+2} is issued as soon as
-//              the softmax has read S_j, ahead of PV_j.
-//   warp 14    TMA producer for the V ring.
+// One CTA = one work item: two 128-row query tiles that read the same key /
+// value tiles -- two query heads of one kv group at the same rows when the
+// group size G is even, else two consecutive query tiles of one head (the
+// second may be absent at the end of a sequence).  Every key tile is loaded
+// and rotated once for both query tiles.  Warp roles:
+//   warps 0-3  softmax warpgroup of query tile 0, warps 4-7 of query tile 1;
+//              thread t owns query row t (TMEM lane t).  Per key tile: row
+//              maximum from a first read of S (TMEM), exponentials from a
+//              second read, 32 columns at a time; P (bf16/fp16) is written in
+//              place over the S columns already read; O is rescaled only when
+//              the maximum grows by > 2^8.  At the end: O / l to global memory.
+//   warps 8-15 two RoPE warpgroups: rotate both query tiles once, then every
+//              key tile, in place in the 128B-swizzled shared-memory layout.
+//              Element i and its rotate-half partner i + D/2 sit at the same
+//              offset of two swizzle atoms (D = 128) or in chunks c and c ^ 4
+//              of one atom (D = 64).  Key angles come from a complex
+//              recurrence in registers when the sequence's positions are
+//              consecutive, else from cos/sin rows that TMA staged beside the
+//              tile; query angles always from staged rows.
+//   warp 16    TMA producer: both query tiles (+ their cos/sin rows, staged in
+//              the first two V slots) once, then key tiles (+ rows when
+//              needed) through a kStages ring.
+//   warp 17    tcgen05 issuer (one thread) and TMEM owner.  Order per key
+//              tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), where
+//              S_i = Q_i' K_j'^T goes to TMEM buffer i and O_i += P_i V_j reads
+//              P_i from that same buffer.  MMAs issued by one thread execute
+//              in issue order, so QK_i(j+1) overwrites P_i only after PV_i(j)
+//              has read it, and S_i(j+1) being complete implies O_i holds
+//              PV_i(j).
+//   warp 18    TMA producer for the V ring.
 // Completion of every async step is tracked by mbarriers; each wait is bounded.
 #pragma once
 #include <cuda.h>
@@ -50,12 +55,14 @@ namespace rfa {
 
 constexpr int kBlockM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per tile
-constexpr int kAttnThreads = 512;
+constexpr int kAttnThreads = 640;
 constexpr int kRopeWarp0 = 8;
-constexpr int kTmaWarp = 12;   // Q, K (+ cos/sin rows)
-constexpr int kMmaWarp = 13;
-constexpr int kTmaVWarp = 14;  // V: its own producer, so K prefetch never waits on a V slot
-// warp 15 only takes part in the block-wide barriers
+constexpr int kRopeWarps = 8;   // two RoPE warpgroups share every tile
+constexpr int kRopeThreads = kRopeWarps * 32;
+constexpr int kTmaWarp = 16;    // Q, K (+ cos/sin rows)
+constexpr int kMmaWarp = 17;
+constexpr int kTmaVWarp = 18;   // V: its own producer, so K prefetch never waits on a V slot
+// warp 19 only takes part in the block-wide barriers
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
 struct AttnArgs {
@@ -65,6 +72,7 @@ struct AttnArgs {
     int32_t B, Hq, Hkv, G;
     int32_t S;       // BNSD sequence length
     int32_t causal;
+    int32_t pair_heads;  // 1: an item's query tiles are heads 2p, 2p+1 at one tile (G even); 0: tiles 2p, 2p+1 of one head
     float scale_log2;  // softmax scale * log2(e)
     int32_t n_items;
     // TND: sequences sorted by length, descending; seg_item0[k] = first work item of sequence k
@@ -76,6 +84,11 @@ struct AttnArgs {
     int32_t seg_orig[16];  // caller's index of sorted sequence k
 };
 
+// Work items of one sequence with nt query tiles.
+__host__ __device__ inline int32_t items_per_sequence(int32_t Hq, int32_t nt, bool pair_heads) {
+    return pair_heads ? (Hq / 2) * nt : Hq * ((nt + 1) / 2);
+}
+
 template <int D>
 struct AttnCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
@@ -84,77 +97,92 @@ struct AttnCfg {
     static constexpr int kTileBytes = kBlockM * D * 2;    // Q, K or V tile
     static constexpr int kTabBytes = kBlockM * D * 2;     // cos/sin rows of a tile: D/2 fp16 cos + D/2 fp16 sin
     static constexpr int kTabBoxes = D / 64;              // 128-byte boxes of 32 (cos, sin) pairs
-    static constexpr int kStages = (D == 64) ? 4 : 2;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;
+    static constexpr int kStages = (D == 64) ? 4 : 2;     // K ring and V ring
+    static constexpr int kTStages = (D == 64) ? 4 : 1;    // cos/sin rows of key tiles (positions not consecutive)
+    static constexpr int kOffQ = 0;                       // two query tiles
+    static constexpr int kOffK = kOffQ + 2 * kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kTileBytes;
     static constexpr int kOffT = kOffV + kStages * kTileBytes;
-    static constexpr int kOffBar = kOffT + kStages * kTabBytes;
+    static constexpr int kOffBar = kOffT + kTStages * kTabBytes;
     // barrier indices
-    static constexpr int kBarQFull = 0, kBarQReady = 1;
+    static constexpr int kBarQFull = 0;  // both query tiles and their cos/sin rows landed
+    static constexpr int kBarQReady = 1; // both rotated (8 RoPE warp arrivals); their rows' V slots are free
     static constexpr int kBarKFull = 2;
     static constexpr int kBarVFull = kBarKFull + kStages;
     static constexpr int kBarKReady = kBarVFull + kStages;
     static constexpr int kBarKEmpty = kBarKReady + kStages;
     static constexpr int kBarVEmpty = kBarKEmpty + kStages;
-    static constexpr int kBarSFull = kBarVEmpty + kStages;  // 2: S_j in TMEM buffer j % 2
-    static constexpr int kBarSEmpty = kBarSFull + 2;        // 2: both warpgroups have read S_j (8 warp arrivals)
-    static constexpr int kBarPFull = kBarSEmpty + 2;        // P_j written (8 warp arrivals)
-    static constexpr int kBarPVDone = kBarPFull + 1;        // PV_j done: O updated, P free
-    static constexpr int kBarMmaFin = kBarPVDone + 1;
-    static constexpr int kBarQRot = kBarMmaFin + 1;         // Q' rotated in shared memory (4 warp arrivals)
-    static constexpr int kNumBars = kBarQRot + 1;
+    static constexpr int kBarSFull = kBarVEmpty + kStages;  // 2: S_i complete (and every earlier MMA)
+    static constexpr int kBarPFull = kBarSFull + 2;         // 2: P_i written, O_i rescaled (4 warp arrivals)
+    static constexpr int kBarOFull = kBarPFull + 2;         // 2: last PV_i complete
+    static constexpr int kBarMmaFin = kBarOFull + 2;
+    static constexpr int kNumBars = kBarMmaFin + 1;
     static constexpr int kOffAbort = kOffBar + 8 * kNumBars;
     static constexpr int kOffTmemSlot = kOffAbort + 16;
-    static constexpr int kOffXchg = kOffTmemSlot + 16;  // float [2 slots][2 halves][128 rows]
     // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (the
     // kernel checks it), so no alignment slack is requested.
-    static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBlockM * 4;
-    // TMEM columns: S/score buffers, O accumulator, Q' and P (16-bit, two per column)
+    static constexpr int kSmemBytes = kOffTmemSlot + 16;
+    // TMEM columns: S_0, S_1 (P_i over the first 64 columns of S_i), O_0, O_1
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS = 0;      // 2 x 128
-    static constexpr uint32_t kColO = 256;    // D
-    static constexpr uint32_t kColQ = 384;    // D / 2
-    static constexpr uint32_t kColP = 448;    // 64
-    static_assert(kColO + D <= kColQ && kColQ + D / 2 <= kColP && kColP + kBlockN / 2 <= kTmemCols, "TMEM budget");
+    static constexpr uint32_t kColS = 0;      // S_i at 128 i
+    static constexpr uint32_t kColO = 256;    // O_i at 256 + D i
+    static_assert(kColO + 2 * D <= kTmemCols, "TMEM budget");
+    static_assert(kStages >= 2 && kTabBytes == kTileBytes, "query cos/sin rows are staged in V slots 0 and 1");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct WorkItem {
-    int32_t orig;  // sequence index in the caller's order
-    int32_t tok0;  // first token of the sequence (BNSD: seq * S)
-    int32_t seq;   // BNSD batch index
-    int32_t L;     // sequence length
-    int32_t h;     // query head
-    int32_t qt;    // query tile index within the sequence
+    int32_t orig;   // sequence index in the caller's order
+    int32_t tok0;   // first token of the sequence (BNSD: seq * S)
+    int32_t seq;    // BNSD batch index / TND sorted sequence index
+    int32_t L;      // sequence length
+    int32_t kvh;    // kv head read by both query tiles
+    int32_t h[2];   // query heads
+    int32_t qt[2];  // query tile indices within the sequence; qt[1] < 0: no second tile
 };
 
-// Head-major order (all query tiles of one head are neighbours, so the CTAs
-// resident at one time share K/V tiles through L2), largest tile first within
-// a head; packed sequences longest first.
+// Head-major order (the items of one head / head pair are neighbours, so the
+// CTAs resident at one time share K/V tiles through L2), largest tiles first;
+// packed sequences longest first.
 __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     WorkItem w;
+    int32_t nt, r;
+    const bool ph = a.pair_heads != 0;
     if (a.layout == 0) {
-        const int32_t nqt = (a.S + kBlockM - 1) / kBlockM;
-        const int32_t bh = x / nqt;
-        w.qt = nqt - 1 - (x - bh * nqt);
-        w.seq = bh / a.Hq;
-        w.h = bh - w.seq * a.Hq;
+        nt = (a.S + kBlockM - 1) / kBlockM;
+        const int32_t per = items_per_sequence(a.Hq, nt, ph);
+        w.seq = x / per;
+        r = x - w.seq * per;
+        w.orig = w.seq;
         w.tok0 = w.seq * a.S;
         w.L = a.S;
-        w.orig = w.seq;
-        return w;
+    } else {
+        int32_t s = 0;
+        while (s + 1 < a.nseg && x >= a.seg_item0[s + 1]) ++s;
+        r = x - a.seg_item0[s];
+        nt = a.seg_tiles[s];
+        w.seq = s;
+        w.orig = a.seg_orig[s];
+        w.tok0 = a.seg_start[s];
+        w.L = a.seg_len[s];
     }
-    int32_t s = 0;
-    while (s + 1 < a.nseg && x >= a.seg_item0[s + 1]) ++s;
-    const int32_t r = x - a.seg_item0[s];
-    const int32_t nt = a.seg_tiles[s];
-    w.h = r / nt;
-    w.qt = nt - 1 - (r - w.h * nt);
-    w.seq = s;
-    w.orig = a.seg_orig[s];
-    w.tok0 = a.seg_start[s];
-    w.L = a.seg_len[s];
+    if (ph) {
+        const int32_t hp = r / nt;
+        const int32_t qt = nt - 1 - (r - hp * nt);
+        w.h[0] = 2 * hp;
+        w.h[1] = 2 * hp + 1;
+        w.qt[0] = qt;
+        w.qt[1] = qt;
+    } else {
+        const int32_t np = (nt + 1) / 2;
+        const int32_t h = r / np;
+        const int32_t p = np - 1 - (r - h * np);
+        w.h[0] = h;
+        w.h[1] = h;
+        w.qt[0] = 2 * p;
+        w.qt[1] = (2 * p + 1 < nt) ? 2 * p + 1 : -1;
+    }
+    w.kvh = w.h[0] / a.G;
     return w;
 }
 
@@ -229,10 +257,10 @@ __device__ __forceinline__ void rotate8(uint4& x1, uint4& x2, const uint4& t0, c
 template <int D, bool kFP16>
 __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t rows, int32_t rt) {
     constexpr int kPairsPerRow = D / 16;  // 16-byte chunk pairs per row
-    constexpr int kIters = kBlockM * kPairsPerRow / 128;
+    constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
 #pragma unroll 1
     for (int it = 0; it < kIters; ++it) {
-        const int task = rt + 128 * it;
+        const int task = rt + kRopeThreads * it;
         const int r = task / kPairsPerRow;
         const int cp = task % kPairsPerRow;
         if (r >= rows) continue;
@@ -285,12 +313,12 @@ template <int D, bool kFP16>
 __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32_t rt, const RecState& z,
                                               const uint64_t (&wc)[4], const uint64_t (&ws)[4]) {
     constexpr int kPairsPerRow = D / 16;
-    constexpr int kIters = kBlockM * kPairsPerRow / 128;
-    constexpr int kStep = 128 / kPairsPerRow;
+    constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
+    constexpr int kStep = kRopeThreads / kPairsPerRow;
     const int cp = rt % kPairsPerRow;
     const int r0 = rt / kPairsPerRow;
     RecState e = z;
-    // Modest unrolling: 16 warps run four roles at once and their hot loops
+    // Modest unrolling: 20 warps run five roles at once and their hot loops
     // must stay resident in the instruction cache.
 #pragma unroll 2
     for (int it = 0; it < kIters; ++it) {
@@ -325,28 +353,6 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
     }
 }
 
-// Copy this thread's row (rt) of a rotated 128-row tile from 128B-swizzled
-// shared memory into TMEM columns col0.. as packed 16-bit pairs (the A-operand
-// layout of tcgen05.mma: lane = row, column c = elements 2c, 2c+1).
-template <int D>
-__device__ __forceinline__ void tile_row_to_tmem(uint32_t tile, uint32_t taddr, int32_t r) {
-    const uint32_t sw = static_cast<uint32_t>(r & 7);
-#pragma unroll 1
-    for (int h = 0; h < D / 32; ++h) {  // 16 columns = 32 elements = 4 chunks per store
-        uint32_t v[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int c = h * 4 + q;  // logical 16-byte chunk of the row
-            const uint4 x = lds128(tile + (c >> 3) * AttnCfg<D>::kAtomBytes + r * 128 + (((c & 7) ^ sw) << 4));
-            v[4 * q + 0] = x.x;
-            v[4 * q + 1] = x.y;
-            v[4 * q + 2] = x.z;
-            v[4 * q + 3] = x.w;
-        }
-        tmem_st16(taddr + h * 16, v);
-    }
-}
-
 // Bounded wait that ignores the abort flag: used to drain in-flight async
 // copies and MMAs before the CTA exits.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
@@ -370,6 +376,7 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
         : "memory");
 }
 
+
 template <int D, bool kFP16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     fused_rope_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -390,29 +397,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const WorkItem w = decode_item(a, blockIdx.x);
-    const int32_t kvh = w.h / a.G;
-    const int32_t n_kv = a.causal ? (w.qt + 1) : (w.L + kBlockN - 1) / kBlockN;
+    const int32_t nq = (w.qt[1] >= 0) ? 2 : 1;  // query tiles in this item
+    const int32_t nkt = (w.L + kBlockN - 1) / kBlockN;
+    // key tiles read by query tile i (0: tile absent)
+    const int32_t n0 = a.causal ? (w.qt[0] + 1) : nkt;
+    const int32_t n1 = (nq == 1) ? 0 : (a.causal ? (w.qt[1] + 1) : nkt);
+    const int32_t n_kv = max(n0, n1);
     // consecutive positions: K angles come from the recurrence, no cos/sin rows per K tile
     const bool rec = a.seeds[w.orig].consecutive != 0;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::kBarQFull), 1);
-        mbar_init(bar(C::kBarQReady), 4);
+        mbar_init(bar(C::kBarQReady), kRopeWarps);
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(bar(C::kBarKFull + s), 1);
             mbar_init(bar(C::kBarVFull + s), 1);
-            mbar_init(bar(C::kBarKReady + s), 4);
+            mbar_init(bar(C::kBarKReady + s), kRopeWarps);
             mbar_init(bar(C::kBarKEmpty + s), 1);
             mbar_init(bar(C::kBarVEmpty + s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(C::kBarSFull + b), 1);
-            mbar_init(bar(C::kBarSEmpty + b), 8);  // one arrival per softmax warp
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(C::kBarSFull + i), 1);
+            mbar_init(bar(C::kBarPFull + i), 4);  // one arrival per warp of softmax warpgroup i
+            mbar_init(bar(C::kBarOFull + i), 1);
         }
-        mbar_init(bar(C::kBarPFull), 8);
-        mbar_init(bar(C::kBarPVDone), 1);
         mbar_init(bar(C::kBarMmaFin), 1);
-        mbar_init(bar(C::kBarQRot), 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -432,8 +441,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmT);
             const bool bnsd = (a.layout == 0);
-            const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h) : w.h;
-            const int32_t kvplane = bnsd ? (w.seq * a.Hkv + kvh) : kvh;
+            const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
             auto load_tile = [&](const CUtensorMap* m, uint32_t dst, uint32_t b, int32_t plane, int32_t row0) {
                 for (int at = 0; at < C::kAtoms; ++at) {
                     if (bnsd)
@@ -446,20 +454,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int bx = 0; bx < C::kTabBoxes; ++bx)
                     tma_load_3d(dst + bx * C::kAtomBytes, &tmT, b, bx * 32, w.tok0 + row0, 0);
             };
+            // query tiles and their cos/sin rows (staged in V slots 0 and 1 until QReady)
+            mbar_expect_tx(bar(C::kBarQFull), static_cast<uint32_t>(nq) * (C::kTileBytes + C::kTabBytes));
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (i >= nq) break;
+                const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
+                load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane, w.qt[i] * kBlockM);
+                load_tab(sbase + C::kOffV + i * C::kTileBytes, bar(C::kBarQFull), w.qt[i] * kBlockM);
+            }
             const uint32_t kbytes = C::kTileBytes + (rec ? 0 : C::kTabBytes);
-            // Q and its cos/sin rows; the rows go to table stage 1, free until K tile 1.
-            mbar_expect_tx(bar(C::kBarQFull), C::kTileBytes + C::kTabBytes);
-            load_tile(&tmQ, sbase + C::kOffQ, bar(C::kBarQFull), qplane, w.qt * kBlockM);
-            load_tab(sbase + C::kOffT + 1 * C::kTabBytes, bar(C::kBarQFull), w.qt * kBlockM);
             int32_t issued_k = 0;
             for (int32_t j = 0; j < n_kv; ++j) {
                 const int s = j % C::kStages;
                 const uint32_t u = static_cast<uint32_t>(j / C::kStages);
-                if (!rec && j == 1 && !mbar_wait(bar(C::kBarQReady), 0, abort_flag)) break;  // Q's rows consumed
                 if (u > 0 && !mbar_wait(bar(C::kBarKEmpty + s), (u - 1) & 1u, abort_flag)) break;
+                if (!rec && j >= C::kTStages) {
+                    // the rows slot held the rows of key tile j - kTStages: wait until that tile is rotated
+                    const int32_t jp = j - C::kTStages;
+                    if (!mbar_wait(bar(C::kBarKReady + jp % C::kStages), static_cast<uint32_t>(jp / C::kStages) & 1u,
+                                   abort_flag))
+                        break;
+                }
                 mbar_expect_tx(bar(C::kBarKFull + s), kbytes);
                 load_tile(&tmK, sbase + C::kOffK + s * C::kTileBytes, bar(C::kBarKFull + s), kvplane, j * kBlockN);
-                if (!rec) load_tab(sbase + C::kOffT + s * C::kTabBytes, bar(C::kBarKFull + s), j * kBlockN);
+                if (!rec) load_tab(sbase + C::kOffT + (j % C::kTStages) * C::kTabBytes, bar(C::kBarKFull + s), j * kBlockN);
                 issued_k = j + 1;
             }
             // Drain: every issued copy must have landed before the CTA exits.
@@ -472,22 +491,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tmV);
             const bool bnsd = (a.layout == 0);
-            const int32_t kvplane = bnsd ? (w.seq * a.Hkv + kvh) : kvh;
+            const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
             int32_t issued_v = 0;
-            for (int32_t j = 0; j < n_kv; ++j) {
-                const int s = j % C::kStages;
-                const uint32_t u = static_cast<uint32_t>(j / C::kStages);
-                if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) break;
-                mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-                const uint32_t dst = sbase + C::kOffV + s * C::kTileBytes;
-                for (int at = 0; at < C::kAtoms; ++at) {
-                    if (bnsd)
-                        tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, j * kBlockN, kvplane);
-                    else
-                        tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, kvplane,
-                                    w.tok0 + j * kBlockN);
+            // V slots 0 and 1 hold the query tiles' cos/sin rows until both are rotated
+            if (mbar_wait(bar(C::kBarQReady), 0, abort_flag)) {
+                for (int32_t j = 0; j < n_kv; ++j) {
+                    const int s = j % C::kStages;
+                    const uint32_t u = static_cast<uint32_t>(j / C::kStages);
+                    if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) break;
+                    mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+                    const uint32_t dst = sbase + C::kOffV + s * C::kTileBytes;
+                    for (int at = 0; at < C::kAtoms; ++at) {
+                        if (bnsd)
+                            tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, j * kBlockN,
+                                        kvplane);
+                        else
+                            tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, kvplane,
+                                        w.tok0 + j * kBlockN);
+                    }
+                    issued_v = j + 1;
                 }
-                issued_v = j + 1;
             }
             for (int32_t j = (issued_v > C::kStages ? issued_v - C::kStages : 0); j < issued_v; ++j)
                 mbar_wait_drain(bar(C::kBarVFull + j % C::kStages), static_cast<uint32_t>(j / C::kStages) & 1u);
@@ -497,113 +520,124 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_f16(IoT<kFP16>::kFmt, 0, 0, kBlockM, kBlockN);
             constexpr uint32_t kIdescPV = idesc_f16(IoT<kFP16>::kFmt, 0, 1, kBlockM, D);
-            auto issue_qk = [&](int32_t j) -> bool {
-                const int s = j % C::kStages;
-                const int b = j & 1;
-                if (!mbar_wait(bar(C::kBarKReady + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag))
-                    return false;
-                // buffer b held S_{j-2}: both softmax warpgroups must have read it
-                if (j >= 2 && !mbar_wait(bar(C::kBarSEmpty + b), static_cast<uint32_t>((j >> 1) - 1) & 1u, abort_flag))
-                    return false;
-                tc_fence_after();
-                const uint32_t kbase = sbase + C::kOffK + s * C::kTileBytes;
+            // S_i = Q_i' K_j'^T into TMEM buffer i (A = Q_i' and B = K_j' from shared memory)
+            auto issue_qk = [&](int i, int32_t j) {
+                const uint32_t kbase = sbase + C::kOffK + (j % C::kStages) * C::kTileBytes;
+                const uint32_t qbase = sbase + C::kOffQ + i * C::kTileBytes;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t koff = (k >> 2) * C::kAtomBytes + (k & 3) * 32;
-                    const uint64_t bd = smem_desc_sw128(kbase + koff, 16, 1024);
-                    // A = Q' from TMEM: 16 elements of K = 8 packed columns per step
-                    umma_ts(tmem + C::kColS + b * kBlockN, tmem + C::kColQ + k * 8, bd, kIdescQK, k > 0 ? 1u : 0u);
+                    umma_ss(tmem + C::kColS + i * kBlockN, smem_desc_sw128(qbase + koff, 16, 1024),
+                            smem_desc_sw128(kbase + koff, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
                 }
-                tc_commit(bar(C::kBarSFull + b));
-                tc_commit(bar(C::kBarKEmpty + s));
-                return true;
+                tc_commit(bar(C::kBarSFull + i));
             };
-            auto issue_pv = [&](int32_t i) -> bool {
-                const int s = i % C::kStages;
-                if (!mbar_wait(bar(C::kBarPFull), static_cast<uint32_t>(i) & 1u, abort_flag)) return false;
-                if (!mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(i / C::kStages) & 1u, abort_flag))
-                    return false;
-                tc_fence_after();
-                const uint32_t vbase = sbase + C::kOffV + s * C::kTileBytes;
+            // O_i += P_i V_j (A = P_i from the first 64 columns of TMEM buffer i, B = V_j from shared memory)
+            auto issue_pv = [&](int i, int32_t j) {
+                const uint32_t vbase = sbase + C::kOffV + (j % C::kStages) * C::kTileBytes;
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k) {
                     const uint64_t bd = smem_desc_sw128(vbase + k * 16 * 128, C::kAtomBytes, 1024);
-                    umma_ts(tmem + C::kColO, tmem + C::kColP + k * 8, bd, kIdescPV, (i > 0 || k > 0) ? 1u : 0u);
+                    umma_ts(tmem + C::kColO + i * D, tmem + C::kColS + i * kBlockN + k * 8, bd, kIdescPV,
+                            (j > 0 || k > 0) ? 1u : 0u);
                 }
-                tc_commit(bar(C::kBarPVDone));
-                tc_commit(bar(C::kBarVEmpty + s));
-                return true;
             };
-            bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag);
+            bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag) && mbar_wait(bar(C::kBarKReady), 0, abort_flag);
             if (ok) {
                 tc_fence_after();
-                ok = issue_qk(0);
-                if (ok && n_kv > 1) ok = issue_qk(1);
-                for (int32_t j = 0; j < n_kv && ok; ++j) {
-                    if (j + 2 < n_kv) ok = issue_qk(j + 2);
-                    if (ok) ok = issue_pv(j);
+                if (n0 > 0) issue_qk(0, 0);
+                if (n1 > 0) issue_qk(1, 0);
+                tc_commit(bar(C::kBarKEmpty));
+            }
+            for (int32_t j = 0; j < n_kv && ok; ++j) {
+                const int s = j % C::kStages;
+                const int32_t jn = j + 1;
+                ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag);
+                if (!ok) break;
+                if (j < n0) {
+                    ok = mbar_wait(bar(C::kBarPFull + 0), static_cast<uint32_t>(j) & 1u, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(0, j);
+                    if (j == n0 - 1) tc_commit(bar(C::kBarOFull + 0));
+                }
+                if (jn < n_kv) {
+                    ok = mbar_wait(bar(C::kBarKReady + jn % C::kStages), static_cast<uint32_t>(jn / C::kStages) & 1u,
+                                   abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (jn < n0) issue_qk(0, jn);
+                }
+                if (j < n1) {
+                    ok = mbar_wait(bar(C::kBarPFull + 1), static_cast<uint32_t>(j) & 1u, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(1, j);
+                    if (j == n1 - 1) tc_commit(bar(C::kBarOFull + 1));
+                }
+                tc_commit(bar(C::kBarVEmpty + s));
+                if (jn < n_kv) {
+                    if (jn < n1) issue_qk(1, jn);
+                    tc_commit(bar(C::kBarKEmpty + jn % C::kStages));
                 }
             }
             tc_commit(bar(C::kBarMmaFin));
             mbar_wait_drain(bar(C::kBarMmaFin), 0);
         }
-    } else if (warp >= kRopeWarp0 && warp < kRopeWarp0 + 4) {
-        // ------------------------------------------------------------ RoPE warpgroup
-        const int32_t rt = threadIdx.x - kRopeWarp0 * 32;  // == TMEM lane of this thread
+    } else if (warp >= kRopeWarp0 && warp < kRopeWarp0 + kRopeWarps) {
+        // ------------------------------------------------------------ RoPE warpgroups
+        const int32_t rt = threadIdx.x - kRopeWarp0 * 32;  // 0..255
         constexpr int kPairsPerRow = D / 16;
+        constexpr int kStep = kRopeThreads / kPairsPerRow;  // rows between a thread's tasks
         RecState z;
-        uint64_t wc[4], ws[4], wc128[4], ws128[4];
+        uint64_t wc[4], ws[4];
+        const RopeSeed* sd = a.seeds + w.orig;
         if (rec) {
-            const RopeSeed* sd = a.seeds + w.orig;
             const int cp = rt % kPairsPerRow;
-            const int r0 = rt / kPairsPerRow;
+            const int r0 = rt / kPairsPerRow;  // < kStep
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int f = 8 * cp + 2 * k;
-                float2 z0 = sd->z0[r0 % kSeedRows][f], z1 = sd->z0[r0 % kSeedRows][f + 1];
+                const float2 z0 = sd->z0[r0 % kSeedRows][f], z1 = sd->z0[r0 % kSeedRows][f + 1];
                 const float2 w0 = sd->w16[f], w1 = sd->w16[f + 1];
-                wc[k] = f2pack(w0.x, w1.x);
-                ws[k] = f2pack(w0.y, w1.y);
+                const uint64_t w16c = f2pack(w0.x, w1.x), w16s = f2pack(w0.y, w1.y);
                 z.c[k] = f2pack(z0.x, z1.x);
                 z.s[k] = f2pack(z0.y, z1.y);
-                if (r0 >= kSeedRows) rec_step(z.c[k], z.s[k], wc[k], ws[k]);  // D = 64: rows 16..31
-                if (D == 64) {  // D = 64 steps by 32 rows: w32 = w16^2
-                    uint64_t c2 = wc[k], s2 = ws[k];
-                    rec_step(c2, s2, wc[k], ws[k]);
-                    wc[k] = c2;
-                    ws[k] = s2;
-                }
-                const float2 v0 = sd->w128[f], v1 = sd->w128[f + 1];
-                wc128[k] = f2pack(v0.x, v1.x);
-                ws128[k] = f2pack(v0.y, v1.y);
+                for (int q = 0; q < r0 / kSeedRows; ++q) rec_step(z.c[k], z.s[k], w16c, w16s);  // rows >= 16
+                // step of kStep rows: w16^(kStep/16)
+                wc[k] = w16c;
+                ws[k] = w16s;
+#pragma unroll
+                for (int q = 1; q < kStep / kSeedRows; ++q) rec_step(wc[k], ws[k], w16c, w16s);
             }
         }
         if (mbar_wait(bar(C::kBarQFull), 0, abort_flag)) {
-            const int32_t q0 = w.qt * kBlockM;
-            rope_tile<D, kFP16>(sbase + C::kOffQ, sbase + C::kOffT + 1 * C::kTabBytes, min(kBlockM, w.L - q0), rt);
-            // all of Q' rotated (by every RoPE warp) before rows are copied to TMEM
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarQRot));
-            const bool qrot = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarQRot), 0, abort_flag));
-            if (qrot) {
-                tile_row_to_tmem<D>(sbase + C::kOffQ, tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + C::kColQ, rt);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::kBarQReady));
+#pragma unroll 1
+            for (int i = 0; i < nq; ++i) {
+                const int32_t q0 = (i == 0 ? w.qt[0] : w.qt[1]) * kBlockM;
+                rope_tile<D, kFP16>(sbase + C::kOffQ + i * C::kTileBytes, sbase + C::kOffV + i * C::kTileBytes,
+                                    min(kBlockM, w.L - q0), rt);
             }
-            for (int32_t j = 0; j < n_kv && qrot; ++j) {
+            fence_proxy_async_smem();  // Q' written by the generic proxy, read by the tensor cores
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::kBarQReady));
+            for (int32_t j = 0; j < n_kv; ++j) {
                 const int s = j % C::kStages;
                 const uint32_t u = static_cast<uint32_t>(j / C::kStages);
                 if (!mbar_wait(bar(C::kBarKFull + s), u & 1u, abort_flag)) break;
                 const int32_t k0 = j * kBlockN;
                 if (rec) {
                     rope_tile_rec<D, kFP16>(sbase + C::kOffK + s * C::kTileBytes, min(kBlockN, w.L - k0), rt, z, wc, ws);
+                    // advance to the next tile by 128 rows (the step is re-read from the cached seed)
+                    const int f0 = 8 * (rt % kPairsPerRow);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) rec_step(z.c[k], z.s[k], wc128[k], ws128[k]);
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 v0 = sd->w128[f0 + 2 * k], v1 = sd->w128[f0 + 2 * k + 1];
+                        rec_step(z.c[k], z.s[k], f2pack(v0.x, v1.x), f2pack(v0.y, v1.y));
+                    }
                 } else {
-                    rope_tile<D, kFP16>(sbase + C::kOffK + s * C::kTileBytes, sbase + C::kOffT + s * C::kTabBytes,
-                                        min(kBlockN, w.L - k0), rt);
+                    rope_tile<D, kFP16>(sbase + C::kOffK + s * C::kTileBytes,
+                                        sbase + C::kOffT + (j % C::kTStages) * C::kTabBytes, min(kBlockN, w.L - k0), rt);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -612,74 +646,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax warpgroups
-        // The two warpgroups meet at named barrier 1 exactly n_kv + 1 times: a
-        // failed (timed-out) wait only turns the remaining work into no-ops,
-        // it never skips a barrier, so the barrier cannot deadlock.
-        const int hf = warp >> 2;            // key-column half of every score tile
+        const int i = warp >> 2;             // query tile of this warpgroup
+        const int32_t n_i = i == 0 ? n0 : n1;
         const int row = threadIdx.x & 127;   // 0..127 == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        float* xmax = reinterpret_cast<float*>(smem + C::kOffXchg);  // [slot][half][row]
-        const int32_t qi = w.qt * kBlockM + row;
+        const uint32_t sc = tmem + lane_off + C::kColS + i * kBlockN;  // S_i, then P_i over its first 64 columns
+        const uint32_t oc = tmem + lane_off + C::kColO + i * D;        // O_i
+        const int32_t qt_i = i == 0 ? w.qt[0] : w.qt[1];
+        const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
+        const int32_t qi = qt_i * kBlockM + row;
+        const int32_t vis = a.causal ? min(qi + 1, w.L) : w.L;  // keys [0, vis) visible to this row
         const float sl2 = a.scale_log2;
-        constexpr int kOHalf = D / 2;        // O columns rescaled / stored by this warpgroup
-        float m = -INFINITY;  // running max of score * scale * log2(e) (same in both warpgroups)
-        float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
-        bool ok = true;       // warp-uniform
-        for (int32_t j = 0; j < n_kv; ++j) {
-            const int b = j & 1;
-            const int slot = j & 1;
-            // tcgen05.ld/st are warp-collective: every decision below is warp-uniform.
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + b), static_cast<uint32_t>(j >> 1) & 1u,
-                                                         abort_flag));
-            uint32_t sr[2][32];
-            float mxh = -INFINITY;
-            if (ok) {
-                tc_fence_after();
-                const uint32_t sc = tmem + lane_off + C::kColS + b * kBlockN + hf * 64;
-                tmem_ld32(sc, sr[0]);
-                tmem_ld32(sc + 32, sr[1]);
+        float m = -INFINITY;  // running max of score * scale * log2(e)
+        float l = 0.0f;       // running sum of exp2(score * scale_log2 - m)
+        bool ok = n_i > 0;    // warp-uniform; tcgen05.ld/st are warp-collective
+        for (int32_t j = 0; j < n_i && ok; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + i), static_cast<uint32_t>(j) & 1u, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const int32_t lim = vis - j * kBlockN;  // columns [0, lim) of this tile are visible
+            // pass 1: row maximum
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t sr[32];
+                tmem_ld32(sc + q * 32, sr);
                 tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::kBarSEmpty + b));  // S_j consumed: the buffer may take S_{j+2}
-
-                // mask: keys [kv0, kv0 + lim) of this half are visible to this row
-                const int32_t kv0 = j * kBlockN + hf * 64;
-                const int32_t lim = (a.causal ? min(qi + 1, w.L) : w.L) - kv0;
-                if (lim < 64) {
+                const int32_t lq = lim - q * 32;
+                if (lq < 32) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+                    for (int c = 0; c < 32; ++c)
+                        if (c >= lq) sr[c] = __float_as_uint(-INFINITY);
                 }
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 64; c += 2)
-                    mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c >> 5][c & 31]),
-                                              __uint_as_float(sr[c >> 5][(c + 1) & 31]));
-                mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+                for (int c = 0; c < 32; c += 2)
+                    mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
             }
-            // exchange half-row maxima with the other warpgroup
-            xmax[(slot * 2 + hf) * kBlockM + row] = mxh;
-            named_bar_sync(1, 256);
-            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
-            if (!ok) continue;
-            const float mx = fmaxf(mxh, xmax[(slot * 2 + (hf ^ 1)) * kBlockM + row]);
-            const float m_new = fmaxf(m, mx * sl2);
-            // PV_{j-1} must be done before P_j overwrites P_{j-1} (and before O is rescaled)
+            const float m_new = fmaxf(m, fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2);
             if (j > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(j - 1) & 1u, abort_flag));
-                if (!ok) continue;
-                tc_fence_after();
+                // O_i already holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
                 const bool need = m_new > m + kRescaleThreshold;
                 if (__any_sync(0xffffffffu, need)) {
                     const float alpha = need ? ex2(m - m_new) : 1.0f;
                     const uint64_t alpha2 = f2pack(alpha, alpha);
                     l *= alpha;
 #pragma unroll 1
-                    for (int q = 0; q < kOHalf / 32; ++q) {
+                    for (int q = 0; q < D / 32; ++q) {
                         uint32_t o[32];
-                        const uint32_t oc = tmem + lane_off + C::kColO + hf * kOHalf + q * 32;
-                        tmem_ld32(oc, o);
+                        tmem_ld32(oc + q * 32, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int c = 0; c < 32; c += 2) {
@@ -687,44 +701,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             o[c] = __float_as_uint(v.x);
                             o[c + 1] = __float_as_uint(v.y);
                         }
-                        tmem_st32(oc, o);
+                        tmem_st32(oc + q * 32, o);
                     }
                     if (need) m = m_new;
                 }
             } else {
                 m = m_new;
             }
+            // pass 2: P = exp2(S * scale_log2 - m), written over S columns already read
             const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-            uint32_t pw[32];
             const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
             uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t sr[32], pw[16];
+                tmem_ld32(sc + q * 32, sr);
+                tmem_wait_ld();
+                const int32_t lq = lim - q * 32;
+                if (lq < 32) {
 #pragma unroll
-            for (int c2 = 0; c2 < 32; ++c2) {
-                const int c = 2 * c2;
-                const uint64_t sv = f2pack(__uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[c >> 5][(c + 1) & 31]));
-                const float2 x = f2unpack(ffma2(sv, sl2x2, negm2));
-                const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
-                l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
-                pw[c2] = pack2<kFP16>(pp);
+                    for (int c = 0; c < 32; ++c)
+                        if (c >= lq) sr[c] = __float_as_uint(-INFINITY);
+                }
+#pragma unroll
+                for (int c2 = 0; c2 < 16; ++c2) {
+                    const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
+                    const float2 x = f2unpack(ffma2(sv, sl2x2, negm2));
+                    const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
+                    l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
+                    pw[c2] = pack2<kFP16>(pp);
+                }
+                // P columns [16q, 16q + 16) lie in S columns [0, 32q + 32), all read by now
+                tmem_st16(sc + q * 16, pw);
             }
             const float2 la = f2unpack(fadd2(l2[0], l2[1]));
             l += la.x + la.y;
-            tmem_st32(tmem + lane_off + C::kColP + hf * 32, pw);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarPFull));
+            if (lane == 0) mbar_arrive(bar(C::kBarPFull + i));
         }
-        // epilogue: combine the partial sums (one more named barrier), out = O / l after the last PV
-        {
-            const int slot = n_kv & 1;  // last read at tile n_kv-2, free for both warpgroups now
-            xmax[(slot * 2 + hf) * kBlockM + row] = l;
-            named_bar_sync(1, 256);
-            l += xmax[(slot * 2 + (hf ^ 1)) * kBlockM + row];
-        }
-        const bool fin = __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
-                         __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone), static_cast<uint32_t>(n_kv - 1) & 1u,
-                                                           abort_flag));
+        // epilogue: out = O / l once the last PV_i is complete
+        const bool fin = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), 0, abort_flag));
         if (fin) {
             tc_fence_after();
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
@@ -732,15 +750,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
             int64_t o_off;
             if (a.layout == 0)
-                o_off = ((static_cast<int64_t>(w.seq) * a.Hq + w.h) * a.S + qi) * D;
+                o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
             else
-                o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + w.h) * D;
-            o_off += hf * kOHalf;
+                o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
             const uint64_t il2 = f2pack(inv_l, inv_l);
 #pragma unroll 1
-            for (int q = 0; q < kOHalf / 32; ++q) {
+            for (int q = 0; q < D / 32; ++q) {
                 uint32_t o[32];
-                tmem_ld32(tmem + lane_off + C::kColO + hf * kOHalf + q * 32, o);
+                tmem_ld32(oc + q * 32, o);
                 tmem_wait_ld();
                 if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);

@@ -89,6 +89,18 @@ int grid_for(int64_t work, int threads) {
     return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, 148LL * 64)));
 }
 
+// Grid of a grid-stride kernel: no more blocks than fit on the device at once
+// (every block then pays its prologue once).
+template <typename K>
+int resident_grid(K kernel, int64_t work, int threads) {
+    int dev = 0, sms = 148, per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const int64_t blocks = (work + threads - 1) / threads;
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(sms) * per_sm)));
+}
+
 // invFreq_j = base^(-2j/D) in fp64, rounded once to fp32.
 void inv_freq_row(double base, int D, float* out) {
     for (int j = 0; j < D / 2; ++j) out[j] = static_cast<float>(std::pow(base, -2.0 * j / static_cast<double>(D)));
@@ -183,21 +195,21 @@ rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, con
     if (headSize < 32 || headSize > 2048 || headSize % 32 != 0) return RFA_ERR_INVALID_ARG;
     if (!aligned(invFreq, 16) || !aligned(sinOut, 16) || !aligned(cosOut, 16)) return RFA_ERR_INVALID_ARG;
     const int64_t work = static_cast<int64_t>(ntokens) * (headSize / 16);
-    const int grid = grid_for(work, 256);
     cudaStream_t st = as_stream(stream);
     switch (outType) {
         case RFA_DT_FP16:
-            rfa::rope_sincos_kernel<__half><<<grid, 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
+            rfa::rope_sincos_kernel<__half><<<resident_grid(rfa::rope_sincos_kernel<__half>, work, 256), 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
                                                                    headSize, static_cast<__half*>(sinOut),
                                                                    static_cast<__half*>(cosOut));
             break;
         case RFA_DT_BF16:
-            rfa::rope_sincos_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            rfa::rope_sincos_kernel<__nv_bfloat16>
+                <<<resident_grid(rfa::rope_sincos_kernel<__nv_bfloat16>, work, 256), 256, 0, st>>>(
                 positionIds, invFreq, seqLens, batch, ntokens, headSize, static_cast<__nv_bfloat16*>(sinOut),
                 static_cast<__nv_bfloat16*>(cosOut));
             break;
         default:
-            rfa::rope_sincos_kernel<float><<<grid, 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
+            rfa::rope_sincos_kernel<float><<<resident_grid(rfa::rope_sincos_kernel<float>, work, 256), 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
                                                                   headSize, static_cast<float*>(sinOut),
                                                                   static_cast<float*>(cosOut));
             break;
@@ -281,6 +293,9 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
     aa.G = p->Hq / p->Hkv;
     aa.S = tnd ? 0 : p->S;
     aa.causal = p->causal ? 1 : 0;
+    // two query tiles per CTA: two heads of one kv group when G is even, else consecutive tiles of one head
+    const bool pair_heads = (aa.G % 2) == 0;
+    aa.pair_heads = pair_heads ? 1 : 0;
     const float scale = p->scale > 0.0f ? p->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
     aa.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     const bool fp16 = p->io_dtype == RFA_DT_FP16;
@@ -289,7 +304,7 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
     bool ok;
     if (!tnd) {
         const int64_t nqt = (p->S + rfa::kBlockM - 1) / rfa::kBlockM;
-        const int64_t items = nqt * p->B * p->Hq;
+        const int64_t items = static_cast<int64_t>(rfa::items_per_sequence(p->Hq, static_cast<int32_t>(nqt), pair_heads)) * p->B;
         if (items > 0x7fffffff) return RFA_ERR_UNSUPPORTED;
         aa.n_items = static_cast<int32_t>(items);
         ok = make_map(&mq, q, fp16, D, p->S, static_cast<uint64_t>(p->B) * p->Hq, D * esz, p->S * D * esz, 64,
@@ -318,7 +333,7 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
             aa.seg_len[i] = seqLens_host[b];
             aa.seg_tiles[i] = (seqLens_host[b] + rfa::kBlockM - 1) / rfa::kBlockM;
             aa.seg_item0[i] = static_cast<int32_t>(std::min<int64_t>(items, 0x7fffffff));
-            items += static_cast<int64_t>(aa.seg_tiles[i]) * p->Hq;
+            items += rfa::items_per_sequence(p->Hq, aa.seg_tiles[i], pair_heads);
         }
         aa.seg_item0[p->B] = static_cast<int32_t>(std::min<int64_t>(items, 0x7fffffff));
         if (items > 0x7fffffff) return RFA_ERR_UNSUPPORTED;

@@ -69,19 +69,25 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
                                                           OutT* __restrict__ cosOut) {
     __shared__ int32_t s_cum[kMaxSeqs + 1];
     __shared__ int32_t s_ok;
-    if (threadIdx.x == 0) {
-        int64_t acc = 0;
-        int32_t ok = 1;
-        for (int32_t b = 0; b < batch; ++b) {
-            const int32_t L = seqLens[b];
-            if (L <= 0) ok = 0;
-            s_cum[b] = static_cast<int32_t>(acc);
-            acc += L;
+    if (threadIdx.x < 32) {
+        // prefix sums of the lengths: one load per lane, then a warp scan
+        const int32_t lane = threadIdx.x;
+        const int64_t L = (lane < batch) ? static_cast<int64_t>(__ldg(seqLens + lane)) : 0;
+        int64_t x = L;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
         }
-        s_cum[batch] = static_cast<int32_t>(acc);
-        if (acc != ntokens) ok = 0;
-        s_ok = ok;
-        if (!ok && blockIdx.x == 0) record_status(1 /* RFA_ERR_INVALID_ARG */);
+        const bool bad = __any_sync(0xffffffffu, lane < batch && L <= 0);
+        const int64_t total = __shfl_sync(0xffffffffu, x, batch - 1);
+        if (lane < batch) s_cum[lane + 1] = static_cast<int32_t>(x);
+        if (lane == 0) {
+            s_cum[0] = 0;
+            const int32_t ok = (!bad && total == ntokens) ? 1 : 0;
+            s_ok = ok;
+            if (!ok && blockIdx.x == 0) record_status(1 /* RFA_ERR_INVALID_ARG */);
+        }
     }
     __syncthreads();
     if (!s_ok) return;
@@ -92,8 +98,11 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
          w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int32_t t = static_cast<int32_t>(w / chunks);
         const int32_t c = static_cast<int32_t>(w - static_cast<int64_t>(t) * chunks);
+        // segment of token t: the last b with s_cum[b] <= t (binary search over at most 16)
         int32_t b = 0;
-        while (b + 1 < batch && t >= s_cum[b + 1]) ++b;
+#pragma unroll
+        for (int step = kMaxSeqs / 2; step > 0; step >>= 1)
+            if (b + step < batch && t >= s_cum[b + step]) b += step;
         float s[8], co[8];
         sincos8(static_cast<float>(__ldg(pos + t)), inv + static_cast<int64_t>(b) * half + 8 * c, s, co);
         const int64_t o = static_cast<int64_t>(t) * headSize + 8 * c;
