@@ -55,7 +55,7 @@ namespace rfa {
 
 constexpr int kBlockM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per tile
-constexpr int kAttnThreads = 640;
+constexpr int kAttnThreads = 640;  // 20 warps: 96 registers per thread
 constexpr int kRopeWarp0 = 8;
 constexpr int kRopeWarps = 8;   // two RoPE warpgroups share every tile
 constexpr int kRopeThreads = kRopeWarps * 32;
@@ -350,6 +350,15 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
 #pragma unroll
             for (int k = 0; k < 4; ++k) rec_step(e.c[k], e.s[k], wc[k], ws[k]);
         }
+    }
+}
+
+// Columns c >= lim of a 32-column slice of S are masked (-inf).
+__device__ __forceinline__ void mask_cols(uint32_t (&sr)[32], int32_t lim) {
+    if (lim < 32) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+            if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
     }
 }
 
@@ -665,76 +674,99 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (!ok) break;
             tc_fence_after();
             const int32_t lim = vis - j * kBlockN;  // columns [0, lim) of this tile are visible
-            // pass 1: row maximum
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (j == 0) {
+                // first tile: the row maximum from a read of all of S_i
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t sr[32];
+                    tmem_ld32(sc + q * 32, sr);
+                    tmem_wait_ld();
+                    mask_cols(sr, lim - q * 32);
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2)
+                        mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                }
+                m = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;
+            }
+            // One pass over S_i, 32 columns at a time: P = exp2(S * scale_log2 - m), written over
+            // S columns already read (P columns [16q, 16q + 16) lie in S columns [0, 32q + 32)).
+            // Later tiles keep the running maximum m unless a chunk exceeds it by more than
+            // 2^kRescaleThreshold; then the warp raises m from the chunks still unread (they hold
+            // that chunk), and rescales the P chunks already written, l and O by exp2(m_old - m).
+            uint64_t l2 = 0ull;  // this tile's row sum as a packed pair (+0.0f, +0.0f)
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
                 uint32_t sr[32];
                 tmem_ld32(sc + q * 32, sr);
                 tmem_wait_ld();
-                const int32_t lq = lim - q * 32;
-                if (lq < 32) {
+                mask_cols(sr, lim - q * 32);
+                if (j > 0) {
+                    float cm = __uint_as_float(sr[0]);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c >= lq) sr[c] = __float_as_uint(-INFINITY);
-                }
-#pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-            }
-            const float m_new = fmaxf(m, fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2);
-            if (j > 0) {
-                // O_i already holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
-                const bool need = m_new > m + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need)) {
-                    const float alpha = need ? ex2(m - m_new) : 1.0f;
-                    const uint64_t alpha2 = f2pack(alpha, alpha);
-                    l *= alpha;
+                    for (int c = 1; c < 31; c += 2) cm = fmax3(cm, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                    cm = fmaxf(cm, __uint_as_float(sr[31]));
+                    const bool viol = cm * sl2 > m + kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, viol)) {
+                        // maximum over S chunks q..3 (all unread so far)
 #pragma unroll 1
-                    for (int q = 0; q < D / 32; ++q) {
-                        uint32_t o[32];
-                        tmem_ld32(oc + q * 32, o);
-                        tmem_wait_ld();
+                        for (int r = q + 1; r < 4; ++r) {
+                            tmem_ld32(sc + r * 32, sr);
+                            tmem_wait_ld();
+                            mask_cols(sr, lim - r * 32);
 #pragma unroll
-                        for (int c = 0; c < 32; c += 2) {
-                            const float2 v = f2unpack(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), alpha2));
-                            o[c] = __float_as_uint(v.x);
-                            o[c + 1] = __float_as_uint(v.y);
+                            for (int c = 0; c < 32; c += 2)
+                                cm = fmax3(cm, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
                         }
-                        tmem_st32(oc + q * 32, o);
-                    }
-                    if (need) m = m_new;
-                }
-            } else {
-                m = m_new;
-            }
-            // pass 2: P = exp2(S * scale_log2 - m), written over S columns already read
-            const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-            const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
-            uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
+                        const float m_new = viol ? cm * sl2 : m;
+                        const float alpha = viol ? ex2(m - m_new) : 1.0f;
+                        const uint64_t alpha2 = f2pack(alpha, alpha);
+                        tmem_wait_st();
+                        uint32_t(&pw)[16] = reinterpret_cast<uint32_t(&)[16]>(sr);
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint32_t sr[32], pw[16];
-                tmem_ld32(sc + q * 32, sr);
-                tmem_wait_ld();
-                const int32_t lq = lim - q * 32;
-                if (lq < 32) {
+                        for (int r = 0; r < q; ++r) {  // P chunks written with the old maximum
+                            tmem_ld16(sc + r * 16, pw);
+                            tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c >= lq) sr[c] = __float_as_uint(-INFINITY);
+                            for (int c = 0; c < 16; ++c) pw[c] = pack2<kFP16>(fmul2(IoT<kFP16>::unpack2(pw[c]), alpha2));
+                            tmem_st16(sc + r * 16, pw);
+                        }
+                        l2 = fmul2(l2, alpha2);
+                        l *= alpha;
+                        // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
+#pragma unroll 1
+                        for (int r = 0; r < D / 32; ++r) {
+                            tmem_ld32(oc + r * 32, sr);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; c += 2) {
+                                const float2 v =
+                                    f2unpack(fmul2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), alpha2));
+                                sr[c] = __float_as_uint(v.x);
+                                sr[c + 1] = __float_as_uint(v.y);
+                            }
+                            tmem_st32(oc + r * 32, sr);
+                        }
+                        m = m_new;
+                        tmem_ld32(sc + q * 32, sr);  // this chunk again
+                        tmem_wait_ld();
+                        mask_cols(sr, lim - q * 32);
+                    }
                 }
+                const float neg_m = (m == -INFINITY) ? 0.0f : -m;
+                const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
+                // packed P words go to sr[0..15], each after the two scores it replaces were read
 #pragma unroll
                 for (int c2 = 0; c2 < 16; ++c2) {
                     const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
                     const float2 x = f2unpack(ffma2(sv, sl2x2, negm2));
                     const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
-                    l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
-                    pw[c2] = pack2<kFP16>(pp);
+                    l2 = fadd2(l2, pp);
+                    sr[c2] = pack2<kFP16>(pp);
                 }
-                // P columns [16q, 16q + 16) lie in S columns [0, 32q + 32), all read by now
-                tmem_st16(sc + q * 16, pw);
+                tmem_st16(sc + q * 16, reinterpret_cast<const uint32_t(&)[16]>(sr));
             }
-            const float2 la = f2unpack(fadd2(l2[0], l2[1]));
+            const float2 la = f2unpack(l2);
             l += la.x + la.y;
             tmem_wait_st();
             tc_fence_before();

@@ -96,6 +96,42 @@ def test_fp16_io(rfa, D):
     full_bnsd(rfa, 1, 4, 4, 260, D, seed=9, dtype=torch.float16)
 
 
+def test_odd_group_size_pairs_query_tiles(rfa):
+    # G = 3 and an odd number of query tiles: the last work item has one tile
+    full_bnsd(rfa, 1, 6, 2, 520, 128, seed=17)
+
+
+@pytest.mark.parametrize("dtype,causal,zero_pos", [(torch.bfloat16, True, True), (torch.float16, False, False)])
+def test_running_max_jumps_within_later_tiles(rfa, dtype, causal, zero_pos):
+    """A few keys far larger than the rest make the row maximum jump by much
+    more than 2^8 inside later key tiles, in different 32-key chunks (keys
+    300, 420, 500, 520, 690: chunks 1, 1, 3, 0, 1 of tiles 2, 3, 3, 4, 5), so
+    the part of the tile already exponentiated, the row sum and O must be
+    rescaled mid-tile.  The large keys share one value row: how the weight
+    splits among them (sensitive to the rounding of the rotated keys at such
+    scores) then does not move the output.  The bf16 case puts every token
+    at position 0, where the rotation is exactly the identity, so that the
+    scores carry no rounding of rotated operands (bf16 keeps 8 bits, and at
+    scores of ~10 that alone moves the weights of keys near the maximum)."""
+    B, Hq, Hkv, S, D = 1, 2, 1, 700, 128
+    big = ((300, 14.0), (420, 20.0), (500, 28.0), (520, 36.0), (690, 50.0))
+    q = workloads.randn16((B, Hq, S, D), 91, dtype)
+    k = workloads.randn16((B, Hkv, S, D), 92, dtype).float()
+    v = workloads.randn16((B, Hkv, S, D), 93, dtype)
+    for t, f in big:
+        k[:, :, t] *= f
+        v[:, :, t] = v[:, :, big[0][0]]
+    k = k.to(dtype)
+    pos = torch.arange(S, dtype=torch.int32).repeat(B, 1).contiguous()
+    if zero_pos:
+        pos.zero_()
+    out = rfa.fused_rope_attention(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), layout="BNSD", causal=causal,
+                                   rope_base=10000.0)
+    assert rfa.get_device_status() == 0
+    ref = oracle.attention_full(q, k, v, pos.numpy(), _inv_rows(B, D, 10000.0), causal=causal)
+    _compare(out.float().cpu().numpy(), ref)
+
+
 def test_mqa_and_scale(rfa):
     full_bnsd(rfa, 1, 8, 1, 200, 128, seed=13, scale=0.05)
 
