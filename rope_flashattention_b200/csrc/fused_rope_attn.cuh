@@ -692,8 +692,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // One pass over S_i, 32 columns at a time: P = exp2(S * scale_log2 - m), written over
             // S columns already read (P columns [16q, 16q + 16) lie in S columns [0, 32q + 32)).
             // Later tiles keep the running maximum m unless a chunk exceeds it by more than
-            // 2^kRescaleThreshold; then the warp raises m from the chunks still unread (they hold
-            // that chunk), and rescales the P chunks already written, l and O by exp2(m_old - m).
+            // 2^kRescaleThreshold.  A chunk is exponentiated with the current m while its maximum
+            // is taken; if any row of the warp exceeds the bound, the warp raises m from the
+            // chunks still unread (they hold the offending one), rescales the P chunks already
+            // written, l and O by exp2(m_old - m), re-reads the chunk (its P is stored only after
+            // the check) and does it again.
             uint64_t l2 = 0ull;  // this tile's row sum as a packed pair (+0.0f, +0.0f)
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
@@ -701,69 +704,73 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_ld32(sc + q * 32, sr);
                 tmem_wait_ld();
                 mask_cols(sr, lim - q * 32);
-                if (j > 0) {
-                    float cm = __uint_as_float(sr[0]);
-#pragma unroll
-                    for (int c = 1; c < 31; c += 2) cm = fmax3(cm, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                    cm = fmaxf(cm, __uint_as_float(sr[31]));
-                    const bool viol = cm * sl2 > m + kRescaleThreshold;
-                    if (__any_sync(0xffffffffu, viol)) {
-                        // maximum over S chunks q..3 (all unread so far)
+                uint64_t lc;
 #pragma unroll 1
-                        for (int r = q + 1; r < 4; ++r) {
-                            tmem_ld32(sc + r * 32, sr);
-                            tmem_wait_ld();
-                            mask_cols(sr, lim - r * 32);
+                for (int attempt = 0;; ++attempt) {
+                    const float neg_m = (m == -INFINITY) ? 0.0f : -m;
+                    const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    uint64_t lc2[2] = {0ull, 0ull};
+                    // packed P words go to sr[0..15], each after the two scores it replaces were read
 #pragma unroll
-                            for (int c = 0; c < 32; c += 2)
-                                cm = fmax3(cm, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                        }
-                        const float m_new = viol ? cm * sl2 : m;
-                        const float alpha = viol ? ex2(m - m_new) : 1.0f;
-                        const uint64_t alpha2 = f2pack(alpha, alpha);
-                        tmem_wait_st();
-                        uint32_t(&pw)[16] = reinterpret_cast<uint32_t(&)[16]>(sr);
-#pragma unroll 1
-                        for (int r = 0; r < q; ++r) {  // P chunks written with the old maximum
-                            tmem_ld16(sc + r * 16, pw);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) pw[c] = pack2<kFP16>(fmul2(IoT<kFP16>::unpack2(pw[c]), alpha2));
-                            tmem_st16(sc + r * 16, pw);
-                        }
-                        l2 = fmul2(l2, alpha2);
-                        l *= alpha;
-                        // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
-#pragma unroll 1
-                        for (int r = 0; r < D / 32; ++r) {
-                            tmem_ld32(oc + r * 32, sr);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int c = 0; c < 32; c += 2) {
-                                const float2 v =
-                                    f2unpack(fmul2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), alpha2));
-                                sr[c] = __float_as_uint(v.x);
-                                sr[c + 1] = __float_as_uint(v.y);
-                            }
-                            tmem_st32(oc + r * 32, sr);
-                        }
-                        m = m_new;
-                        tmem_ld32(sc + q * 32, sr);  // this chunk again
-                        tmem_wait_ld();
-                        mask_cols(sr, lim - q * 32);
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        const float a0 = __uint_as_float(sr[2 * c2]), a1 = __uint_as_float(sr[2 * c2 + 1]);
+                        mx[c2 & 3] = fmax3(mx[c2 & 3], a0, a1);
+                        const float2 x = f2unpack(ffma2(f2pack(a0, a1), sl2x2, negm2));
+                        const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
+                        lc2[c2 & 1] = fadd2(lc2[c2 & 1], pp);
+                        sr[c2] = pack2<kFP16>(pp);
                     }
-                }
-                const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-                const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
-                // packed P words go to sr[0..15], each after the two scores it replaces were read
+                    lc = fadd2(lc2[0], lc2[1]);
+                    if (j == 0 || attempt > 0) break;
+                    const float cm = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+                    const bool viol = cm * sl2 > m + kRescaleThreshold;
+                    if (!__any_sync(0xffffffffu, viol)) break;
+                    // maximum over S chunks q..3 (all unread so far; chunk q's P is not stored yet)
+                    float cmx = cm;
+#pragma unroll 1
+                    for (int r = q + 1; r < 4; ++r) {
+                        tmem_ld32(sc + r * 32, sr);
+                        tmem_wait_ld();
+                        mask_cols(sr, lim - r * 32);
 #pragma unroll
-                for (int c2 = 0; c2 < 16; ++c2) {
-                    const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
-                    const float2 x = f2unpack(ffma2(sv, sl2x2, negm2));
-                    const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
-                    l2 = fadd2(l2, pp);
-                    sr[c2] = pack2<kFP16>(pp);
+                        for (int c = 0; c < 32; c += 2) cmx = fmax3(cmx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                    }
+                    const float m_new = viol ? cmx * sl2 : m;
+                    const float alpha = viol ? ex2(m - m_new) : 1.0f;
+                    const uint64_t alpha2 = f2pack(alpha, alpha);
+                    tmem_wait_st();
+                    uint32_t(&pw)[16] = reinterpret_cast<uint32_t(&)[16]>(sr);
+#pragma unroll 1
+                    for (int r = 0; r < q; ++r) {  // P chunks written with the old maximum
+                        tmem_ld16(sc + r * 16, pw);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) pw[c] = pack2<kFP16>(fmul2(IoT<kFP16>::unpack2(pw[c]), alpha2));
+                        tmem_st16(sc + r * 16, pw);
+                    }
+                    l2 = fmul2(l2, alpha2);
+                    l *= alpha;
+                    // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
+#pragma unroll 1
+                    for (int r = 0; r < D / 32; ++r) {
+                        tmem_ld32(oc + r * 32, sr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            const float2 v =
+                                f2unpack(fmul2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), alpha2));
+                            sr[c] = __float_as_uint(v.x);
+                            sr[c + 1] = __float_as_uint(v.y);
+                        }
+                        tmem_st32(oc + r * 32, sr);
+                    }
+                    m = m_new;
+                    tmem_ld32(sc + q * 32, sr);  // this chunk again
+                    tmem_wait_ld();
+                    mask_cols(sr, lim - q * 32);
                 }
+                l2 = fadd2(l2, lc);
                 tmem_st16(sc + q * 16, reinterpret_cast<const uint32_t(&)[16]>(sr));
             }
             const float2 la = f2unpack(l2);
