@@ -16,12 +16,14 @@
 // second may be absent at the end of a sequence).  Every key tile is loaded
 // and rotated once for both query tiles.  Warp roles:
 //   warps 0-3  softmax warpgroup of query tile 0, warps 4-7 of query tile 1;
-//              thread t owns query row t (TMEM lane t).  Per key tile: row
-//              maximum from a first read of S (TMEM), exponentials from a
-//              second read, 32 columns at a time; P (bf16/fp16) is written in
-//              place over the S columns already read; O is rescaled only when
-//              the maximum grows by > 2^8.  At the end: O / l to global memory.
-//   warps 8-15 two RoPE warpgroups: rotate both query tiles once, then every
+//              thread t owns query row t (TMEM lane t).  Per key tile, 32
+//              columns of S (TMEM) at a time: exponentials against the running
+//              maximum, which the first tile takes from a separate read and
+//              later tiles raise only when a chunk exceeds it by > 2^8 (then
+//              what was written, l and O are rescaled).  P (bf16/fp16) is
+//              written in place over the S columns already read.  At the end:
+//              O / l to global memory.
+//   warps 8-11 RoPE warpgroup: rotates both query tiles once, then every
 //              key tile, in place in the 128B-swizzled shared-memory layout.
 //              Element i and its rotate-half partner i + D/2 sit at the same
 //              offset of two swizzle atoms (D = 128) or in chunks c and c ^ 4
@@ -29,17 +31,17 @@
 //              recurrence in registers when the sequence's positions are
 //              consecutive, else from cos/sin rows that TMA staged beside the
 //              tile; query angles always from staged rows.
-//   warp 16    TMA producer: both query tiles (+ their cos/sin rows, staged in
+//   warp 12    TMA producer: both query tiles (+ their cos/sin rows, staged in
 //              the first two V slots) once, then key tiles (+ rows when
 //              needed) through a kStages ring.
-//   warp 17    tcgen05 issuer (one thread) and TMEM owner.  Order per key
+//   warp 13    tcgen05 issuer (one thread) and TMEM owner.  Order per key
 //              tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), where
 //              S_i = Q_i' K_j'^T goes to TMEM buffer i and O_i += P_i V_j reads
 //              P_i from that same buffer.  MMAs issued by one thread execute
 //              in issue order, so QK_i(j+1) overwrites P_i only after PV_i(j)
 //              has read it, and S_i(j+1) being complete implies O_i holds
 //              PV_i(j).
-//   warp 18    TMA producer for the V ring.
+//   warp 14    TMA producer for the V ring.
 // Completion of every async step is tracked by mbarriers; each wait is bounded.
 #pragma once
 #include <cuda.h>
@@ -55,14 +57,14 @@ namespace rfa {
 
 constexpr int kBlockM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per tile
-constexpr int kAttnThreads = 640;  // 20 warps: 96 registers per thread
+constexpr int kAttnThreads = 512;  // 16 warps: 128 registers per thread
 constexpr int kRopeWarp0 = 8;
-constexpr int kRopeWarps = 8;   // two RoPE warpgroups share every tile
+constexpr int kRopeWarps = 4;      // one RoPE warpgroup
 constexpr int kRopeThreads = kRopeWarps * 32;
-constexpr int kTmaWarp = 16;    // Q, K (+ cos/sin rows)
-constexpr int kMmaWarp = 17;
-constexpr int kTmaVWarp = 18;   // V: its own producer, so K prefetch never waits on a V slot
-// warp 19 only takes part in the block-wide barriers
+constexpr int kTmaWarp = 12;       // Q, K (+ cos/sin rows)
+constexpr int kMmaWarp = 13;
+constexpr int kTmaVWarp = 14;      // V: its own producer, so K prefetch never waits on a V slot
+// warp 15 only takes part in the block-wide barriers
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
 struct AttnArgs {
@@ -318,7 +320,7 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
     const int cp = rt % kPairsPerRow;
     const int r0 = rt / kPairsPerRow;
     RecState e = z;
-    // Modest unrolling: 20 warps run five roles at once and their hot loops
+    // Modest unrolling: 16 warps run five roles at once and their hot loops
     // must stay resident in the instruction cache.
 #pragma unroll 2
     for (int it = 0; it < kIters; ++it) {
