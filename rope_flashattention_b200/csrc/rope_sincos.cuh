@@ -48,7 +48,27 @@ struct Pack8<float> {
     }
 };
 
-// sin/cos of the fp32 angles position * invFreq[j], j = j0 .. j0+7.
+// sin/cos of the angles position * invFreq[j], j = j0 .. j0+7.
+// The fp32 product x = p * w is reduced by 2*pi with the two-constant
+// Cody-Waite scheme (W. J. Cody and W. Waite, "Software Manual for the
+// Elementary Functions", 1980): k = round(x / 2pi), r = (x - k C1) - k C2 with
+// C1 + C2 = 2pi to ~7e-15 (both products exact inside fma).  The rounding error
+// of x itself, recovered exactly as fma(p, w, -x), is added back to r, so the
+// angle carries no error from the fp32 product.  The SFU then evaluates sin and
+// cos of r, which lies in [-pi, pi] up to a few ulps for |x| below ~1e6 (beyond
+// that the quotient's rounding can leave |r| a few multiples of 2pi larger, still
+// within the SFU's accurate range for the 16-bit outputs).
+constexpr float kTwoPiHi = 6.2831854820251465f;      // fp32 nearest to 2 pi
+constexpr float kTwoPiLo = -1.7484555314695172e-07f;  // 2 pi - kTwoPiHi, rounded to fp32
+constexpr float kInvTwoPi = 0.15915493667125702f;     // fp32 nearest to 1 / (2 pi)
+__device__ __forceinline__ void sincos_reduced(float p, float w, float& s, float& c) {
+    const float x = p * w;
+    const float xe = fmaf(p, w, -x);  // p * w - x, exactly
+    const float k = rintf(x * kInvTwoPi);
+    const float r = fmaf(-k, kTwoPiLo, fmaf(-k, kTwoPiHi, x)) + xe;
+    __sincosf(r, &s, &c);
+}
+
 __device__ __forceinline__ void sincos8(float position, const float* inv, float (&s)[8], float (&c)[8]) {
     // Generic loads: `inv` points either to global memory or into the
     // kernel's parameter block (host-derived frequencies).
@@ -56,7 +76,7 @@ __device__ __forceinline__ void sincos8(float position, const float* inv, float 
     const float4 i1 = reinterpret_cast<const float4*>(inv)[1];
     const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) sincosf(position * iv[k], &s[k], &c[k]);
+    for (int k = 0; k < 8; ++k) sincos_reduced(position, iv[k], s[k], c[k]);
 }
 
 // Public table: sin/cos [ntokens, headSize] from device positions, invFreq
@@ -92,12 +112,12 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
     __syncthreads();
     if (!s_ok) return;
     const int32_t half = headSize >> 1;
-    const int32_t chunks = half >> 3;
-    const int64_t work = static_cast<int64_t>(ntokens) * chunks;
-    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < work;
-         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t chunks = static_cast<uint32_t>(half >> 3);
+    // ntokens <= 256000 and chunks <= 128: the work index fits 32 bits
+    const uint32_t work = static_cast<uint32_t>(ntokens) * chunks;
+    for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < work; w += gridDim.x * blockDim.x) {
         const int32_t t = static_cast<int32_t>(w / chunks);
-        const int32_t c = static_cast<int32_t>(w - static_cast<int64_t>(t) * chunks);
+        const int32_t c = static_cast<int32_t>(w - static_cast<uint32_t>(t) * chunks);
         // segment of token t: the last b with s_cum[b] <= t (binary search over at most 16)
         int32_t b = 0;
 #pragma unroll

@@ -83,6 +83,22 @@ def test_ceiling_shape_sampled(rfa):
     _check(rfa, pos, inv, lens, 128, torch.float16, rows=rows)
 
 
+def test_large_angles_fp32_accuracy(rfa):
+    """Angles up to 1e6 rad (positions up to +-1e6, frequencies in [0.5, 1]):
+    the angle is reduced by 2 pi with the fp32 product's rounding error carried
+    along, so fp32 outputs stay within 2e-6 of the exact values (rounding the
+    product to fp32 alone would err by up to 3e-2 here)."""
+    g = workloads.gen(17)
+    T, D = 4096, 64
+    pos = torch.randint(-1000000, 1000001, (T,), generator=g, dtype=torch.int32)
+    inv = 0.5 + 0.5 * torch.rand(1, D // 2, generator=g, dtype=torch.float32)
+    lens = torch.tensor([T], dtype=torch.int32)
+    s, c = _run(rfa, pos, inv, lens, D, torch.float32)
+    rs, rc = oracle.rope_sincos(pos.numpy(), inv.double().numpy(), lens.numpy(), D)
+    assert np.abs(s.cpu().numpy() - rs).max() <= 2e-6
+    assert np.abs(c.cpu().numpy() - rc).max() <= 2e-6
+
+
 def test_segment_indexing_exact(rfa):
     # row b of invFreq = 2^-(b+1): each token's angle identifies its batch exactly
     lens = torch.tensor([3, 9, 1, 20], dtype=torch.int32)
