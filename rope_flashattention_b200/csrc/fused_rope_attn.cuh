@@ -57,14 +57,15 @@ namespace rfa {
 
 constexpr int kBlockM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;  // keys per tile
-constexpr int kAttnThreads = 512;  // 16 warps: 128 registers per thread
-constexpr int kRopeWarp0 = 8;
+constexpr int kAttnThreads = 768;  // 24 warps: 80 registers per thread
+constexpr int kSoftmaxWarps = 16;  // 8 per query tile: 4 TMEM lane groups x 2 column halves
+constexpr int kRopeWarp0 = 16;
 constexpr int kRopeWarps = 4;      // one RoPE warpgroup
 constexpr int kRopeThreads = kRopeWarps * 32;
-constexpr int kTmaWarp = 12;       // Q, K (+ cos/sin rows)
-constexpr int kMmaWarp = 13;
-constexpr int kTmaVWarp = 14;      // V: its own producer, so K prefetch never waits on a V slot
-// warp 15 only takes part in the block-wide barriers
+constexpr int kTmaWarp = 20;       // Q, K (+ cos/sin rows)
+constexpr int kMmaWarp = 21;
+constexpr int kTmaVWarp = 22;      // V: its own producer, so K prefetch never waits on a V slot
+// warp 23 only takes part in the block-wide barriers
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
 struct AttnArgs {
@@ -115,15 +116,16 @@ struct AttnCfg {
     static constexpr int kBarKEmpty = kBarKReady + kStages;
     static constexpr int kBarVEmpty = kBarKEmpty + kStages;
     static constexpr int kBarSFull = kBarVEmpty + kStages;  // 2: S_i complete (and every earlier MMA)
-    static constexpr int kBarPFull = kBarSFull + 2;         // 2: P_i written, O_i rescaled (4 warp arrivals)
+    static constexpr int kBarPFull = kBarSFull + 2;         // 2: P_i written, O_i rescaled (8 warp arrivals)
     static constexpr int kBarOFull = kBarPFull + 2;         // 2: last PV_i complete
     static constexpr int kBarMmaFin = kBarOFull + 2;
     static constexpr int kNumBars = kBarMmaFin + 1;
     static constexpr int kOffAbort = kOffBar + 8 * kNumBars;
     static constexpr int kOffTmemSlot = kOffAbort + 16;
+    static constexpr int kOffXchg = kOffTmemSlot + 16;  // float [2 query tiles][2 column halves][128 rows]
     // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (the
     // kernel checks it), so no alignment slack is requested.
-    static constexpr int kSmemBytes = kOffTmemSlot + 16;
+    static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBlockM * 4;
     // TMEM columns: S_0, S_1 (P_i over the first 64 columns of S_i), O_0, O_1
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;      // S_i at 128 i
@@ -429,7 +431,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(C::kBarSFull + i), 1);
-            mbar_init(bar(C::kBarPFull + i), 4);  // one arrival per warp of softmax warpgroup i
+            mbar_init(bar(C::kBarPFull + i), 8);  // one arrival per softmax warp of query tile i
             mbar_init(bar(C::kBarOFull + i), 1);
         }
         mbar_init(bar(C::kBarMmaFin), 1);
@@ -532,26 +534,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             constexpr uint32_t kIdescQK = idesc_f16(IoT<kFP16>::kFmt, 0, 0, kBlockM, kBlockN);
             constexpr uint32_t kIdescPV = idesc_f16(IoT<kFP16>::kFmt, 0, 1, kBlockM, D);
             // S_i = Q_i' K_j'^T into TMEM buffer i (A = Q_i' and B = K_j' from shared memory)
+            // The issuing thread must keep up with the tensor pipe (one 128x128x16 MMA per ~64
+            // cycles): a tile's descriptors are built once and each k-step adds its byte offset
+            // >> 4 to the start-address field (shared addresses < 256 KB: no carry out of it).
             auto issue_qk = [&](int i, int32_t j) {
-                const uint32_t kbase = sbase + C::kOffK + (j % C::kStages) * C::kTileBytes;
-                const uint32_t qbase = sbase + C::kOffQ + i * C::kTileBytes;
+                const uint64_t kd = smem_desc_sw128(sbase + C::kOffK + (j % C::kStages) * C::kTileBytes, 16, 1024);
+                const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + i * C::kTileBytes, 16, 1024);
+                const uint32_t dS = tmem + C::kColS + i * kBlockN;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t koff = (k >> 2) * C::kAtomBytes + (k & 3) * 32;
-                    umma_ss(tmem + C::kColS + i * kBlockN, smem_desc_sw128(qbase + koff, 16, 1024),
-                            smem_desc_sw128(kbase + koff, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+                    const uint32_t koff16 = ((k >> 2) * C::kAtomBytes + (k & 3) * 32) >> 4;
+                    umma_ss(dS, qd + koff16, kd + koff16, kIdescQK, k > 0 ? 1u : 0u);
                 }
                 tc_commit(bar(C::kBarSFull + i));
             };
-            // O_i += P_i V_j (A = P_i from the first 64 columns of TMEM buffer i, B = V_j from shared memory)
+            // O_i += P_i V_j (A = P_i from TMEM buffer i: keys [64h, 64h + 64) at columns [64h, 64h + 32);
+            // B = V_j from shared memory)
             auto issue_pv = [&](int i, int32_t j) {
-                const uint32_t vbase = sbase + C::kOffV + (j % C::kStages) * C::kTileBytes;
+                const uint64_t vd = smem_desc_sw128(sbase + C::kOffV + (j % C::kStages) * C::kTileBytes, C::kAtomBytes, 1024);
+                const uint32_t dO = tmem + C::kColO + i * D, aP = tmem + C::kColS + i * kBlockN;
 #pragma unroll
-                for (int k = 0; k < kBlockN / 16; ++k) {
-                    const uint64_t bd = smem_desc_sw128(vbase + k * 16 * 128, C::kAtomBytes, 1024);
-                    umma_ts(tmem + C::kColO + i * D, tmem + C::kColS + i * kBlockN + k * 8, bd, kIdescPV,
+                for (int k = 0; k < kBlockN / 16; ++k)
+                    umma_ts(dO, aP + (k >> 2) * 64 + (k & 3) * 8, vd + ((k * 16 * 128) >> 4), kIdescPV,
                             (j > 0 || k > 0) ? 1u : 0u);
-                }
             };
             bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag) && mbar_wait(bar(C::kBarKReady), 0, abort_flag);
             if (ok) {
@@ -655,32 +660,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (lane == 0) mbar_arrive(bar(C::kBarKReady + s));
             }
         }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ softmax warpgroups
-        const int i = warp >> 2;             // query tile of this warpgroup
+    } else if (warp < kSoftmaxWarps) {
+        // ------------------------------------------------------------ softmax warps
+        // Query tile i has 8 warps: warp w covers TMEM lanes (rows) 32 (w % 4) .. + 31 and key
+        // columns [64 hf, 64 hf + 64) of every score tile, hf = (w / 4) % 2.  The two warps of a
+        // row exchange half-row maxima (then row sums) through shared memory at named barrier
+        // 1 + i (256 threads), executed exactly n_i + 2 times by every one of them: a failed
+        // (timed-out) wait only turns the remaining work into no-ops, it never skips a barrier.
+        // A slot written at tile j + 1 was read at tile j before the reader arrived on PFull_i(j),
+        // which S_i(j + 1) waits for, so one slot per row and half suffices.
+        const int i = warp >> 3;             // query tile
+        const int hf = (warp >> 2) & 1;      // key-column half
         const int32_t n_i = i == 0 ? n0 : n1;
-        const int row = threadIdx.x & 127;   // 0..127 == TMEM lane
+        const int row = ((warp & 3) << 5) + lane;  // 0..127 == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t sc = tmem + lane_off + C::kColS + i * kBlockN;  // S_i, then P_i over its first 64 columns
-        const uint32_t oc = tmem + lane_off + C::kColO + i * D;        // O_i
+        const uint32_t sc = tmem + lane_off + C::kColS + i * kBlockN + hf * 64;  // this half of S_i; P over [0, 32)
+        constexpr int kOHalf = D / 2;                                           // O_i columns rescaled / stored
+        const uint32_t oc = tmem + lane_off + C::kColO + i * D + hf * kOHalf;
+        float* xch = reinterpret_cast<float*>(smem + C::kOffXchg) + i * 2 * kBlockM;  // [half][row]
+        const uint32_t nb = 1u + static_cast<uint32_t>(i);
         const int32_t qt_i = i == 0 ? w.qt[0] : w.qt[1];
-        const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
         const int32_t qi = qt_i * kBlockM + row;
         const int32_t vis = a.causal ? min(qi + 1, w.L) : w.L;  // keys [0, vis) visible to this row
         const float sl2 = a.scale_log2;
-        float m = -INFINITY;  // running max of score * scale * log2(e)
-        float l = 0.0f;       // running sum of exp2(score * scale_log2 - m)
-        bool ok = n_i > 0;    // warp-uniform; tcgen05.ld/st are warp-collective
-        for (int32_t j = 0; j < n_i && ok; ++j) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + i), static_cast<uint32_t>(j) & 1u, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            const int32_t lim = vis - j * kBlockN;  // columns [0, lim) of this tile are visible
-            if (j == 0) {
-                // first tile: the row maximum from a read of all of S_i
+        float m = -INFINITY;  // running max of score * scale * log2(e) (identical in both halves)
+        float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
+        bool ok = true;       // warp-uniform; tcgen05.ld/st are warp-collective
+        for (int32_t j = 0; j < n_i; ++j) {
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + i), static_cast<uint32_t>(j) & 1u, abort_flag));
+            const int32_t lim = vis - j * kBlockN - hf * 64;  // columns [0, lim) of this half are visible
+            float mxh = -INFINITY;
+            if (ok) {
+                tc_fence_after();
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     uint32_t sr[32];
                     tmem_ld32(sc + q * 32, sr);
                     tmem_wait_ld();
@@ -689,103 +703,77 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int c = 0; c < 32; c += 2)
                         mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
                 }
-                m = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;
+                mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
             }
-            // One pass over S_i, 32 columns at a time: P = exp2(S * scale_log2 - m), written over
-            // S columns already read (P columns [16q, 16q + 16) lie in S columns [0, 32q + 32)).
-            // Later tiles keep the running maximum m unless a chunk exceeds it by more than
-            // 2^kRescaleThreshold.  A chunk is exponentiated with the current m while its maximum
-            // is taken; if any row of the warp exceeds the bound, the warp raises m from the
-            // chunks still unread (they hold the offending one), rescales the P chunks already
-            // written, l and O by exp2(m_old - m), re-reads the chunk (its P is stored only after
-            // the check) and does it again.
-            uint64_t l2 = 0ull;  // this tile's row sum as a packed pair (+0.0f, +0.0f)
+            xch[hf * kBlockM + row] = mxh;
+            named_bar_sync(nb, 256);
+            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
+            if (!ok) continue;
+            const float m_new = fmaxf(m, fmaxf(mxh, xch[(hf ^ 1) * kBlockM + row]) * sl2);
+            if (j > 0) {
+                // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
+                const bool need = m_new > m + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float alpha = need ? ex2(m - m_new) : 1.0f;
+                    const uint64_t alpha2 = f2pack(alpha, alpha);
+                    l *= alpha;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < kOHalf / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32(oc + q * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            const float2 v = f2unpack(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), alpha2));
+                            o[c] = __float_as_uint(v.x);
+                            o[c + 1] = __float_as_uint(v.y);
+                        }
+                        tmem_st32(oc + q * 32, o);
+                    }
+                    if (need) m = m_new;
+                }
+            } else {
+                m = m_new;
+            }
+            // P = exp2(S * scale_log2 - m) over this half, 32 columns at a time, written over
+            // the half's S columns already read (P columns [16q, 16q + 16) lie in [0, 32q + 32))
+            const float neg_m = (m == -INFINITY) ? 0.0f : -m;
+            const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
+            uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
+#pragma unroll 1
+            for (int q = 0; q < 2; ++q) {
                 uint32_t sr[32];
                 tmem_ld32(sc + q * 32, sr);
                 tmem_wait_ld();
                 mask_cols(sr, lim - q * 32);
-                uint64_t lc;
-#pragma unroll 1
-                for (int attempt = 0;; ++attempt) {
-                    const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-                    const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
-                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    uint64_t lc2[2] = {0ull, 0ull};
-                    // packed P words go to sr[0..15], each after the two scores it replaces were read
 #pragma unroll
-                    for (int c2 = 0; c2 < 16; ++c2) {
-                        const float a0 = __uint_as_float(sr[2 * c2]), a1 = __uint_as_float(sr[2 * c2 + 1]);
-                        mx[c2 & 3] = fmax3(mx[c2 & 3], a0, a1);
-                        const float2 x = f2unpack(ffma2(f2pack(a0, a1), sl2x2, negm2));
-                        const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
-                        lc2[c2 & 1] = fadd2(lc2[c2 & 1], pp);
-                        sr[c2] = pack2<kFP16>(pp);
-                    }
-                    lc = fadd2(lc2[0], lc2[1]);
-                    if (j == 0 || attempt > 0) break;
-                    const float cm = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-                    const bool viol = cm * sl2 > m + kRescaleThreshold;
-                    if (!__any_sync(0xffffffffu, viol)) break;
-                    // maximum over S chunks q..3 (all unread so far; chunk q's P is not stored yet)
-                    float cmx = cm;
-#pragma unroll 1
-                    for (int r = q + 1; r < 4; ++r) {
-                        tmem_ld32(sc + r * 32, sr);
-                        tmem_wait_ld();
-                        mask_cols(sr, lim - r * 32);
-#pragma unroll
-                        for (int c = 0; c < 32; c += 2) cmx = fmax3(cmx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                    }
-                    const float m_new = viol ? cmx * sl2 : m;
-                    const float alpha = viol ? ex2(m - m_new) : 1.0f;
-                    const uint64_t alpha2 = f2pack(alpha, alpha);
-                    tmem_wait_st();
-                    uint32_t(&pw)[16] = reinterpret_cast<uint32_t(&)[16]>(sr);
-#pragma unroll 1
-                    for (int r = 0; r < q; ++r) {  // P chunks written with the old maximum
-                        tmem_ld16(sc + r * 16, pw);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) pw[c] = pack2<kFP16>(fmul2(IoT<kFP16>::unpack2(pw[c]), alpha2));
-                        tmem_st16(sc + r * 16, pw);
-                    }
-                    l2 = fmul2(l2, alpha2);
-                    l *= alpha;
-                    // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
-#pragma unroll 1
-                    for (int r = 0; r < D / 32; ++r) {
-                        tmem_ld32(oc + r * 32, sr);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; c += 2) {
-                            const float2 v =
-                                f2unpack(fmul2(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), alpha2));
-                            sr[c] = __float_as_uint(v.x);
-                            sr[c + 1] = __float_as_uint(v.y);
-                        }
-                        tmem_st32(oc + r * 32, sr);
-                    }
-                    m = m_new;
-                    tmem_ld32(sc + q * 32, sr);  // this chunk again
-                    tmem_wait_ld();
-                    mask_cols(sr, lim - q * 32);
+                for (int c2 = 0; c2 < 16; ++c2) {
+                    const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
+                    const float2 x = f2unpack(ffma2(sv, sl2x2, negm2));
+                    const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
+                    l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
+                    sr[c2] = pack2<kFP16>(pp);
                 }
-                l2 = fadd2(l2, lc);
                 tmem_st16(sc + q * 16, reinterpret_cast<const uint32_t(&)[16]>(sr));
             }
-            const float2 la = f2unpack(l2);
+            const float2 la = f2unpack(fadd2(l2[0], l2[1]));
             l += la.x + la.y;
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::kBarPFull + i));
         }
-        // epilogue: out = O / l once the last PV_i is complete
-        const bool fin = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), 0, abort_flag));
+        // epilogue: combine the two halves' row sums (the slot may still hold a maximum the
+        // other half has yet to read, hence the barrier before writing), then out = O / l
+        named_bar_sync(nb, 256);
+        xch[hf * kBlockM + row] = l;
+        named_bar_sync(nb, 256);
+        l += xch[(hf ^ 1) * kBlockM + row];
+        const bool fin = n_i > 0 && __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
+                         __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), 0, abort_flag));
         if (fin) {
             tc_fence_after();
+            const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
             const bool valid = qi < w.L;
             uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
@@ -794,9 +782,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
             else
                 o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
+            o_off += hf * kOHalf;
             const uint64_t il2 = f2pack(inv_l, inv_l);
 #pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
+            for (int q = 0; q < kOHalf / 32; ++q) {
                 uint32_t o[32];
                 tmem_ld32(oc + q * 32, o);
                 tmem_wait_ld();
