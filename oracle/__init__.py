@@ -18,6 +18,10 @@ computes, with the passage it follows:
 * ``rope_sincos``  freq = outer(positionIds_b, invFreq_b); emb = cat(freq, freq);
   sin/cos of emb -- page "DynamicNTKOperation", computation process.
 * ``rope_rotate``  rotate-half: x' = x*cos + rotate_half(x)*sin.
+* ``rope_apply``   the Rope operator on given sin/cos tables: q, k, sin, cos
+  in, rotated q, k out -- page "DynamicNTKOperation", operator context;
+  out = x*cos + rot(x)*sin with rotate-half pairs, or adjacent pairs
+  (x1,x2),(x3,x4),... -- page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 6.
 * ``attention_rows`` / ``attention_probs``  softmax(Q'K'^T * scale) V with the
   full score row, two passes -- page "FlashAttention in ops-transformer", the
   attention formula; GQA grouping from page "RoPE, RMSNorm, GQA/MQA", sec. 12.
@@ -83,6 +87,8 @@ def _load():
             lib.oracle_rope_sincos.restype = ctypes.c_int
             lib.oracle_rope_rotate.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, P]
             lib.oracle_rope_rotate.restype = None
+            lib.oracle_rope_apply.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, P, ctypes.c_int32, P]
+            lib.oracle_rope_apply.restype = None
             lib.oracle_attention_rows.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P, P, ctypes.c_int64, P]
             lib.oracle_attention_rows.restype = ctypes.c_int
             lib.oracle_attention_probs.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, ctypes.c_int32,
@@ -148,6 +154,21 @@ def rope_rotate(x, pos, inv_freq_row):
     assert p.shape == (n,) and inv.shape == (D // 2,)
     out = np.empty_like(x)
     _load().oracle_rope_rotate(_ptr(x), n, D, _ptr(p), _ptr(inv), _ptr(out))
+    return out
+
+
+def rope_apply(x, sin_t, cos_t, table_rows, interleaved: bool = False):
+    """Rows x [n, D] (fp64) rotated with table rows sin_t/cos_t[table_rows[r]]
+    ([*, D], fp64; 16-bit tables are widened exactly by the caller)."""
+    x = _c(x, np.float64)
+    n, D = x.shape
+    s = _c(sin_t, np.float64)
+    c = _c(cos_t, np.float64)
+    tr = _c(table_rows, np.int64)
+    assert s.shape == c.shape and s.shape[1] == D and tr.shape == (n,)
+    assert n == 0 or (tr.min() >= 0 and tr.max() < s.shape[0])
+    out = np.empty_like(x)
+    _load().oracle_rope_apply(_ptr(x), n, D, _ptr(s), _ptr(c), _ptr(tr), 1 if interleaved else 0, _ptr(out))
     return out
 
 

@@ -112,6 +112,32 @@ void oracle_rope_rotate(const double* x, int64_t n, int32_t D, const int32_t* po
     }
 }
 
+/* The Rope operator of page "DynamicNTKOperation" (operator context: q, k,
+ * sin and cos go in, rotated q and k come out), for n rows of width D whose
+ * row r uses table row trow[r] of sin/cos [*, D]:
+ *   out[j] = x[j] * cos[j] + rot(x)[j] * sin[j]
+ * rotate-half pairs (interleaved == 0): rot(x) = (-x[D/2..D), x[0..D/2));
+ * adjacent pairs (interleaved != 0, the (x1,x2),(x3,x4),... blocks of page
+ * "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 6): rot(x)[2i] = -x[2i+1],
+ * rot(x)[2i+1] = x[2i]. */
+void oracle_rope_apply(const double* x, int64_t n, int32_t D, const double* sin_t, const double* cos_t,
+                       const int64_t* trow, int32_t interleaved, double* out) {
+    const int32_t half = D / 2;
+    for (int64_t r = 0; r < n; ++r) {
+        const double* xr = x + r * D;
+        const double* s = sin_t + trow[r] * D;
+        const double* c = cos_t + trow[r] * D;
+        for (int32_t j = 0; j < D; ++j) {
+            double rx;
+            if (interleaved)
+                rx = (j & 1) ? xr[j - 1] : -xr[j + 1];
+            else
+                rx = (j < half) ? -xr[j + half] : xr[j - half];
+            out[r * D + j] = xr[j] * c[j] + rx * s[j];
+        }
+    }
+}
+
 typedef struct {
     int32_t layout;  /* ORC_BNSD: q [B,Hq,S,D], k/v [B,Hkv,S,D], pos [B,S]
                         ORC_TND : q [T,Hq,D],   k/v [T,Hkv,D],   pos [T]   */

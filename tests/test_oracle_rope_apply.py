@@ -1,0 +1,94 @@
+"""Pins of oracle.rope_apply, the Rope operator on given sin/cos tables (page
+"DynamicNTKOperation", operator context: q, k, sin, cos in, rotated q, k out;
+adjacent-pair variant from page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 6).
+
+Each pin checks it against something other than its own formula: complex
+multiplication in numpy, the pinned position-based rotation, the bare pair
+permutation written with numpy slicing, and invariants of a rotation.
+"""
+import numpy as np
+
+import oracle
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _angles(n, half, seed):
+    return _rng(seed).uniform(-50.0, 50.0, (n, half))
+
+
+def test_rotate_half_is_complex_multiplication():
+    n, D = 7, 16
+    x = _rng(1).standard_normal((n, D))
+    th = _angles(n, D // 2, 2)
+    sin_t = np.concatenate([np.sin(th), np.sin(th)], axis=1)
+    cos_t = np.concatenate([np.cos(th), np.cos(th)], axis=1)
+    got = oracle.rope_apply(x, sin_t, cos_t, np.arange(n))
+    z = (x[:, : D // 2] + 1j * x[:, D // 2:]) * np.exp(1j * th)
+    np.testing.assert_allclose(got, np.concatenate([z.real, z.imag], axis=1), rtol=0, atol=1e-12)
+
+
+def test_adjacent_pairs_are_complex_multiplication():
+    n, D = 5, 12
+    x = _rng(3).standard_normal((n, D))
+    th = _angles(n, D // 2, 4)
+    sin_t = np.repeat(np.sin(th), 2, axis=1)  # cos/sin of pair i at columns 2i and 2i+1
+    cos_t = np.repeat(np.cos(th), 2, axis=1)
+    got = oracle.rope_apply(x, sin_t, cos_t, np.arange(n), interleaved=True)
+    z = (x[:, 0::2] + 1j * x[:, 1::2]) * np.exp(1j * th)
+    want = np.empty_like(x)
+    want[:, 0::2], want[:, 1::2] = z.real, z.imag
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_dynamic_ntk_tables_reproduce_position_rotation():
+    # tables from the pinned sin/cos table, rows looked up per token: the same
+    # as rotating by the positions directly
+    D, lens = 32, np.array([3, 5], np.int32)
+    pos = np.array([0, 1, 2, 100, -7, 3, 4, 65535], np.int32)
+    inv = np.stack([oracle.inv_freq(10000.0, D), oracle.inv_freq(500000.0, D)])
+    s, c = oracle.rope_sincos(pos, inv, lens, D)
+    x = _rng(5).standard_normal((len(pos), D))
+    got = oracle.rope_apply(x, s, c, np.arange(len(pos)))
+    seg = np.repeat(np.arange(2), lens)
+    want = np.concatenate([oracle.rope_rotate(x[t:t + 1], pos[t:t + 1], inv[seg[t]]) for t in range(len(pos))])
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_quarter_turn_is_the_pair_permutation():
+    n, D = 4, 10
+    x = _rng(6).standard_normal((n, D))
+    ones, zeros = np.ones((1, D)), np.zeros((1, D))
+    rows = np.zeros(n, np.int64)
+    half = oracle.rope_apply(x, ones, zeros, rows)
+    np.testing.assert_array_equal(half, np.concatenate([-x[:, D // 2:], x[:, : D // 2]], axis=1))
+    adj = oracle.rope_apply(x, ones, zeros, rows, interleaved=True)
+    want = np.empty_like(x)
+    want[:, 0::2], want[:, 1::2] = -x[:, 1::2], x[:, 0::2]
+    np.testing.assert_array_equal(adj, want)
+
+
+def test_zero_sine_scales_elementwise_and_zero_angle_is_identity():
+    n, D = 3, 8
+    x = _rng(7).standard_normal((n, D))
+    c = _rng(8).standard_normal((2, D))
+    rows = np.array([1, 0, 1])
+    for inter in (False, True):
+        np.testing.assert_array_equal(oracle.rope_apply(x, np.zeros((2, D)), c, rows, inter), x * c[rows])
+        np.testing.assert_array_equal(oracle.rope_apply(x, np.zeros((1, D)), np.ones((1, D)), np.zeros(n, np.int64),
+                                                        inter), x)
+
+
+def test_pair_norms_preserved():
+    n, D = 6, 16
+    x = _rng(9).standard_normal((n, D))
+    th = _angles(n, D // 2, 10)
+    s2 = np.concatenate([np.sin(th)] * 2, axis=1)
+    c2 = np.concatenate([np.cos(th)] * 2, axis=1)
+    out = oracle.rope_apply(x, s2, c2, np.arange(n))
+    np.testing.assert_allclose(out[:, :8] ** 2 + out[:, 8:] ** 2, x[:, :8] ** 2 + x[:, 8:] ** 2, rtol=1e-12)
+    s1, c1 = np.repeat(np.sin(th), 2, axis=1), np.repeat(np.cos(th), 2, axis=1)
+    out = oracle.rope_apply(x, s1, c1, np.arange(n), interleaved=True)
+    np.testing.assert_allclose(out[:, 0::2] ** 2 + out[:, 1::2] ** 2, x[:, 0::2] ** 2 + x[:, 1::2] ** 2, rtol=1e-12)
