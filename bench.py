@@ -359,6 +359,36 @@ def sincos_bench(rfa, dev):
             "read_flushed_us": t_rf * 1e6, "read_flushed_GB/s": byts / t_rf / 1e9}
 
 
+def rope_apply_bench(rfa, dev):
+    """rope_apply on the Qwen-7B-shaped prefill's tokens (T = 8192, 32 query +
+    32 kv heads, D = 128, bf16, fp16 DynamicNTK tables): GB/s of algorithmic
+    bytes (q and k read and written, sin and cos read), 272 MB per launch, so
+    launches run back to back without an L2 flush."""
+    T, Hq, Hkv, D = 8192, 32, 32, 128
+    q = workloads.randn16((T, Hq, D), 21).to(dev)
+    k = workloads.randn16((T, Hkv, D), 22).to(dev)
+    pos = torch.arange(T, dtype=torch.int32, device=dev) % 2048
+    inv = torch.from_numpy((10000.0 ** (-np.arange(0, D, 2) / D)).astype(np.float32))[None].to(dev)
+    s, c = rfa.rope_sincos(pos, inv, torch.tensor([T], dtype=torch.int32, device=dev), D, out_dtype=torch.float16)
+    qo, ko = torch.empty_like(q), torch.empty_like(k)
+    for _ in range(3):
+        rfa.rope_apply(q, k, s, c, q_out=qo, k_out=ko)
+    torch.cuda.synchronize()
+    n = 50
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        rfa.rope_apply(q, k, s, c, q_out=qo, k_out=ko)
+    e1.record()
+    torch.cuda.synchronize()
+    assert rfa.get_device_status() == 0
+    t = e0.elapsed_time(e1) * 1e-3 / n
+    byts = 2 * (q.numel() + k.numel()) * 2 + 2 * T * D * 2
+    return {"shape": "T=8192, Hq=32, Hkv=32, D=128, bf16, fp16 tables, rotate-half", "bytes": byts,
+            "us": t * 1e6, "GB/s": byts / t / 1e9, "timing": f"{n} launches back to back (data > L2)"}
+
+
 def unfused_context(w, q, k, v, pos, dev, iters=20):
     """Unfused GPU context: rope with torch ops (rotated q/k written to HBM)
     then torch scaled_dot_product_attention."""
@@ -481,6 +511,8 @@ def run_gpu(args, world, rank, local):
     if rank == 0 and world == 1:
         extra["sincos"] = sincos_bench(rfa, dev)
         extra["sincos"]["frac_hbm"] = extra["sincos"]["GB/s"] / peaks["hbm_gbs"]
+        extra["rope_apply"] = rope_apply_bench(rfa, dev)
+        extra["rope_apply"]["frac_hbm"] = extra["rope_apply"]["GB/s"] / peaks["hbm_gbs"]
         if not args.no_context:
             try:
                 extra["context_unfused"] = unfused_context(w, q, k, v, pos, dev)

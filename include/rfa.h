@@ -72,8 +72,11 @@ typedef enum { RFA_LAYOUT_BNSD = 0, RFA_LAYOUT_TND = 1 } rfa_layout;
  *   sinOut,cosOut dev [ntokens, headSize] of outType, written in full;
  *                columns j and j+headSize/2 are bit-identical.
  *
- * The angle is the fp32 product position*invFreq (as in the page's einsum on
- * fp32 tensors); sin/cos are evaluated in fp32 and rounded to nearest even.
+ * The angle is position*invFreq taken exactly (the fp32 product plus its
+ * rounding error, reduced by 2*pi with the two-constant Cody-Waite scheme);
+ * sin/cos of the reduced angle are evaluated in fp32 (max abs error below
+ * 2e-6 for angles up to 1e6) and rounded to nearest even.  Positions beyond
+ * +-2^24 lose low bits in the int32 -> fp32 conversion.
  * Returns RFA_ERR_INVALID_ARG / RFA_ERR_UNSUPPORTED on host-checkable errors.
  * seqLens lives on the device, so its sum is checked by the kernel: if it is
  * not ntokens (or a length is <= 0) nothing is written and the status word
@@ -82,6 +85,49 @@ typedef enum { RFA_LAYOUT_BNSD = 0, RFA_LAYOUT_TND = 1 } rfa_layout;
 RFA_API rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, const int32_t* seqLens,
                            int32_t batch, int32_t ntokens, int32_t headSize, rfa_dtype outType,
                            void* sinOut, void* cosOut, void* stream);
+
+/* Parameters of rfa_rope_apply (plain old data). */
+typedef struct {
+    int32_t layout;       /* RFA_LAYOUT_TND: x [T, H, D], token t uses table row t;
+                             RFA_LAYOUT_BNSD: x [B, H, S, D], token (b, s) uses table row b*S + s */
+    int32_t T;            /* TND: tokens (>= 1) */
+    int32_t B, S;         /* BNSD: batch, sequence length (>= 1 each) */
+    int32_t Hq, Hkv;      /* heads of q and of k (>= 1; 0 when that tensor is not given) */
+    int32_t D;            /* head dim: even, multiple of 16, <= 512 */
+    int32_t io_dtype;     /* RFA_DT_BF16 | RFA_DT_FP16: q, k, outputs and the cache */
+    int32_t table_dtype;  /* RFA_DT_FP16 | RFA_DT_BF16 | RFA_DT_FP32: sin, cos */
+    int32_t interleaved;  /* 0: rotate-half pairs (j, j + D/2); 1: adjacent pairs (2i, 2i+1) */
+} rfa_rope_apply_params;
+
+/*
+ * rfa_rope_apply -- the Rope operator: q, k, sin and cos in, rotated q and k
+ * out (page "DynamicNTKOperation", operator context: DynamicNTK outputs sin
+ * and cos, which go with q and k into the Rope operator), optionally writing
+ * the rotated keys into a KV cache.  For every row x of width D of q and k and
+ * its token's table rows:
+ *     out[j] = x[j] * cos[j] + rot(x)[j] * sin[j]
+ * with rot(x) = (-x[D/2..D), x[0..D/2)) for rotate-half pairs, or
+ * rot(x)[2i] = -x[2i+1], rot(x)[2i+1] = x[2i] for adjacent pairs (the
+ * (x1,x2),(x3,x4),... blocks of page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE",
+ * sec. 6; such tables hold the angle of pair i in columns 2i and 2i+1).
+ * Arithmetic in fp32, outputs rounded to nearest even.
+ *
+ *   q, k          dev  io_dtype [T, Hq|Hkv, D] (TND) or [B, Hq|Hkv, S, D] (BNSD);
+ *                 either may be NULL (then its heads must be 0)
+ *   sin, cos      dev  table_dtype [T or B*S, D], e.g. rfa_rope_sincos's output
+ *   q_out, k_out  dev  like q, k; may equal q, k (in place); k_out may be NULL
+ *                 when the rotated keys only go to the cache
+ *   cache_slots   dev  int32 [T or B*S] or NULL: token t's rotated keys go to
+ *                 k_cache row cache_slots[t]; negative slots are skipped
+ *   k_cache       dev  io_dtype [cache_rows, Hkv, D] (NULL iff cache_slots NULL)
+ *   cache_rows    rows of k_cache; a slot >= cache_rows is not written and the
+ *                 status word becomes RFA_ERR_INVALID_ARG
+ * Pointers 16-byte aligned.  Returns RFA_ERR_INVALID_ARG for null/misaligned
+ * pointers or bad sizes, RFA_ERR_UNSUPPORTED for other dtypes.
+ */
+RFA_API rfa_status rfa_rope_apply(const rfa_rope_apply_params* p, const void* q, const void* k, const void* sin,
+                                  const void* cos, void* q_out, void* k_out, const int32_t* cache_slots,
+                                  void* k_cache, int64_t cache_rows, void* stream);
 
 /* Parameters of rfa_fused_rope_attention (plain old data). */
 typedef struct {

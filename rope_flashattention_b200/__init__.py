@@ -8,6 +8,7 @@ kernels.  There is no CPU fallback: if librfa.so is missing the import fails.
 
 Entry points (C name without the ``rfa_`` prefix):
     rope_sincos(position_ids, inv_freq, seq_lens, head_size, out_dtype)
+    rope_apply(q, k, sin, cos, ...)   rotated q, k (and a KV-cache write)
     fused_rope_attention(q, k, v, position, ...)
     fused_rope_attention_workspace(...)
     get_device_status()
@@ -25,8 +26,8 @@ import torch
 __all__ = [
     "RfaError", "LIB_PATH", "EXPORTS", "load_library", "rope_sincos", "fused_rope_attention",
     "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
-    "fused_rope_attention_noalloc",
-    "get_device_status", "status_string", "AttnParams",
+    "fused_rope_attention_noalloc", "rope_apply",
+    "get_device_status", "status_string", "AttnParams", "RopeApplyParams",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa.so")
@@ -34,6 +35,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa.so")
 # Every symbol include/rfa.h declares.
 EXPORTS = (
     "rfa_rope_sincos",
+    "rfa_rope_apply",
     "rfa_fused_rope_attention_workspace",
     "rfa_fused_rope_attention",
     "rfa_rope_attention_table",
@@ -75,6 +77,22 @@ class AttnParams(ctypes.Structure):
     ]
 
 
+class RopeApplyParams(ctypes.Structure):
+    """Mirror of rfa_rope_apply_params."""
+    _fields_ = [
+        ("layout", ctypes.c_int32),
+        ("T", ctypes.c_int32),
+        ("B", ctypes.c_int32),
+        ("S", ctypes.c_int32),
+        ("Hq", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("io_dtype", ctypes.c_int32),
+        ("table_dtype", ctypes.c_int32),
+        ("interleaved", ctypes.c_int32),
+    ]
+
+
 _lib = None
 
 
@@ -99,6 +117,8 @@ def load_library():
     lib.rfa_fused_rope_attention_with_table.restype = ctypes.c_int
     lib.rfa_fused_rope_attention_noalloc.argtypes = [ctypes.POINTER(AttnParams), P, P, P, P, P, P, P, P]
     lib.rfa_fused_rope_attention_noalloc.restype = ctypes.c_int
+    lib.rfa_rope_apply.argtypes = [ctypes.POINTER(RopeApplyParams), P, P, P, P, P, P, P, P, I64, P]
+    lib.rfa_rope_apply.restype = ctypes.c_int
     lib.rfa_get_device_status.argtypes = [P]
     lib.rfa_get_device_status.restype = ctypes.c_int
     lib.rfa_status_string.argtypes = [ctypes.c_int]
@@ -154,6 +174,71 @@ def rope_sincos(position_ids: torch.Tensor, inv_freq: torch.Tensor, seq_lens: to
         _dev(sin_out, "sin_out"), _dev(cos_out, "cos_out"), _stream_ptr(stream))
     _check(code, "rfa_rope_sincos")
     return sin_out, cos_out
+
+
+def rope_apply(q: Optional[torch.Tensor], k: Optional[torch.Tensor], sin: torch.Tensor, cos: torch.Tensor, *,
+               layout: str = "TND", interleaved: bool = False, inplace: bool = False,
+               q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None,
+               cache_slots: Optional[torch.Tensor] = None, k_cache: Optional[torch.Tensor] = None,
+               keys_out: bool = True, stream=None):
+    """Rotated (q, k) from sin/cos tables [tokens, D] (rfa_rope_apply).
+
+    layout "TND": q [T, Hq, D], k [T, Hkv, D]; "BNSD": q [B, Hq, S, D],
+    k [B, Hkv, S, D] with table row b*S + s.  Either of q, k may be None.
+    inplace writes over q and k.  cache_slots (int32 [tokens]) and k_cache
+    ([rows, Hkv, D]) also write the rotated keys to k_cache[cache_slots[t]]
+    (negative slots skipped); keys_out=False then skips the separate k output.
+    Returns (q_out, k_out) (None where not produced).
+    """
+    x0 = q if q is not None else k
+    if x0 is None:
+        raise ValueError("q or k is required")
+    if layout == "TND":
+        if x0.dim() != 3:
+            raise ValueError("TND tensors are [T, H, D]")
+        T, D = x0.shape[0], x0.shape[2]
+        B = S = 0
+        rows = T
+    elif layout == "BNSD":
+        if x0.dim() != 4:
+            raise ValueError("BNSD tensors are [B, H, S, D]")
+        B, S, D = x0.shape[0], x0.shape[2], x0.shape[3]
+        T = 0
+        rows = B * S
+    else:
+        raise ValueError(f"layout {layout!r}")
+    io = _TORCH_DT.get(x0.dtype)
+    if io not in (DT_FP16, DT_BF16):
+        raise TypeError("q/k must be float16 or bfloat16")
+    tab = _TORCH_DT.get(sin.dtype)
+    if tab is None or cos.dtype != sin.dtype:
+        raise TypeError("sin/cos must share one of float16, bfloat16, float32")
+    if tuple(sin.shape) != (rows, D) or tuple(cos.shape) != (rows, D):
+        raise ValueError(f"sin/cos must be [{rows}, {D}]")
+    hax = 1
+    Hq = int(q.shape[hax]) if q is not None else 0
+    Hkv = int(k.shape[hax]) if k is not None else 0
+    for t, name in ((q, "q"), (k, "k")):
+        if t is not None and (t.dtype != x0.dtype or t.dim() != x0.dim()):
+            raise ValueError(f"{name} must match the other input's dtype and layout")
+    if q is not None:
+        q_out = q if inplace else (q_out if q_out is not None else torch.empty_like(q))
+    if k is not None and (keys_out or k_cache is None):
+        k_out = k if inplace else (k_out if k_out is not None else torch.empty_like(k))
+    else:
+        k_out = None
+    p = RopeApplyParams(LAYOUT_TND if layout == "TND" else LAYOUT_BNSD, T, B, S, Hq, Hkv, D, io, tab,
+                        1 if interleaved else 0)
+    nul = ctypes.c_void_p(None)
+    slots_p = _dev(cache_slots, "cache_slots", torch.int32) if cache_slots is not None else nul
+    cache_p = _dev(k_cache, "k_cache", x0.dtype) if k_cache is not None else nul
+    rows_cache = int(k_cache.shape[0]) if k_cache is not None else 0
+    code = load_library().rfa_rope_apply(
+        ctypes.byref(p), _dev(q, "q") if q is not None else nul, _dev(k, "k") if k is not None else nul,
+        _dev(sin, "sin"), _dev(cos, "cos"), _dev(q_out, "q_out") if q is not None else nul,
+        _dev(k_out, "k_out") if k_out is not None else nul, slots_p, cache_p, rows_cache, _stream_ptr(stream))
+    _check(code, "rfa_rope_apply")
+    return (q_out if q is not None else None), k_out
 
 
 def _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor) -> AttnParams:

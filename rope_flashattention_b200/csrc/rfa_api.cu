@@ -12,6 +12,7 @@
 
 #include "fused_rope_attn.cuh"
 #include "rfa.h"
+#include "rope_apply.cuh"
 #include "rope_sincos.cuh"
 
 namespace {
@@ -212,6 +213,94 @@ rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, con
             rfa::rope_sincos_kernel<float><<<resident_grid(rfa::rope_sincos_kernel<float>, work, 256), 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
                                                                   headSize, static_cast<float*>(sinOut),
                                                                   static_cast<float*>(cosOut));
+            break;
+    }
+    return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+
+template <bool kFP16, typename TabT>
+void launch_rope_apply(const rfa::RopeApplyArgs& a, bool interleaved, uint32_t work, cudaStream_t st) {
+    if (interleaved) {
+        auto kern = rfa::rope_apply_kernel<kFP16, TabT, true>;
+        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
+    } else {
+        auto kern = rfa::rope_apply_kernel<kFP16, TabT, false>;
+        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+rfa_status rfa_rope_apply(const rfa_rope_apply_params* p, const void* q, const void* k, const void* sin,
+                          const void* cos, void* q_out, void* k_out, const int32_t* cache_slots, void* k_cache,
+                          int64_t cache_rows, void* stream) {
+    if (!p || !sin || !cos) return RFA_ERR_INVALID_ARG;
+    if (p->layout != RFA_LAYOUT_BNSD && p->layout != RFA_LAYOUT_TND) return RFA_ERR_INVALID_ARG;
+    const bool bnsd = p->layout == RFA_LAYOUT_BNSD;
+    int64_t R;
+    if (bnsd) {
+        if (p->B < 1 || p->S < 1) return RFA_ERR_INVALID_ARG;
+        R = static_cast<int64_t>(p->B) * p->S;
+    } else {
+        if (p->T < 1) return RFA_ERR_INVALID_ARG;
+        R = p->T;
+    }
+    if (p->Hq < 0 || p->Hkv < 0 || p->Hq + p->Hkv < 1) return RFA_ERR_INVALID_ARG;
+    if (p->D < 16 || p->D > 512 || p->D % 16 != 0) return RFA_ERR_INVALID_ARG;
+    if (p->interleaved != 0 && p->interleaved != 1) return RFA_ERR_INVALID_ARG;
+    if (p->io_dtype != RFA_DT_BF16 && p->io_dtype != RFA_DT_FP16)
+        return p->io_dtype == RFA_DT_FP32 ? RFA_ERR_UNSUPPORTED : RFA_ERR_INVALID_ARG;
+    if (p->table_dtype != RFA_DT_BF16 && p->table_dtype != RFA_DT_FP16 && p->table_dtype != RFA_DT_FP32)
+        return RFA_ERR_INVALID_ARG;
+    // q: given exactly when it has heads, with somewhere to write; k likewise (k_out and/or the cache)
+    if ((q != nullptr) != (p->Hq > 0) || (p->Hq > 0 && !q_out)) return RFA_ERR_INVALID_ARG;
+    if ((k != nullptr) != (p->Hkv > 0)) return RFA_ERR_INVALID_ARG;
+    if ((cache_slots != nullptr) != (k_cache != nullptr)) return RFA_ERR_INVALID_ARG;
+    if (k_cache && (p->Hkv < 1 || cache_rows < 1)) return RFA_ERR_INVALID_ARG;
+    if (p->Hkv > 0 && !k_out && !k_cache) return RFA_ERR_INVALID_ARG;
+    for (const void* ptr : {static_cast<const void*>(q), k, sin, cos, static_cast<const void*>(q_out),
+                            static_cast<const void*>(k_out), static_cast<const void*>(k_cache)})
+        if (ptr && !aligned(ptr, 16)) return RFA_ERR_INVALID_ARG;
+    if (cache_slots && !aligned(cache_slots, 4)) return RFA_ERR_INVALID_ARG;
+    const int64_t hgroups = (p->Hq + p->Hkv + rfa::kApplyHeads - 1) / rfa::kApplyHeads;
+    const int64_t work = R * hgroups * (p->D / 16);
+    if (work >= (int64_t{1} << 31)) return RFA_ERR_UNSUPPORTED;
+    rfa::RopeApplyArgs a;
+    a.q = q;
+    a.k = k;
+    a.sin_t = sin;
+    a.cos_t = cos;
+    a.q_out = q_out;
+    a.k_out = k_out;
+    a.slots = cache_slots;
+    a.cache = k_cache;
+    a.cache_rows = cache_rows;
+    a.bnsd = bnsd ? 1 : 0;
+    a.R = static_cast<int32_t>(R);
+    a.S = bnsd ? p->S : 1;
+    a.Hq = p->Hq;
+    a.Hkv = p->Hkv;
+    a.D = p->D;
+    const bool fp16 = p->io_dtype == RFA_DT_FP16;
+    const bool inter = p->interleaved != 0;
+    const uint32_t w = static_cast<uint32_t>(work);
+    cudaStream_t st = as_stream(stream);
+    switch (p->table_dtype) {
+        case RFA_DT_FP16:
+            fp16 ? launch_rope_apply<true, __half>(a, inter, w, st) : launch_rope_apply<false, __half>(a, inter, w, st);
+            break;
+        case RFA_DT_BF16:
+            fp16 ? launch_rope_apply<true, __nv_bfloat16>(a, inter, w, st)
+                 : launch_rope_apply<false, __nv_bfloat16>(a, inter, w, st);
+            break;
+        default:
+            fp16 ? launch_rope_apply<true, float>(a, inter, w, st) : launch_rope_apply<false, float>(a, inter, w, st);
             break;
     }
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;

@@ -1,0 +1,186 @@
+// rope_apply.cuh -- the Rope operator: q, k and their tokens' sin/cos table
+// rows in, rotated q and k out (page "DynamicNTKOperation", operator context:
+// DynamicNTK's sin and cos go with q and k into the Rope operator), with an
+// optional write of the rotated keys into a KV cache.
+//
+//   out[j] = x[j] * cos[j] + rot(x)[j] * sin[j]
+//   rotate-half pairs: rot(x) = (-x[D/2..D), x[0..D/2))
+//   adjacent pairs (page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 6):
+//                      rot(x)[2i] = -x[2i+1], rot(x)[2i+1] = x[2i]
+//
+// HBM-bound elementwise work.  A thread owns one token row, one 8-element
+// chunk in each half of D (elements 8c.. and D/2 + 8c..) and a group of up to
+// kApplyHeads heads: it reads its 2 x 8 cos and sin values once, then rotates
+// that chunk pair of each head with 16-byte loads and stores.  Eight
+// consecutive threads cover one 256-byte row (D = 128), so accesses coalesce.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace rfa {
+
+constexpr int kApplyHeads = 8;  // heads per thread
+
+struct RopeApplyArgs {
+    const void* q;
+    const void* k;
+    const void* sin_t;
+    const void* cos_t;
+    void* q_out;
+    void* k_out;
+    const int32_t* slots;  // [R] or nullptr
+    void* cache;           // [cache_rows, Hkv, D] or nullptr
+    int64_t cache_rows;
+    int32_t bnsd;          // 1: x [B, H, S, D]; 0: x [R, H, D]
+    int32_t R;             // token rows (T, or B * S)
+    int32_t S;             // BNSD sequence length
+    int32_t Hq, Hkv, D;
+};
+
+// 8 consecutive table values as fp32
+template <typename TabT>
+struct Tab8;
+template <>
+struct Tab8<__half> {
+    static __device__ __forceinline__ void load(const void* p, float (&v)[8]) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+        }
+    }
+};
+template <>
+struct Tab8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const void* p, float (&v)[8]) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+template <>
+struct Tab8<float> {
+    static __device__ __forceinline__ void load(const void* p, float (&v)[8]) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+
+// 8 bf16 / fp16 values <-> fp32
+template <bool kFP16>
+__device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if constexpr (kFP16) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+        } else {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+}
+template <bool kFP16>
+__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if constexpr (kFP16) {
+            const __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        } else {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <bool kFP16, typename TabT, bool kInterleaved>
+__global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyArgs a) {
+    const uint32_t chunks = static_cast<uint32_t>(a.D) / 16u;  // chunk pairs per row
+    const int32_t H = a.Hq + a.Hkv;
+    const uint32_t hgroups = static_cast<uint32_t>((H + kApplyHeads - 1) / kApplyHeads);
+    const uint32_t work = static_cast<uint32_t>(a.R) * hgroups * chunks;  // < 2^31, checked on the host
+    const int32_t half = a.D / 2;
+    for (uint32_t w = blockIdx.x * blockDim.x + threadIdx.x; w < work; w += gridDim.x * blockDim.x) {
+        const uint32_t c = w % chunks;
+        const uint32_t rem = w / chunks;
+        const int32_t hg = static_cast<int32_t>(rem % hgroups);
+        const int32_t r = static_cast<int32_t>(rem / hgroups);
+        const int32_t e0 = 8 * static_cast<int32_t>(c), e1 = half + e0;
+        const size_t tsz = sizeof(TabT);
+        const char* srow = static_cast<const char*>(a.sin_t) + static_cast<size_t>(r) * a.D * tsz;
+        const char* crow = static_cast<const char*>(a.cos_t) + static_cast<size_t>(r) * a.D * tsz;
+        float s0[8], s1[8], c0[8], c1[8];
+        Tab8<TabT>::load(srow + e0 * tsz, s0);
+        Tab8<TabT>::load(srow + e1 * tsz, s1);
+        Tab8<TabT>::load(crow + e0 * tsz, c0);
+        Tab8<TabT>::load(crow + e1 * tsz, c1);
+        const int32_t h0 = hg * kApplyHeads;
+        const int32_t h1 = min(h0 + kApplyHeads, H);
+        int32_t slot = -1;
+        if (a.slots != nullptr && h1 > a.Hq) slot = __ldg(a.slots + r);
+        const int32_t b = a.bnsd ? r / a.S : 0, s = a.bnsd ? r - b * a.S : 0;
+#pragma unroll 2
+        for (int32_t h = h0; h < h1; ++h) {
+            const bool is_k = h >= a.Hq;
+            const int32_t hx = is_k ? h - a.Hq : h;
+            const int32_t Hx = is_k ? a.Hkv : a.Hq;
+            const int64_t row = a.bnsd ? (static_cast<int64_t>(b) * Hx + hx) * a.S + s
+                                       : static_cast<int64_t>(r) * Hx + hx;
+            const uint16_t* src = static_cast<const uint16_t*>(is_k ? a.k : a.q) + row * a.D;
+            float x0[8], x1[8], o0[8], o1[8];
+            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e0), x0);
+            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e1), x1);
+            if constexpr (kInterleaved) {
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    o0[i] = fmaf(x0[i], c0[i], -x0[i + 1] * s0[i]);
+                    o0[i + 1] = fmaf(x0[i + 1], c0[i + 1], x0[i] * s0[i + 1]);
+                    o1[i] = fmaf(x1[i], c1[i], -x1[i + 1] * s1[i]);
+                    o1[i + 1] = fmaf(x1[i + 1], c1[i + 1], x1[i] * s1[i + 1]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    o0[i] = fmaf(x0[i], c0[i], -x1[i] * s0[i]);
+                    o1[i] = fmaf(x1[i], c1[i], x0[i] * s1[i]);
+                }
+            }
+            const uint4 p0 = pack8<kFP16>(o0), p1 = pack8<kFP16>(o1);
+            void* dst = is_k ? a.k_out : a.q_out;
+            if (dst != nullptr) {
+                uint16_t* d = static_cast<uint16_t*>(dst) + row * a.D;
+                *reinterpret_cast<uint4*>(d + e0) = p0;
+                *reinterpret_cast<uint4*>(d + e1) = p1;
+            }
+            if (is_k && slot >= 0) {
+                if (slot < a.cache_rows) {
+                    uint16_t* d = static_cast<uint16_t*>(a.cache) + (static_cast<int64_t>(slot) * a.Hkv + hx) * a.D;
+                    *reinterpret_cast<uint4*>(d + e0) = p0;
+                    *reinterpret_cast<uint4*>(d + e1) = p1;
+                } else {
+                    record_status(1 /* RFA_ERR_INVALID_ARG */);
+                }
+            }
+        }
+    }
+}
+
+}  // namespace rfa

@@ -156,3 +156,53 @@ def test_product_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.lower().replace("the oracle", ""), f
+
+
+def _ra(**kw):
+    p = rfa.RopeApplyParams()
+    p.layout, p.T, p.B, p.S, p.Hq, p.Hkv, p.D = rfa.LAYOUT_TND, 16, 0, 0, 2, 1, 64
+    p.io_dtype, p.table_dtype, p.interleaved = rfa.DT_BF16, rfa.DT_FP16, 0
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_rope_apply_params_struct_matches_c_layout():
+    assert ctypes.sizeof(rfa.RopeApplyParams) == 40
+    assert rfa.RopeApplyParams.interleaved.offset == 36
+
+
+MIS = ctypes.c_void_p(0x10002)  # not 16-byte aligned
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=24), rfa.RFA_ERR_INVALID_ARG),            # D % 16
+    (dict(D=528), rfa.RFA_ERR_INVALID_ARG),           # D <= 512
+    (dict(D=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(io_dtype=rfa.DT_FP32), rfa.RFA_ERR_UNSUPPORTED),
+    (dict(io_dtype=rfa.DT_UNDEFINED), rfa.RFA_ERR_INVALID_ARG),
+    (dict(table_dtype=rfa.DT_UNDEFINED), rfa.RFA_ERR_INVALID_ARG),
+    (dict(interleaved=2), rfa.RFA_ERR_INVALID_ARG),
+    (dict(T=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(layout=rfa.LAYOUT_BNSD, B=2, S=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(layout=7), rfa.RFA_ERR_INVALID_ARG),
+    (dict(Hq=0), rfa.RFA_ERR_INVALID_ARG),            # q given without heads
+    (dict(Hq=-1), rfa.RFA_ERR_INVALID_ARG),
+])
+def test_rope_apply_rejects_invalid_params(lib, kw, code):
+    p = _ra(**kw)
+    rc = lib.rfa_rope_apply(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, None)
+    assert rc == code
+
+
+def test_rope_apply_rejects_bad_pointers(lib):
+    p = _ra()
+    call = lambda *a: lib.rfa_rope_apply(ctypes.byref(p), *a, None)
+    assert call(FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, 0) == rfa.RFA_ERR_INVALID_ARG   # no sin
+    assert call(FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, 0) == rfa.RFA_ERR_INVALID_ARG   # no q_out
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 0) == rfa.RFA_ERR_INVALID_ARG   # keys go nowhere
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 8) == rfa.RFA_ERR_INVALID_ARG   # slots without cache
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0) == rfa.RFA_ERR_INVALID_ARG   # cache of 0 rows
+    assert call(FAKE, FAKE, MIS, FAKE, FAKE, FAKE, None, None, 0) == rfa.RFA_ERR_INVALID_ARG    # misaligned table
+    assert call(FAKE, None, FAKE, FAKE, FAKE, FAKE, None, None, 0) == rfa.RFA_ERR_INVALID_ARG   # k heads, no k
+    assert lib.rfa_rope_apply(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, None) == rfa.RFA_ERR_INVALID_ARG
