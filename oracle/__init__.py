@@ -69,6 +69,7 @@ class _Desc(ctypes.Structure):
         ("causal", ctypes.c_int32),
         ("scale", ctypes.c_double),
         ("nthreads", ctypes.c_int32),
+        ("interleaved", ctypes.c_int32),
     ]
 
 
@@ -191,13 +192,13 @@ def _dtype_code(t) -> int:
     return BF16 if t.dtype == torch.bfloat16 else FP16
 
 
-def _desc(layout, dtype, B, Hq, Hkv, S, D, causal, scale, nthreads):
+def _desc(layout, dtype, B, Hq, Hkv, S, D, causal, scale, nthreads, interleaved=False):
     return _Desc(layout, dtype, B, Hq, Hkv, S, D, int(bool(causal)), float(scale),
-                 int(nthreads or default_threads()))
+                 int(nthreads or default_threads()), int(bool(interleaved)))
 
 
 def attention_rows(q, k, v, position, inv_freq_rows, rows, *, layout=BNSD, seq_lens=None, causal=True,
-                   scale=None, nthreads=None) -> np.ndarray:
+                   scale=None, nthreads=None, interleaved=False) -> np.ndarray:
     """fp64 attention output for the given (b, h, i) rows -> [nrows, D].
 
     BNSD: q [B,Hq,S,D], k/v [B,Hkv,S,D], position [B,S].
@@ -216,7 +217,7 @@ def attention_rows(q, k, v, position, inv_freq_rows, rows, *, layout=BNSD, seq_l
         B, S = sl.shape[0], 0
     if scale is None:
         scale = 1.0 / np.sqrt(D)
-    d = _desc(layout, dt, B, Hq, Hkv, S, D, causal, scale, nthreads)
+    d = _desc(layout, dt, B, Hq, Hkv, S, D, causal, scale, nthreads, interleaved)
     qb, kb, vb = _bits16(q), _bits16(k), _bits16(v)
     pos = _c(np.asarray(position), np.int32).reshape(-1)
     inv = _c(inv_freq_rows, np.float64).reshape(B, D // 2)
@@ -230,7 +231,7 @@ def attention_rows(q, k, v, position, inv_freq_rows, rows, *, layout=BNSD, seq_l
 
 
 def attention_probs(q, k, position, inv_freq_rows, b, h, i, *, layout=BNSD, seq_lens=None, causal=True,
-                    scale=None) -> np.ndarray:
+                    scale=None, interleaved=False) -> np.ndarray:
     """One full softmax row P[b,h,i,:] in fp64."""
     dt = _dtype_code(q)
     if layout == BNSD:
@@ -246,7 +247,7 @@ def attention_probs(q, k, position, inv_freq_rows, b, h, i, *, layout=BNSD, seq_
         L = int(sl[b])
     if scale is None:
         scale = 1.0 / np.sqrt(D)
-    d = _desc(layout, dt, B, Hq, Hkv, S, D, causal, scale, 1)
+    d = _desc(layout, dt, B, Hq, Hkv, S, D, causal, scale, 1, interleaved)
     qb, kb = _bits16(q), _bits16(k)
     pos = _c(np.asarray(position), np.int32).reshape(-1)
     inv = _c(inv_freq_rows, np.float64).reshape(B, D // 2)
@@ -270,19 +271,19 @@ def all_rows(B: int, Hq: int, lens) -> np.ndarray:
 
 
 def attention_full(q, k, v, position, inv_freq_rows, *, layout=BNSD, seq_lens=None, causal=True, scale=None,
-                   nthreads=None) -> np.ndarray:
+                   nthreads=None, interleaved=False) -> np.ndarray:
     """Full fp64 output in the layout of q."""
     if layout == BNSD:
         B, Hq, S, D = q.shape
         rows = all_rows(B, Hq, [S] * B)
         out = attention_rows(q, k, v, position, inv_freq_rows, rows, layout=layout, causal=causal, scale=scale,
-                             nthreads=nthreads)
+                             nthreads=nthreads, interleaved=interleaved)
         return out.reshape(B, Hq, S, D)
     T, Hq, D = q.shape
     sl = np.asarray(seq_lens, np.int64)
     rows = all_rows(len(sl), Hq, sl)
     out = attention_rows(q, k, v, position, inv_freq_rows, rows, layout=layout, seq_lens=seq_lens, causal=causal,
-                         scale=scale, nthreads=nthreads)
+                         scale=scale, nthreads=nthreads, interleaved=interleaved)
     full = np.zeros((T, Hq, D), np.float64)
     t0 = np.concatenate([[0], np.cumsum(sl)])
     tok = t0[rows[:, 0]] + rows[:, 2]

@@ -149,7 +149,25 @@ typedef struct {
     int32_t causal;
     double scale;    /* multiplies q'.k' */
     int32_t nthreads;
+    int32_t interleaved; /* 0: rotate-half pairs (i, i + D/2); 1: adjacent pairs (2i, 2i+1) */
 } oracle_attn_desc;
+
+/* RoPE of one row at position pos: rotate-half, or adjacent pairs (the
+ * (x1,x2),(x3,x4),... blocks of page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE",
+ * sec. 6), pair i turned by pos * invFreq[i]. */
+static void rotate_row(const oracle_attn_desc* d, const double* x, int32_t pos, const double* invFreq, double* out) {
+    if (!d->interleaved) {
+        oracle_rope_rotate(x, 1, d->D, &pos, invFreq, out);
+        return;
+    }
+    for (int32_t i = 0; i < d->D / 2; ++i) {
+        double a = (double)pos * invFreq[i];
+        double c = cos(a), s = sin(a);
+        double x1 = x[2 * i], x2 = x[2 * i + 1];
+        out[2 * i] = x1 * c - x2 * s;
+        out[2 * i + 1] = x2 * c + x1 * s;
+    }
+}
 
 typedef struct {
     const oracle_attn_desc* d;
@@ -192,7 +210,7 @@ static void* prep_kv(void* arg) {
             g->Vd[(int64_t)j * D + c] = widen16(g->v[o + c], d->dtype);
         }
         int32_t p = pos_at(d, g->pos, g->tok0, g->b, j);
-        oracle_rope_rotate(xk, 1, D, &p, g->invFreq + (int64_t)g->b * (D / 2), g->Kr + (int64_t)j * D);
+        rotate_row(d, xk, p, g->invFreq + (int64_t)g->b * (D / 2), g->Kr + (int64_t)j * D);
     }
     free(xk);
     return NULL;
@@ -213,7 +231,7 @@ static void* rows_job(void* arg) {
         int64_t qo = q_off(d, g->tok0, g->b, h, i);
         for (int32_t c = 0; c < D; ++c) xq[c] = widen16(g->q[qo + c], d->dtype);
         int32_t p = pos_at(d, g->pos, g->tok0, g->b, i);
-        oracle_rope_rotate(xq, 1, D, &p, g->invFreq + (int64_t)g->b * (D / 2), qr);
+        rotate_row(d, xq, p, g->invFreq + (int64_t)g->b * (D / 2), qr);
         int32_t jmax = d->causal ? i + 1 : g->len;
         /* pass 1: scores and their maximum */
         double m = -INFINITY;
@@ -347,7 +365,7 @@ int oracle_attention_probs(const oracle_attn_desc* d, const uint16_t* q, const u
     for (int32_t c = 0; c < D; ++c) x[c] = widen16(q[qo + c], d->dtype);
     int32_t pq = pos_at(d, pos, t0, b, i);
     const double* inv = invFreq + (int64_t)b * (D / 2);
-    oracle_rope_rotate(x, 1, D, &pq, inv, qr);
+    rotate_row(d, x, pq, inv, qr);
     int32_t jmax = d->causal ? i + 1 : len;
     double m = -INFINITY;
     for (int32_t j = 0; j < len; ++j) {
@@ -358,7 +376,7 @@ int oracle_attention_probs(const oracle_attn_desc* d, const uint16_t* q, const u
         int64_t ko = kv_off(d, t0, b, kvh, j);
         for (int32_t c = 0; c < D; ++c) x[c] = widen16(k[ko + c], d->dtype);
         int32_t pk = pos_at(d, pos, t0, b, j);
-        oracle_rope_rotate(x, 1, D, &pk, inv, kr);
+        rotate_row(d, x, pk, inv, kr);
         double acc = 0.0;
         for (int32_t c = 0; c < D; ++c) acc += qr[c] * kr[c];
         p[j] = acc * d->scale;

@@ -92,3 +92,24 @@ def test_pair_norms_preserved():
     s1, c1 = np.repeat(np.sin(th), 2, axis=1), np.repeat(np.cos(th), 2, axis=1)
     out = oracle.rope_apply(x, s1, c1, np.arange(n), interleaved=True)
     np.testing.assert_allclose(out[:, 0::2] ** 2 + out[:, 1::2] ** 2, x[:, 0::2] ** 2 + x[:, 1::2] ** 2, rtol=1e-12)
+
+
+def test_attention_adjacent_pairs_is_rotate_half_on_permuted_dims():
+    # pair (2i, 2i+1) of the adjacent variant is pair (i, i + D/2) once the
+    # dims are reordered even-then-odd; q.k is unchanged by reordering both
+    import torch
+
+    import workloads
+
+    B, Hq, Hkv, S, D = 1, 2, 1, 37, 16
+    q = workloads.randn16((B, Hq, S, D), 31)
+    k = workloads.randn16((B, Hkv, S, D), 32)
+    v = workloads.randn16((B, Hkv, S, D), 33)
+    pos = torch.arange(S, dtype=torch.int32)[None] * 3 - 5
+    inv = oracle.inv_freq(100.0, D)[None]
+    perm = np.concatenate([np.arange(0, D, 2), np.arange(1, D, 2)])
+    got = oracle.attention_full(q, k, v, pos.numpy(), inv, interleaved=True)
+    want = oracle.attention_full(q[..., perm].contiguous(), k[..., perm].contiguous(), v, pos.numpy(), inv)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    # and it is a different operation from rotate-half on the original order
+    assert np.abs(got - oracle.attention_full(q, k, v, pos.numpy(), inv)).max() > 1e-3
