@@ -141,6 +141,10 @@ typedef struct {
     int32_t causal;        /* 1: key index > query index (within a sequence) masked */
     int32_t io_dtype;      /* RFA_DT_BF16 or RFA_DT_FP16 for q, k, v and out */
     float scale;           /* softmax scale; 0 -> 1/sqrt(D) */
+    int32_t rope_interleaved; /* 0: rotate-half pairs (i, i + D/2); 1: adjacent pairs
+                              (2i, 2i+1), the (x1,x2),(x3,x4),... blocks of page "RoPE,
+                              RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 6; pair i turns by
+                              position * invFreq_i in both */
     double rope_base;      /* invFreq_j = base^(-2j/D) (page "RoPE fused into
                               attention on Ascend", section 1.2), e.g. 10000 */
     int32_t ntk_enable;    /* dynamic NTK (page "DynamicNTKOperation", function

@@ -70,6 +70,7 @@ class AttnParams(ctypes.Structure):
         ("causal", ctypes.c_int32),
         ("io_dtype", ctypes.c_int32),
         ("scale", ctypes.c_float),
+        ("rope_interleaved", ctypes.c_int32),
         ("rope_base", ctypes.c_double),
         ("ntk_enable", ctypes.c_int32),
         ("ntk_train_len", ctypes.c_int32),
@@ -241,7 +242,8 @@ def rope_apply(q: Optional[torch.Tensor], k: Optional[torch.Tensor], sin: torch.
     return (q_out if q is not None else None), k_out
 
 
-def _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor) -> AttnParams:
+def _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor,
+            interleaved=False) -> AttnParams:
     if layout == "BNSD":
         B, Hq, S, D = q.shape
         Hkv = k.shape[1]
@@ -261,12 +263,13 @@ def _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk
     p.ntk_enable = 1 if ntk_train_len else 0
     p.ntk_train_len = int(ntk_train_len or 0)
     p.ntk_factor = float(ntk_factor)
+    p.rope_interleaved = 1 if interleaved else 0
     return p
 
 
 def fused_rope_attention_workspace(q, k, *, layout="BNSD", seq_lens=None, causal=True, scale=None,
-                                   rope_base=10000.0, ntk_train_len=0, ntk_factor=1.0) -> int:
-    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+                                   rope_base=10000.0, ntk_train_len=0, ntk_factor=1.0, interleaved=False) -> int:
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     T = p.B * p.S if layout == "BNSD" else int(sum(int(x) for x in seq_lens))
     return int(load_library().rfa_fused_rope_attention_workspace(ctypes.byref(p), T))
 
@@ -293,10 +296,11 @@ def _ptr_or_null(arr):
 def rope_attention_table(q, k, position: torch.Tensor, *, layout: str = "BNSD", seq_lens=None, causal=True,
                          scale=None, rope_base: float = 10000.0, ntk_train_len: int = 0, ntk_factor: float = 1.0,
                          inv_freq: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                         stream=None) -> torch.Tensor:
+                         interleaved: bool = False, stream=None) -> torch.Tensor:
     """Build the cos/sin table of this batch's positions into a workspace
-    tensor (returned), for reuse by fused_rope_attention_with_table."""
-    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    tensor (returned), for reuse by fused_rope_attention_with_table (the table
+    is the same for both pairings)."""
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, T = _lens_arg(layout, seq_lens, p)
     need = _need(p, T)
     if workspace is None:
@@ -312,9 +316,9 @@ def rope_attention_table(q, k, position: torch.Tensor, *, layout: str = "BNSD", 
 def fused_rope_attention_with_table(q, k, v, table: torch.Tensor, *, layout: str = "BNSD", seq_lens=None,
                                     causal=True, scale=None, rope_base: float = 10000.0, ntk_train_len: int = 0,
                                     ntk_factor: float = 1.0, out: Optional[torch.Tensor] = None,
-                                    stream=None) -> torch.Tensor:
+                                    interleaved: bool = False, stream=None) -> torch.Tensor:
     """The attention kernel alone, reading a table from rope_attention_table."""
-    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, T = _lens_arg(layout, seq_lens, p)
     if out is None:
         out = torch.empty_like(q)
@@ -331,15 +335,16 @@ def fused_rope_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, posi
                          scale: Optional[float] = None, rope_base: float = 10000.0, ntk_train_len: int = 0,
                          ntk_factor: float = 1.0, inv_freq: Optional[torch.Tensor] = None,
                          out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                         stream=None) -> torch.Tensor:
+                         interleaved: bool = False, stream=None) -> torch.Tensor:
     """softmax(rope(q) rope(k)^T * scale) v, rotated q/k kept on chip.
 
     BNSD: q [B,Hq,S,D], k/v [B,Hkv,S,D], position int32 [B,S].
     TND : q [T,Hq,D], k/v [T,Hkv,D], position int32 [T], seq_lens (host ints).
     ntk_train_len > 0 enables dynamic NTK with factor ntk_factor.
+    interleaved: adjacent pairs (2i, 2i+1) instead of rotate-half pairs.
     inv_freq: optional fp32 [B, D/2] on the GPU.
     """
-    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, T = _lens_arg(layout, seq_lens, p)
     need = _need(p, T)
     if workspace is None:
@@ -361,12 +366,12 @@ def fused_rope_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
                                  layout: str = "BNSD", seq_lens: Optional[Sequence[int]] = None, causal: bool = True,
                                  scale: Optional[float] = None, rope_base: float = 10000.0, ntk_train_len: int = 0,
                                  ntk_factor: float = 1.0, inv_freq: Optional[torch.Tensor] = None,
-                                 out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                                 out: Optional[torch.Tensor] = None, interleaved: bool = False, stream=None) -> torch.Tensor:
     """fused_rope_attention with the library's fixed internal scratch instead of
     a caller workspace (for callers that cannot allocate device memory; see
     rfa_fused_rope_attention_noalloc in include/rfa.h for limits and the
     one-scratch-per-device rule)."""
-    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor)
+    p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, _ = _lens_arg(layout, seq_lens, p)
     if out is None:
         out = torch.empty_like(q)

@@ -254,11 +254,53 @@ __device__ __forceinline__ void rotate8(uint4& x1, uint4& x2, const uint4& t0, c
     }
 }
 
+// One adjacent pair (x[2i], x[2i+1]) held in a 32-bit word, turned by angle
+// (c, s):  (x0 c - x1 s, x1 c + x0 s).
+template <bool kFP16>
+__device__ __forceinline__ uint32_t rot_adj(uint32_t w, float c, float s) {
+    const float2 v = f2unpack(IoT<kFP16>::unpack2(w));
+    return IoT<kFP16>::pack(fmaf(v.x, c, -v.y * s), fmaf(v.y, c, v.x * s));
+}
+
+// Rotate 8 adjacent pairs held in two 16-byte chunks (x1: pairs i..i+3, x2:
+// pairs i+4..i+7), angles from the same table words as rotate8 (t0: pairs
+// i..i+3, t1: pairs i+4..i+7).
+template <bool kFP16>
+__device__ __forceinline__ void rotate8_adj(uint4& x1, uint4& x2, const uint4& t0, const uint4& t1) {
+    uint32_t* a = reinterpret_cast<uint32_t*>(&x1);
+    uint32_t* b = reinterpret_cast<uint32_t*>(&x2);
+    const uint32_t u0[4] = {t0.x, t0.y, t0.z, t0.w}, u1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 c0 = __half22float2(*reinterpret_cast<const __half2*>(&u0[(k >> 1) * 2]));
+        const float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&u0[(k >> 1) * 2 + 1]));
+        const float2 c1 = __half22float2(*reinterpret_cast<const __half2*>(&u1[(k >> 1) * 2]));
+        const float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&u1[(k >> 1) * 2 + 1]));
+        a[k] = rot_adj<kFP16>(a[k], (k & 1) ? c0.y : c0.x, (k & 1) ? s0.y : s0.x);
+        b[k] = rot_adj<kFP16>(b[k], (k & 1) ? c1.y : c1.x, (k & 1) ? s1.y : s1.x);
+    }
+}
+
+// Shared-memory address of logical 16-byte chunk L of row r of a 128-row
+// tile: 128B swizzle within 128-row atoms of 8 chunks.
+template <int D>
+__device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int32_t r, int32_t L) {
+    return tile + static_cast<uint32_t>(L >> 3) * AttnCfg<D>::kAtomBytes + static_cast<uint32_t>(r) * 128u +
+           ((static_cast<uint32_t>(L & 7) ^ static_cast<uint32_t>(r & 7)) << 4);
+}
+// The two chunks a RoPE task rotates together hold the 8 pairs of frequencies
+// 8cp..8cp+7: chunks cp and cp + D/16 (rotate-half) or 2cp and 2cp + 1 (adjacent pairs).
+template <int D, bool kAdj>
+__device__ __forceinline__ void task_chunks(uint32_t tile, int32_t r, int cp, uint32_t& o1, uint32_t& o2) {
+    o1 = chunk_addr<D>(tile, r, kAdj ? 2 * cp : cp);
+    o2 = chunk_addr<D>(tile, r, kAdj ? 2 * cp + 1 : cp + D / 16);
+}
+
 // Rotate the first `rows` rows of a 128-row tile in shared memory with the
 // cos/sin rows staged at `tab`.  128B swizzle: 16-byte chunk c of row r sits at
 // r*128 + ((c ^ (r&7)) << 4) within its 128-row atom.  The table's atoms hold
 // 32 (cos, sin) pairs per row, 4 pairs per chunk.
-template <int D, bool kFP16>
+template <int D, bool kFP16, bool kAdj>
 __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t rows, int32_t rt) {
     constexpr int kPairsPerRow = D / 16;  // 16-byte chunk pairs per row
     constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
@@ -270,13 +312,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t r
         if (r >= rows) continue;
         const uint32_t sw = static_cast<uint32_t>(r & 7);
         uint32_t o1, o2;
-        if constexpr (D == 128) {
-            o1 = tile + r * 128 + ((cp ^ sw) << 4);
-            o2 = o1 + AttnCfg<D>::kAtomBytes;
-        } else {
-            o1 = tile + r * 128 + ((cp ^ sw) << 4);
-            o2 = tile + r * 128 + (((cp + 4) ^ sw) << 4);
-        }
+        task_chunks<D, kAdj>(tile, r, cp, o1, o2);
         uint4 t0, t1;
         if constexpr (D == 128) {
             // row layout of the table: chunk cp of atom 0 = pairs 8cp..8cp+3,
@@ -292,7 +328,10 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t r
             t1 = lds128(tb + (((tc + 1) ^ sw) << 4));
         }
         uint4 x1 = lds128(o1), x2 = lds128(o2);
-        rotate8<kFP16>(x1, x2, t0, t1);
+        if constexpr (kAdj)
+            rotate8_adj<kFP16>(x1, x2, t0, t1);
+        else
+            rotate8<kFP16>(x1, x2, t0, t1);
         sts128(o1, x1);
         sts128(o2, x2);
     }
@@ -313,7 +352,7 @@ __device__ __forceinline__ void rec_step(uint64_t& c, uint64_t& s, uint64_t wc, 
 // Rotate a key tile whose rows hold consecutive positions, without a table.
 // This thread's rows are r0, r0 + step, ...; z holds the angles of row r0 and
 // (wc, ws) advance them by `step` rows.
-template <int D, bool kFP16>
+template <int D, bool kFP16, bool kAdj>
 __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32_t rt, const RecState& z,
                                               const uint64_t (&wc)[4], const uint64_t (&ws)[4]) {
     constexpr int kPairsPerRow = D / 16;
@@ -328,24 +367,28 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
     for (int it = 0; it < kIters; ++it) {
         const int r = r0 + it * kStep;
         if (r < rows) {
-            const uint32_t sw = static_cast<uint32_t>(r & 7);
             uint32_t o1, o2;
-            if constexpr (D == 128) {
-                o1 = tile + r * 128 + ((cp ^ sw) << 4);
-                o2 = o1 + AttnCfg<D>::kAtomBytes;
-            } else {
-                o1 = tile + r * 128 + ((cp ^ sw) << 4);
-                o2 = tile + r * 128 + (((cp + 4) ^ sw) << 4);
-            }
+            task_chunks<D, kAdj>(tile, r, cp, o1, o2);
             uint4 x1 = lds128(o1), x2 = lds128(o2);
             uint32_t* xa = reinterpret_cast<uint32_t*>(&x1);
             uint32_t* xb = reinterpret_cast<uint32_t*>(&x2);
+            if constexpr (kAdj) {
+                // word k of x1 is pair 8cp + k, of x2 pair 8cp + 4 + k
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t X1 = IoT<kFP16>::unpack2(xa[k]);
-                const uint64_t X2 = IoT<kFP16>::unpack2(xb[k]);
-                xa[k] = pack2<kFP16>(fsub2(fmul2(X1, e.c[k]), fmul2(X2, e.s[k])));  // x1 cos - x2 sin
-                xb[k] = pack2<kFP16>(ffma2(X2, e.c[k], fmul2(X1, e.s[k])));        // x2 cos + x1 sin
+                for (int k = 0; k < 4; ++k) {
+                    const float2 ca = f2unpack(e.c[k >> 1]), sa = f2unpack(e.s[k >> 1]);
+                    const float2 cb = f2unpack(e.c[2 + (k >> 1)]), sb = f2unpack(e.s[2 + (k >> 1)]);
+                    xa[k] = rot_adj<kFP16>(xa[k], (k & 1) ? ca.y : ca.x, (k & 1) ? sa.y : sa.x);
+                    xb[k] = rot_adj<kFP16>(xb[k], (k & 1) ? cb.y : cb.x, (k & 1) ? sb.y : sb.x);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t X1 = IoT<kFP16>::unpack2(xa[k]);
+                    const uint64_t X2 = IoT<kFP16>::unpack2(xb[k]);
+                    xa[k] = pack2<kFP16>(fsub2(fmul2(X1, e.c[k]), fmul2(X2, e.s[k])));  // x1 cos - x2 sin
+                    xb[k] = pack2<kFP16>(ffma2(X2, e.c[k], fmul2(X1, e.s[k])));        // x2 cos + x1 sin
+                }
             }
             sts128(o1, x1);
             sts128(o2, x2);
@@ -390,7 +433,7 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 }
 
 
-template <int D, bool kFP16>
+template <int D, bool kFP16, bool kAdj>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     fused_rope_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmT,
@@ -631,7 +674,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
             for (int i = 0; i < nq; ++i) {
                 const int32_t q0 = (i == 0 ? w.qt[0] : w.qt[1]) * kBlockM;
-                rope_tile<D, kFP16>(sbase + C::kOffQ + i * C::kTileBytes, sbase + C::kOffV + i * C::kTileBytes,
+                rope_tile<D, kFP16, kAdj>(sbase + C::kOffQ + i * C::kTileBytes, sbase + C::kOffV + i * C::kTileBytes,
                                     min(kBlockM, w.L - q0), rt);
             }
             fence_proxy_async_smem();  // Q' written by the generic proxy, read by the tensor cores
@@ -643,7 +686,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!mbar_wait(bar(C::kBarKFull + s), u & 1u, abort_flag)) break;
                 const int32_t k0 = j * kBlockN;
                 if (rec) {
-                    rope_tile_rec<D, kFP16>(sbase + C::kOffK + s * C::kTileBytes, min(kBlockN, w.L - k0), rt, z, wc, ws);
+                    rope_tile_rec<D, kFP16, kAdj>(sbase + C::kOffK + s * C::kTileBytes, min(kBlockN, w.L - k0), rt, z, wc, ws);
                     // advance to the next tile by 128 rows (the step is re-read from the cached seed)
                     const int f0 = 8 * (rt % kPairsPerRow);
 #pragma unroll
@@ -652,7 +695,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         rec_step(z.c[k], z.s[k], f2pack(v0.x, v1.x), f2pack(v0.y, v1.y));
                     }
                 } else {
-                    rope_tile<D, kFP16>(sbase + C::kOffK + s * C::kTileBytes,
+                    rope_tile<D, kFP16, kAdj>(sbase + C::kOffK + s * C::kTileBytes,
                                         sbase + C::kOffT + (j % C::kTStages) * C::kTabBytes, min(kBlockN, w.L - k0), rt);
                 }
                 fence_proxy_async_smem();

@@ -129,6 +129,7 @@ rfa_status validate_attn(const rfa_attn_params* p) {
     if (p->ntk_enable && (p->ntk_train_len < 1 || !(p->ntk_factor >= 1.0) || !std::isfinite(p->ntk_factor)))
         return RFA_ERR_INVALID_ARG;
     if ((p->D & 1) != 0) return RFA_ERR_INVALID_ARG;
+    if (p->rope_interleaved != 0 && p->rope_interleaved != 1) return RFA_ERR_INVALID_ARG;
     if (p->D != 64 && p->D != 128) return RFA_ERR_UNSUPPORTED;
     return RFA_OK;
 }
@@ -148,12 +149,12 @@ size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * 
 size_t seeds_bytes(int nseg) { return round_up(static_cast<size_t>(nseg) * sizeof(rfa::RopeSeed), 256); }
 size_t workspace_bytes(int64_t T, int D, int nseg) { return table_bytes(T, D) + seeds_bytes(nseg); }
 
-template <int D, bool kFP16>
+template <int D, bool kFP16, bool kAdj>
 rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mt,
                        const rfa::AttnArgs& args, cudaStream_t st) {
-    auto kern = rfa::fused_rope_attn_fwd_kernel<D, kFP16>;
+    auto kern = rfa::fused_rope_attn_fwd_kernel<D, kFP16, kAdj>;
     constexpr int smem = rfa::AttnCfg<D>::kSmemBytes;
-    if (ensure_smem_attr<D * 2 + (kFP16 ? 1 : 0)>(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
+    if (ensure_smem_attr<D * 4 + (kFP16 ? 2 : 0) + (kAdj ? 1 : 0)>(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
     kern<<<args.n_items, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, mt, args);
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
@@ -437,9 +438,19 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
     CUtensorMap mt;
     ok = ok && make_table_map(&mt, table, static_cast<uint64_t>(T), D);
     if (!ok) return RFA_ERR_CUDA;
-    if (D == 128)
-        return fp16 ? launch_attn<128, true>(mq, mk, mv, mt, aa, st) : launch_attn<128, false>(mq, mk, mv, mt, aa, st);
-    return fp16 ? launch_attn<64, true>(mq, mk, mv, mt, aa, st) : launch_attn<64, false>(mq, mk, mv, mt, aa, st);
+    const bool adj = p->rope_interleaved != 0;
+    if (D == 128) {
+        if (adj)
+            return fp16 ? launch_attn<128, true, true>(mq, mk, mv, mt, aa, st)
+                        : launch_attn<128, false, true>(mq, mk, mv, mt, aa, st);
+        return fp16 ? launch_attn<128, true, false>(mq, mk, mv, mt, aa, st)
+                    : launch_attn<128, false, false>(mq, mk, mv, mt, aa, st);
+    }
+    if (adj)
+        return fp16 ? launch_attn<64, true, true>(mq, mk, mv, mt, aa, st)
+                    : launch_attn<64, false, true>(mq, mk, mv, mt, aa, st);
+    return fp16 ? launch_attn<64, true, false>(mq, mk, mv, mt, aa, st)
+                : launch_attn<64, false, false>(mq, mk, mv, mt, aa, st);
 }
 
 }  // namespace

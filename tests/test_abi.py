@@ -65,6 +65,7 @@ def test_params_struct_matches_c_layout():
     assert ctypes.sizeof(rfa.AttnParams) == 64
     assert rfa.AttnParams.rope_base.offset == 40
     assert rfa.AttnParams.ntk_factor.offset == 56
+    assert rfa.AttnParams.rope_interleaved.offset == 36
 
 
 def _ru(x, a=256):

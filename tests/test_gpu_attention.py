@@ -48,13 +48,13 @@ def _compare(got, ref):
 
 
 def run_bnsd(rfa, B, Hq, Hkv, S, D, *, seed=0, base=10000.0, causal=True, dtype=torch.bfloat16, ntk=None,
-             pos=None, inv=None, scale=None):
+             pos=None, inv=None, scale=None, interleaved=False):
     q = workloads.randn16((B, Hq, S, D), seed, dtype)
     k = workloads.randn16((B, Hkv, S, D), seed + 1, dtype)
     v = workloads.randn16((B, Hkv, S, D), seed + 2, dtype)
     if pos is None:
         pos = torch.arange(S, dtype=torch.int32).repeat(B, 1).contiguous()
-    kw = dict(layout="BNSD", causal=causal, rope_base=base, scale=scale)
+    kw = dict(layout="BNSD", causal=causal, rope_base=base, scale=scale, interleaved=interleaved)
     if ntk is not None:
         kw.update(ntk_train_len=ntk[0], ntk_factor=ntk[1])
     if inv is not None:
@@ -67,7 +67,8 @@ def run_bnsd(rfa, B, Hq, Hkv, S, D, *, seed=0, base=10000.0, causal=True, dtype=
 
 def full_bnsd(rfa, B, Hq, Hkv, S, D, **kw):
     q, k, v, pos, inv, got = run_bnsd(rfa, B, Hq, Hkv, S, D, **kw)
-    ref = oracle.attention_full(q, k, v, pos.numpy(), inv, causal=kw.get("causal", True), scale=kw.get("scale"))
+    ref = oracle.attention_full(q, k, v, pos.numpy(), inv, causal=kw.get("causal", True), scale=kw.get("scale"),
+                                interleaved=kw.get("interleaved", False))
     return _compare(got, ref)
 
 
@@ -132,6 +133,20 @@ def test_running_max_jumps_within_later_tiles(rfa, dtype, causal, zero_pos):
     _compare(out.float().cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("D,S,dtype", [(128, 300, torch.bfloat16), (64, 257, torch.bfloat16), (128, 200, torch.float16)])
+def test_adjacent_pairs(rfa, D, S, dtype):
+    # RoPE on pairs (2i, 2i+1): recurrence path (consecutive positions)
+    full_bnsd(rfa, 2, 4, 2, S, D, seed=200 + D, dtype=dtype, interleaved=True)
+
+
+def test_adjacent_pairs_arbitrary_positions(rfa):
+    # table path (positions not consecutive)
+    B, S, D = 1, 290, 128
+    g = workloads.gen(23)
+    pos = torch.randint(-5000, 90000, (B, S), generator=g, dtype=torch.int32)
+    full_bnsd(rfa, B, 6, 3, S, D, seed=24, pos=pos, interleaved=True)
+
+
 def test_mqa_and_scale(rfa):
     full_bnsd(rfa, 1, 8, 1, 200, 128, seed=13, scale=0.05)
 
@@ -160,13 +175,14 @@ def test_position_shift_invariance(rfa):
     assert d.max() <= MAX_ABS
 
 
-def _packed(rfa, lens, Hq, Hkv, D, *, seed, base=10000.0, random_inv=False, ntk=None, rows=None, dtype=torch.bfloat16):
+def _packed(rfa, lens, Hq, Hkv, D, *, seed, base=10000.0, random_inv=False, ntk=None, rows=None, dtype=torch.bfloat16,
+            interleaved=False):
     T = int(sum(lens))
     q = workloads.randn16((T, Hq, D), seed, dtype)
     k = workloads.randn16((T, Hkv, D), seed + 1, dtype)
     v = workloads.randn16((T, Hkv, D), seed + 2, dtype)
     pos = torch.cat([torch.arange(int(n), dtype=torch.int32) for n in lens])
-    kw = dict(layout="TND", seq_lens=[int(x) for x in lens], rope_base=base)
+    kw = dict(layout="TND", seq_lens=[int(x) for x in lens], rope_base=base, interleaved=interleaved)
     inv_t = None
     if random_inv:
         inv_t = torch.rand(len(lens), D // 2, generator=workloads.gen(seed + 3), dtype=torch.float32)
@@ -178,9 +194,10 @@ def _packed(rfa, lens, Hq, Hkv, D, *, seed, base=10000.0, random_inv=False, ntk=
     got = out.float().cpu().numpy()
     inv = inv_t.double().numpy() if random_inv else _inv_rows(len(lens), D, base, lens, ntk)
     if rows is None:
-        ref = oracle.attention_full(q, k, v, pos.numpy(), inv, layout=oracle.TND, seq_lens=lens)
+        ref = oracle.attention_full(q, k, v, pos.numpy(), inv, layout=oracle.TND, seq_lens=lens, interleaved=interleaved)
         return _compare(got, ref)
-    ref = oracle.attention_rows(q, k, v, pos.numpy(), inv, rows, layout=oracle.TND, seq_lens=lens)
+    ref = oracle.attention_rows(q, k, v, pos.numpy(), inv, rows, layout=oracle.TND, seq_lens=lens,
+                                interleaved=interleaved)
     t0 = np.concatenate([[0], np.cumsum(lens)])
     return _compare(got[t0[rows[:, 0]] + rows[:, 2], rows[:, 1]], ref)
 
@@ -191,6 +208,10 @@ def test_packed_ragged_sequences(rfa):
 
 def test_packed_d64_random_inv(rfa):
     _packed(rfa, [64, 1, 200], 2, 2, 64, seed=50, random_inv=True)
+
+
+def test_packed_adjacent_pairs(rfa):
+    _packed(rfa, [130, 5, 260], 4, 1, 128, seed=65, interleaved=True)
 
 
 def test_packed_per_sequence_ntk(rfa):
