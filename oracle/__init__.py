@@ -22,6 +22,12 @@ computes, with the passage it follows:
   in, rotated q, k out -- page "DynamicNTKOperation", operator context;
   out = x*cos + rot(x)*sin with rotate-half pairs, or adjacent pairs
   (x1,x2),(x3,x4),... -- page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 6.
+* ``rms_norm``     gamma * x / sqrt(mean(x^2) + eps) -- same page, sec. 8.
+* ``kv_rms_norm_rope_cache``  the fused cache-write op named on page "RoPE
+  fused into attention on Ascend" (sec. 5.2, kv_rms_norm_rope_cache): per
+  token and kv head, RMSNorm of k, then the Rope operator, into the K cache at
+  the token's slot; v into the V cache at the same slot; negative slots are
+  skipped.  Its composition is the reading taken (the page names the op only).
 * ``attention_rows`` / ``attention_probs``  softmax(Q'K'^T * scale) V with the
   full score row, two passes -- page "FlashAttention in ops-transformer", the
   attention formula; GQA grouping from page "RoPE, RMSNorm, GQA/MQA", sec. 12.
@@ -90,6 +96,8 @@ def _load():
             lib.oracle_rope_rotate.restype = None
             lib.oracle_rope_apply.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, P, ctypes.c_int32, P]
             lib.oracle_rope_apply.restype = None
+            lib.oracle_rms_norm.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, ctypes.c_double, P]
+            lib.oracle_rms_norm.restype = None
             lib.oracle_attention_rows.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, P, P, ctypes.c_int64, P]
             lib.oracle_attention_rows.restype = ctypes.c_int
             lib.oracle_attention_probs.argtypes = [ctypes.POINTER(_Desc), P, P, P, P, P, ctypes.c_int32,
@@ -171,6 +179,35 @@ def rope_apply(x, sin_t, cos_t, table_rows, interleaved: bool = False):
     out = np.empty_like(x)
     _load().oracle_rope_apply(_ptr(x), n, D, _ptr(s), _ptr(c), _ptr(tr), 1 if interleaved else 0, _ptr(out))
     return out
+
+
+def rms_norm(x, gamma, eps: float):
+    """Rows x [n, D] (fp64) -> gamma * x / sqrt(mean(x^2) + eps)."""
+    x = _c(x, np.float64)
+    n, D = x.shape
+    g = _c(gamma, np.float64)
+    assert g.shape == (D,)
+    out = np.empty_like(x)
+    _load().oracle_rms_norm(_ptr(x), n, D, _ptr(g), float(eps), _ptr(out))
+    return out
+
+
+def kv_rms_norm_rope_cache(k, v, gamma, eps, sin_t, cos_t, slots, k_cache, v_cache, interleaved=False):
+    """k, v [T, Hkv, D] (fp64 values), tables [T, D]; writes rows into copies
+    of k_cache / v_cache [rows, Hkv, D] and returns them (fp64)."""
+    k = _c(k, np.float64)
+    v = _c(v, np.float64)
+    T, H, D = k.shape
+    kc = np.array(k_cache, dtype=np.float64, copy=True)
+    vc = np.array(v_cache, dtype=np.float64, copy=True)
+    kn = rms_norm(k.reshape(T * H, D), gamma, eps)
+    kr = rope_apply(kn, sin_t, cos_t, np.repeat(np.arange(T), H), interleaved).reshape(T, H, D)
+    for t in range(T):
+        sl = int(slots[t])
+        if sl >= 0:
+            kc[sl] = kr[t]
+            vc[sl] = v[t]
+    return kc, vc
 
 
 def _bits16(t) -> np.ndarray:

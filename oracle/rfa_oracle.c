@@ -138,6 +138,17 @@ void oracle_rope_apply(const double* x, int64_t n, int32_t D, const double* sin_
     }
 }
 
+/* RMSNorm of n rows of width D (page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE",
+ * sec. 8): out = gamma * x / sqrt(mean(x^2) + eps). */
+void oracle_rms_norm(const double* x, int64_t n, int32_t D, const double* gamma, double eps, double* out) {
+    for (int64_t r = 0; r < n; ++r) {
+        double ss = 0.0;
+        for (int32_t j = 0; j < D; ++j) ss += x[r * D + j] * x[r * D + j];
+        const double inv = 1.0 / sqrt(ss / (double)D + eps);
+        for (int32_t j = 0; j < D; ++j) out[r * D + j] = gamma[j] * (x[r * D + j] * inv);
+    }
+}
+
 typedef struct {
     int32_t layout;  /* ORC_BNSD: q [B,Hq,S,D], k/v [B,Hkv,S,D], pos [B,S]
                         ORC_TND : q [T,Hq,D],   k/v [T,Hkv,D],   pos [T]   */

@@ -113,3 +113,42 @@ def test_attention_adjacent_pairs_is_rotate_half_on_permuted_dims():
     np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
     # and it is a different operation from rotate-half on the original order
     assert np.abs(got - oracle.attention_full(q, k, v, pos.numpy(), inv)).max() > 1e-3
+
+
+def test_rms_norm_pins():
+    import torch
+
+    x = _rng(40).standard_normal((9, 24)) * 3.0
+    g = _rng(41).uniform(0.5, 2.0, 24)
+    # a library routine as the reference: torch's rms_norm in fp64
+    want = torch.nn.functional.rms_norm(torch.from_numpy(x), (24,), torch.from_numpy(g), eps=1e-5).numpy()
+    np.testing.assert_allclose(oracle.rms_norm(x, g, 1e-5), want, rtol=1e-13, atol=1e-13)
+    # closed forms: unit RMS with gamma = 1, eps = 0; invariant to a positive scale; gamma elementwise
+    one = oracle.rms_norm(x, np.ones(24), 0.0)
+    np.testing.assert_allclose(np.sqrt((one ** 2).mean(axis=1)), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(oracle.rms_norm(7.5 * x, np.ones(24), 0.0), one, rtol=1e-13)
+    np.testing.assert_allclose(oracle.rms_norm(x, g, 0.0), one * g, rtol=1e-13)
+
+
+def test_kv_cache_op_is_norm_then_rope_at_slots():
+    T, H, D, rows = 5, 2, 16, 8
+    k = _rng(42).standard_normal((T, H, D))
+    v = _rng(43).standard_normal((T, H, D))
+    g = _rng(44).uniform(0.5, 2.0, D)
+    th = _angles(T, D // 2, 45)
+    s = np.concatenate([np.sin(th)] * 2, axis=1)
+    c = np.concatenate([np.cos(th)] * 2, axis=1)
+    slots = np.array([3, -1, 0, 7, 5])
+    kc0, vc0 = np.full((rows, H, D), 9.0), np.full((rows, H, D), -9.0)
+    kc, vc = oracle.kv_rms_norm_rope_cache(k, v, g, 1e-6, s, c, slots, kc0, vc0)
+    for t, sl in enumerate(slots):
+        if sl < 0:
+            continue
+        # rotate-half via complex multiplication of the normalised row
+        kn = oracle.rms_norm(k[t], g, 1e-6)
+        z = (kn[:, : D // 2] + 1j * kn[:, D // 2:]) * np.exp(1j * th[t])
+        np.testing.assert_allclose(kc[sl], np.concatenate([z.real, z.imag], axis=1), rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(vc[sl], v[t])
+    untouched = [r for r in range(rows) if r not in set(slots[slots >= 0].tolist())]
+    np.testing.assert_array_equal(kc[untouched], kc0[untouched])
+    np.testing.assert_array_equal(vc[untouched], vc0[untouched])
