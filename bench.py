@@ -389,6 +389,38 @@ def rope_apply_bench(rfa, dev):
             "us": t * 1e6, "GB/s": byts / t / 1e9, "timing": f"{n} launches back to back (data > L2)"}
 
 
+def kv_cache_bench(rfa, dev):
+    """kv_rms_norm_rope_cache writing 32768 tokens x 8 kv heads x D 128 (bf16,
+    fp16 tables) into caches of as many rows: GB/s of algorithmic bytes (k, v,
+    gamma, tables and slots read; both caches written), 285 MB per launch, so
+    launches run back to back without an L2 flush."""
+    T, Hkv, D = 32768, 8, 128
+    k = workloads.randn16((T, Hkv, D), 31).to(dev)
+    v = workloads.randn16((T, Hkv, D), 32).to(dev)
+    gamma = torch.ones(D, dtype=torch.float32, device=dev)
+    pos = torch.arange(T, dtype=torch.int32, device=dev)
+    inv = torch.from_numpy((10000.0 ** (-np.arange(0, D, 2) / D)).astype(np.float32))[None].to(dev)
+    s, c = rfa.rope_sincos(pos, inv, torch.tensor([T], dtype=torch.int32, device=dev), D, out_dtype=torch.float16)
+    slots = torch.randperm(T, generator=workloads.gen(33)).to(torch.int32).to(dev)
+    kc, vc = torch.empty_like(k), torch.empty_like(v)
+    for _ in range(3):
+        rfa.kv_rms_norm_rope_cache(k, v, gamma, 1e-6, s, c, slots, kc, vc)
+    torch.cuda.synchronize()
+    n = 50
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        rfa.kv_rms_norm_rope_cache(k, v, gamma, 1e-6, s, c, slots, kc, vc)
+    e1.record()
+    torch.cuda.synchronize()
+    assert rfa.get_device_status() == 0
+    t = e0.elapsed_time(e1) * 1e-3 / n
+    byts = 2 * 2 * k.numel() * 2 + 2 * T * D * 2 + T * 4 + D * 4
+    return {"shape": "T=32768, Hkv=8, D=128, bf16, fp16 tables, slots a permutation", "bytes": byts,
+            "us": t * 1e6, "GB/s": byts / t / 1e9, "timing": f"{n} launches back to back (data > L2)"}
+
+
 def unfused_context(w, q, k, v, pos, dev, iters=20):
     """Unfused GPU context: rope with torch ops (rotated q/k written to HBM)
     then torch scaled_dot_product_attention."""
@@ -513,6 +545,8 @@ def run_gpu(args, world, rank, local):
         extra["sincos"]["frac_hbm"] = extra["sincos"]["GB/s"] / peaks["hbm_gbs"]
         extra["rope_apply"] = rope_apply_bench(rfa, dev)
         extra["rope_apply"]["frac_hbm"] = extra["rope_apply"]["GB/s"] / peaks["hbm_gbs"]
+        extra["kv_rms_norm_rope_cache"] = kv_cache_bench(rfa, dev)
+        extra["kv_rms_norm_rope_cache"]["frac_hbm"] = extra["kv_rms_norm_rope_cache"]["GB/s"] / peaks["hbm_gbs"]
         if not args.no_context:
             try:
                 extra["context_unfused"] = unfused_context(w, q, k, v, pos, dev)

@@ -129,6 +129,44 @@ RFA_API rfa_status rfa_rope_apply(const rfa_rope_apply_params* p, const void* q,
                                   const void* cos, void* q_out, void* k_out, const int32_t* cache_slots,
                                   void* k_cache, int64_t cache_rows, void* stream);
 
+/* Parameters of rfa_kv_rms_norm_rope_cache (plain old data). */
+typedef struct {
+    int32_t T;            /* tokens (>= 1) */
+    int32_t Hkv;          /* kv heads (>= 1) */
+    int32_t D;            /* head dim: 16, 32, 64, 128, 256 or 512 */
+    int32_t io_dtype;     /* RFA_DT_BF16 | RFA_DT_FP16: k, v and both caches */
+    int32_t table_dtype;  /* RFA_DT_FP16 | RFA_DT_BF16 | RFA_DT_FP32: sin, cos */
+    int32_t interleaved;  /* 0: rotate-half pairs; 1: adjacent pairs (as rfa_rope_apply) */
+    float eps;            /* RMSNorm epsilon, finite and >= 0 */
+} rfa_kv_cache_params;
+
+/*
+ * rfa_kv_rms_norm_rope_cache -- RMSNorm, RoPE and the KV-cache write in one
+ * pass: the kv_rms_norm_rope_cache op of page "RoPE fused into attention on
+ * Ascend" (sec. 5.2), which names it without stating its formula; the reading
+ * taken: for token t and kv head h,
+ *     k_cache[slots[t], h, :] = rope(gamma * k[t,h,:] / sqrt(mean(k[t,h,:]^2) + eps))
+ *     v_cache[slots[t], h, :] = v[t,h,:]
+ * with RMSNorm as on page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE" (sec. 8) and
+ * rope() the Rope operator of rfa_rope_apply on the token's table row.
+ * Tokens with slots[t] < 0 are skipped.  Arithmetic in fp32, cache rows
+ * rounded to nearest even; v rows are copied bit for bit.
+ *
+ *   k, v          dev  io_dtype [T, Hkv, D]
+ *   gamma         dev  fp32 [D]
+ *   sin, cos      dev  table_dtype [T, D]
+ *   slots         dev  int32 [T]
+ *   k_cache, v_cache dev io_dtype [cache_rows, Hkv, D]
+ *   cache_rows    >= 1; a slot >= cache_rows is not written and the status word
+ *                 becomes RFA_ERR_INVALID_ARG
+ * Pointers 16-byte aligned (slots 4-byte).  Returns RFA_ERR_INVALID_ARG for
+ * null/misaligned pointers or bad sizes.
+ */
+RFA_API rfa_status rfa_kv_rms_norm_rope_cache(const rfa_kv_cache_params* p, const void* k, const void* v,
+                                              const float* gamma, const void* sin, const void* cos,
+                                              const int32_t* slots, void* k_cache, void* v_cache,
+                                              int64_t cache_rows, void* stream);
+
 /* Parameters of rfa_fused_rope_attention (plain old data). */
 typedef struct {
     int32_t B;             /* BNSD: batch size; TND: number of packed sequences (1..16) */

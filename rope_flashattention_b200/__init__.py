@@ -9,6 +9,7 @@ kernels.  There is no CPU fallback: if librfa.so is missing the import fails.
 Entry points (C name without the ``rfa_`` prefix):
     rope_sincos(position_ids, inv_freq, seq_lens, head_size, out_dtype)
     rope_apply(q, k, sin, cos, ...)   rotated q, k (and a KV-cache write)
+    kv_rms_norm_rope_cache(k, v, gamma, eps, sin, cos, slots, k_cache, v_cache)
     fused_rope_attention(q, k, v, position, ...)
     fused_rope_attention_workspace(...)
     get_device_status()
@@ -26,7 +27,7 @@ import torch
 __all__ = [
     "RfaError", "LIB_PATH", "EXPORTS", "load_library", "rope_sincos", "fused_rope_attention",
     "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
-    "fused_rope_attention_noalloc", "rope_apply",
+    "fused_rope_attention_noalloc", "rope_apply", "kv_rms_norm_rope_cache", "KvCacheParams",
     "get_device_status", "status_string", "AttnParams", "RopeApplyParams",
 ]
 
@@ -36,6 +37,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa.so")
 EXPORTS = (
     "rfa_rope_sincos",
     "rfa_rope_apply",
+    "rfa_kv_rms_norm_rope_cache",
     "rfa_fused_rope_attention_workspace",
     "rfa_fused_rope_attention",
     "rfa_rope_attention_table",
@@ -94,6 +96,19 @@ class RopeApplyParams(ctypes.Structure):
     ]
 
 
+class KvCacheParams(ctypes.Structure):
+    """Mirror of rfa_kv_cache_params."""
+    _fields_ = [
+        ("T", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("io_dtype", ctypes.c_int32),
+        ("table_dtype", ctypes.c_int32),
+        ("interleaved", ctypes.c_int32),
+        ("eps", ctypes.c_float),
+    ]
+
+
 _lib = None
 
 
@@ -120,6 +135,8 @@ def load_library():
     lib.rfa_fused_rope_attention_noalloc.restype = ctypes.c_int
     lib.rfa_rope_apply.argtypes = [ctypes.POINTER(RopeApplyParams), P, P, P, P, P, P, P, P, I64, P]
     lib.rfa_rope_apply.restype = ctypes.c_int
+    lib.rfa_kv_rms_norm_rope_cache.argtypes = [ctypes.POINTER(KvCacheParams), P, P, P, P, P, P, P, P, I64, P]
+    lib.rfa_kv_rms_norm_rope_cache.restype = ctypes.c_int
     lib.rfa_get_device_status.argtypes = [P]
     lib.rfa_get_device_status.restype = ctypes.c_int
     lib.rfa_status_string.argtypes = [ctypes.c_int]
@@ -291,6 +308,35 @@ def _need(p, T) -> int:
 
 def _ptr_or_null(arr):
     return None if arr is None else ctypes.cast(arr, ctypes.c_void_p)
+
+
+def kv_rms_norm_rope_cache(k: torch.Tensor, v: torch.Tensor, gamma: torch.Tensor, eps: float, sin: torch.Tensor,
+                           cos: torch.Tensor, slots: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *,
+                           interleaved: bool = False, stream=None):
+    """RMSNorm(k) * gamma, rotated with the token's sin/cos row, into
+    k_cache[slots[t]]; v into v_cache[slots[t]] (rfa_kv_rms_norm_rope_cache).
+    k, v [T, Hkv, D]; gamma fp32 [D]; sin/cos [T, D]; slots int32 [T];
+    caches [rows, Hkv, D].  Writes the caches in place and returns them."""
+    if k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("k and v must both be [T, Hkv, D]")
+    T, Hkv, D = k.shape
+    io = _TORCH_DT.get(k.dtype)
+    if io not in (DT_FP16, DT_BF16):
+        raise TypeError("k/v must be float16 or bfloat16")
+    tab = _TORCH_DT.get(sin.dtype)
+    if tab is None or cos.dtype != sin.dtype:
+        raise TypeError("sin/cos must share one of float16, bfloat16, float32")
+    if tuple(sin.shape) != (T, D) or tuple(cos.shape) != (T, D):
+        raise ValueError(f"sin/cos must be [{T}, {D}]")
+    if k_cache.dim() != 3 or tuple(k_cache.shape[1:]) != (Hkv, D) or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [rows, Hkv, D]")
+    p = KvCacheParams(T, Hkv, D, io, tab, 1 if interleaved else 0, float(eps))
+    code = load_library().rfa_kv_rms_norm_rope_cache(
+        ctypes.byref(p), _dev(k, "k"), _dev(v, "v", k.dtype), _dev(gamma, "gamma", torch.float32), _dev(sin, "sin"),
+        _dev(cos, "cos"), _dev(slots, "slots", torch.int32), _dev(k_cache, "k_cache", k.dtype),
+        _dev(v_cache, "v_cache", k.dtype), int(k_cache.shape[0]), _stream_ptr(stream))
+    _check(code, "rfa_kv_rms_norm_rope_cache")
+    return k_cache, v_cache
 
 
 def rope_attention_table(q, k, position: torch.Tensor, *, layout: str = "BNSD", seq_lens=None, causal=True,

@@ -307,6 +307,75 @@ rfa_status rfa_rope_apply(const rfa_rope_apply_params* p, const void* q, const v
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+template <bool kFP16, typename TabT>
+void launch_kv_cache(const rfa::KvCacheArgs& a, bool interleaved, uint32_t work, cudaStream_t st) {
+    if (interleaved) {
+        auto kern = rfa::kv_norm_rope_cache_kernel<kFP16, TabT, true>;
+        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
+    } else {
+        auto kern = rfa::kv_norm_rope_cache_kernel<kFP16, TabT, false>;
+        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+rfa_status rfa_kv_rms_norm_rope_cache(const rfa_kv_cache_params* p, const void* k, const void* v, const float* gamma,
+                                      const void* sin, const void* cos, const int32_t* slots, void* k_cache,
+                                      void* v_cache, int64_t cache_rows, void* stream) {
+    if (!p || !k || !v || !gamma || !sin || !cos || !slots || !k_cache || !v_cache) return RFA_ERR_INVALID_ARG;
+    if (p->T < 1 || p->Hkv < 1 || cache_rows < 1) return RFA_ERR_INVALID_ARG;
+    if (p->D < 16 || p->D > 512 || (p->D & (p->D - 1)) != 0) return RFA_ERR_INVALID_ARG;
+    if (p->interleaved != 0 && p->interleaved != 1) return RFA_ERR_INVALID_ARG;
+    if (!(p->eps >= 0.0f) || !std::isfinite(p->eps)) return RFA_ERR_INVALID_ARG;
+    if (p->io_dtype != RFA_DT_BF16 && p->io_dtype != RFA_DT_FP16)
+        return p->io_dtype == RFA_DT_FP32 ? RFA_ERR_UNSUPPORTED : RFA_ERR_INVALID_ARG;
+    if (p->table_dtype != RFA_DT_BF16 && p->table_dtype != RFA_DT_FP16 && p->table_dtype != RFA_DT_FP32)
+        return RFA_ERR_INVALID_ARG;
+    for (const void* ptr : {k, v, static_cast<const void*>(gamma), sin, cos, static_cast<const void*>(k_cache),
+                            static_cast<const void*>(v_cache)})
+        if (!aligned(ptr, 16)) return RFA_ERR_INVALID_ARG;
+    if (!aligned(slots, 4)) return RFA_ERR_INVALID_ARG;
+    const int64_t work = static_cast<int64_t>(p->T) * p->Hkv * (p->D / 16);
+    if (work >= (int64_t{1} << 31)) return RFA_ERR_UNSUPPORTED;
+    rfa::KvCacheArgs a;
+    a.k = k;
+    a.v = v;
+    a.gamma = gamma;
+    a.sin_t = sin;
+    a.cos_t = cos;
+    a.slots = slots;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.cache_rows = cache_rows;
+    a.T = p->T;
+    a.Hkv = p->Hkv;
+    a.D = p->D;
+    a.eps = p->eps;
+    const bool fp16 = p->io_dtype == RFA_DT_FP16, inter = p->interleaved != 0;
+    const uint32_t w = static_cast<uint32_t>(work);
+    cudaStream_t st = as_stream(stream);
+    switch (p->table_dtype) {
+        case RFA_DT_FP16:
+            fp16 ? launch_kv_cache<true, __half>(a, inter, w, st) : launch_kv_cache<false, __half>(a, inter, w, st);
+            break;
+        case RFA_DT_BF16:
+            fp16 ? launch_kv_cache<true, __nv_bfloat16>(a, inter, w, st)
+                 : launch_kv_cache<false, __nv_bfloat16>(a, inter, w, st);
+            break;
+        default:
+            fp16 ? launch_kv_cache<true, float>(a, inter, w, st) : launch_kv_cache<false, float>(a, inter, w, st);
+            break;
+    }
+    return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+}
+
 size_t rfa_fused_rope_attention_workspace(const rfa_attn_params* p, int64_t ntokens) {
     if (validate_attn(p) != RFA_OK || ntokens < 1) return 0;
     return workspace_bytes(ntokens, p->D, p->B);

@@ -183,4 +183,104 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyArgs a) 
     }
 }
 
+// RMSNorm + RoPE + KV-cache write (the kv_rms_norm_rope_cache op named on page
+// "RoPE fused into attention on Ascend", sec. 5.2; RMSNorm from page "RoPE,
+// RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 8): for token t and kv head h,
+//   k_cache[slot_t, h] = rope(gamma * k[t,h] / sqrt(mean(k[t,h]^2) + eps))
+//   v_cache[slot_t, h] = v[t,h]
+// slots < 0 are skipped.  Same thread layout as rope_apply_kernel (one thread
+// per row and chunk pair); a row's D/16 threads are consecutive lanes of one
+// warp and sum their squares with shuffles, so D/16 must be a power of two
+// dividing 32.  The grid-stride loop advances whole warps: every lane of a
+// warp runs the same iterations (lanes past the end carry zeros).
+struct KvCacheArgs {
+    const void* k;
+    const void* v;
+    const float* gamma;
+    const void* sin_t;
+    const void* cos_t;
+    const int32_t* slots;
+    void* k_cache;
+    void* v_cache;
+    int64_t cache_rows;
+    int32_t T, Hkv, D;
+    float eps;
+};
+
+template <bool kFP16, typename TabT, bool kInterleaved>
+__global__ void __launch_bounds__(256) kv_norm_rope_cache_kernel(const KvCacheArgs a) {
+    const uint32_t chunks = static_cast<uint32_t>(a.D) / 16u;  // power of two <= 32
+    const uint32_t work = static_cast<uint32_t>(a.T) * static_cast<uint32_t>(a.Hkv) * chunks;
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t stride = gridDim.x * blockDim.x;
+    const int32_t half = a.D / 2;
+    for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < work; base += stride) {
+        const uint32_t w = base + lane;
+        const bool act = w < work;
+        const uint32_t c = w % chunks;
+        const uint32_t row = w / chunks;  // t * Hkv + h
+        const int32_t t = act ? static_cast<int32_t>(row / static_cast<uint32_t>(a.Hkv)) : 0;
+        const int32_t h = act ? static_cast<int32_t>(row - static_cast<uint32_t>(t) * a.Hkv) : 0;
+        const int32_t e0 = 8 * static_cast<int32_t>(c), e1 = half + e0;
+        float x0[8] = {}, x1[8] = {};
+        const int64_t off = (static_cast<int64_t>(t) * a.Hkv + h) * a.D;
+        if (act) {
+            const uint16_t* src = static_cast<const uint16_t*>(a.k) + off;
+            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e0), x0);
+            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e1), x1);
+        }
+        float ss = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(x0[i], x0[i], fmaf(x1[i], x1[i], ss));
+        for (uint32_t o = chunks >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (!act) continue;
+        const int32_t slot = __ldg(a.slots + t);
+        if (slot < 0) continue;
+        if (slot >= a.cache_rows) {
+            record_status(1 /* RFA_ERR_INVALID_ARG */);
+            continue;
+        }
+        const float inv = rsqrtf(ss / static_cast<float>(a.D) + a.eps);
+        float g0[8], g1[8];
+        Tab8<float>::load(a.gamma + e0, g0);
+        Tab8<float>::load(a.gamma + e1, g1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            x0[i] = g0[i] * (x0[i] * inv);
+            x1[i] = g1[i] * (x1[i] * inv);
+        }
+        const size_t tsz = sizeof(TabT);
+        const char* srow = static_cast<const char*>(a.sin_t) + static_cast<size_t>(t) * a.D * tsz;
+        const char* crow = static_cast<const char*>(a.cos_t) + static_cast<size_t>(t) * a.D * tsz;
+        float s0[8], s1[8], c0[8], c1[8], o0[8], o1[8];
+        Tab8<TabT>::load(srow + e0 * tsz, s0);
+        Tab8<TabT>::load(srow + e1 * tsz, s1);
+        Tab8<TabT>::load(crow + e0 * tsz, c0);
+        Tab8<TabT>::load(crow + e1 * tsz, c1);
+        if constexpr (kInterleaved) {
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                o0[i] = fmaf(x0[i], c0[i], -x0[i + 1] * s0[i]);
+                o0[i + 1] = fmaf(x0[i + 1], c0[i + 1], x0[i] * s0[i + 1]);
+                o1[i] = fmaf(x1[i], c1[i], -x1[i + 1] * s1[i]);
+                o1[i + 1] = fmaf(x1[i + 1], c1[i + 1], x1[i] * s1[i + 1]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                o0[i] = fmaf(x0[i], c0[i], -x1[i] * s0[i]);
+                o1[i] = fmaf(x1[i], c1[i], x0[i] * s1[i]);
+            }
+        }
+        const int64_t dst = (static_cast<int64_t>(slot) * a.Hkv + h) * a.D;
+        uint16_t* kd = static_cast<uint16_t*>(a.k_cache) + dst;
+        *reinterpret_cast<uint4*>(kd + e0) = pack8<kFP16>(o0);
+        *reinterpret_cast<uint4*>(kd + e1) = pack8<kFP16>(o1);
+        const uint16_t* vs = static_cast<const uint16_t*>(a.v) + off;
+        uint16_t* vd = static_cast<uint16_t*>(a.v_cache) + dst;
+        *reinterpret_cast<uint4*>(vd + e0) = *reinterpret_cast<const uint4*>(vs + e0);
+        *reinterpret_cast<uint4*>(vd + e1) = *reinterpret_cast<const uint4*>(vs + e1);
+    }
+}
+
 }  // namespace rfa

@@ -207,3 +207,43 @@ def test_rope_apply_rejects_bad_pointers(lib):
     assert call(FAKE, FAKE, MIS, FAKE, FAKE, FAKE, None, None, 0) == rfa.RFA_ERR_INVALID_ARG    # misaligned table
     assert call(FAKE, None, FAKE, FAKE, FAKE, FAKE, None, None, 0) == rfa.RFA_ERR_INVALID_ARG   # k heads, no k
     assert lib.rfa_rope_apply(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, None) == rfa.RFA_ERR_INVALID_ARG
+
+
+def _kv(**kw):
+    p = rfa.KvCacheParams(8, 2, 64, rfa.DT_BF16, rfa.DT_FP16, 0, 1e-6)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_kv_cache_params_struct_matches_c_layout():
+    assert ctypes.sizeof(rfa.KvCacheParams) == 28
+    assert rfa.KvCacheParams.eps.offset == 24
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=48), rfa.RFA_ERR_INVALID_ARG),           # D a power of two
+    (dict(D=8), rfa.RFA_ERR_INVALID_ARG),
+    (dict(D=1024), rfa.RFA_ERR_INVALID_ARG),
+    (dict(T=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(Hkv=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(eps=-1.0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), rfa.RFA_ERR_INVALID_ARG),
+    (dict(interleaved=3), rfa.RFA_ERR_INVALID_ARG),
+    (dict(io_dtype=rfa.DT_FP32), rfa.RFA_ERR_UNSUPPORTED),
+    (dict(table_dtype=rfa.DT_UNDEFINED), rfa.RFA_ERR_INVALID_ARG),
+])
+def test_kv_cache_rejects_invalid_params(lib, kw, code):
+    p = _kv(**kw)
+    assert lib.rfa_kv_rms_norm_rope_cache(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+                                          None) == code
+
+
+def test_kv_cache_rejects_bad_pointers(lib):
+    p = _kv()
+    call = lambda *a: lib.rfa_kv_rms_norm_rope_cache(ctypes.byref(p), *a, None)
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0) == rfa.RFA_ERR_INVALID_ARG      # no cache rows
+    assert call(FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, 16) == rfa.RFA_ERR_INVALID_ARG     # no gamma
+    assert call(FAKE, FAKE, MIS, FAKE, FAKE, FAKE, FAKE, FAKE, 16) == rfa.RFA_ERR_INVALID_ARG      # misaligned
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16) == rfa.RFA_ERR_INVALID_ARG     # no slots
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 16) == rfa.RFA_ERR_INVALID_ARG     # no v cache

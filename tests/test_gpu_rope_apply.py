@@ -156,3 +156,43 @@ def test_gqa_prefill_size(rfa):
     assert rfa.get_device_status() == 0
     _close(qo, _ref_rows(q, s, c, False, "TND"), torch.bfloat16)
     _close(ko, _ref_rows(k, s, c, False, "TND"), torch.bfloat16)
+
+
+# ---------------------------------------------------------------- RMSNorm + RoPE + KV-cache write
+@pytest.mark.parametrize("io,tab,inter,D", [
+    (torch.bfloat16, torch.float16, False, 128),
+    (torch.bfloat16, torch.float32, True, 64),
+    (torch.float16, torch.bfloat16, False, 256),
+])
+def test_kv_rms_norm_rope_cache(rfa, io, tab, inter, D):
+    T, Hkv, rows = 97, 4, 160
+    k = (workloads.randn16((T, Hkv, D), 50, io).float() * 3.0).to(io).cuda()
+    v = workloads.randn16((T, Hkv, D), 51, io).cuda()
+    gamma = (0.5 + torch.rand(D, generator=workloads.gen(52))).float().cuda()
+    s, c = _tables(rfa, T, D, 53, tab, inter)
+    g = workloads.gen(54)
+    slots = torch.randperm(rows, generator=g)[:T].to(torch.int32)
+    slots[::5] = -1
+    kc = torch.full((rows, Hkv, D), 3.0, dtype=io).cuda()
+    vc = torch.full((rows, Hkv, D), -3.0, dtype=io).cuda()
+    kc0, vc0 = kc.clone(), vc.clone()
+    rfa.kv_rms_norm_rope_cache(k, v, gamma, 1e-6, s, c, slots.cuda(), kc, vc, interleaved=inter)
+    assert rfa.get_device_status() == 0
+    rk, rv = oracle.kv_rms_norm_rope_cache(_f64(k), _f64(v), gamma.double().cpu().numpy(), 1e-6, _f64(s), _f64(c),
+                                           slots.numpy(), _f64(kc0), _f64(vc0), inter)
+    _close(kc, rk, io)
+    assert np.array_equal(_f64(vc), rv)  # values copied bit for bit (and untouched rows kept)
+
+
+def test_kv_cache_op_slot_beyond_cache_sets_status(rfa):
+    T, Hkv, D, rows = 4, 1, 64, 2
+    k = workloads.randn16((T, Hkv, D), 55).cuda()
+    v = workloads.randn16((T, Hkv, D), 56).cuda()
+    s, c = _tables(rfa, T, D, 57, torch.float16, False)
+    kc = torch.zeros((rows, Hkv, D), dtype=torch.bfloat16).cuda()
+    vc = torch.zeros_like(kc)
+    slots = torch.tensor([1, 2, 0, 7], dtype=torch.int32).cuda()
+    rfa.kv_rms_norm_rope_cache(k, v, torch.ones(D).cuda(), 0.0, s, c, slots, kc, vc)
+    assert rfa.get_device_status() == rfa.RFA_ERR_INVALID_ARG
+    assert rfa.get_device_status() == 0
+    assert torch.equal(vc[1], v[0]) and torch.equal(vc[0], v[2])
