@@ -23,6 +23,13 @@ computes, with the passage it follows:
   out = x*cos + rot(x)*sin with rotate-half pairs, or adjacent pairs
   (x1,x2),(x3,x4),... -- page "RoPE, RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 6.
 * ``rms_norm``     gamma * x / sqrt(mean(x^2) + eps) -- same page, sec. 8.
+* ``decode_attention``  the decode step over a KV cache (page "RoPE, RMSNorm,
+  GQA/MQA, SwiGLU, MoE", sec. 12-13: every decode step reads the cached K/V,
+  shared by a group of query heads): the Sq new tokens' queries, rotated at
+  their positions, attend to the cached keys (rotated when written) and
+  values; new token s of a sequence with L cached keys sees keys [0, L-Sq+s]
+  (its own and earlier positions: the new tokens are the last Sq entries).
+  Plain numpy in fp64, full score rows, two-pass softmax.
 * ``kv_rms_norm_rope_cache``  the fused cache-write op named on page "RoPE
   fused into attention on Ascend" (sec. 5.2, kv_rms_norm_rope_cache): per
   token and kv head, RMSNorm of k, then the Rope operator, into the K cache at
@@ -208,6 +215,53 @@ def kv_rms_norm_rope_cache(k, v, gamma, eps, sin_t, cos_t, slots, k_cache, v_cac
             kc[sl] = kr[t]
             vc[sl] = v[t]
     return kc, vc
+
+
+def decode_attention(q, k_cache, v_cache, q_pos, kv_lens, inv_freq_rows, *, causal=True, scale=None,
+                     interleaved=False) -> np.ndarray:
+    """q [B, Hq, Sq, D] (new tokens, not rotated), caches [B, Smax, Hkv, D]
+    (keys already rotated), q_pos [B, Sq], kv_lens [B], inv_freq_rows [B, D/2]
+    -> out [B, Hq, Sq, D] in fp64."""
+    qf = _f64_values(q)
+    kf = _f64_values(k_cache)
+    vf = _f64_values(v_cache)
+    B, Hq, Sq, D = qf.shape
+    Hkv = kf.shape[2]
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    pos = np.asarray(q_pos, np.int64).reshape(B, Sq)
+    inv = np.asarray(inv_freq_rows, np.float64).reshape(B, D // 2)
+    out = np.zeros((B, Hq, Sq, D), np.float64)
+    for b in range(B):
+        L = int(kv_lens[b])
+        for h in range(Hq):
+            kvh = h // G
+            K = kf[b, :L, kvh, :]
+            V = vf[b, :L, kvh, :]
+            for s in range(Sq):
+                th = pos[b, s] * inv[b]  # angle of pair i
+                x = qf[b, h, s]
+                if interleaved:
+                    z = (x[0::2] + 1j * x[1::2]) * np.exp(1j * th)
+                    qr = np.empty(D)
+                    qr[0::2], qr[1::2] = z.real, z.imag
+                else:
+                    z = (x[: D // 2] + 1j * x[D // 2:]) * np.exp(1j * th)
+                    qr = np.concatenate([z.real, z.imag])
+                sc = (K @ qr) * scale
+                if causal:
+                    sc[L - Sq + s + 1:] = -np.inf
+                p = np.exp(sc - sc.max())
+                out[b, h, s] = (p / p.sum()) @ V
+    return out
+
+
+def _f64_values(t) -> np.ndarray:
+    """bf16/fp16 torch tensors (or numpy arrays) as fp64 values, widened exactly."""
+    if hasattr(t, "float"):
+        return t.float().cpu().numpy().astype(np.float64)
+    return np.asarray(t, np.float64)
 
 
 def _bits16(t) -> np.ndarray:

@@ -152,3 +152,34 @@ def test_kv_cache_op_is_norm_then_rope_at_slots():
     untouched = [r for r in range(rows) if r not in set(slots[slots >= 0].tolist())]
     np.testing.assert_array_equal(kc[untouched], kc0[untouched])
     np.testing.assert_array_equal(vc[untouched], vc0[untouched])
+
+
+def test_decode_equals_last_rows_of_full_attention():
+    # a cache filled with keys rotated by the pinned Rope operator at positions
+    # 0..L-1: decoding the last Sq tokens reproduces the last Sq rows of the
+    # pinned full causal attention, for both pairings and with GQA
+    import torch
+
+    import workloads
+
+    B, Hq, Hkv, D, L, Sq = 2, 4, 2, 16, 23, 3
+    for inter in (False, True):
+        q = workloads.randn16((B, Hq, L, D), 60)
+        k = workloads.randn16((B, Hkv, L, D), 61)
+        v = workloads.randn16((B, Hkv, L, D), 62)
+        pos = np.tile(np.arange(L, dtype=np.int32), (B, 1))
+        inv = np.stack([oracle.inv_freq(100.0, D)] * B)
+        full = oracle.attention_full(q, k, v, pos, inv, interleaved=inter)
+        # rotated keys, token-major cache [B, L, Hkv, D]
+        th = pos[..., None] * inv[:, None, :]                       # [B, L, D/2]
+        if inter:
+            s_t, c_t = np.repeat(np.sin(th), 2, -1), np.repeat(np.cos(th), 2, -1)
+        else:
+            s_t, c_t = np.concatenate([np.sin(th)] * 2, -1), np.concatenate([np.cos(th)] * 2, -1)
+        kf = k.float().numpy().astype(np.float64).transpose(0, 2, 1, 3)  # [B, L, Hkv, D]
+        rows = np.repeat(np.arange(B * L), Hkv)
+        kr = oracle.rope_apply(kf.reshape(-1, D), s_t.reshape(-1, D), c_t.reshape(-1, D), rows, inter)
+        kc = kr.reshape(B, L, Hkv, D)
+        vc = v.float().numpy().astype(np.float64).transpose(0, 2, 1, 3)
+        got = oracle.decode_attention(q[:, :, L - Sq:], kc, vc, pos[:, L - Sq:], [L] * B, inv, interleaved=inter)
+        np.testing.assert_allclose(got, full[:, :, L - Sq:], rtol=0, atol=1e-12)
