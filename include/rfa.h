@@ -167,6 +167,52 @@ RFA_API rfa_status rfa_kv_rms_norm_rope_cache(const rfa_kv_cache_params* p, cons
                                               const int32_t* slots, void* k_cache, void* v_cache,
                                               int64_t cache_rows, void* stream);
 
+/* Parameters of rfa_decode_rope_attention (plain old data). */
+typedef struct {
+    int32_t B;                /* sequences (>= 1) */
+    int32_t Hq, Hkv;          /* query / kv heads; Hq % Hkv == 0, G = Hq / Hkv */
+    int32_t Sq;               /* new tokens per sequence (>= 1); G * Sq <= 128 */
+    int32_t D;                /* head dim: 64 or 128 */
+    int32_t Smax;             /* cache rows per sequence */
+    int32_t max_kv_len;       /* bound on kv_lens (Sq..Smax), used to split the keys across CTAs */
+    int32_t causal;           /* 1: new token s sees keys [0, kv_len - Sq + s]; 0: all kv_len keys */
+    int32_t io_dtype;         /* RFA_DT_BF16 | RFA_DT_FP16: q, caches and out */
+    int32_t rope_interleaved; /* 0: rotate-half pairs; 1: adjacent pairs (as the cache was written) */
+    float scale;              /* softmax scale; 0 -> 1/sqrt(D) */
+    int32_t pad_;             /* unused, keep 0 */
+    double rope_base;         /* invFreq_j = base^(-2j/D) when invFreq is NULL */
+} rfa_decode_params;
+
+/*
+ * rfa_decode_rope_attention -- a decode step over a KV cache: the Sq new
+ * tokens of each sequence attend to its cached keys and values (page "RoPE,
+ * RMSNorm, GQA/MQA, SwiGLU, MoE", sec. 12-13: every decode step reads the
+ * cached K/V, shared by a group of query heads).  The new queries are rotated
+ * in the kernel at their positions; the cached keys are taken as stored (they
+ * were rotated when written, e.g. by rfa_rope_apply or
+ * rfa_kv_rms_norm_rope_cache with slot = b * Smax + t).  The new tokens are
+ * the last Sq of the kv_len cached entries:
+ *     out[b,h,s] = softmax_j(rope(q[b,h,s], q_pos[b,s]) . K[b,j,h/G] * scale) V[b,j,h/G]
+ * over j in [0, kv_len_b - Sq + s] (causal) or [0, kv_len_b).
+ *
+ *   q, out        dev io_dtype [B, Hq, Sq, D]
+ *   k_cache, v_cache dev io_dtype [B, Smax, Hkv, D]
+ *   q_pos         dev int32 [B, Sq]
+ *   kv_lens       dev int32 [B]; each in [Sq, max_kv_len], else the status word
+ *                 becomes RFA_ERR_INVALID_ARG (the length is clamped)
+ *   invFreq       dev fp32 [B, D/2] or NULL (then base^(-2j/D) from rope_base)
+ *   workspace     dev, 256-byte aligned, >= rfa_decode_rope_attention_workspace(p)
+ *                 bytes: the queries' cos/sin rows and, when the keys are split
+ *                 across CTAs, fp32 partial results merged by a second kernel
+ * Returns RFA_ERR_INVALID_ARG / RFA_ERR_UNSUPPORTED / RFA_ERR_WORKSPACE on
+ * host-checkable errors; nothing is enqueued then.
+ */
+RFA_API size_t rfa_decode_rope_attention_workspace(const rfa_decode_params* p);
+RFA_API rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* q_pos, const int32_t* kv_lens,
+                                             const float* invFreq, void* out, void* workspace, size_t ws_bytes,
+                                             void* stream);
+
 /* Parameters of rfa_fused_rope_attention (plain old data). */
 typedef struct {
     int32_t B;             /* BNSD: batch size; TND: number of packed sequences (1..16) */

@@ -10,6 +10,7 @@ Entry points (C name without the ``rfa_`` prefix):
     rope_sincos(position_ids, inv_freq, seq_lens, head_size, out_dtype)
     rope_apply(q, k, sin, cos, ...)   rotated q, k (and a KV-cache write)
     kv_rms_norm_rope_cache(k, v, gamma, eps, sin, cos, slots, k_cache, v_cache)
+    decode_rope_attention(q, k_cache, v_cache, q_pos, kv_lens, ...)
     fused_rope_attention(q, k, v, position, ...)
     fused_rope_attention_workspace(...)
     get_device_status()
@@ -28,6 +29,7 @@ __all__ = [
     "RfaError", "LIB_PATH", "EXPORTS", "load_library", "rope_sincos", "fused_rope_attention",
     "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
     "fused_rope_attention_noalloc", "rope_apply", "kv_rms_norm_rope_cache", "KvCacheParams",
+    "decode_rope_attention", "DecodeParams",
     "get_device_status", "status_string", "AttnParams", "RopeApplyParams",
 ]
 
@@ -38,6 +40,8 @@ EXPORTS = (
     "rfa_rope_sincos",
     "rfa_rope_apply",
     "rfa_kv_rms_norm_rope_cache",
+    "rfa_decode_rope_attention_workspace",
+    "rfa_decode_rope_attention",
     "rfa_fused_rope_attention_workspace",
     "rfa_fused_rope_attention",
     "rfa_rope_attention_table",
@@ -109,6 +113,25 @@ class KvCacheParams(ctypes.Structure):
     ]
 
 
+class DecodeParams(ctypes.Structure):
+    """Mirror of rfa_decode_params."""
+    _fields_ = [
+        ("B", ctypes.c_int32),
+        ("Hq", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32),
+        ("Sq", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("Smax", ctypes.c_int32),
+        ("max_kv_len", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
+        ("io_dtype", ctypes.c_int32),
+        ("rope_interleaved", ctypes.c_int32),
+        ("scale", ctypes.c_float),
+        ("pad_", ctypes.c_int32),
+        ("rope_base", ctypes.c_double),
+    ]
+
+
 _lib = None
 
 
@@ -137,6 +160,10 @@ def load_library():
     lib.rfa_rope_apply.restype = ctypes.c_int
     lib.rfa_kv_rms_norm_rope_cache.argtypes = [ctypes.POINTER(KvCacheParams), P, P, P, P, P, P, P, P, I64, P]
     lib.rfa_kv_rms_norm_rope_cache.restype = ctypes.c_int
+    lib.rfa_decode_rope_attention_workspace.argtypes = [ctypes.POINTER(DecodeParams)]
+    lib.rfa_decode_rope_attention_workspace.restype = SZ
+    lib.rfa_decode_rope_attention.argtypes = [ctypes.POINTER(DecodeParams), P, P, P, P, P, P, P, P, SZ, P]
+    lib.rfa_decode_rope_attention.restype = ctypes.c_int
     lib.rfa_get_device_status.argtypes = [P]
     lib.rfa_get_device_status.restype = ctypes.c_int
     lib.rfa_status_string.argtypes = [ctypes.c_int]
@@ -337,6 +364,44 @@ def kv_rms_norm_rope_cache(k: torch.Tensor, v: torch.Tensor, gamma: torch.Tensor
         _dev(v_cache, "v_cache", k.dtype), int(k_cache.shape[0]), _stream_ptr(stream))
     _check(code, "rfa_kv_rms_norm_rope_cache")
     return k_cache, v_cache
+
+
+def decode_rope_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, q_pos: torch.Tensor,
+                          kv_lens: torch.Tensor, *, max_kv_len: Optional[int] = None, causal: bool = True,
+                          scale: Optional[float] = None, rope_base: float = 10000.0,
+                          inv_freq: Optional[torch.Tensor] = None, interleaved: bool = False,
+                          out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """A decode step over a KV cache (rfa_decode_rope_attention).
+
+    q [B, Hq, Sq, D] new tokens (rotated in the kernel at q_pos [B, Sq]);
+    k_cache / v_cache [B, Smax, Hkv, D] with keys already rotated; kv_lens
+    int32 [B] on the GPU (each in [Sq, max_kv_len]; max_kv_len defaults to
+    Smax).  Returns out [B, Hq, Sq, D].
+    """
+    if q.dim() != 4 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q [B, Hq, Sq, D]; caches [B, Smax, Hkv, D]")
+    B, Hq, Sq, D = q.shape
+    Smax, Hkv = int(k_cache.shape[1]), int(k_cache.shape[2])
+    p = DecodeParams(B, Hq, Hkv, Sq, D, Smax, int(max_kv_len if max_kv_len is not None else Smax), 1 if causal else 0,
+                     _TORCH_DT.get(q.dtype, DT_UNDEFINED), 1 if interleaved else 0,
+                     0.0 if scale is None else float(scale), 0, float(rope_base))
+    lib = load_library()
+    need = int(lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)))
+    if need == 0:
+        _check(RFA_ERR_INVALID_ARG, "rfa_decode_rope_attention_workspace")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    io = (torch.bfloat16, torch.float16)
+    code = lib.rfa_decode_rope_attention(
+        ctypes.byref(p), _dev(q, "q", io), _dev(k_cache, "k_cache", q.dtype), _dev(v_cache, "v_cache", q.dtype),
+        _dev(q_pos, "q_pos", torch.int32), _dev(kv_lens, "kv_lens", torch.int32),
+        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(out, "out", q.dtype),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(code, "rfa_decode_rope_attention")
+    return out
 
 
 def rope_attention_table(q, k, position: torch.Tensor, *, layout: str = "BNSD", seq_lens=None, causal=True,

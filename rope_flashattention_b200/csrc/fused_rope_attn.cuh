@@ -85,6 +85,17 @@ struct AttnArgs {
     int32_t seg_tiles[16];
     int32_t seg_item0[17];
     int32_t seg_orig[16];  // caller's index of sorted sequence k
+    // decode over a KV cache (kernel instantiated with kDecode): work item =
+    // (batch, kv head, split of the cache); the query tile holds the G heads x
+    // Sq new tokens of that kv group, rows of q viewed as [B*Hq*Sq, D]
+    int32_t dec_Sq;          // new tokens per sequence
+    int32_t dec_Smax;        // cache rows per sequence (cache viewed as [B*Smax, Hkv, D])
+    int32_t dec_splits;      // splits of each sequence's keys
+    int32_t dec_chunk;       // keys per split, a multiple of kBlockN
+    int32_t dec_max_len;     // upper bound of kv_lens (host planning)
+    const int32_t* kv_lens;  // [B] keys in each sequence's cache, Sq <= len <= dec_max_len
+    float* part_o;           // splits > 1: [splits][B*Hq*Sq][D] unnormalised O
+    float* part_ml;          // splits > 1: [splits][B*Hq*Sq][2] (running max, row sum)
 };
 
 // Work items of one sequence with nt query tiles.
@@ -136,6 +147,8 @@ struct AttnCfg {
 };
 
 struct WorkItem {
+    int32_t qrow0;  // decode: first row of the query tile in q viewed as [B*Hq*Sq, D]
+    int32_t split;  // decode: split index
     int32_t orig;   // sequence index in the caller's order
     int32_t tok0;   // first token of the sequence (BNSD: seq * S)
     int32_t seq;    // BNSD batch index / TND sorted sequence index
@@ -148,8 +161,28 @@ struct WorkItem {
 // Head-major order (the items of one head / head pair are neighbours, so the
 // CTAs resident at one time share K/V tiles through L2), largest tiles first;
 // packed sequences longest first.
+__device__ __forceinline__ WorkItem decode_item_kv(const AttnArgs& a, int32_t x) {
+    WorkItem w;
+    w.split = x % a.dec_splits;
+    const int32_t bk = x / a.dec_splits;
+    w.kvh = bk % a.Hkv;
+    w.seq = bk / a.Hkv;
+    w.orig = w.seq;
+    w.h[0] = w.h[1] = w.kvh * a.G;
+    w.qt[0] = 0;
+    w.qt[1] = -1;
+    w.qrow0 = (w.seq * a.Hq + w.kvh * a.G) * a.dec_Sq;
+    const int32_t k0 = w.split * a.dec_chunk;
+    const int32_t len = min(max(a.kv_lens[w.seq], 0), a.dec_Smax);
+    w.tok0 = w.seq * a.dec_Smax + k0;  // first key of the split in the cache
+    w.L = max(0, min(len - k0, a.dec_chunk));
+    return w;
+}
+
 __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     WorkItem w;
+    w.qrow0 = 0;
+    w.split = 0;
     int32_t nt, r;
     const bool ph = a.pair_heads != 0;
     if (a.layout == 0) {
@@ -433,7 +466,7 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 }
 
 
-template <int D, bool kFP16, bool kAdj>
+template <int D, bool kFP16, bool kAdj, bool kDecode>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     fused_rope_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmT,
@@ -452,15 +485,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const WorkItem w = decode_item(a, blockIdx.x);
+    const WorkItem w = kDecode ? decode_item_kv(a, blockIdx.x) : decode_item(a, blockIdx.x);
     const int32_t nq = (w.qt[1] >= 0) ? 2 : 1;  // query tiles in this item
     const int32_t nkt = (w.L + kBlockN - 1) / kBlockN;
     // key tiles read by query tile i (0: tile absent)
-    const int32_t n0 = a.causal ? (w.qt[0] + 1) : nkt;
+    const int32_t n0 = (a.causal && !kDecode) ? (w.qt[0] + 1) : nkt;
     const int32_t n1 = (nq == 1) ? 0 : (a.causal ? (w.qt[1] + 1) : nkt);
     const int32_t n_kv = max(n0, n1);
     // consecutive positions: K angles come from the recurrence, no cos/sin rows per K tile
-    const bool rec = a.seeds[w.orig].consecutive != 0;
+    // (decode: the cached keys are already rotated)
+    const bool rec = !kDecode && a.seeds[w.orig].consecutive != 0;
+    if constexpr (kDecode) {
+        if (threadIdx.x == 0 && w.split == 0) {
+            const int32_t len = a.kv_lens[w.seq];
+            if (len < a.dec_Sq || len > a.dec_max_len) record_status(1 /* RFA_ERR_INVALID_ARG */);
+        }
+        if (n_kv == 0) {
+            // no keys in this split (past the sequence's length): an empty partial, or, with
+            // one split, zero rows; the CTA returns before any barrier or TMEM is set up
+            const int32_t rq = a.Hq * a.dec_Sq * a.B;
+            for (int r = threadIdx.x; r < a.G * a.dec_Sq; r += blockDim.x) {
+                if (a.dec_splits > 1) {
+                    const int64_t pr = static_cast<int64_t>(w.split) * rq + w.qrow0 + r;
+                    a.part_ml[2 * pr] = -INFINITY;
+                    a.part_ml[2 * pr + 1] = 0.0f;
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) +
+                                                          static_cast<int64_t>(w.qrow0 + r) * D);
+                    for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            return;
+        }
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::kBarQFull), 1);
@@ -515,17 +572,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 if (i >= nq) break;
-                const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
-                load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane, w.qt[i] * kBlockM);
-                load_tab(sbase + C::kOffV + i * C::kTileBytes, bar(C::kBarQFull), w.qt[i] * kBlockM);
+                if constexpr (kDecode) {  // q viewed as [B*Hq*Sq, D]: the group's rows from qrow0
+                    for (int at = 0; at < C::kAtoms; ++at)
+                        tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64, 0, w.qrow0);
+                    for (int bx = 0; bx < C::kTabBoxes; ++bx)
+                        tma_load_3d(sbase + C::kOffV + bx * C::kAtomBytes, &tmT, bar(C::kBarQFull), bx * 32, w.qrow0, 0);
+                } else {
+                    const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
+                    load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane, w.qt[i] * kBlockM);
+                    load_tab(sbase + C::kOffV + i * C::kTileBytes, bar(C::kBarQFull), w.qt[i] * kBlockM);
+                }
             }
-            const uint32_t kbytes = C::kTileBytes + (rec ? 0 : C::kTabBytes);
+            const bool ktab = !kDecode && !rec;  // cos/sin rows staged beside each K tile
+            const uint32_t kbytes = C::kTileBytes + (ktab ? C::kTabBytes : 0);
             int32_t issued_k = 0;
             for (int32_t j = 0; j < n_kv; ++j) {
                 const int s = j % C::kStages;
                 const uint32_t u = static_cast<uint32_t>(j / C::kStages);
                 if (u > 0 && !mbar_wait(bar(C::kBarKEmpty + s), (u - 1) & 1u, abort_flag)) break;
-                if (!rec && j >= C::kTStages) {
+                if (ktab && j >= C::kTStages) {
                     // the rows slot held the rows of key tile j - kTStages: wait until that tile is rotated
                     const int32_t jp = j - C::kTStages;
                     if (!mbar_wait(bar(C::kBarKReady + jp % C::kStages), static_cast<uint32_t>(jp / C::kStages) & 1u,
@@ -534,7 +599,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 mbar_expect_tx(bar(C::kBarKFull + s), kbytes);
                 load_tile(&tmK, sbase + C::kOffK + s * C::kTileBytes, bar(C::kBarKFull + s), kvplane, j * kBlockN);
-                if (!rec) load_tab(sbase + C::kOffT + (j % C::kTStages) * C::kTabBytes, bar(C::kBarKFull + s), j * kBlockN);
+                if (ktab) load_tab(sbase + C::kOffT + (j % C::kTStages) * C::kTabBytes, bar(C::kBarKFull + s), j * kBlockN);
                 issued_k = j + 1;
             }
             // Drain: every issued copy must have landed before the CTA exits.
@@ -675,7 +740,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int i = 0; i < nq; ++i) {
                 const int32_t q0 = (i == 0 ? w.qt[0] : w.qt[1]) * kBlockM;
                 rope_tile<D, kFP16, kAdj>(sbase + C::kOffQ + i * C::kTileBytes, sbase + C::kOffV + i * C::kTileBytes,
-                                    min(kBlockM, w.L - q0), rt);
+                                          kDecode ? kBlockM : min(kBlockM, w.L - q0), rt);
             }
             fence_proxy_async_smem();  // Q' written by the generic proxy, read by the tensor cores
             __syncwarp();
@@ -685,7 +750,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint32_t u = static_cast<uint32_t>(j / C::kStages);
                 if (!mbar_wait(bar(C::kBarKFull + s), u & 1u, abort_flag)) break;
                 const int32_t k0 = j * kBlockN;
-                if (rec) {
+                if constexpr (kDecode) {
+                    // cached keys are already rotated: hand the tile on as it is
+                } else if (rec) {
                     rope_tile_rec<D, kFP16, kAdj>(sbase + C::kOffK + s * C::kTileBytes, min(kBlockN, w.L - k0), rt, z, wc, ws);
                     // advance to the next tile by 128 rows (the step is re-read from the cached seed)
                     const int f0 = 8 * (rt % kPairsPerRow);
@@ -724,7 +791,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t nb = 1u + static_cast<uint32_t>(i);
         const int32_t qt_i = i == 0 ? w.qt[0] : w.qt[1];
         const int32_t qi = qt_i * kBlockM + row;
-        const int32_t vis = a.causal ? min(qi + 1, w.L) : w.L;  // keys [0, vis) visible to this row
+        int32_t vis = a.causal ? min(qi + 1, w.L) : w.L;  // keys [0, vis) visible to this row
+        if constexpr (kDecode) {
+            // row = g * Sq + s: new token s of the sequence's last Sq sees keys up to len - Sq + s
+            // (bottom-right causal), relative to this split's first key
+            const int32_t len = min(max(a.kv_lens[w.seq], 0), a.dec_Smax);
+            vis = a.causal ? min(w.L, len - a.dec_Sq + row % a.dec_Sq + 1 - w.split * a.dec_chunk) : w.L;
+        }
         const float sl2 = a.scale_log2;
         float m = -INFINITY;  // running max of score * scale * log2(e) (identical in both halves)
         float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
@@ -818,13 +891,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_fence_after();
             const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
             const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-            const bool valid = qi < w.L;
+            bool valid = qi < w.L;
             uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
             int64_t o_off;
             if (a.layout == 0)
                 o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
             else
                 o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
+            bool partial = false;
+            if constexpr (kDecode) {
+                // output rows of q viewed as [B*Hq*Sq, D]; with several splits, unnormalised
+                // fp32 O and (m, l) go to the partials that the combine kernel merges
+                valid = row < a.G * a.dec_Sq;
+                o_off = static_cast<int64_t>(w.qrow0 + row) * D;
+                partial = a.dec_splits > 1;
+                if (partial) {
+                    const int64_t pr = static_cast<int64_t>(w.split) * (a.B * a.Hq * a.dec_Sq) + w.qrow0 + row;
+                    o_off = pr * D;
+                    if (valid && hf == 0) {
+                        a.part_ml[2 * pr] = (l > 0.0f) ? m : -INFINITY;
+                        a.part_ml[2 * pr + 1] = l;
+                    }
+                }
+            }
             o_off += hf * kOHalf;
             const uint64_t il2 = f2pack(inv_l, inv_l);
 #pragma unroll 1
@@ -832,7 +921,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 uint32_t o[32];
                 tmem_ld32(oc + q * 32, o);
                 tmem_wait_ld();
-                if (valid) {
+                if (kDecode && partial) {
+                    if (valid) {
+                        float4* dst = reinterpret_cast<float4*>(a.part_o + o_off + q * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 8; ++v4)
+                            dst[v4] = make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
+                                                  __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
+                    }
+                } else if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
@@ -855,6 +952,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// Merge the split partials of decode attention: for every query row,
+// out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s over the splits with
+// l_s > 0 (M their largest m_s), rounded to bf16/fp16.  One thread per row and
+// 8 consecutive columns.
+template <bool kFP16>
+__global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ part_o,
+                                                             const float* __restrict__ part_ml, void* out,
+                                                             int32_t rows, int32_t D, int32_t splits) {
+    const int32_t per_row = D / 8;
+    const int64_t work = static_cast<int64_t>(rows) * per_row;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < work;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int32_t r = static_cast<int32_t>(w / per_row);
+        const int32_t c = static_cast<int32_t>(w - static_cast<int64_t>(r) * per_row) * 8;
+        float M = -INFINITY;
+        for (int32_t s = 0; s < splits; ++s) {
+            const int64_t pr = static_cast<int64_t>(s) * rows + r;
+            if (part_ml[2 * pr + 1] > 0.0f) M = fmaxf(M, part_ml[2 * pr]);
+        }
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float den = 0.0f;
+        for (int32_t s = 0; s < splits; ++s) {
+            const int64_t pr = static_cast<int64_t>(s) * rows + r;
+            const float ls = part_ml[2 * pr + 1];
+            if (!(ls > 0.0f)) continue;
+            const float wgt = exp2f(part_ml[2 * pr] - M);
+            den = fmaf(wgt, ls, den);
+            const float4* src = reinterpret_cast<const float4*>(part_o + pr * D + c);
+            const float4 u = src[0], v = src[1];
+            acc[0] = fmaf(wgt, u.x, acc[0]); acc[1] = fmaf(wgt, u.y, acc[1]);
+            acc[2] = fmaf(wgt, u.z, acc[2]); acc[3] = fmaf(wgt, u.w, acc[3]);
+            acc[4] = fmaf(wgt, v.x, acc[4]); acc[5] = fmaf(wgt, v.y, acc[5]);
+            acc[6] = fmaf(wgt, v.z, acc[6]); acc[7] = fmaf(wgt, v.w, acc[7]);
+        }
+        const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+        uint32_t wv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wv[e] = IoT<kFP16>::pack(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(r) * D + c) =
+            make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
 }
 

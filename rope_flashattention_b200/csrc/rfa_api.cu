@@ -149,12 +149,13 @@ size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * 
 size_t seeds_bytes(int nseg) { return round_up(static_cast<size_t>(nseg) * sizeof(rfa::RopeSeed), 256); }
 size_t workspace_bytes(int64_t T, int D, int nseg) { return table_bytes(T, D) + seeds_bytes(nseg); }
 
-template <int D, bool kFP16, bool kAdj>
+template <int D, bool kFP16, bool kAdj, bool kDecode = false>
 rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mt,
                        const rfa::AttnArgs& args, cudaStream_t st) {
-    auto kern = rfa::fused_rope_attn_fwd_kernel<D, kFP16, kAdj>;
+    auto kern = rfa::fused_rope_attn_fwd_kernel<D, kFP16, kAdj, kDecode>;
     constexpr int smem = rfa::AttnCfg<D>::kSmemBytes;
-    if (ensure_smem_attr<D * 4 + (kFP16 ? 2 : 0) + (kAdj ? 1 : 0)>(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
+    constexpr int kTag = ((D * 4 + (kFP16 ? 2 : 0) + (kAdj ? 1 : 0)) << 1) + (kDecode ? 1 : 0);
+    if (ensure_smem_attr<kTag>(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
     kern<<<args.n_items, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, mt, args);
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
@@ -634,6 +635,155 @@ rfa_status rfa_fused_rope_attention_noalloc(const rfa_attn_params* p, const void
     r = enqueue_table(p, T, position, seqLens_host, invFreq, scratch, st);
     if (r != RFA_OK) return r;
     return enqueue_attention(p, T, q, k, v, seqLens_host, out, scratch, st);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- decode over a KV cache
+namespace {
+
+struct DecodePlan {
+    int32_t splits, chunk;
+    int64_t rq;  // query rows B * Hq * Sq
+    size_t tab_bytes, po_bytes, pml_bytes, total;
+};
+
+rfa_status decode_validate(const rfa_decode_params* p) {
+    if (!p) return RFA_ERR_INVALID_ARG;
+    if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->Sq < 1 || p->Smax < 1) return RFA_ERR_INVALID_ARG;
+    if (p->Hq % p->Hkv != 0) return RFA_ERR_INVALID_ARG;
+    if (p->max_kv_len < p->Sq || p->max_kv_len > p->Smax) return RFA_ERR_INVALID_ARG;
+    if (p->io_dtype != RFA_DT_BF16 && p->io_dtype != RFA_DT_FP16)
+        return p->io_dtype == RFA_DT_UNDEFINED ? RFA_ERR_INVALID_ARG : RFA_ERR_UNSUPPORTED;
+    if (p->rope_interleaved != 0 && p->rope_interleaved != 1) return RFA_ERR_INVALID_ARG;
+    if (!(p->scale >= 0.0f) || !std::isfinite(p->scale)) return RFA_ERR_INVALID_ARG;
+    if (!(p->rope_base > 0.0) || !std::isfinite(p->rope_base)) return RFA_ERR_INVALID_ARG;
+    if ((p->D & 1) != 0 || p->D < 1) return RFA_ERR_INVALID_ARG;
+    if (p->D != 64 && p->D != 128) return RFA_ERR_UNSUPPORTED;
+    if ((p->Hq / p->Hkv) * p->Sq > rfa::kBlockM) return RFA_ERR_UNSUPPORTED;  // one query tile per kv group
+    if (static_cast<int64_t>(p->B) * p->Smax >= (int64_t{1} << 31)) return RFA_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(p->B) * p->Hq * p->Sq >= (int64_t{1} << 31) / 256) return RFA_ERR_UNSUPPORTED;
+    return RFA_OK;
+}
+
+// Keys of a sequence are split so that about two CTAs per SM have work
+// (B * Hkv * splits of them); each split is a whole number of key tiles.
+DecodePlan decode_plan(const rfa_decode_params* p) {
+    DecodePlan pl;
+    pl.rq = static_cast<int64_t>(p->B) * p->Hq * p->Sq;
+    const int64_t groups = static_cast<int64_t>(p->B) * p->Hkv;
+    const int32_t tiles = (p->max_kv_len + rfa::kBlockN - 1) / rfa::kBlockN;
+    int64_t want = (2 * 148 + groups - 1) / groups;
+    const int32_t splits0 = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(want, tiles)));
+    const int32_t per = (tiles + splits0 - 1) / splits0;
+    pl.chunk = per * rfa::kBlockN;
+    pl.splits = (p->max_kv_len + pl.chunk - 1) / pl.chunk;
+    pl.tab_bytes = round_up(static_cast<size_t>(pl.rq) * p->D * 2, 256);
+    pl.po_bytes = pl.splits > 1 ? round_up(static_cast<size_t>(pl.splits) * pl.rq * p->D * 4, 256) : 0;
+    pl.pml_bytes = pl.splits > 1 ? round_up(static_cast<size_t>(pl.splits) * pl.rq * 2 * 4, 256) : 0;
+    pl.total = pl.tab_bytes + pl.po_bytes + pl.pml_bytes;
+    return pl;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rfa_decode_rope_attention_workspace(const rfa_decode_params* p) {
+    if (decode_validate(p) != RFA_OK) return 0;
+    return decode_plan(p).total;
+}
+
+rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* q_pos, const int32_t* kv_lens,
+                                     const float* invFreq, void* out, void* workspace, size_t ws_bytes,
+                                     void* stream) {
+    rfa_status vs = decode_validate(p);
+    if (vs != RFA_OK) return vs;
+    if (!q || !k_cache || !v_cache || !q_pos || !kv_lens || !out) return RFA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+        return RFA_ERR_INVALID_ARG;
+    if (invFreq && !aligned(invFreq, 16)) return RFA_ERR_INVALID_ARG;
+    const DecodePlan pl = decode_plan(p);
+    if (!workspace || ws_bytes < pl.total || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
+    const int D = p->D, half = D / 2;
+    const bool fp16 = p->io_dtype == RFA_DT_FP16;
+    cudaStream_t st = as_stream(stream);
+    char* ws = static_cast<char*>(workspace);
+    // cos/sin rows of every query row (b, h, s), in the layout the attention kernel reads
+    rfa::TableArgs ta;
+    std::memset(&ta, 0, sizeof ta);
+    ta.pos = q_pos;
+    ta.inv_dev = invFreq;
+    ta.table = reinterpret_cast<uint32_t*>(ws);
+    ta.ntokens = static_cast<int32_t>(pl.rq);
+    ta.half = half;
+    ta.nseg = 1;
+    ta.uniform_len = p->Hq * p->Sq;  // row t belongs to sequence t / (Hq * Sq)
+    ta.pos_sq = p->Sq;               // and reads position q_pos[b, t % Sq]
+    if (!invFreq) {
+        ta.inv_host_rows = 1;
+        inv_freq_row(p->rope_base, D, ta.inv_host);
+    }
+    rfa::rope_table_kernel<<<grid_for(pl.rq * (half / 8), 256), 256, 0, st>>>(ta);
+    if (cudaGetLastError() != cudaSuccess) return RFA_ERR_CUDA;
+
+    rfa::AttnArgs aa;
+    std::memset(&aa, 0, sizeof aa);
+    aa.out = out;
+    aa.seeds = nullptr;
+    aa.layout = 1;  // cache rows token-major: [B * Smax, Hkv, D]
+    aa.B = p->B;
+    aa.Hq = p->Hq;
+    aa.Hkv = p->Hkv;
+    aa.G = p->Hq / p->Hkv;
+    aa.causal = p->causal ? 1 : 0;
+    const float scale = p->scale > 0.0f ? p->scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    aa.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    aa.n_items = p->B * p->Hkv * pl.splits;
+    aa.dec_Sq = p->Sq;
+    aa.dec_Smax = p->Smax;
+    aa.dec_splits = pl.splits;
+    aa.dec_chunk = pl.chunk;
+    aa.dec_max_len = p->max_kv_len;
+    aa.kv_lens = kv_lens;
+    aa.part_o = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.tab_bytes) : nullptr;
+    aa.part_ml = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.tab_bytes + pl.po_bytes) : nullptr;
+    const uint64_t esz = 2, rows_cache = static_cast<uint64_t>(p->B) * p->Smax;
+    CUtensorMap mq, mk, mv, mt;
+    bool ok = make_map(&mq, q, fp16, D, 1, static_cast<uint64_t>(pl.rq), D * esz, D * esz, 64, 1, rfa::kBlockM) &&
+              make_map(&mk, k_cache, fp16, D, p->Hkv, rows_cache, D * esz, static_cast<uint64_t>(p->Hkv) * D * esz, 64,
+                       1, rfa::kBlockN) &&
+              make_map(&mv, v_cache, fp16, D, p->Hkv, rows_cache, D * esz, static_cast<uint64_t>(p->Hkv) * D * esz, 64,
+                       1, rfa::kBlockN) &&
+              make_table_map(&mt, ws, static_cast<uint64_t>(pl.rq), D);
+    if (!ok) return RFA_ERR_CUDA;
+    const bool adj = p->rope_interleaved != 0;
+    rfa_status r;
+    if (D == 128) {
+        if (adj)
+            r = fp16 ? launch_attn<128, true, true, true>(mq, mk, mv, mt, aa, st)
+                     : launch_attn<128, false, true, true>(mq, mk, mv, mt, aa, st);
+        else
+            r = fp16 ? launch_attn<128, true, false, true>(mq, mk, mv, mt, aa, st)
+                     : launch_attn<128, false, false, true>(mq, mk, mv, mt, aa, st);
+    } else {
+        if (adj)
+            r = fp16 ? launch_attn<64, true, true, true>(mq, mk, mv, mt, aa, st)
+                     : launch_attn<64, false, true, true>(mq, mk, mv, mt, aa, st);
+        else
+            r = fp16 ? launch_attn<64, true, false, true>(mq, mk, mv, mt, aa, st)
+                     : launch_attn<64, false, false, true>(mq, mk, mv, mt, aa, st);
+    }
+    if (r != RFA_OK || pl.splits == 1) return r;
+    const int grid = grid_for(pl.rq * (D / 8), 256);
+    if (fp16)
+        rfa::decode_combine_kernel<true><<<grid, 256, 0, st>>>(aa.part_o, aa.part_ml, out, static_cast<int32_t>(pl.rq),
+                                                                D, pl.splits);
+    else
+        rfa::decode_combine_kernel<false><<<grid, 256, 0, st>>>(aa.part_o, aa.part_ml, out,
+                                                                 static_cast<int32_t>(pl.rq), D, pl.splits);
+    return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -167,6 +167,7 @@ struct TableArgs {
     int32_t nseg;
     int32_t uniform_len;
     int32_t inv_host_rows;  // 1: one row shared by all segments; else one per segment
+    int32_t pos_sq;         // > 0: row t reads pos[(t / uniform_len) * pos_sq + t % pos_sq] (decode query rows)
     int32_t cum[kMaxSeqs + 1];
     alignas(16) float inv_host[kMaxSeqs * kMaxHalfHost];
 };
@@ -188,7 +189,8 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
         const float* inv = a.inv_dev ? a.inv_dev + static_cast<int64_t>(b) * a.half
                                      : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
         float s[8], co[8];
-        sincos8(static_cast<float>(__ldg(a.pos + t)), inv + 8 * c, s, co);
+        const int32_t pt = a.pos_sq > 0 ? (t / a.uniform_len) * a.pos_sq + t % a.pos_sq : t;
+        sincos8(static_cast<float>(__ldg(a.pos + pt)), inv + 8 * c, s, co);
         uint32_t pr[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {

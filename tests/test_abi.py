@@ -247,3 +247,52 @@ def test_kv_cache_rejects_bad_pointers(lib):
     assert call(FAKE, FAKE, MIS, FAKE, FAKE, FAKE, FAKE, FAKE, 16) == rfa.RFA_ERR_INVALID_ARG      # misaligned
     assert call(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16) == rfa.RFA_ERR_INVALID_ARG     # no slots
     assert call(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 16) == rfa.RFA_ERR_INVALID_ARG     # no v cache
+
+
+def _dp(**kw):
+    p = rfa.DecodeParams(2, 8, 2, 1, 128, 1024, 1024, 1, rfa.DT_BF16, 0, 0.0, 0, 10000.0)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_decode_params_struct_matches_c_layout():
+    assert ctypes.sizeof(rfa.DecodeParams) == 56
+    assert rfa.DecodeParams.rope_base.offset == 48
+
+
+def test_decode_workspace_plans_splits(lib):
+    # 2 x 2 kv groups over 1024 keys (8 tiles): split into single tiles -> 8 splits
+    p = _dp()
+    rq, D = 2 * 8 * 1, 128
+    tab = _ru(rq * D * 2)
+    assert lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)) == tab + _ru(8 * rq * D * 4) + _ru(8 * rq * 2 * 4)
+    # 64 x 8 groups: enough CTAs without splitting, so only the query table
+    p = _dp(B=64, Hq=32, Hkv=8, Sq=1)
+    assert lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)) == _ru(64 * 32 * 128 * 2)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=6, Hkv=4), rfa.RFA_ERR_INVALID_ARG),       # Hq % Hkv
+    (dict(Sq=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(max_kv_len=2048), rfa.RFA_ERR_INVALID_ARG),   # > Smax
+    (dict(Sq=4, max_kv_len=3), rfa.RFA_ERR_INVALID_ARG),
+    (dict(D=96), rfa.RFA_ERR_UNSUPPORTED),
+    (dict(Hq=64, Hkv=1, Sq=4), rfa.RFA_ERR_UNSUPPORTED),  # G * Sq > 128
+    (dict(io_dtype=rfa.DT_UNDEFINED), rfa.RFA_ERR_INVALID_ARG),
+    (dict(rope_interleaved=2), rfa.RFA_ERR_INVALID_ARG),
+    (dict(rope_base=0.0), rfa.RFA_ERR_INVALID_ARG),
+])
+def test_decode_rejects_invalid_params(lib, kw, code):
+    p = _dp(**kw)
+    assert lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)) == 0
+    assert lib.rfa_decode_rope_attention(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30,
+                                         None) == code
+
+
+def test_decode_rejects_null_and_workspace(lib):
+    p = _dp()
+    call = lambda *a: lib.rfa_decode_rope_attention(ctypes.byref(p), *a, None)
+    assert call(FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, 1 << 30) == rfa.RFA_ERR_INVALID_ARG   # no q_pos
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16) == rfa.RFA_ERR_WORKSPACE          # too small
+    assert call(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, 1 << 30) == rfa.RFA_ERR_WORKSPACE     # none
