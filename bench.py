@@ -421,6 +421,37 @@ def kv_cache_bench(rfa, dev):
             "us": t * 1e6, "GB/s": byts / t / 1e9, "timing": f"{n} launches back to back (data > L2)"}
 
 
+def decode_bench(rfa, dev):
+    """decode_rope_attention: 8 sequences x 32 query / 8 kv heads x D 128, one
+    new token each, over 32768 cached tokens (bf16): GB/s of algorithmic bytes
+    (the K and V caches read once, plus q, out and the queries' cos/sin rows),
+    1.07 GB per launch, launches back to back."""
+    B, Hq, Hkv, Sq, D, L = 8, 32, 8, 1, 128, 32768
+    q = workloads.randn16((B, Hq, Sq, D), 41).to(dev)
+    kc = workloads.randn16((B, L, Hkv, D), 42).to(dev)
+    vc = workloads.randn16((B, L, Hkv, D), 43).to(dev)
+    q_pos = torch.full((B, Sq), L - 1, dtype=torch.int32, device=dev)
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    ws = None
+    for _ in range(3):
+        rfa.decode_rope_attention(q, kc, vc, q_pos, lens, out=out)
+    torch.cuda.synchronize()
+    n = 20
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        rfa.decode_rope_attention(q, kc, vc, q_pos, lens, out=out, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    assert rfa.get_device_status() == 0
+    t = e0.elapsed_time(e1) * 1e-3 / n
+    byts = 2 * kc.numel() * 2 + 2 * q.numel() * 2 + B * Hq * Sq * D * 2
+    return {"shape": "B=8, Hq=32, Hkv=8, Sq=1, D=128, 32768 cached tokens, bf16", "bytes": byts, "us": t * 1e6,
+            "GB/s": byts / t / 1e9, "tokens/s": B * Sq / t, "timing": f"{n} launches back to back (data > L2)"}
+
+
 def unfused_context(w, q, k, v, pos, dev, iters=20):
     """Unfused GPU context: rope with torch ops (rotated q/k written to HBM)
     then torch scaled_dot_product_attention."""
@@ -547,6 +578,8 @@ def run_gpu(args, world, rank, local):
         extra["rope_apply"]["frac_hbm"] = extra["rope_apply"]["GB/s"] / peaks["hbm_gbs"]
         extra["kv_rms_norm_rope_cache"] = kv_cache_bench(rfa, dev)
         extra["kv_rms_norm_rope_cache"]["frac_hbm"] = extra["kv_rms_norm_rope_cache"]["GB/s"] / peaks["hbm_gbs"]
+        extra["decode"] = decode_bench(rfa, dev)
+        extra["decode"]["frac_hbm"] = extra["decode"]["GB/s"] / peaks["hbm_gbs"]
         if not args.no_context:
             try:
                 extra["context_unfused"] = unfused_context(w, q, k, v, pos, dev)

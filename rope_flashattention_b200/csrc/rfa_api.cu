@@ -666,14 +666,16 @@ rfa_status decode_validate(const rfa_decode_params* p) {
     return RFA_OK;
 }
 
-// Keys of a sequence are split so that about two CTAs per SM have work
-// (B * Hkv * splits of them); each split is a whole number of key tiles.
+// Keys of a sequence are split so that about four CTAs per SM have work
+// (B * Hkv * splits of them, one resident per SM at a time: measured best
+// against 1, 2, 8 and 16 on an 8-sequence, 32K-key decode); each split is a
+// whole number of key tiles.
 DecodePlan decode_plan(const rfa_decode_params* p) {
     DecodePlan pl;
     pl.rq = static_cast<int64_t>(p->B) * p->Hq * p->Sq;
     const int64_t groups = static_cast<int64_t>(p->B) * p->Hkv;
     const int32_t tiles = (p->max_kv_len + rfa::kBlockN - 1) / rfa::kBlockN;
-    int64_t want = (2 * 148 + groups - 1) / groups;
+    int64_t want = (4 * 148 + groups - 1) / groups;
     const int32_t splits0 = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(want, tiles)));
     const int32_t per = (tiles + splits0 - 1) / splits0;
     pl.chunk = per * rfa::kBlockN;

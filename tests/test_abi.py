@@ -267,9 +267,9 @@ def test_decode_workspace_plans_splits(lib):
     rq, D = 2 * 8 * 1, 128
     tab = _ru(rq * D * 2)
     assert lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)) == tab + _ru(8 * rq * D * 4) + _ru(8 * rq * 2 * 4)
-    # 64 x 8 groups: enough CTAs without splitting, so only the query table
-    p = _dp(B=64, Hq=32, Hkv=8, Sq=1)
-    assert lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)) == _ru(64 * 32 * 128 * 2)
+    # 128 x 8 groups: enough CTAs without splitting, so only the query table
+    p = _dp(B=128, Hq=32, Hkv=8, Sq=1)
+    assert lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)) == _ru(128 * 32 * 128 * 2)
 
 
 @pytest.mark.parametrize("kw,code", [
