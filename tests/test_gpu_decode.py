@@ -59,9 +59,9 @@ def test_gqa_single_token_split_keys(rfa):
 
 
 def test_many_groups_one_split(rfa):
-    # 40 x 8 kv groups fill the GPU without splitting the keys
-    lens = [int(x) for x in np.random.default_rng(2).integers(1, 700, 40)]
-    got, ref, st = _case(rfa, 40, 16, 8, 1, 128, 700, lens, seed=3)
+    # 80 x 8 kv groups fill the GPU without splitting the keys
+    lens = [int(x) for x in np.random.default_rng(2).integers(1, 700, 80)]
+    got, ref, st = _case(rfa, 80, 16, 8, 1, 128, 700, lens, seed=3)
     assert st == 0
     _compare(got, ref)
 
