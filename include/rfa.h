@@ -326,6 +326,15 @@ RFA_API rfa_status rfa_fused_rope_attention_noalloc(const rfa_attn_params* p, co
  * synchronisation itself failed. */
 RFA_API rfa_status rfa_get_device_status(void* stream);
 
+/* Sets, on the current device, how long a kernel role waits for another
+ * (an mbarrier phase) before giving up: on expiry the kernel records
+ * RFA_ERR_TIMEOUT, its roles stop, its in-flight copies and MMAs are drained
+ * (those drains keep their own 2 s limit) and it returns.  0 restores the
+ * default of 2 s.  Meant for failure-detection tests, which lower it so that
+ * waits run out on purpose; synchronous; must not overlap running kernels of
+ * this library.  RFA_ERR_CUDA if the device variable cannot be written. */
+RFA_API rfa_status rfa_set_wait_limit_ns(uint64_t ns);
+
 /* Static, human-readable name of a status code. */
 RFA_API const char* rfa_status_string(rfa_status s);
 

@@ -30,7 +30,7 @@ __all__ = [
     "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
     "fused_rope_attention_noalloc", "rope_apply", "kv_rms_norm_rope_cache", "KvCacheParams",
     "decode_rope_attention", "DecodeParams",
-    "get_device_status", "status_string", "AttnParams", "RopeApplyParams",
+    "get_device_status", "set_wait_limit_ns", "status_string", "AttnParams", "RopeApplyParams",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa.so")
@@ -48,6 +48,7 @@ EXPORTS = (
     "rfa_fused_rope_attention_with_table",
     "rfa_fused_rope_attention_noalloc",
     "rfa_get_device_status",
+    "rfa_set_wait_limit_ns",
     "rfa_status_string",
     "rfa_version",
 )
@@ -164,6 +165,8 @@ def load_library():
     lib.rfa_decode_rope_attention_workspace.restype = SZ
     lib.rfa_decode_rope_attention.argtypes = [ctypes.POINTER(DecodeParams), P, P, P, P, P, P, P, P, SZ, P]
     lib.rfa_decode_rope_attention.restype = ctypes.c_int
+    lib.rfa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.rfa_set_wait_limit_ns.restype = ctypes.c_int
     lib.rfa_get_device_status.argtypes = [P]
     lib.rfa_get_device_status.restype = ctypes.c_int
     lib.rfa_status_string.argtypes = [ctypes.c_int]
@@ -172,6 +175,12 @@ def load_library():
     lib.rfa_version.restype = I32
     _lib = lib
     return lib
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Kernel role-to-role wait limit on the current device (0: default 2 s);
+    for failure-detection tests (rfa_set_wait_limit_ns)."""
+    _check(load_library().rfa_set_wait_limit_ns(int(ns)), "rfa_set_wait_limit_ns")
 
 
 def status_string(code: int) -> str:

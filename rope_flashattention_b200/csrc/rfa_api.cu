@@ -187,6 +187,12 @@ rfa_status rfa_get_device_status(void* stream) {
     return static_cast<rfa_status>(v);
 }
 
+rfa_status rfa_set_wait_limit_ns(uint64_t ns) {
+    const uint64_t v = ns == 0 ? rfa::kWaitLimitNs : ns;
+    if (cudaDeviceSynchronize() != cudaSuccess) return RFA_ERR_CUDA;
+    return cudaMemcpyToSymbol(rfa::g_wait_limit_ns, &v, sizeof v) == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+}
+
 rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, const int32_t* seqLens, int32_t batch,
                            int32_t ntokens, int32_t headSize, rfa_dtype outType, void* sinOut, void* cosOut,
                            void* stream) {

@@ -51,6 +51,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wall-clock limit of one wait.  Legitimate waits last microseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Limit of the role-to-role waits below (the drains before a CTA exits keep
+// kWaitLimitNs).  Host code may lower it through rfa_set_wait_limit_ns to make
+// waits run out on purpose (failure-detection tests).
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 // Bounded wait for the phase of `bar` with parity `parity` to complete.
 // Returns false (and raises *abort) if the wait timed out or another role of
@@ -58,12 +62,13 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // spin loop is one shared out-of-line copy, so warps waiting at different
 // places do not each keep their own copy of it in the instruction cache.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int32_t* abort) {
-    uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = *static_cast<volatile uint64_t*>(&g_wait_limit_ns);
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u) {
+        if ((it & 255u) == 1u) {  // after the first failed poll, then every 256
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit) {
                 *abort = 1;
                 record_status(5 /* RFA_ERR_TIMEOUT */);
                 return false;
