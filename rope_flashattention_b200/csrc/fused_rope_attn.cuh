@@ -158,9 +158,7 @@ struct WorkItem {
     int32_t qt[2];  // query tile indices within the sequence; qt[1] < 0: no second tile
 };
 
-// Head-major order (the items of one head / head pair are neighbours, so the
-// CTAs resident at one time share K/V tiles through L2), largest tiles first;
-// packed sequences longest first.
+// Decode: item x = (sequence, kv head, split), splits of one kv group adjacent.
 __device__ __forceinline__ WorkItem decode_item_kv(const AttnArgs& a, int32_t x) {
     WorkItem w;
     w.split = x % a.dec_splits;
@@ -179,6 +177,13 @@ __device__ __forceinline__ WorkItem decode_item_kv(const AttnArgs& a, int32_t x)
     return w;
 }
 
+// BNSD: heads (head pairs when G is even) are taken in groups of
+// kOrderGroup; within a group, items run longest first across its heads (a
+// list schedule near its lower bound on causal masks, where items range from
+// 1 to S/128 key tiles), and a group's K/V stays in L2 while its items run.
+// Packed sequences: longest sequence first, head-major within a sequence
+// (its items share K/V tiles through L2), largest tiles first.
+constexpr int kOrderGroup = 16;
 __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     WorkItem w;
     w.qrow0 = 0;
@@ -187,12 +192,20 @@ __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     const bool ph = a.pair_heads != 0;
     if (a.layout == 0) {
         nt = (a.S + kBlockM - 1) / kBlockM;
-        const int32_t per = items_per_sequence(a.Hq, nt, ph);
-        w.seq = x / per;
-        r = x - w.seq * per;
+        const int32_t per_unit = ph ? nt : (nt + 1) / 2;  // items of one head (pair)
+        const int32_t units_seq = ph ? a.Hq / 2 : a.Hq;   // head (pair) units per sequence
+        const int32_t units = a.B * units_seq;
+        const int32_t g = x / (kOrderGroup * per_unit);
+        const int32_t rg = x - g * kOrderGroup * per_unit;
+        const int32_t ng = min(kOrderGroup, units - g * kOrderGroup);  // units in this group
+        const int32_t rank = rg / ng;                                 // 0: each unit's longest item
+        const int32_t u = g * kOrderGroup + (rg - rank * ng);
+        w.seq = u / units_seq;
         w.orig = w.seq;
         w.tok0 = w.seq * a.S;
         w.L = a.S;
+        // unit u's rank-th item in the per-sequence numbering below (longest first)
+        r = (u - w.seq * units_seq) * per_unit + rank;
     } else {
         int32_t s = 0;
         while (s + 1 < a.nseg && x >= a.seg_item0[s + 1]) ++s;
