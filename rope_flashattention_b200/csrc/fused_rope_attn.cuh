@@ -181,8 +181,8 @@ __device__ __forceinline__ WorkItem decode_item_kv(const AttnArgs& a, int32_t x)
 // kOrderGroup; within a group, items run longest first across its heads (a
 // list schedule near its lower bound on causal masks, where items range from
 // 1 to S/128 key tiles), and a group's K/V stays in L2 while its items run.
-// Packed sequences: longest sequence first, head-major within a sequence
-// (its items share K/V tiles through L2), largest tiles first.
+// Packed sequences: longest sequence first, the same grouped longest-first
+// order over the heads within a sequence.
 constexpr int kOrderGroup = 16;
 __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     WorkItem w;
@@ -209,12 +209,20 @@ __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     } else {
         int32_t s = 0;
         while (s + 1 < a.nseg && x >= a.seg_item0[s + 1]) ++s;
-        r = x - a.seg_item0[s];
+        const int32_t rs = x - a.seg_item0[s];
         nt = a.seg_tiles[s];
         w.seq = s;
         w.orig = a.seg_orig[s];
         w.tok0 = a.seg_start[s];
         w.L = a.seg_len[s];
+        // within the sequence, the same grouped longest-first order over its heads
+        const int32_t per_unit = ph ? nt : (nt + 1) / 2;
+        const int32_t units = ph ? a.Hq / 2 : a.Hq;
+        const int32_t g = rs / (kOrderGroup * per_unit);
+        const int32_t rg = rs - g * kOrderGroup * per_unit;
+        const int32_t ng = min(kOrderGroup, units - g * kOrderGroup);
+        const int32_t rank = rg / ng;
+        r = (g * kOrderGroup + (rg - rank * ng)) * per_unit + rank;
     }
     if (ph) {
         const int32_t hp = r / nt;
