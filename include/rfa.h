@@ -179,7 +179,9 @@ typedef struct {
     int32_t io_dtype;         /* RFA_DT_BF16 | RFA_DT_FP16: q, caches and out */
     int32_t rope_interleaved; /* 0: rotate-half pairs; 1: adjacent pairs (as the cache was written) */
     float scale;              /* softmax scale; 0 -> 1/sqrt(D) */
-    int32_t pad_;             /* unused, keep 0 */
+    int32_t num_splits;       /* parts each sequence's keys are split into across CTAs (whole
+                                 128-key tiles; clamped to the tiles of max_kv_len);
+                                 0 -> the library's plan; < 0 -> RFA_ERR_INVALID_ARG */
     double rope_base;         /* invFreq_j = base^(-2j/D) when invFreq is NULL */
 } rfa_decode_params;
 

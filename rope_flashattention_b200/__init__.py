@@ -128,7 +128,7 @@ class DecodeParams(ctypes.Structure):
         ("io_dtype", ctypes.c_int32),
         ("rope_interleaved", ctypes.c_int32),
         ("scale", ctypes.c_float),
-        ("pad_", ctypes.c_int32),
+        ("num_splits", ctypes.c_int32),
         ("rope_base", ctypes.c_double),
     ]
 
@@ -379,14 +379,15 @@ def decode_rope_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
                           kv_lens: torch.Tensor, *, max_kv_len: Optional[int] = None, causal: bool = True,
                           scale: Optional[float] = None, rope_base: float = 10000.0,
                           inv_freq: Optional[torch.Tensor] = None, interleaved: bool = False,
-                          out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                          stream=None) -> torch.Tensor:
+                          num_splits: int = 0, out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """A decode step over a KV cache (rfa_decode_rope_attention).
 
     q [B, Hq, Sq, D] new tokens (rotated in the kernel at q_pos [B, Sq]);
     k_cache / v_cache [B, Smax, Hkv, D] with keys already rotated; kv_lens
     int32 [B] on the GPU (each in [Sq, max_kv_len]; max_kv_len defaults to
-    Smax).  Returns out [B, Hq, Sq, D].
+    Smax).  num_splits: parts each sequence's keys are split into across CTAs
+    (0: the library's plan).  Returns out [B, Hq, Sq, D].
     """
     if q.dim() != 4 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
         raise ValueError("q [B, Hq, Sq, D]; caches [B, Smax, Hkv, D]")
@@ -394,7 +395,7 @@ def decode_rope_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
     Smax, Hkv = int(k_cache.shape[1]), int(k_cache.shape[2])
     p = DecodeParams(B, Hq, Hkv, Sq, D, Smax, int(max_kv_len if max_kv_len is not None else Smax), 1 if causal else 0,
                      _TORCH_DT.get(q.dtype, DT_UNDEFINED), 1 if interleaved else 0,
-                     0.0 if scale is None else float(scale), 0, float(rope_base))
+                     0.0 if scale is None else float(scale), int(num_splits), float(rope_base))
     lib = load_library()
     need = int(lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)))
     if need == 0:

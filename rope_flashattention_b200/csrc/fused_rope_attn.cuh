@@ -493,6 +493,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmT,
                                const __grid_constant__ AttnArgs a) {
     using C = AttnCfg<D>;
+    static_assert(C::kTabBytes <= C::kTileBytes, "decode stages the queries' cos/sin rows in a query slot");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     if ((sbase & 1023u) != 0u) {  // 128B-swizzled TMA/UMMA tiles need 1024-byte alignment
@@ -509,10 +510,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const WorkItem w = kDecode ? decode_item_kv(a, blockIdx.x) : decode_item(a, blockIdx.x);
     const int32_t nq = (w.qt[1] >= 0) ? 2 : 1;  // query tiles in this item
     const int32_t nkt = (w.L + kBlockN - 1) / kBlockN;
-    // key tiles read by query tile i (0: tile absent)
-    const int32_t n0 = (a.causal && !kDecode) ? (w.qt[0] + 1) : nkt;
-    const int32_t n1 = (nq == 1) ? 0 : (a.causal ? (w.qt[1] + 1) : nkt);
-    const int32_t n_kv = max(n0, n1);
+    // key tiles read by query tile i (0: tile absent).  Decode has one query tile and two
+    // independent chains over alternate key tiles: tile j goes to S/O buffer j % 2, and the
+    // two buffers' results are merged before the store.
+    const int32_t n0 = kDecode ? (nkt + 1) / 2 : (a.causal ? (w.qt[0] + 1) : nkt);
+    const int32_t n1 = kDecode ? nkt / 2 : ((nq == 1) ? 0 : (a.causal ? (w.qt[1] + 1) : nkt));
+    const int32_t n_kv = kDecode ? nkt : max(n0, n1);
     // consecutive positions: K angles come from the recurrence, no cos/sin rows per K tile
     // (decode: the cached keys are already rotated)
     const bool rec = !kDecode && a.seeds[w.orig].consecutive != 0;
@@ -588,7 +591,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int bx = 0; bx < C::kTabBoxes; ++bx)
                     tma_load_3d(dst + bx * C::kAtomBytes, &tmT, b, bx * 32, w.tok0 + row0, 0);
             };
-            // query tiles and their cos/sin rows (staged in V slots 0 and 1 until QReady)
+            // query tiles and their cos/sin rows (staged in V slots 0 and 1 until QReady; decode:
+            // in the second query tile's slot, which it does not otherwise use, so V loads need not
+            // wait)
             mbar_expect_tx(bar(C::kBarQFull), static_cast<uint32_t>(nq) * (C::kTileBytes + C::kTabBytes));
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
@@ -597,7 +602,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int at = 0; at < C::kAtoms; ++at)
                         tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64, 0, w.qrow0);
                     for (int bx = 0; bx < C::kTabBoxes; ++bx)
-                        tma_load_3d(sbase + C::kOffV + bx * C::kAtomBytes, &tmT, bar(C::kBarQFull), bx * 32, w.qrow0, 0);
+                        tma_load_3d(sbase + C::kOffQ + C::kTileBytes + bx * C::kAtomBytes, &tmT, bar(C::kBarQFull),
+                                    bx * 32, w.qrow0, 0);
                 } else {
                     const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
                     load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane, w.qt[i] * kBlockM);
@@ -635,8 +641,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const bool bnsd = (a.layout == 0);
             const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
             int32_t issued_v = 0;
-            // V slots 0 and 1 hold the query tiles' cos/sin rows until both are rotated
-            if (mbar_wait(bar(C::kBarQReady), 0, abort_flag)) {
+            // V slots 0 and 1 hold the query tiles' cos/sin rows until both are rotated (not in decode)
+            if (kDecode || mbar_wait(bar(C::kBarQReady), 0, abort_flag)) {
                 for (int32_t j = 0; j < n_kv; ++j) {
                     const int s = j % C::kStages;
                     const uint32_t u = static_cast<uint32_t>(j / C::kStages);
@@ -668,7 +674,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // >> 4 to the start-address field (shared addresses < 256 KB: no carry out of it).
             auto issue_qk = [&](int i, int32_t j) {
                 const uint64_t kd = smem_desc_sw128(sbase + C::kOffK + (j % C::kStages) * C::kTileBytes, 16, 1024);
-                const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + i * C::kTileBytes, 16, 1024);
+                const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + (kDecode ? 0 : i) * C::kTileBytes, 16, 1024);
                 const uint32_t dS = tmem + C::kColS + i * kBlockN;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
@@ -679,51 +685,88 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             };
             // O_i += P_i V_j (A = P_i from TMEM buffer i: keys [64h, 64h + 64) at columns [64h, 64h + 32);
             // B = V_j from shared memory)
-            auto issue_pv = [&](int i, int32_t j) {
+            // (acc: O_i already holds a partial sum)
+            auto issue_pv = [&](int i, int32_t j, bool acc) {
                 const uint64_t vd = smem_desc_sw128(sbase + C::kOffV + (j % C::kStages) * C::kTileBytes, C::kAtomBytes, 1024);
                 const uint32_t dO = tmem + C::kColO + i * D, aP = tmem + C::kColS + i * kBlockN;
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k)
                     umma_ts(dO, aP + (k >> 2) * 64 + (k & 3) * 8, vd + ((k * 16 * 128) >> 4), kIdescPV,
-                            (j > 0 || k > 0) ? 1u : 0u);
+                            (acc || k > 0) ? 1u : 0u);
             };
-            bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag) && mbar_wait(bar(C::kBarKReady), 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                if (n0 > 0) issue_qk(0, 0);
-                if (n1 > 0) issue_qk(1, 0);
-                tc_commit(bar(C::kBarKEmpty));
-            }
-            for (int32_t j = 0; j < n_kv && ok; ++j) {
-                const int s = j % C::kStages;
-                const int32_t jn = j + 1;
-                ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag);
-                if (!ok) break;
-                if (j < n0) {
-                    ok = mbar_wait(bar(C::kBarPFull + 0), static_cast<uint32_t>(j) & 1u, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(0, j);
-                    if (j == n0 - 1) tc_commit(bar(C::kBarOFull + 0));
-                }
-                if (jn < n_kv) {
-                    ok = mbar_wait(bar(C::kBarKReady + jn % C::kStages), static_cast<uint32_t>(jn / C::kStages) & 1u,
+            if constexpr (kDecode) {
+                // Two chains over alternate key tiles (tile j into buffer j % 2, its t = j / 2-th
+                // tile).  QK_i of tile j + 2 reuses S_i: it is issued after PV_i of tile j, which
+                // read P_i, and MMAs from this thread execute in order.
+                bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag);
+                for (int32_t j = 0; j < 2 && j < n_kv && ok; ++j) {
+                    ok = mbar_wait(bar(C::kBarKReady + j % C::kStages), static_cast<uint32_t>(j / C::kStages) & 1u,
                                    abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    if (jn < n0) issue_qk(0, jn);
+                    issue_qk(j, j);
+                    tc_commit(bar(C::kBarKEmpty + j % C::kStages));
                 }
-                if (j < n1) {
-                    ok = mbar_wait(bar(C::kBarPFull + 1), static_cast<uint32_t>(j) & 1u, abort_flag);
+                for (int32_t j = 0; j < n_kv && ok; ++j) {
+                    const int s = j % C::kStages;
+                    const int i = j & 1;
+                    const int32_t t = j >> 1;
+                    ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag) &&
+                         mbar_wait(bar(C::kBarPFull + i), static_cast<uint32_t>(t) & 1u, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(1, j);
-                    if (j == n1 - 1) tc_commit(bar(C::kBarOFull + 1));
+                    issue_pv(i, j, t > 0);
+                    if (j + 2 >= n_kv) tc_commit(bar(C::kBarOFull + i));  // last tile of buffer i
+                    tc_commit(bar(C::kBarVEmpty + s));
+                    const int32_t jn = j + 2;
+                    if (jn < n_kv) {
+                        ok = mbar_wait(bar(C::kBarKReady + jn % C::kStages), static_cast<uint32_t>(jn / C::kStages) & 1u,
+                                       abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_qk(i, jn);
+                        tc_commit(bar(C::kBarKEmpty + jn % C::kStages));
+                    }
                 }
-                tc_commit(bar(C::kBarVEmpty + s));
-                if (jn < n_kv) {
-                    if (jn < n1) issue_qk(1, jn);
-                    tc_commit(bar(C::kBarKEmpty + jn % C::kStages));
+            } else {
+                bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag) && mbar_wait(bar(C::kBarKReady), 0, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    if (n0 > 0) issue_qk(0, 0);
+                    if (n1 > 0) issue_qk(1, 0);
+                    tc_commit(bar(C::kBarKEmpty));
+                }
+                for (int32_t j = 0; j < n_kv && ok; ++j) {
+                    const int s = j % C::kStages;
+                    const int32_t jn = j + 1;
+                    ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag);
+                    if (!ok) break;
+                    if (j < n0) {
+                        ok = mbar_wait(bar(C::kBarPFull + 0), static_cast<uint32_t>(j) & 1u, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(0, j, j > 0);
+                        if (j == n0 - 1) tc_commit(bar(C::kBarOFull + 0));
+                    }
+                    if (jn < n_kv) {
+                        ok = mbar_wait(bar(C::kBarKReady + jn % C::kStages), static_cast<uint32_t>(jn / C::kStages) & 1u,
+                                       abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (jn < n0) issue_qk(0, jn);
+                    }
+                    if (j < n1) {
+                        ok = mbar_wait(bar(C::kBarPFull + 1), static_cast<uint32_t>(j) & 1u, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(1, j, j > 0);
+                        if (j == n1 - 1) tc_commit(bar(C::kBarOFull + 1));
+                    }
+                    tc_commit(bar(C::kBarVEmpty + s));
+                    if (jn < n_kv) {
+                        if (jn < n1) issue_qk(1, jn);
+                        tc_commit(bar(C::kBarKEmpty + jn % C::kStages));
+                    }
                 }
             }
             tc_commit(bar(C::kBarMmaFin));
@@ -760,8 +803,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
             for (int i = 0; i < nq; ++i) {
                 const int32_t q0 = (i == 0 ? w.qt[0] : w.qt[1]) * kBlockM;
-                rope_tile<D, kFP16, kAdj>(sbase + C::kOffQ + i * C::kTileBytes, sbase + C::kOffV + i * C::kTileBytes,
-                                          kDecode ? kBlockM : min(kBlockM, w.L - q0), rt);
+                // decode: only the group's G * Sq rows of the tile are queries of this item
+                rope_tile<D, kFP16, kAdj>(sbase + C::kOffQ + i * C::kTileBytes,
+                                          sbase + (kDecode ? C::kOffQ + C::kTileBytes : C::kOffV + i * C::kTileBytes),
+                                          kDecode ? a.G * a.dec_Sq : min(kBlockM, w.L - q0), rt);
             }
             fence_proxy_async_smem();  // Q' written by the generic proxy, read by the tensor cores
             __syncwarp();
@@ -825,7 +870,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool ok = true;       // warp-uniform; tcgen05.ld/st are warp-collective
         for (int32_t j = 0; j < n_i; ++j) {
             ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + i), static_cast<uint32_t>(j) & 1u, abort_flag));
-            const int32_t lim = vis - j * kBlockN - hf * 64;  // columns [0, lim) of this half are visible
+            const int32_t kt = kDecode ? 2 * j + i : j;          // key tile of this step
+            const int32_t lim = vis - kt * kBlockN - hf * 64;  // columns [0, lim) of this half are visible
             float mxh = -INFINITY;
             if (ok) {
                 tc_fence_after();
@@ -906,61 +952,115 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         xch[hf * kBlockM + row] = l;
         named_bar_sync(nb, 256);
         l += xch[(hf ^ 1) * kBlockM + row];
-        const bool fin = n_i > 0 && __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
-                         __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), 0, abort_flag));
-        if (fin) {
-            tc_fence_after();
-            const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
-            const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-            bool valid = qi < w.L;
-            uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
-            int64_t o_off;
-            if (a.layout == 0)
-                o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
-            else
-                o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
-            bool partial = false;
-            if constexpr (kDecode) {
-                // output rows of q viewed as [B*Hq*Sq, D]; with several splits, unnormalised
-                // fp32 O and (m, l) go to the partials that the combine kernel merges
-                valid = row < a.G * a.dec_Sq;
-                o_off = static_cast<int64_t>(w.qrow0 + row) * D;
-                partial = a.dec_splits > 1;
+        if constexpr (kDecode) {
+            // The two buffers hold alternate key tiles of this split.  With M = max(m_0, m_1) and
+            // c_b = 2^(m_b - M) (0 where l_b = 0): O = c_0 O_0 + c_1 O_1, l = c_0 l_0 + c_1 l_1.
+            // Warp (i, hf) merges column quarter 2 i + hf of its lane group's rows.  (m, l) pass
+            // through the K-tile cos/sin slot, which decode uses for nothing else: a buffer with
+            // no tiles reaches this point while the query tile may still be in flight.
+            float* mlx = reinterpret_cast<float*>(smem + C::kOffT);  // [m_0, m_1, l_0, l_1][row]
+            if (hf == 0) {
+                mlx[i * kBlockM + row] = m;
+                mlx[(2 + i) * kBlockM + row] = l;
+            }
+            named_bar_sync(3, kSoftmaxWarps * 32);
+            const float m0 = mlx[row], m1 = mlx[kBlockM + row];
+            const float l0 = mlx[2 * kBlockM + row], l1 = mlx[3 * kBlockM + row];
+            const bool fin = __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
+                             __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + 0), 0, abort_flag)) &&
+                             (n1 == 0 || __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + 1), 0, abort_flag)));
+            if (fin) {
+                tc_fence_after();
+                const float M = fmaxf(m0, m1);
+                const float c0 = (l0 > 0.0f) ? ex2(m0 - M) : 0.0f;
+                const float c1 = (l1 > 0.0f) ? ex2(m1 - M) : 0.0f;
+                const float lt = c0 * l0 + c1 * l1;
+                // rows of q viewed as [B*Hq*Sq, D]; with several splits, unnormalised fp32 O and
+                // (m, l) go to the partials that the combine kernel merges
+                const bool valid = row < a.G * a.dec_Sq;
+                const bool partial = a.dec_splits > 1;
+                int64_t o_off = static_cast<int64_t>(w.qrow0 + row) * D;
                 if (partial) {
                     const int64_t pr = static_cast<int64_t>(w.split) * (a.B * a.Hq * a.dec_Sq) + w.qrow0 + row;
                     o_off = pr * D;
-                    if (valid && hf == 0) {
-                        a.part_ml[2 * pr] = (l > 0.0f) ? m : -INFINITY;
-                        a.part_ml[2 * pr + 1] = l;
+                    if (valid && i == 0 && hf == 0) {
+                        a.part_ml[2 * pr] = (lt > 0.0f) ? M : -INFINITY;
+                        a.part_ml[2 * pr + 1] = lt;
+                    }
+                }
+                const float sc = partial ? 1.0f : ((lt > 0.0f) ? 1.0f / lt : 0.0f);
+                const float w0 = c0 * sc, w1 = c1 * sc;
+                constexpr int kOQ = D / 4;  // columns per warp
+                const int c_lo = (2 * i + hf) * kOQ;
+                const uint32_t o0c = tmem + lane_off + C::kColO + c_lo;  // O_1 is D columns further
+#pragma unroll 1
+                for (int q = 0; q < kOQ / 16; ++q) {
+                    uint32_t o0[16], o1[16];
+                    tmem_ld16(o0c + q * 16, o0);
+                    if (n1 > 0) {
+                        tmem_ld16(o0c + D + q * 16, o1);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o1[e] = 0u;
+                    }
+                    tmem_wait_ld();
+                    float v[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)  // a buffer with l = 0 contributes nothing (its O may be unset)
+                        v[e] = (c0 > 0.0f ? w0 * __uint_as_float(o0[e]) : 0.0f) +
+                               (c1 > 0.0f ? w1 * __uint_as_float(o1[e]) : 0.0f);
+                    if (!valid) continue;
+                    if (partial) {
+                        float4* dst = reinterpret_cast<float4*>(a.part_o + o_off + c_lo + q * 16);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_float4(v[4 * v4], v[4 * v4 + 1], v[4 * v4 + 2], v[4 * v4 + 3]);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + o_off + c_lo + q * 16);
+#pragma unroll
+                        for (int v4 = 0; v4 < 2; ++v4) {
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                wv[e] = pack2<kFP16>(f2pack(v[8 * v4 + 2 * e], v[8 * v4 + 2 * e + 1]));
+                            dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        }
                     }
                 }
             }
-            o_off += hf * kOHalf;
-            const uint64_t il2 = f2pack(inv_l, inv_l);
+        } else {
+            const bool fin = n_i > 0 && __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
+                             __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), 0, abort_flag));
+            if (fin) {
+                tc_fence_after();
+                const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
+                const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+                const bool valid = qi < w.L;
+                uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
+                int64_t o_off;
+                if (a.layout == 0)
+                    o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
+                else
+                    o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
+                o_off += hf * kOHalf;
+                const uint64_t il2 = f2pack(inv_l, inv_l);
 #pragma unroll 1
-            for (int q = 0; q < kOHalf / 32; ++q) {
-                uint32_t o[32];
-                tmem_ld32(oc + q * 32, o);
-                tmem_wait_ld();
-                if (kDecode && partial) {
+                for (int q = 0; q < kOHalf / 32; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(oc + q * 32, o);
+                    tmem_wait_ld();
                     if (valid) {
-                        float4* dst = reinterpret_cast<float4*>(a.part_o + o_off + q * 32);
+                        uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);
 #pragma unroll
-                        for (int v4 = 0; v4 < 8; ++v4)
-                            dst[v4] = make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
-                                                  __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
-                    }
-                } else if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            uint32_t wv[4];
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        uint32_t wv[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = 8 * v4 + 2 * e;
-                            wv[e] = pack2<kFP16>(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), il2));
+                            for (int e = 0; e < 4; ++e) {
+                                const int c = 8 * v4 + 2 * e;
+                                wv[e] = pack2<kFP16>(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), il2));
+                            }
+                            dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                         }
-                        dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                     }
                 }
             }

@@ -664,6 +664,7 @@ rfa_status decode_validate(const rfa_decode_params* p) {
     if (p->rope_interleaved != 0 && p->rope_interleaved != 1) return RFA_ERR_INVALID_ARG;
     if (!(p->scale >= 0.0f) || !std::isfinite(p->scale)) return RFA_ERR_INVALID_ARG;
     if (!(p->rope_base > 0.0) || !std::isfinite(p->rope_base)) return RFA_ERR_INVALID_ARG;
+    if (p->num_splits < 0) return RFA_ERR_INVALID_ARG;
     if ((p->D & 1) != 0 || p->D < 1) return RFA_ERR_INVALID_ARG;
     if (p->D != 64 && p->D != 128) return RFA_ERR_UNSUPPORTED;
     if ((p->Hq / p->Hkv) * p->Sq > rfa::kBlockM) return RFA_ERR_UNSUPPORTED;  // one query tile per kv group
@@ -672,18 +673,40 @@ rfa_status decode_validate(const rfa_decode_params* p) {
     return RFA_OK;
 }
 
-// Keys of a sequence are split so that about four CTAs per SM have work
-// (B * Hkv * splits of them, one resident per SM at a time: measured best
-// against 1, 2, 8 and 16 on an 8-sequence, 32K-key decode); each split is a
-// whole number of key tiles.
+// Keys of a sequence are split into whole key tiles across CTAs; one CTA is
+// resident per SM, so B * Hkv * splits CTAs run in ceil(that / 148) waves of
+// about tiles / splits key tiles each.  The plan takes the split count with the
+// least waves x (tiles per split + kSplitCost), kSplitCost being the fixed cost
+// of a CTA (setup, query load and rotation, pipeline fill and drain, merge and
+// store) in key tiles; ties go to fewer splits.  kSplitCost = 6 fits timings of
+// 1 to 64 sequences over 4K-32K cached keys (32 query / 8 kv heads, D 128):
+// e.g. 8 sequences x 32K keys run fastest as 2 splits, one wave of 128 CTAs
+// that already saturates HBM.
+constexpr int64_t kSplitCost = 6;
+constexpr int64_t kNumSMs = 148;
 DecodePlan decode_plan(const rfa_decode_params* p) {
     DecodePlan pl;
     pl.rq = static_cast<int64_t>(p->B) * p->Hq * p->Sq;
     const int64_t groups = static_cast<int64_t>(p->B) * p->Hkv;
     const int32_t tiles = (p->max_kv_len + rfa::kBlockN - 1) / rfa::kBlockN;
-    int64_t want = (4 * 148 + groups - 1) / groups;
-    const int32_t splits0 = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(want, tiles)));
-    const int32_t per = (tiles + splits0 - 1) / splits0;
+    int32_t per = tiles;
+    if (p->num_splits > 0) {
+        per = (tiles + std::min(p->num_splits, tiles) - 1) / std::min(p->num_splits, tiles);
+    } else {
+        // beyond about 8 waves more splits only add CTA costs
+        const int64_t s_max = std::min<int64_t>(tiles, std::max<int64_t>(1, (8 * kNumSMs + groups - 1) / groups));
+        int64_t best = -1;
+        for (int32_t s = 1; s <= s_max; ++s) {
+            const int32_t ps = (tiles + s - 1) / s;
+            if (s > 1 && ps == (tiles + s - 2) / (s - 1)) continue;  // same split as s - 1
+            const int64_t n = (tiles + ps - 1) / ps;
+            const int64_t cost = ((groups * n + kNumSMs - 1) / kNumSMs) * (ps + kSplitCost);
+            if (best < 0 || cost < best) {
+                best = cost;
+                per = ps;
+            }
+        }
+    }
     pl.chunk = per * rfa::kBlockN;
     pl.splits = (p->max_kv_len + pl.chunk - 1) / pl.chunk;
     pl.tab_bytes = round_up(static_cast<size_t>(pl.rq) * p->D * 2, 256);

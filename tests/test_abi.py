@@ -258,6 +258,7 @@ def _dp(**kw):
 
 def test_decode_params_struct_matches_c_layout():
     assert ctypes.sizeof(rfa.DecodeParams) == 56
+    assert rfa.DecodeParams.num_splits.offset == 44
     assert rfa.DecodeParams.rope_base.offset == 48
 
 
@@ -272,6 +273,38 @@ def test_decode_workspace_plans_splits(lib):
     assert lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)) == _ru(128 * 32 * 128 * 2)
 
 
+def _decode_ws(lib, splits, **kw):
+    p = _dp(**kw)
+    rq = p.B * p.Hq * p.Sq
+    tab = _ru(rq * p.D * 2)
+    want = tab + (_ru(splits * rq * p.D * 4) + _ru(splits * rq * 2 * 4) if splits > 1 else 0)
+    return lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)), want
+
+
+def test_decode_plan_weighs_waves_against_cta_cost(lib):
+    # Cost of a plan: waves x (tiles per split + 6), one CTA per SM on 148 SMs.
+    # 8 x 8 kv groups over 32768 keys (256 tiles): 2 splits of 128 tiles, one wave of
+    # 128 CTAs (cost 134), beat 4 of 64 (2 waves, 140), 9 of 29 (4 waves, 140) and 3 of
+    # 86 (192 CTAs: 2 waves, 184)
+    got, want = _decode_ws(lib, 2, B=8, Hq=32, Hkv=8, Sq=1, Smax=32768, max_kv_len=32768)
+    assert got == want
+    # one sequence, 8 kv groups over 256 tiles: 18 splits of 15 tiles fill one wave
+    # (144 CTAs, cost 21); 37 of 7 take two (26), 9 of 29 one (35)
+    got, want = _decode_ws(lib, 18, B=1, Hq=32, Hkv=8, Sq=1, Smax=32768, max_kv_len=32768)
+    assert got == want
+    # 32 x 8 groups over 4096 keys (32 tiles): no split (2 waves, 76) against 2 (4 waves, 88)
+    got, want = _decode_ws(lib, 1, B=32, Hq=32, Hkv=8, Sq=1, Smax=4096, max_kv_len=4096)
+    assert got == want
+
+
+@pytest.mark.parametrize("n,splits", [(1, 1), (3, 3), (7, 4), (100, 8)])
+def test_decode_num_splits_is_taken_as_given(lib, n, splits):
+    # 1024 keys = 8 tiles, split into parts of ceil(8 / n) whole tiles: 7 asked -> parts of
+    # 2 tiles -> 4 splits; more parts than tiles -> one tile each
+    got, want = _decode_ws(lib, splits, num_splits=n)
+    assert got == want
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(Hq=6, Hkv=4), rfa.RFA_ERR_INVALID_ARG),       # Hq % Hkv
     (dict(Sq=0), rfa.RFA_ERR_INVALID_ARG),
@@ -282,6 +315,7 @@ def test_decode_workspace_plans_splits(lib):
     (dict(io_dtype=rfa.DT_UNDEFINED), rfa.RFA_ERR_INVALID_ARG),
     (dict(rope_interleaved=2), rfa.RFA_ERR_INVALID_ARG),
     (dict(rope_base=0.0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(num_splits=-1), rfa.RFA_ERR_INVALID_ARG),
 ])
 def test_decode_rejects_invalid_params(lib, kw, code):
     p = _dp(**kw)

@@ -26,14 +26,14 @@ def rfa():
 
 
 def _case(rfa, B, Hq, Hkv, Sq, D, Smax, lens, *, seed, dtype=torch.bfloat16, causal=True, interleaved=False,
-          base=10000.0, inv=None, max_len=None):
+          base=10000.0, inv=None, max_len=None, num_splits=0):
     q = workloads.randn16((B, Hq, Sq, D), seed, dtype)
     kc = workloads.randn16((B, Smax, Hkv, D), seed + 1, dtype)
     vc = workloads.randn16((B, Smax, Hkv, D), seed + 2, dtype)
     lens_t = torch.tensor(lens, dtype=torch.int32)
     # new tokens sit at the last Sq positions of each sequence
     q_pos = torch.stack([torch.arange(L - Sq, L, dtype=torch.int32) for L in lens])
-    kw = dict(causal=causal, interleaved=interleaved, rope_base=base, max_kv_len=max_len)
+    kw = dict(causal=causal, interleaved=interleaved, rope_base=base, max_kv_len=max_len, num_splits=num_splits)
     if inv is not None:
         kw["inv_freq"] = inv.cuda()
     out = rfa.decode_rope_attention(q.cuda(), kc.cuda(), vc.cuda(), q_pos.cuda(), lens_t.cuda(), **kw)
@@ -66,9 +66,13 @@ def test_many_groups_one_split(rfa):
     _compare(got, ref)
 
 
-def test_several_new_tokens_d64(rfa):
-    # Sq = 4 new tokens with G = 8 (32 query rows per tile), ragged lengths, partial last tiles
-    got, ref, st = _case(rfa, 3, 16, 2, 4, 64, 600, [300, 129, 5], seed=4)
+@pytest.mark.parametrize("D", [64, 128])
+def test_several_new_tokens(rfa, D):
+    # Sq = 4 new tokens with G = 8 (32 query rows per tile), ragged lengths, partial last tiles;
+    # one key tile per split, so the second chain of every CTA is empty and reaches the merge
+    # while the first still runs (the rows it exchanges must not share shared memory with the
+    # query tile's cos/sin rows)
+    got, ref, st = _case(rfa, 3, 16, 2, 4, D, 600, [300, 129, 5], seed=4)
     assert st == 0
     _compare(got, ref)
 
@@ -99,3 +103,27 @@ def test_lengths_outside_the_bound_set_status(rfa):
         assert rfa.get_device_status() == rfa.RFA_ERR_INVALID_ARG
         assert torch.isfinite(out.float()).all()
     assert rfa.get_device_status() == 0
+
+
+# A CTA runs its split's key tiles in two chains (tile j into score/accumulator
+# buffer j % 2) and merges them before the store: one-tile splits leave buffer 1
+# empty, odd tile counts give buffer 0 one tile more, ragged tails and the
+# bottom-right causal edge fall in either buffer.
+@pytest.mark.parametrize("lens,Smax,num_splits,Sq", [
+    ([1000, 3001], 3072, 1, 1),     # one split: 8 and 24 tiles, direct store
+    ([129, 3001], 3072, 24, 1),     # one tile per split: buffer 1 never used
+    ([640, 1663], 2048, 3, 1),      # 6 tiles per split: even, the last split ragged
+    ([1100, 1999], 2048, 2, 3),     # 8 tiles per split, 3 new tokens on the causal edge
+    ([300, 700], 768, 6, 4),        # one tile per split, short sequences, empty splits
+])
+def test_two_chain_merge_and_given_splits(rfa, lens, Smax, num_splits, Sq):
+    got, ref, st = _case(rfa, 2, 32, 8, Sq, 128, Smax, lens, seed=11 + num_splits, num_splits=num_splits)
+    assert st == 0
+    _compare(got, ref)
+
+
+def test_two_chain_merge_d64_fp16_noncausal(rfa):
+    got, ref, st = _case(rfa, 3, 16, 4, 2, 64, 1500, [1500, 385, 2], seed=21, dtype=torch.float16, causal=False,
+                         num_splits=2)
+    assert st == 0
+    _compare(got, ref)
