@@ -24,6 +24,7 @@
 namespace rfa {
 
 constexpr int kApplyHeads = 8;  // heads per thread
+constexpr int kApplyBatch = 4;  // heads whose loads are in flight together
 
 struct RopeApplyArgs {
     const void* q;
@@ -137,46 +138,68 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyArgs a) 
         int32_t slot = -1;
         if (a.slots != nullptr && h1 > a.Hq) slot = __ldg(a.slots + r);
         const int32_t b = a.bnsd ? r / a.S : 0, s = a.bnsd ? r - b * a.S : 0;
-#pragma unroll 2
-        for (int32_t h = h0; h < h1; ++h) {
-            const bool is_k = h >= a.Hq;
-            const int32_t hx = is_k ? h - a.Hq : h;
+        auto row_of = [&](int32_t h, bool& is_k, int32_t& hx) -> int64_t {
+            is_k = h >= a.Hq;
+            hx = is_k ? h - a.Hq : h;
             const int32_t Hx = is_k ? a.Hkv : a.Hq;
-            const int64_t row = a.bnsd ? (static_cast<int64_t>(b) * Hx + hx) * a.S + s
-                                       : static_cast<int64_t>(r) * Hx + hx;
-            const uint16_t* src = static_cast<const uint16_t*>(is_k ? a.k : a.q) + row * a.D;
-            float x0[8], x1[8], o0[8], o1[8];
-            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e0), x0);
-            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e1), x1);
-            if constexpr (kInterleaved) {
+            return a.bnsd ? (static_cast<int64_t>(b) * Hx + hx) * a.S + s : static_cast<int64_t>(r) * Hx + hx;
+        };
+        // Heads in batches of kApplyBatch: every load of a batch is issued before its first
+        // store, so each thread keeps kApplyBatch x 32 bytes in flight (the outputs may alias
+        // the inputs, which stops the compiler from hoisting loads above stores itself).
+#pragma unroll 1
+        for (int32_t hb = h0; hb < h1; hb += kApplyBatch) {
+            uint4 xa[kApplyBatch], xb[kApplyBatch];
 #pragma unroll
-                for (int i = 0; i < 8; i += 2) {
-                    o0[i] = fmaf(x0[i], c0[i], -x0[i + 1] * s0[i]);
-                    o0[i + 1] = fmaf(x0[i + 1], c0[i + 1], x0[i] * s0[i + 1]);
-                    o1[i] = fmaf(x1[i], c1[i], -x1[i + 1] * s1[i]);
-                    o1[i + 1] = fmaf(x1[i + 1], c1[i + 1], x1[i] * s1[i + 1]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    o0[i] = fmaf(x0[i], c0[i], -x1[i] * s0[i]);
-                    o1[i] = fmaf(x1[i], c1[i], x0[i] * s1[i]);
+            for (int u = 0; u < kApplyBatch; ++u) {
+                if (hb + u < h1) {
+                    bool is_k;
+                    int32_t hx;
+                    const int64_t row = row_of(hb + u, is_k, hx);
+                    const uint16_t* src = static_cast<const uint16_t*>(is_k ? a.k : a.q) + row * a.D;
+                    xa[u] = *reinterpret_cast<const uint4*>(src + e0);
+                    xb[u] = *reinterpret_cast<const uint4*>(src + e1);
                 }
             }
-            const uint4 p0 = pack8<kFP16>(o0), p1 = pack8<kFP16>(o1);
-            void* dst = is_k ? a.k_out : a.q_out;
-            if (dst != nullptr) {
-                uint16_t* d = static_cast<uint16_t*>(dst) + row * a.D;
-                *reinterpret_cast<uint4*>(d + e0) = p0;
-                *reinterpret_cast<uint4*>(d + e1) = p1;
-            }
-            if (is_k && slot >= 0) {
-                if (slot < a.cache_rows) {
-                    uint16_t* d = static_cast<uint16_t*>(a.cache) + (static_cast<int64_t>(slot) * a.Hkv + hx) * a.D;
+#pragma unroll
+            for (int u = 0; u < kApplyBatch; ++u) {
+                if (hb + u >= h1) break;
+                bool is_k;
+                int32_t hx;
+                const int64_t row = row_of(hb + u, is_k, hx);
+                float x0[8], x1[8], o0[8], o1[8];
+                unpack8<kFP16>(xa[u], x0);
+                unpack8<kFP16>(xb[u], x1);
+                if constexpr (kInterleaved) {
+#pragma unroll
+                    for (int i = 0; i < 8; i += 2) {
+                        o0[i] = fmaf(x0[i], c0[i], -x0[i + 1] * s0[i]);
+                        o0[i + 1] = fmaf(x0[i + 1], c0[i + 1], x0[i] * s0[i + 1]);
+                        o1[i] = fmaf(x1[i], c1[i], -x1[i + 1] * s1[i]);
+                        o1[i + 1] = fmaf(x1[i + 1], c1[i + 1], x1[i] * s1[i + 1]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        o0[i] = fmaf(x0[i], c0[i], -x1[i] * s0[i]);
+                        o1[i] = fmaf(x1[i], c1[i], x0[i] * s1[i]);
+                    }
+                }
+                const uint4 p0 = pack8<kFP16>(o0), p1 = pack8<kFP16>(o1);
+                void* dst = is_k ? a.k_out : a.q_out;
+                if (dst != nullptr) {
+                    uint16_t* d = static_cast<uint16_t*>(dst) + row * a.D;
                     *reinterpret_cast<uint4*>(d + e0) = p0;
                     *reinterpret_cast<uint4*>(d + e1) = p1;
-                } else {
-                    record_status(1 /* RFA_ERR_INVALID_ARG */);
+                }
+                if (is_k && slot >= 0) {
+                    if (slot < a.cache_rows) {
+                        uint16_t* d = static_cast<uint16_t*>(a.cache) + (static_cast<int64_t>(slot) * a.Hkv + hx) * a.D;
+                        *reinterpret_cast<uint4*>(d + e0) = p0;
+                        *reinterpret_cast<uint4*>(d + e1) = p1;
+                    } else {
+                        record_status(1 /* RFA_ERR_INVALID_ARG */);
+                    }
                 }
             }
         }
