@@ -159,8 +159,9 @@ typedef struct {
  *   k_cache, v_cache dev io_dtype [cache_rows, Hkv, D]
  *   cache_rows    >= 1; a slot >= cache_rows is not written and the status word
  *                 becomes RFA_ERR_INVALID_ARG
- * Pointers 16-byte aligned (slots 4-byte).  Returns RFA_ERR_INVALID_ARG for
- * null/misaligned pointers or bad sizes.
+ * The caches must not overlap k or v (the rows are read ahead of the cache
+ * writes).  Pointers 16-byte aligned (slots 4-byte).  Returns
+ * RFA_ERR_INVALID_ARG for null/misaligned pointers or bad sizes.
  */
 RFA_API rfa_status rfa_kv_rms_norm_rope_cache(const rfa_kv_cache_params* p, const void* k, const void* v,
                                               const float* gamma, const void* sin, const void* cos,

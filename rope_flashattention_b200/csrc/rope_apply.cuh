@@ -231,7 +231,7 @@ struct KvCacheArgs {
 };
 
 template <bool kFP16, typename TabT, bool kInterleaved>
-__global__ void __launch_bounds__(256) kv_norm_rope_cache_kernel(const KvCacheArgs a) {
+__global__ void __launch_bounds__(256, 4) kv_norm_rope_cache_kernel(const KvCacheArgs a) {
     const uint32_t chunks = static_cast<uint32_t>(a.D) / 16u;  // power of two <= 32
     const uint32_t work = static_cast<uint32_t>(a.T) * static_cast<uint32_t>(a.Hkv) * chunks;
     const uint32_t lane = threadIdx.x & 31u;
@@ -245,20 +245,28 @@ __global__ void __launch_bounds__(256) kv_norm_rope_cache_kernel(const KvCacheAr
         const int32_t t = act ? static_cast<int32_t>(row / static_cast<uint32_t>(a.Hkv)) : 0;
         const int32_t h = act ? static_cast<int32_t>(row - static_cast<uint32_t>(t) * a.Hkv) : 0;
         const int32_t e0 = 8 * static_cast<int32_t>(c), e1 = half + e0;
-        float x0[8] = {}, x1[8] = {};
         const int64_t off = (static_cast<int64_t>(t) * a.Hkv + h) * a.D;
+        // k, v and the slot are loaded together, before any store of this iteration (the
+        // caches do not overlap k and v), so their latencies overlap
+        uint4 ka = make_uint4(0u, 0u, 0u, 0u), kb = ka, va = ka, vb = ka;
+        int32_t slot = -1;
         if (act) {
             const uint16_t* src = static_cast<const uint16_t*>(a.k) + off;
-            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e0), x0);
-            unpack8<kFP16>(*reinterpret_cast<const uint4*>(src + e1), x1);
+            const uint16_t* vs = static_cast<const uint16_t*>(a.v) + off;
+            ka = *reinterpret_cast<const uint4*>(src + e0);
+            kb = *reinterpret_cast<const uint4*>(src + e1);
+            va = *reinterpret_cast<const uint4*>(vs + e0);
+            vb = *reinterpret_cast<const uint4*>(vs + e1);
+            slot = __ldg(a.slots + t);
         }
+        float x0[8], x1[8];
+        unpack8<kFP16>(ka, x0);
+        unpack8<kFP16>(kb, x1);
         float ss = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) ss = fmaf(x0[i], x0[i], fmaf(x1[i], x1[i], ss));
         for (uint32_t o = chunks >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (!act) continue;
-        const int32_t slot = __ldg(a.slots + t);
-        if (slot < 0) continue;
+        if (!act || slot < 0) continue;
         if (slot >= a.cache_rows) {
             record_status(1 /* RFA_ERR_INVALID_ARG */);
             continue;
@@ -299,10 +307,9 @@ __global__ void __launch_bounds__(256) kv_norm_rope_cache_kernel(const KvCacheAr
         uint16_t* kd = static_cast<uint16_t*>(a.k_cache) + dst;
         *reinterpret_cast<uint4*>(kd + e0) = pack8<kFP16>(o0);
         *reinterpret_cast<uint4*>(kd + e1) = pack8<kFP16>(o1);
-        const uint16_t* vs = static_cast<const uint16_t*>(a.v) + off;
         uint16_t* vd = static_cast<uint16_t*>(a.v_cache) + dst;
-        *reinterpret_cast<uint4*>(vd + e0) = *reinterpret_cast<const uint4*>(vs + e0);
-        *reinterpret_cast<uint4*>(vd + e1) = *reinterpret_cast<const uint4*>(vs + e1);
+        *reinterpret_cast<uint4*>(vd + e0) = va;
+        *reinterpret_cast<uint4*>(vd + e1) = vb;
     }
 }
 
