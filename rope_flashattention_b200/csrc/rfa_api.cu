@@ -90,14 +90,28 @@ int grid_for(int64_t work, int threads) {
     return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, 148LL * 64)));
 }
 
+// SMs of the current device; 148 (a B200) when no device is visible, so that
+// host-only planning (workspace sizes) matches the GPU it is meant for.
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+        (void)cudaGetLastError();  // not a launch error: leave no error behind
+        return 148;
+    }
+    return sms;
+}
+
 // Grid of a grid-stride kernel: no more blocks than fit on the device at once
 // (every block then pays its prologue once).
 template <typename K>
 int resident_grid(K kernel, int64_t work, int threads) {
-    int dev = 0, sms = 148, per_sm = 1;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+    const int sms = device_sms();
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1) {
+        (void)cudaGetLastError();
         per_sm = 1;
+    }
     const int64_t blocks = (work + threads - 1) / threads;
     return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(sms) * per_sm)));
 }
@@ -674,7 +688,7 @@ rfa_status decode_validate(const rfa_decode_params* p) {
 }
 
 // Keys of a sequence are split into whole key tiles across CTAs; one CTA is
-// resident per SM, so B * Hkv * splits CTAs run in ceil(that / 148) waves of
+// resident per SM, so B * Hkv * splits CTAs run in ceil(that / SMs) waves of
 // about tiles / splits key tiles each.  The plan takes the split count with the
 // least waves x (tiles per split + kSplitCost), kSplitCost being the fixed cost
 // of a CTA (setup, query load and rotation, pipeline fill and drain, merge and
@@ -683,24 +697,24 @@ rfa_status decode_validate(const rfa_decode_params* p) {
 // e.g. 8 sequences x 32K keys run fastest as 2 splits, one wave of 128 CTAs
 // that already saturates HBM.
 constexpr int64_t kSplitCost = 6;
-constexpr int64_t kNumSMs = 148;
 DecodePlan decode_plan(const rfa_decode_params* p) {
     DecodePlan pl;
     pl.rq = static_cast<int64_t>(p->B) * p->Hq * p->Sq;
     const int64_t groups = static_cast<int64_t>(p->B) * p->Hkv;
     const int32_t tiles = (p->max_kv_len + rfa::kBlockN - 1) / rfa::kBlockN;
+    const int64_t sms = device_sms();
     int32_t per = tiles;
     if (p->num_splits > 0) {
         per = (tiles + std::min(p->num_splits, tiles) - 1) / std::min(p->num_splits, tiles);
     } else {
         // beyond about 8 waves more splits only add CTA costs
-        const int64_t s_max = std::min<int64_t>(tiles, std::max<int64_t>(1, (8 * kNumSMs + groups - 1) / groups));
+        const int64_t s_max = std::min<int64_t>(tiles, std::max<int64_t>(1, (8 * sms + groups - 1) / groups));
         int64_t best = -1;
         for (int32_t s = 1; s <= s_max; ++s) {
             const int32_t ps = (tiles + s - 1) / s;
             if (s > 1 && ps == (tiles + s - 2) / (s - 1)) continue;  // same split as s - 1
             const int64_t n = (tiles + ps - 1) / ps;
-            const int64_t cost = ((groups * n + kNumSMs - 1) / kNumSMs) * (ps + kSplitCost);
+            const int64_t cost = ((groups * n + sms - 1) / sms) * (ps + kSplitCost);
             if (best < 0 || cost < best) {
                 best = cost;
                 per = ps;
