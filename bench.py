@@ -578,31 +578,65 @@ def run_gpu(args, world, rank, local):
     value = job_throughput(flops, world, ms) / 1e12
 
     # ---------------- end to end: host buffers through the C ABI
-    qp, kp, vp, posp = (x.pin_memory() for x in (q_h, k_h, v_h, pos_h))
-    outp = torch.empty(q_h.shape, dtype=q_h.dtype).pin_memory()
+    # Every step copies its inputs in from pinned host memory, runs the public
+    # call, and copies its result back out.  Steps are pipelined as a serving
+    # loop would run them: uploads on one copy stream, downloads on another
+    # (PCIe is full duplex), compute on the current stream, inputs and outputs
+    # double-buffered on the device and guarded by events.
+    host_in = [x.pin_memory() for x in (q_h, k_h, v_h, pos_h)]
+    host_out = [torch.empty(q_h.shape, dtype=q_h.dtype).pin_memory() for _ in range(2)]
+    slots = [([torch.empty(x.shape, dtype=x.dtype, device=dev) for x in host_in], torch.empty_like(q))
+             for _ in range(2)]
     ws = torch.empty_like(table)
+    main = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     K2 = max(3, min(K, 30))
 
-    def e2e_step():
-        qd, kd, vd, pd = (x.to(dev, non_blocking=True) for x in (qp, kp, vp, posp))
-        o = rfa.fused_rope_attention(qd, kd, vd, pd, inv_freq=inv, workspace=ws, **kw)
-        outp.copy_(o, non_blocking=True)
+    def e2e_run(nsteps, e_begin=None):
+        if e_begin is not None:
+            s_in.wait_event(e_begin)
+            s_out.wait_event(e_begin)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        for i in range(nsteps):
+            b = i % 2
+            dins, dout = slots[b]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_comp[b])  # step i - 2 has read this slot's inputs
+                for dst, src in zip(dins, host_in):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[b].record(s_in)
+            main.wait_event(ev_in[b])
+            if i >= 2:
+                main.wait_event(ev_out[b])  # step i - 2's result has left this slot
+            rfa.fused_rope_attention(*dins, inv_freq=inv, workspace=ws, out=dout, **kw)
+            ev_comp[b].record(main)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b])
+                host_out[b].copy_(dout, non_blocking=True)
+                ev_out[b].record(s_out)
+        main.wait_stream(s_in)
+        main.wait_stream(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_run(2)
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(K2):
-        e2e_step()
-    e1.record()
+    e0.record(main)
+    e2e_run(K2, e0)
+    e1.record(main)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K2, world)
-    h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp, posp))
-    d2h = outp.numel() * outp.element_size()
+    # the pipelined result is the plain call's result, bit for bit
+    ref = rfa.fused_rope_attention(q, k, v, pos, inv_freq=inv, workspace=ws, **kw)
+    if not torch.equal(host_out[(K2 - 1) % 2], ref.cpu()):
+        raise RuntimeError("end-to-end pipeline result differs from the plain call")
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = host_out[0].numel() * host_out[0].element_size()
 
     extra = {}
     if rank == 0 and world == 1:
