@@ -221,6 +221,18 @@ def oracle_rows_sample(w, n_rows: int, seed: int):
     return np.stack([b, h, i], axis=1).astype(np.int32)
 
 
+def oracle_rows_sample_group(w, n_rows: int, seed: int):
+    """n_rows random query rows of one random (sequence, kv head) group: an
+    oracle call on them prepares that group's keys and values only."""
+    lens = workloads.seq_lengths(w)
+    rng = np.random.default_rng(seed)
+    b = int(rng.integers(0, w.B))
+    G = w.Hq // w.Hkv
+    h = int(rng.integers(0, w.Hkv)) * G + rng.integers(0, G, n_rows)
+    i = rng.integers(0, lens[b], n_rows)
+    return np.stack([np.full(n_rows, b), h, i], axis=1).astype(np.int32)
+
+
 def rows_flops(w, rows) -> float:
     lens = workloads.seq_lengths(w)
     keys = [(int(i) + 1 if w.causal else lens[int(b)]) for b, _, i in rows]
@@ -322,13 +334,22 @@ def run_reference(args, world, rank):
         return 0
     w = workloads.BY_KEY[args.workload]
     r = OracleRunner(w)
-    per_step = max(1.0, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
-    rows = r.calibrated_rows(per_step)
+    # The whole run (warm-up + steps) takes about 150 s of oracle time whatever
+    # the step count: each step is a sample of rows of one (sequence, kv head)
+    # group, sized to its share (at least one row, at most 65536).
+    per_step = min(6.0, 150.0 / max(1, args.steps + args.warmup))
+    n = 1
+    while True:
+        dt = r.run(oracle_rows_sample_group(w, n, 7))
+        if dt >= per_step / 4 or n >= 65536:
+            break
+        n *= 4
+    n = int(min(65536, max(1, n * per_step / max(dt, 1e-6))))
     for i in range(args.warmup):
-        r.run(oracle_rows_sample(w, len(rows), 100 + i))
+        r.run(oracle_rows_sample_group(w, n, 100 + i))
     times, flops = [], 0.0
     for i in range(args.steps):
-        rs = oracle_rows_sample(w, len(rows), 1000 + i)
+        rs = oracle_rows_sample_group(w, n, 1000 + i)
         times.append(r.run(rs))
         flops += rows_flops(w, rs)
     tot = sum(times)
@@ -340,7 +361,8 @@ def run_reference(args, world, rank):
         "config": config_of(w, {"impl_note": "fp64 CPU oracle (plain loops, pthreads), each step a bounded "
                                              "random row sample of the workload"}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": r.threads, "kind": "oracle",
-                         "sample": f"{len(rows)} random query rows per step"},
+                         "sample": f"{n} random query rows of one random (sequence, kv head) group per step, "
+                                   f"{tot:.1f} s over {args.steps} steps"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }

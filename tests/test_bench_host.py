@@ -34,3 +34,13 @@ def test_row_sample_stays_inside_the_workload():
     rows = bench.oracle_rows_sample(w, 2000, 3)
     lens = np.array(workloads.seq_lengths(w))
     assert (rows[:, 2] < lens[rows[:, 0]]).all() and (rows[:, 1] < w.Hq).all()
+
+
+def test_group_sample_stays_in_one_kv_group():
+    w = workloads.BY_KEY["gqa8k"]
+    G = w.Hq // w.Hkv
+    for seed in range(5):
+        rows = bench.oracle_rows_sample_group(w, 500, seed)
+        assert len(set(rows[:, 0].tolist())) == 1
+        assert len(set((rows[:, 1] // G).tolist())) == 1
+        assert (rows[:, 2] >= 0).all() and (rows[:, 2] < workloads.seq_lengths(w)[rows[0, 0]]).all()
