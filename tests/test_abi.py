@@ -103,6 +103,12 @@ FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails va
     (dict(scale=-0.5), rfa.RFA_ERR_INVALID_ARG),
     (dict(ntk_enable=1, ntk_train_len=0), rfa.RFA_ERR_INVALID_ARG),
     (dict(ntk_enable=1, ntk_train_len=8, ntk_factor=0.5), rfa.RFA_ERR_INVALID_ARG),
+    (dict(rope_interleaved=2), rfa.RFA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), rfa.RFA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), rfa.RFA_ERR_INVALID_ARG),
+    (dict(rope_base=float("inf")), rfa.RFA_ERR_INVALID_ARG),
+    (dict(B=0), rfa.RFA_ERR_INVALID_ARG),
+    (dict(Hq=0), rfa.RFA_ERR_INVALID_ARG),
 ])
 def test_attention_rejects_invalid_params(lib, kw, code):
     rc = lib.rfa_fused_rope_attention(ctypes.byref(_p(**kw)), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
