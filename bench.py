@@ -74,7 +74,7 @@ def kernel_hash() -> str:
 def profiled_traffic(workload_key: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it
     was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    path = os.path.join(ROOT, "profiles", "fused_rope_attn_dram-traffic.txt")
     if not os.path.exists(path):
         return None
     kh = kernel_hash()
