@@ -695,7 +695,7 @@ def run_gpu(args, world, rank, local):
                      "kernel": "fused_rope_attn_fwd_kernel", "kernel_ms": attn_ms, "kernel_source": kernel_hash()},
         "e2e": {"value": job_throughput(flops, world, e2e_ms) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * K,
+        "gpu_launches": 3 * K,  # per step: rope_table_kernel, rope_seed_kernel, fused_rope_attn_fwd_kernel
         "clocks": clk,
         "tok_per_s": job_throughput(workloads.ntokens(w), world, ms),
     }
