@@ -3,14 +3,22 @@
 plus the DynamicNTK sin/cos table (GB/s).
 
 One step = the whole hot path over one batch of the workload: the cos/sin
-table kernel followed by the fused RoPE + attention kernel, inputs resident in
-HBM.  Inputs (q, k, v) are larger than L2, so no flush is needed between
-steps.  Prints one JSON line (rank 0).
+table kernels followed by the fused RoPE + attention kernel, inputs resident
+in HBM.  Inputs (q, k, v) are larger than L2, so no flush is needed between
+steps.  The default workload is the largest that fits one GPU: 16K tokens, 64
+query / 8 kv heads, dynamic NTK.  The same run adds, for each other full-size
+workload (Qwen-7B-shaped 2K prefill, GQA 8K prefill, packed 16 sequences), the
+attention kernel alone timed for about a second with its own clock record,
+then the sin/cos table, the Rope operator, the cache op and decode.  Prints
+one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload KEY] [--impl rfa|reference]
+  python bench.py --only attention|sincos|sincos_ceiling|rope_apply|kv_cache|decode [--workload KEY] [--reps R]
 
 --impl reference times the fp64 CPU oracle on the host cores on bounded row
 samples of the same workload (the comparison program for this method).
+--only runs one kernel alone (2 warm-up + R timed launches) for profiler
+captures.
 Multi-GPU (torchrun): the path shards into independent problems with no data
 exchange, so every rank runs its own replica of the workload (weak scaling);
 ranks only meet for the barrier and the max-over-ranks of the timings.
@@ -41,17 +49,27 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = ["rope_flashattention_b200/csrc/fused_rope_attn.cuh", "rope_flashattention_b200/csrc/sm100_ptx.cuh"]
 
 
-def parse_args():
+ONLY_MODES = ("attention", "sincos", "sincos_ceiling", "rope_apply", "kv_cache", "decode")
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="qwen7b", choices=sorted(workloads.BY_KEY))
+    # the largest workload that fits one GPU (16K tokens, 64 query heads, dynamic NTK)
+    ap.add_argument("--workload", default="ntk16k", choices=sorted(workloads.BY_KEY))
     ap.add_argument("--impl", default="rfa", choices=["rfa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true", help="skip the unfused torch context line")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the per-workload kernel lines")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-oracle sample time")
-    return ap.parse_args()
+    ap.add_argument("--workload-seconds", type=float, default=1.0,
+                    help="timed seconds of each per-workload kernel line")
+    ap.add_argument("--only", choices=ONLY_MODES, default=None,
+                    help="run one kernel alone (for profiler captures) and print its figures")
+    ap.add_argument("--reps", type=int, default=3, help="--only: timed launches after 2 warm-up launches")
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -88,12 +106,20 @@ def profiled_traffic(workload_key: str):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """nvidia-smi samples of the SM clock, power and throttle reasons, taken
+    every 20 ms by a reader thread.  The constructor returns once the first
+    sample has arrived (so the sampler is live when the timed region starts);
+    stop() keeps the samples taken between construction and stop()."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 20
 
     def __init__(self, device_index: int):
+        import threading
+
         self.proc = None
+        self.lines = []
         sel = []
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
@@ -102,24 +128,41 @@ class ClockSampler:
             sel = []
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
+                                          "-lms", str(self.INTERVAL_MS), *sel], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append((time.perf_counter(), line))
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        t0 = time.perf_counter()
+        while not self.lines and time.perf_counter() - t0 < 3.0 and self.proc.poll() is None:
+            time.sleep(0.005)
+        self.t_start = time.perf_counter()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        t_end = time.perf_counter()
+        time.sleep(2.5 * self.INTERVAL_MS / 1000.0)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+            self.proc.wait()
+        self.thread.join(timeout=5)
+        # samples whose reading time falls in the timed region (plus one interval of lag)
+        lag = self.INTERVAL_MS / 1000.0
+        window = [ln for t, ln in self.lines if self.t_start <= t <= t_end + lag]
         sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.splitlines():
+        for line in window:
             p = [x.strip() for x in line.split(",")]
             if len(p) < 9:
                 continue
@@ -133,10 +176,12 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
+                    "window_s": t_end - self.t_start}
         loaded = [s for s, pw in zip(sm, power) if pw > 250.0] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "samples": len(sm),
-                "power_w_max": max(power), "reasons": sorted(reasons)}
+                "samples_under_load": len([pw for pw in power if pw > 250.0]), "power_w_max": max(power),
+                "reasons": sorted(reasons), "window_s": t_end - self.t_start}
 
 
 # ------------------------------------------------------------------ distributed
@@ -198,16 +243,16 @@ def workload_flops(w) -> float:
     return rfa.attention_flops(workloads.seq_lengths(w), w.Hq, w.D, w.causal)
 
 
-def config_of(w, extra=None):
+def config_of(w, world: int = 1):
+    """The workload description; both arms print exactly this dict."""
     c = {"workload": w.name, "layout": w.layout, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
          "S": w.S if w.layout == "BNSD" else None, "D": w.D, "causal": w.causal, "rope_base": w.rope_base,
-         "ntokens": workloads.ntokens(w), "l2": "inputs larger than L2 (126 MB); no flush between steps"}
+         "ntokens": workloads.ntokens(w), "l2": "inputs larger than L2 (126 MB); no flush between steps",
+         "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
     if w.ntk_train_len:
         c["ntk"] = {"train_len": w.ntk_train_len, "factor": w.ntk_factor}
     if w.layout == "TND":
         c["seq_lens"] = workloads.seq_lengths(w)
-    if extra:
-        c.update(extra)
     return c
 
 
@@ -358,8 +403,8 @@ def run_reference(args, world, rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": config_of(w, {"impl_note": "fp64 CPU oracle (plain loops, pthreads), each step a bounded "
-                                             "random row sample of the workload"}),
+        "impl_note": "fp64 CPU oracle (plain loops, pthreads), each step a bounded random row sample of the workload",
+        "config": config_of(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": r.threads, "kind": "oracle",
                          "sample": f"{n} random query rows of one random (sequence, kv head) group per step, "
                                    f"{tot:.1f} s over {args.steps} steps"},
@@ -371,48 +416,80 @@ def run_reference(args, world, rank):
 
 
 # ------------------------------------------------------------------ GPU arm
-def sincos_bench(rfa, dev):
-    """rope_sincos at the operator's ceiling shape (T=256000, D=128, fp16): GB/s
-    of algorithmic bytes (positions + invFreq + lengths read, sin + cos written).
-
-    The 131 MB of outputs exceed L2 (126 MB), so launches run back to back and
-    each one evicts (writes back) the previous one's output: the primary figure.
-    Also reported: one launch after L2 was filled with clean lines by reading a
-    256 MB buffer.  (Flushing by writing a buffer would leave ~126 MB of dirty
-    lines that this write-only kernel would have to write back for it.)"""
-    pos, inv, lens = workloads.sincos_problem(256000, 128, 16, seed=7)
-    pos, inv, lens = pos.to(dev), inv.to(dev), lens.to(dev)
-    s = torch.empty((256000, 128), dtype=torch.float16, device=dev)
-    c = torch.empty_like(s)
-    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)  # 256 MB, read to clear L2
+def _sincos_time(rfa, pos, inv, lens, D, s, c, flush, back_to_back: bool):
+    """Seconds per rope_sincos launch: back to back (outputs larger than L2),
+    else the median of single launches each after a 256 MB read flush."""
     for _ in range(3):
-        rfa.rope_sincos(pos, inv, lens, 128, torch.float16, s, c)
+        rfa.rope_sincos(pos, inv, lens, D, torch.float16, s, c)
     torch.cuda.synchronize()
-    n = 50
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(n):
-        rfa.rope_sincos(pos, inv, lens, 128, torch.float16, s, c)
-    e1.record()
-    torch.cuda.synchronize()
-    t_b2b = e0.elapsed_time(e1) * 1e-3 / n
+    if back_to_back:
+        n = 50
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            rfa.rope_sincos(pos, inv, lens, D, torch.float16, s, c)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e-3 / n, f"{n} launches back to back (outputs > L2)"
     times = []
-    for _ in range(20):
+    for _ in range(30):
         flush.sum()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
-        rfa.rope_sincos(pos, inv, lens, 128, torch.float16, s, c)
+        rfa.rope_sincos(pos, inv, lens, D, torch.float16, s, c)
         b.record()
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b) * 1e-3)
+    return statistics.median(times), "median of 30 single launches, each after a 256 MB read that clears L2"
+
+
+def _sincos_bytes(T: int, D: int, batch: int) -> int:
+    """Algorithmic bytes: positions, invFreq rows and lengths read; sin and cos written (fp16)."""
+    return T * 4 + 2 * T * D * 2 + batch * (D // 2) * 4 + batch * 4
+
+
+def sincos_bench(rfa, dev):
+    """rope_sincos on the packed workload's own input: its 16 sequence lengths
+    (T = 57,209 at seed 5), positions = arange per sequence, its invFreq rows
+    (U[0,1) fp32), headSize 128, fp16 out.  The 29.5 MB of outputs fit in L2
+    (126 MB), so each timed launch follows a 256 MB read that leaves L2 holding
+    clean lines only; the launch is short enough (a few microseconds) that
+    launch latency shows."""
+    w = workloads.PACKED
+    lens_l = workloads.seq_lengths(w)
+    T = sum(lens_l)
+    pos = workloads.positions(w).to(dev)
+    inv = workloads.random_inv_freq(w).to(dev)
+    lens = torch.tensor(lens_l, dtype=torch.int32, device=dev)
+    s = torch.empty((T, w.D), dtype=torch.float16, device=dev)
+    c = torch.empty_like(s)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    t, how = _sincos_time(rfa, pos, inv, lens, w.D, s, c, flush, back_to_back=False)
     assert rfa.get_device_status() == 0
-    byts = 256000 * 4 + 2 * 256000 * 128 * 2 + 16 * 64 * 4 + 16 * 4
-    t_rf = statistics.median(times)
-    return {"shape": "T=256000 (16 x 16000), headSize 128, fp16", "bytes": byts, "us": t_b2b * 1e6,
-            "GB/s": byts / t_b2b / 1e9, "timing": f"{n} launches back to back (outputs > L2)",
-            "read_flushed_us": t_rf * 1e6, "read_flushed_GB/s": byts / t_rf / 1e9}
+    byts = _sincos_bytes(T, w.D, w.B)
+    return {"shape": f"packed workload: T={T} over {w.B} sequences (seed {w.seed}), headSize {w.D}, fp16",
+            "bytes": byts, "us": t * 1e6, "GB/s": byts / t / 1e9, "timing": how}
+
+
+def sincos_ceiling_bench(rfa, dev):
+    """rope_sincos at the operator's ceiling (T = 256000 = 16 x 16000 tokens,
+    the most the DynamicNTK operator accepts, headSize 128, fp16): 132 MB of
+    outputs exceed L2, so launches run back to back, each evicting the
+    previous one's output.  Also: single launches after a 256 MB read flush."""
+    pos, inv, lens = workloads.sincos_problem(256000, 128, 16, seed=7)
+    pos, inv, lens = pos.to(dev), inv.to(dev), lens.to(dev)
+    s = torch.empty((256000, 128), dtype=torch.float16, device=dev)
+    c = torch.empty_like(s)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    t_b2b, how = _sincos_time(rfa, pos, inv, lens, 128, s, c, flush, back_to_back=True)
+    t_rf, _ = _sincos_time(rfa, pos, inv, lens, 128, s, c, flush, back_to_back=False)
+    assert rfa.get_device_status() == 0
+    byts = _sincos_bytes(256000, 128, 16)
+    return {"shape": "T=256000 (16 x 16000, the operator's ceiling), headSize 128, fp16", "bytes": byts,
+            "us": t_b2b * 1e6, "GB/s": byts / t_b2b / 1e9, "timing": how, "read_flushed_us": t_rf * 1e6,
+            "read_flushed_GB/s": byts / t_rf / 1e9}
 
 
 def rope_apply_bench(rfa, dev):
@@ -545,33 +622,125 @@ def unfused_context(w, q, k, v, pos, dev, iters=20):
             "TFLOP/s": workload_flops(w) / t / 1e12, "ms": t * 1e3}
 
 
+class AttnInputs:
+    """A workload's inputs resident on the device, its cos/sin table built."""
+
+    def __init__(self, rfa, w, dev):
+        self.rfa, self.w, self.dev = rfa, w, dev
+        self.kw = workload_kwargs(w)
+        self.q_h, self.k_h, self.v_h = workloads.make_qkv(w)
+        self.pos_h = workloads.positions(w)
+        inv_h = workloads.random_inv_freq(w)
+        self.q, self.k, self.v = self.q_h.to(dev), self.k_h.to(dev), self.v_h.to(dev)
+        self.pos = self.pos_h.to(dev)
+        self.inv = inv_h.to(dev) if inv_h is not None else None
+        self.out = torch.empty_like(self.q)
+        self.table = rfa.rope_attention_table(self.q, self.k, self.pos, inv_freq=self.inv, **self.kw)
+        self.flops = workload_flops(w)
+
+    def step(self, ev=None):
+        """One pass of the hot path: the cos/sin table kernels, then the fused
+        attention kernel (bracketed by `ev`, if given)."""
+        self.rfa.rope_attention_table(self.q, self.k, self.pos, inv_freq=self.inv, workspace=self.table, **self.kw)
+        if ev is not None:
+            ev[0].record()
+        self.attention()
+        if ev is not None:
+            ev[1].record()
+
+    def attention(self):
+        self.rfa.fused_rope_attention_with_table(self.q, self.k, self.v, self.table, out=self.out, **self.kw)
+
+
+def pick_peak(peaks, clk):
+    """The burst GEMM peak applies unless the clock record shows the part held
+    below its maximum clock (power-capped), where the sustained figure does."""
+    sm, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    sustained = bool(sm and smax and sm < 0.9 * smax)
+    return peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"], (
+        "bf16_tflops_sustained" if sustained else "bf16_tflops")
+
+
+def attention_line(rfa, w, dev, peaks, peak_src, seconds: float):
+    """The fused attention kernel alone on workload w, launched back to back
+    for about `seconds` (inputs larger than L2), each launch bracketed by CUDA
+    events on the launching stream, with its own clock record."""
+    a = AttnInputs(rfa, w, dev)
+    for _ in range(3):
+        a.step()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    a.attention()
+    torch.cuda.synchronize()
+    est = max(time.perf_counter() - t0, 1e-5)
+    n = int(max(20, min(20000, seconds / est)))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    for e in evs:
+        e[0].record()
+        a.attention()
+        e[1].record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    st = rfa.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status ({w.name}): {rfa.status_string(st)}")
+    ms = statistics.mean(x.elapsed_time(y) for x, y in evs)
+    peak, which = pick_peak(peaks, clk)
+    tf = a.flops / (ms * 1e-3) / 1e12
+    del a
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "kernel": "fused_rope_attn_fwd_kernel", "launches": n, "kernel_ms": ms,
+            "TFLOP/s": tf, "flops": workload_flops(w), "peak": peak, "peak_source": f"{peak_src} {which}",
+            "frac": tf / peak, "tok_per_s": workloads.ntokens(w) / (ms * 1e-3), "clocks": clk}
+
+
+def run_only(args, dev):
+    """One kernel alone: `--reps` timed launches after 2 warm-up launches, for
+    profiler captures (a figure printed under a profiler is not a bench value)."""
+    import rope_flashattention_b200 as rfa
+
+    rfa.load_library()
+    if args.only == "attention":
+        w = workloads.BY_KEY[args.workload]
+        a = AttnInputs(rfa, w, dev)
+        for _ in range(2):
+            a.attention()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.reps):
+            a.attention()
+        e1.record()
+        torch.cuda.synchronize()
+        st = rfa.get_device_status()
+        ms = e0.elapsed_time(e1) / max(1, args.reps)
+        res = {"only": "attention", "workload": w.name, "kernel_ms": ms, "TFLOP/s": a.flops / (ms * 1e-3) / 1e12,
+               "status": rfa.status_string(st)}
+    else:
+        fn = {"sincos": sincos_bench, "sincos_ceiling": sincos_ceiling_bench, "rope_apply": rope_apply_bench,
+              "kv_cache": kv_cache_bench, "decode": decode_bench}[args.only]
+        res = dict(fn(rfa, dev), only=args.only)
+    print(json.dumps(res), flush=True)
+    return 0
+
+
 def run_gpu(args, world, rank, local):
     import rope_flashattention_b200 as rfa
 
     rfa.load_library()
     dev = torch.device("cuda", local)
+    if args.only:
+        return run_only(args, dev)
     w = workloads.BY_KEY[args.workload]
     peaks, peak_src = load_peaks()
-    kw = workload_kwargs(w)
-    q_h, k_h, v_h = workloads.make_qkv(w)
-    pos_h = workloads.positions(w)
-    inv_h = workloads.random_inv_freq(w)
-    q, k, v, pos = q_h.to(dev), k_h.to(dev), v_h.to(dev), pos_h.to(dev)
-    inv = inv_h.to(dev) if inv_h is not None else None
-    out = torch.empty_like(q)
-    table = rfa.rope_attention_table(q, k, pos, inv_freq=inv, **kw)
-    flops = workload_flops(w)
-
-    def step(ev=None):
-        rfa.rope_attention_table(q, k, pos, inv_freq=inv, workspace=table, **kw)
-        if ev is not None:
-            ev[0].record()
-        rfa.fused_rope_attention_with_table(q, k, v, table, out=out, **kw)
-        if ev is not None:
-            ev[1].record()
+    a = AttnInputs(rfa, w, dev)
+    kw, q, k, v, pos, inv = a.kw, a.q, a.k, a.v, a.pos, a.inv
+    flops = a.flops
 
     for _ in range(max(3, args.warmup)):
-        step()
+        a.step()
     torch.cuda.synchronize()
     st = rfa.get_device_status()
     if st != 0:
@@ -585,7 +754,7 @@ def run_gpu(args, world, rank, local):
     clocks = ClockSampler(local)
     e_start.record()
     for i in range(K):
-        step(evs[i])
+        a.step(evs[i])
     e_end.record()
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -594,7 +763,7 @@ def run_gpu(args, world, rank, local):
     if st != 0:
         raise RuntimeError(f"device status after timing: {rfa.status_string(st)}")
     ms_local = e_start.elapsed_time(e_end) / K
-    attn_ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    attn_ms_local = statistics.mean(x.elapsed_time(y) for x, y in evs)
     ms = max_over_ranks(ms_local, world)
     attn_ms = max_over_ranks(attn_ms_local, world)
     value = job_throughput(flops, world, ms) / 1e12
@@ -605,11 +774,11 @@ def run_gpu(args, world, rank, local):
     # loop would run them: uploads on one copy stream, downloads on another
     # (PCIe is full duplex), compute on the current stream, inputs and outputs
     # double-buffered on the device and guarded by events.
-    host_in = [x.pin_memory() for x in (q_h, k_h, v_h, pos_h)]
-    host_out = [torch.empty(q_h.shape, dtype=q_h.dtype).pin_memory() for _ in range(2)]
+    host_in = [x.pin_memory() for x in (a.q_h, a.k_h, a.v_h, a.pos_h)]
+    host_out = [torch.empty(a.q_h.shape, dtype=a.q_h.dtype).pin_memory() for _ in range(2)]
     slots = [([torch.empty(x.shape, dtype=x.dtype, device=dev) for x in host_in], torch.empty_like(q))
              for _ in range(2)]
-    ws = torch.empty_like(table)
+    ws = torch.empty_like(a.table)
     main = torch.cuda.current_stream(dev)
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     K2 = max(3, min(K, 30))
@@ -659,39 +828,43 @@ def run_gpu(args, world, rank, local):
         raise RuntimeError("end-to-end pipeline result differs from the plain call")
     h2d = sum(x.numel() * x.element_size() for x in host_in)
     d2h = host_out[0].numel() * host_out[0].element_size()
+    del slots, host_in, host_out, ws, ref
 
     extra = {}
+    if rank == 0 and world == 1 and not args.no_context:
+        try:
+            extra["context_unfused"] = unfused_context(w, q, k, v, pos, dev)
+        except Exception as e:  # context only; never fails the bench
+            extra["context_unfused"] = {"error": str(e)[:200]}
+    traffic = profiled_traffic(args.workload)
+    del a, q, k, v, pos
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1:
+        if not args.no_workloads:
+            # the other full-size workloads: the attention kernel alone, each timed for about a second
+            extra["workloads"] = {key: attention_line(rfa, wl, dev, peaks, peak_src, args.workload_seconds)
+                                  for key, wl in workloads.BY_KEY.items() if key not in ("tiny", args.workload)}
         extra["sincos"] = sincos_bench(rfa, dev)
         extra["sincos"]["frac_hbm"] = extra["sincos"]["GB/s"] / peaks["hbm_gbs"]
+        extra["sincos_ceiling"] = sincos_ceiling_bench(rfa, dev)
+        extra["sincos_ceiling"]["frac_hbm"] = extra["sincos_ceiling"]["GB/s"] / peaks["hbm_gbs"]
         extra["rope_apply"] = rope_apply_bench(rfa, dev)
         extra["rope_apply"]["frac_hbm"] = extra["rope_apply"]["GB/s"] / peaks["hbm_gbs"]
         extra["kv_rms_norm_rope_cache"] = kv_cache_bench(rfa, dev)
         extra["kv_rms_norm_rope_cache"]["frac_hbm"] = extra["kv_rms_norm_rope_cache"]["GB/s"] / peaks["hbm_gbs"]
         extra["decode"] = decode_bench(rfa, dev)
         extra["decode"]["frac_hbm"] = extra["decode"]["GB/s"] / peaks["hbm_gbs"]
-        if not args.no_context:
-            try:
-                extra["context_unfused"] = unfused_context(w, q, k, v, pos, dev)
-            except Exception as e:  # context only; never fails the bench
-                extra["context_unfused"] = {"error": str(e)[:200]}
 
-    # The burst GEMM peak applies unless the clock record shows the part held
-    # below its maximum clock (power-capped), where the sustained figure does.
-    sm, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz")
-    sustained = bool(sm and smax and sm < 0.9 * smax)
-    peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    peak, which = pick_peak(peaks, clk)
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    traffic = profiled_traffic(args.workload)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "impl": "rfa",
-        "config": config_of(w, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                                "step": "cos/sin table kernel + fused RoPE/attention kernel"}),
+        "step": "cos/sin table kernels + fused RoPE/attention kernel",
+        "config": config_of(w, world),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                     "traffic": traffic,
-                     "peak_source": f"{peak_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}",
+                     "traffic": traffic, "peak_source": f"{peak_src} {which}",
                      "kernel": "fused_rope_attn_fwd_kernel", "kernel_ms": attn_ms, "kernel_source": kernel_hash()},
         "e2e": {"value": job_throughput(flops, world, e2e_ms) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2, "ms_per_step": e2e_ms},

@@ -61,16 +61,18 @@ BF16, FP16 = 0, 1
 BNSD, TND = 0, 1
 
 
-# Test hook: a prebuilt oracle library to load instead of this one (the mutation
-# tests point it at copies of rfa_oracle.c with planted mistakes).
-_LIB_ENV = "RFA_ORACLE_LIB"
+# Test hook for the mutation tests only: a prebuilt library (a copy of
+# rfa_oracle.c with one planted mistake) to load instead of this one.  It is a
+# module attribute, not read from the environment: only the mutation tests'
+# pytest plugin sets it, in the subprocesses that run the pins against a
+# mutant, so no other process can have its checker swapped.
+_lib_override = None
 
 
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (only if missing or stale)."""
-    override = os.environ.get(_LIB_ENV)
-    if override:
-        return override
+    if _lib_override:
+        return _lib_override
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread", _SRC, "-lm", "-o", tmp])

@@ -1,9 +1,10 @@
 """B200-native rotary position embedding fused into FlashAttention forward.
 
 Thin ctypes binding over librfa.so (C ABI in include/rfa.h).  This module only
-marshals arguments: it checks tensor devices, dtypes and contiguity, passes
-raw pointers and torch's current CUDA stream, and turns status codes into
-exceptions.  Every step of the computation runs in the library's CUDA
+marshals arguments: it checks that every tensor of a call sits on one CUDA
+device (and runs the call with that device current), checks dtypes and
+contiguity, passes raw pointers and torch's current CUDA stream of that
+device, and turns status codes into exceptions.  Every step of the computation runs in the library's CUDA
 kernels.  There is no CPU fallback: if librfa.so is missing the import fails.
 
 Entry points (C name without the ``rfa_`` prefix):
@@ -192,8 +193,13 @@ def _check(code: int, where: str):
         raise RfaError(code, where)
 
 
-def _stream_ptr(stream=None):
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _stream_ptr(stream=None, device: Optional[torch.device] = None):
+    """The stream the library enqueues on: `stream`, else torch's current
+    stream of `device`.  A stream of another device is refused (the library
+    launches on the current device, which _on_device makes `device`)."""
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    if device is not None and s.device != device:
+        raise ValueError(f"stream is on {s.device}, the tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -207,6 +213,36 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _same_device(**tensors) -> torch.device:
+    """The one CUDA device every given tensor (None entries skipped) lives on.
+
+    The library reads its pointers on the current device (TMA tensor maps
+    included), so a tensor on another GPU would be dereferenced as peer
+    memory; such a call is refused here instead."""
+    pairs = []
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        pairs.append((name, t.device))
+    return _one_device(pairs)
+
+
+def _one_device(pairs) -> torch.device:
+    """The device shared by every (name, device) pair; raises if they differ."""
+    dev = None
+    first = None
+    for name, d in pairs:
+        if dev is None:
+            dev, first = d, name
+        elif d != dev:
+            raise ValueError(f"{name} is on {d}, {first} on {dev}: all tensors must be on one GPU")
+    if dev is None:
+        raise ValueError("no CUDA tensor given")
+    return dev
+
+
 def rope_sincos(position_ids: torch.Tensor, inv_freq: torch.Tensor, seq_lens: torch.Tensor, head_size: int,
                 out_dtype=torch.float16, sin_out: Optional[torch.Tensor] = None,
                 cos_out: Optional[torch.Tensor] = None, stream=None):
@@ -217,15 +253,18 @@ def rope_sincos(position_ids: torch.Tensor, inv_freq: torch.Tensor, seq_lens: to
     """
     T = position_ids.numel()
     batch = seq_lens.numel()
-    dev = position_ids.device
+    dev = _same_device(position_ids=position_ids, inv_freq=inv_freq, seq_lens=seq_lens, sin_out=sin_out,
+                       cos_out=cos_out)
     if sin_out is None:
         sin_out = torch.empty((T, head_size), dtype=out_dtype, device=dev)
     if cos_out is None:
         cos_out = torch.empty((T, head_size), dtype=out_dtype, device=dev)
-    code = load_library().rfa_rope_sincos(
-        _dev(position_ids, "position_ids", torch.int32), _dev(inv_freq, "inv_freq", torch.float32),
-        _dev(seq_lens, "seq_lens", torch.int32), batch, T, int(head_size), _TORCH_DT.get(sin_out.dtype, DT_UNDEFINED),
-        _dev(sin_out, "sin_out"), _dev(cos_out, "cos_out"), _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = load_library().rfa_rope_sincos(
+            _dev(position_ids, "position_ids", torch.int32), _dev(inv_freq, "inv_freq", torch.float32),
+            _dev(seq_lens, "seq_lens", torch.int32), batch, T, int(head_size),
+            _TORCH_DT.get(sin_out.dtype, DT_UNDEFINED), _dev(sin_out, "sin_out"), _dev(cos_out, "cos_out"),
+            _stream_ptr(stream, dev))
     _check(code, "rfa_rope_sincos")
     return sin_out, cos_out
 
@@ -283,14 +322,18 @@ def rope_apply(q: Optional[torch.Tensor], k: Optional[torch.Tensor], sin: torch.
         k_out = None
     p = RopeApplyParams(LAYOUT_TND if layout == "TND" else LAYOUT_BNSD, T, B, S, Hq, Hkv, D, io, tab,
                         1 if interleaved else 0)
+    dev = _same_device(q=q, k=k, sin=sin, cos=cos, q_out=q_out if q is not None else None, k_out=k_out,
+                       cache_slots=cache_slots, k_cache=k_cache)
     nul = ctypes.c_void_p(None)
     slots_p = _dev(cache_slots, "cache_slots", torch.int32) if cache_slots is not None else nul
     cache_p = _dev(k_cache, "k_cache", x0.dtype) if k_cache is not None else nul
     rows_cache = int(k_cache.shape[0]) if k_cache is not None else 0
-    code = load_library().rfa_rope_apply(
-        ctypes.byref(p), _dev(q, "q") if q is not None else nul, _dev(k, "k") if k is not None else nul,
-        _dev(sin, "sin"), _dev(cos, "cos"), _dev(q_out, "q_out") if q is not None else nul,
-        _dev(k_out, "k_out") if k_out is not None else nul, slots_p, cache_p, rows_cache, _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = load_library().rfa_rope_apply(
+            ctypes.byref(p), _dev(q, "q") if q is not None else nul, _dev(k, "k") if k is not None else nul,
+            _dev(sin, "sin"), _dev(cos, "cos"), _dev(q_out, "q_out") if q is not None else nul,
+            _dev(k_out, "k_out") if k_out is not None else nul, slots_p, cache_p, rows_cache,
+            _stream_ptr(stream, dev))
     _check(code, "rfa_rope_apply")
     return (q_out if q is not None else None), k_out
 
@@ -367,10 +410,12 @@ def kv_rms_norm_rope_cache(k: torch.Tensor, v: torch.Tensor, gamma: torch.Tensor
     if k_cache.dim() != 3 or tuple(k_cache.shape[1:]) != (Hkv, D) or v_cache.shape != k_cache.shape:
         raise ValueError("caches must be [rows, Hkv, D]")
     p = KvCacheParams(T, Hkv, D, io, tab, 1 if interleaved else 0, float(eps))
-    code = load_library().rfa_kv_rms_norm_rope_cache(
-        ctypes.byref(p), _dev(k, "k"), _dev(v, "v", k.dtype), _dev(gamma, "gamma", torch.float32), _dev(sin, "sin"),
-        _dev(cos, "cos"), _dev(slots, "slots", torch.int32), _dev(k_cache, "k_cache", k.dtype),
-        _dev(v_cache, "v_cache", k.dtype), int(k_cache.shape[0]), _stream_ptr(stream))
+    dev = _same_device(k=k, v=v, gamma=gamma, sin=sin, cos=cos, slots=slots, k_cache=k_cache, v_cache=v_cache)
+    with torch.cuda.device(dev):
+        code = load_library().rfa_kv_rms_norm_rope_cache(
+            ctypes.byref(p), _dev(k, "k"), _dev(v, "v", k.dtype), _dev(gamma, "gamma", torch.float32),
+            _dev(sin, "sin"), _dev(cos, "cos"), _dev(slots, "slots", torch.int32), _dev(k_cache, "k_cache", k.dtype),
+            _dev(v_cache, "v_cache", k.dtype), int(k_cache.shape[0]), _stream_ptr(stream, dev))
     _check(code, "rfa_kv_rms_norm_rope_cache")
     return k_cache, v_cache
 
@@ -397,19 +442,22 @@ def decode_rope_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
                      _TORCH_DT.get(q.dtype, DT_UNDEFINED), 1 if interleaved else 0,
                      0.0 if scale is None else float(scale), int(num_splits), float(rope_base))
     lib = load_library()
-    need = int(lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)))
-    if need == 0:
-        _check(RFA_ERR_INVALID_ARG, "rfa_decode_rope_attention_workspace")
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty_like(q)
-    io = (torch.bfloat16, torch.float16)
-    code = lib.rfa_decode_rope_attention(
-        ctypes.byref(p), _dev(q, "q", io), _dev(k_cache, "k_cache", q.dtype), _dev(v_cache, "v_cache", q.dtype),
-        _dev(q_pos, "q_pos", torch.int32), _dev(kv_lens, "kv_lens", torch.int32),
-        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(out, "out", q.dtype),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    dev = _same_device(q=q, k_cache=k_cache, v_cache=v_cache, q_pos=q_pos, kv_lens=kv_lens, inv_freq=inv_freq,
+                       out=out, workspace=workspace)
+    with torch.cuda.device(dev):
+        need = int(lib.rfa_decode_rope_attention_workspace(ctypes.byref(p)))
+        if need == 0:
+            _check(RFA_ERR_INVALID_ARG, "rfa_decode_rope_attention_workspace")
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        if out is None:
+            out = torch.empty_like(q)
+        io = (torch.bfloat16, torch.float16)
+        code = lib.rfa_decode_rope_attention(
+            ctypes.byref(p), _dev(q, "q", io), _dev(k_cache, "k_cache", q.dtype), _dev(v_cache, "v_cache", q.dtype),
+            _dev(q_pos, "q_pos", torch.int32), _dev(kv_lens, "kv_lens", torch.int32),
+            None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(out, "out", q.dtype),
+            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
     _check(code, "rfa_decode_rope_attention")
     return out
 
@@ -423,13 +471,15 @@ def rope_attention_table(q, k, position: torch.Tensor, *, layout: str = "BNSD", 
     is the same for both pairings)."""
     p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, T = _lens_arg(layout, seq_lens, p)
+    dev = _same_device(q=q, k=k, position=position, inv_freq=inv_freq, workspace=workspace)
     need = _need(p, T)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    code = load_library().rfa_rope_attention_table(
-        ctypes.byref(p), _dev(position, "position", torch.int32), _ptr_or_null(lens),
-        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        code = load_library().rfa_rope_attention_table(
+            ctypes.byref(p), _dev(position, "position", torch.int32), _ptr_or_null(lens),
+            None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(workspace, "workspace"),
+            workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
     _check(code, "rfa_rope_attention_table")
     return workspace
 
@@ -441,12 +491,15 @@ def fused_rope_attention_with_table(q, k, v, table: torch.Tensor, *, layout: str
     """The attention kernel alone, reading a table from rope_attention_table."""
     p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, T = _lens_arg(layout, seq_lens, p)
+    dev = _same_device(q=q, k=k, v=v, table=table, out=out)
     if out is None:
         out = torch.empty_like(q)
     io = (torch.bfloat16, torch.float16)
-    code = load_library().rfa_fused_rope_attention_with_table(
-        ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _ptr_or_null(lens),
-        _dev(out, "out", q.dtype), _dev(table, "table"), table.numel() * table.element_size(), _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = load_library().rfa_fused_rope_attention_with_table(
+            ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _ptr_or_null(lens),
+            _dev(out, "out", q.dtype), _dev(table, "table"), table.numel() * table.element_size(),
+            _stream_ptr(stream, dev))
     _check(code, "rfa_fused_rope_attention_with_table")
     return out
 
@@ -467,18 +520,20 @@ def fused_rope_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, posi
     """
     p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, T = _lens_arg(layout, seq_lens, p)
+    dev = _same_device(q=q, k=k, v=v, position=position, inv_freq=inv_freq, out=out, workspace=workspace)
     need = _need(p, T)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     if out is None:
         out = torch.empty_like(q)
     io = (torch.bfloat16, torch.float16)
-    code = load_library().rfa_fused_rope_attention(
-        ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
-        _dev(position, "position", torch.int32), _ptr_or_null(lens),
-        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32),
-        _dev(out, "out", q.dtype), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = load_library().rfa_fused_rope_attention(
+            ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+            _dev(position, "position", torch.int32), _ptr_or_null(lens),
+            None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32),
+            _dev(out, "out", q.dtype), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            _stream_ptr(stream, dev))
     _check(code, "rfa_fused_rope_attention")
     return out
 
@@ -494,21 +549,29 @@ def fused_rope_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     one-scratch-per-device rule)."""
     p = _params(q, k, layout, seq_lens, causal, scale, rope_base, ntk_train_len, ntk_factor, interleaved)
     lens, _ = _lens_arg(layout, seq_lens, p)
+    dev = _same_device(q=q, k=k, v=v, position=position, inv_freq=inv_freq, out=out)
     if out is None:
         out = torch.empty_like(q)
     io = (torch.bfloat16, torch.float16)
-    code = load_library().rfa_fused_rope_attention_noalloc(
-        ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
-        _dev(position, "position", torch.int32), _ptr_or_null(lens),
-        None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(out, "out", q.dtype),
-        _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = load_library().rfa_fused_rope_attention_noalloc(
+            ctypes.byref(p), _dev(q, "q", io), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+            _dev(position, "position", torch.int32), _ptr_or_null(lens),
+            None if inv_freq is None else _dev(inv_freq, "inv_freq", torch.float32), _dev(out, "out", q.dtype),
+            _stream_ptr(stream, dev))
     _check(code, "rfa_fused_rope_attention_noalloc")
     return out
 
 
-def get_device_status(stream=None) -> int:
-    """Synchronise the stream and return/clear the device status word."""
-    return int(load_library().rfa_get_device_status(_stream_ptr(stream)))
+def get_device_status(stream=None, device=None) -> int:
+    """Synchronise the stream and return/clear the status word of its device
+    (the stream's device, else `device`, else the current device)."""
+    if stream is not None:
+        device = stream.device
+    if device is None:
+        return int(load_library().rfa_get_device_status(_stream_ptr(stream)))
+    with torch.cuda.device(device):
+        return int(load_library().rfa_get_device_status(_stream_ptr(stream, torch.device(device))))
 
 
 # C names, for callers that prefer them.

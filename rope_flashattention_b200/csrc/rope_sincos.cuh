@@ -227,8 +227,9 @@ __global__ void __launch_bounds__(256) rope_seed_kernel(const __grid_constant__ 
     RopeSeed* sd = a.seeds + b;
     if (blockIdx.y == 0) {
         int ok = 1;
+        // compared in 64 bits: positions near INT32_MAX that wrap around are not consecutive
         for (int32_t i = threadIdx.x; i < len; i += blockDim.x)
-            if (__ldg(a.pos + tok0 + i) != p0 + i) ok = 0;
+            if (static_cast<int64_t>(__ldg(a.pos + tok0 + i)) != static_cast<int64_t>(p0) + i) ok = 0;
         ok = __syncthreads_and(ok);
         if (threadIdx.x == 0) {
             sd->consecutive = ok;

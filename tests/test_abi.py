@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import rope_flashattention_b200 as rfa
 
@@ -163,6 +164,19 @@ def test_product_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.lower().replace("the oracle", ""), f
+
+
+def test_binding_refuses_tensors_on_several_devices():
+    """Every pointer of a call is read on one device; the binding refuses a
+    call whose tensors sit on different GPUs (no compute, no GPU needed)."""
+    d0, d1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    assert rfa._one_device([("q", d0), ("k", d0), ("v", d0)]) == d0
+    with pytest.raises(ValueError, match="one GPU"):
+        rfa._one_device([("q", d0), ("k", d0), ("out", d1)])
+    with pytest.raises(ValueError):
+        rfa._one_device([])
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        rfa._same_device(q=torch.zeros(4), k=None)
 
 
 def _ra(**kw):

@@ -67,3 +67,30 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    import bench
+
+    args = bench.parse_args([])
+    assert args.workload == "ntk16k" and args.only is None
+    flops = {k: bench.workload_flops(w) for k, w in workloads.BY_KEY.items()}
+    assert max(flops, key=flops.get) == args.workload
+
+
+def test_both_arms_print_the_same_config():
+    """The reference arm's config dict is the one the GPU arm prints (same
+    keys and values), so the two lines describe one workload."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    import bench
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--steps", "1",
+                        "--warmup", "0"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][0])
+    assert d["config"] == json.loads(json.dumps(bench.config_of(workloads.TINY, 1)))

@@ -218,22 +218,41 @@ def test_packed_per_sequence_ntk(rfa):
     _packed(rfa, [100, 700, 300], 4, 1, 128, seed=60, ntk=(256, 2.0))
 
 
-# ---------------------------------------------------------------- full workload sizes, sampled rows
-def _sample_rows(B, Hq, lens, n, seed):
-    rng = np.random.default_rng(seed)
-    rows = []
-    for _ in range(n):
-        b = int(rng.integers(B))
-        rows.append((b, int(rng.integers(Hq)), int(rng.integers(lens[b]))))
-    for b in range(B):  # first/last rows of each sequence and of its last tile
-        L = int(lens[b])
-        for i in {0, L - 1, max(0, (L - 1) // 128 * 128), min(L - 1, 127)}:
-            rows.append((b, int(rng.integers(Hq)), i))
-    return np.array(rows, np.int32)
+# ---------------------------------------------------------------- full workload sizes, every output element
+class _Err:
+    """Max abs error and relative Frobenius error accumulated over chunks."""
+
+    def __init__(self):
+        self.max_abs, self.d2, self.r2 = 0.0, 0.0, 0.0
+
+    def add(self, got, ref):
+        got = np.asarray(got, np.float64)
+        assert np.all(np.isfinite(got))
+        d = got - ref
+        self.max_abs = max(self.max_abs, float(np.abs(d).max()))
+        self.d2 += float((d * d).sum())
+        self.r2 += float((ref * ref).sum())
+
+    def check(self):
+        fro = (self.d2 / max(self.r2, 1e-300)) ** 0.5
+        assert self.max_abs <= MAX_ABS, f"max abs {self.max_abs:.3e}"
+        assert fro <= REL_FRO, f"rel fro {fro:.3e}"
+        return self.max_abs, fro
+
+
+def _bench_path(rfa, q, k, v, pos, inv, kw):
+    """The launch sequence bench.py times: the cos/sin table kernels into a
+    workspace, then the fused attention kernel reading it."""
+    table = rfa.rope_attention_table(q, k, pos, inv_freq=inv, **kw)
+    out = rfa.fused_rope_attention_with_table(q, k, v, table, **kw)
+    assert rfa.get_device_status() == 0
+    return out
 
 
 @pytest.mark.parametrize("key", ["qwen7b", "gqa8k", "ntk16k"])
-def test_full_size_bnsd_sampled(rfa, key):
+def test_full_size_bnsd_every_element(rfa, key):
+    """The whole output of a full-size BNSD workload against the oracle, one
+    kv group of query heads at a time (every row, every column)."""
     w = workloads.BY_KEY[key]
     q, k, v = workloads.make_qkv(w)
     pos = workloads.positions(w)
@@ -242,18 +261,77 @@ def test_full_size_bnsd_sampled(rfa, key):
     if w.ntk_train_len:
         kw.update(ntk_train_len=w.ntk_train_len, ntk_factor=w.ntk_factor)
         ntk = (w.ntk_train_len, w.ntk_factor)
-    out = rfa.fused_rope_attention(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), **kw)
-    assert rfa.get_device_status() == 0
-    got = out.float().cpu().numpy()
-    assert np.all(np.isfinite(got))
-    rows = _sample_rows(w.B, w.Hq, [w.S] * w.B, 96, seed=w.seed)
+    got = _bench_path(rfa, q.cuda(), k.cuda(), v.cuda(), pos.cuda(), None, kw).float().cpu().numpy()
     inv = _inv_rows(w.B, w.D, w.rope_base, [w.S] * w.B, ntk)
-    ref = oracle.attention_rows(q, k, v, pos.numpy(), inv, rows)
+    G = w.Hq // w.Hkv
+    err = _Err()
+    for b in range(w.B):
+        for kvh in range(w.Hkv):
+            heads = np.arange(kvh * G, (kvh + 1) * G)
+            hh, ii = np.meshgrid(heads, np.arange(w.S), indexing="ij")
+            rows = np.stack([np.full(hh.size, b), hh.ravel(), ii.ravel()], axis=1).astype(np.int32)
+            ref = oracle.attention_rows(q, k, v, pos.numpy(), inv, rows)
+            err.add(got[b, heads].reshape(-1, w.D), ref)
+    err.check()
+
+
+def test_full_size_packed_every_element(rfa):
+    """The whole output of the packed workload (16 sequences, T = 57,209,
+    per-sequence invFreq rows) against the oracle, one sequence and kv group
+    at a time."""
+    w = workloads.PACKED
+    lens = workloads.seq_lengths(w)
+    q, k, v = workloads.make_qkv(w)
+    pos = workloads.positions(w)
+    inv_t = workloads.random_inv_freq(w)
+    kw = dict(layout="TND", seq_lens=lens, rope_base=w.rope_base)
+    got = _bench_path(rfa, q.cuda(), k.cuda(), v.cuda(), pos.cuda(), inv_t.cuda(), kw).float().cpu().numpy()
+    inv = inv_t.double().numpy()
+    t0 = np.concatenate([[0], np.cumsum(lens)])
+    G = w.Hq // w.Hkv
+    err = _Err()
+    for b in range(w.B):
+        for kvh in range(w.Hkv):
+            heads = np.arange(kvh * G, (kvh + 1) * G)
+            hh, ii = np.meshgrid(heads, np.arange(lens[b]), indexing="ij")
+            rows = np.stack([np.full(hh.size, b), hh.ravel(), ii.ravel()], axis=1).astype(np.int32)
+            ref = oracle.attention_rows(q, k, v, pos.numpy(), inv, rows, layout=oracle.TND, seq_lens=lens)
+            err.add(got[t0[b] + rows[:, 2], rows[:, 1]], ref)
+    err.check()
+
+
+def test_long_sequence_65536_last_tiles(rfa):
+    """S = 65536 (512 key tiles): the key angles advance through 512 steps of
+    the recurrence.  Every row of the last two query tiles (which read all 512
+    key tiles) and one seeded row of every other query tile, both heads."""
+    B, Hq, Hkv, S, D = 1, 2, 1, 65536, 128
+    base = 500000.0
+    q = workloads.randn16((B, Hq, S, D), 301)
+    k = workloads.randn16((B, Hkv, S, D), 302)
+    v = workloads.randn16((B, Hkv, S, D), 303)
+    pos = torch.arange(S, dtype=torch.int32)[None].contiguous()
+    kw = dict(layout="BNSD", rope_base=base)
+    got = _bench_path(rfa, q.cuda(), k.cuda(), v.cuda(), pos.cuda(), None, kw).float().cpu().numpy()
+    rng = np.random.default_rng(304)
+    rows = []
+    for h in range(Hq):
+        rows += [(0, h, i) for i in range(S - 256, S)]
+        rows += [(0, h, t * 128 + int(rng.integers(128))) for t in range(S // 128 - 2)]
+    rows = np.array(rows, np.int32)
+    ref = oracle.attention_rows(q, k, v, pos.numpy(), _inv_rows(B, D, base), rows)
     _compare(got[rows[:, 0], rows[:, 1], rows[:, 2]], ref)
 
 
-def test_full_size_packed_sampled(rfa):
-    w = workloads.PACKED
-    lens = workloads.seq_lengths(w)
-    rows = _sample_rows(w.B, w.Hq, lens, 96, seed=w.seed)
-    _packed(rfa, lens, w.Hq, w.Hkv, w.D, seed=w.seed, random_inv=True, rows=rows)
+def test_positions_wrapping_past_int32_max(rfa):
+    """Positions p0 + i counted past INT32_MAX wrap to negative int32 values,
+    so the sequence's positions are not consecutive and its keys must take
+    their angles from the table, not the recurrence (which would continue past
+    the wrap, 2^32 * invFreq radians away).  Small inverse frequencies keep the
+    angles of positions near 2^31 accurate in fp32."""
+    B, Hq, Hkv, S, D = 1, 2, 1, 300, 128
+    p0 = 2**31 - 150
+    wrapped = (torch.arange(S, dtype=torch.int64) + p0 + 2**31) % 2**32 - 2**31
+    pos = wrapped.to(torch.int32)[None].contiguous()
+    assert int(pos[0, -1]) < 0 < int(pos[0, 0])
+    inv = (torch.linspace(0.5, 1.0, D // 2) * 1e-9)[None].to(torch.float32).contiguous()
+    full_bnsd(rfa, B, Hq, Hkv, S, D, seed=310, pos=pos, inv=inv)

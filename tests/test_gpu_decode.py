@@ -127,3 +127,23 @@ def test_two_chain_merge_d64_fp16_noncausal(rfa):
                          num_splits=2)
     assert st == 0
     _compare(got, ref)
+
+
+def test_benchmarked_shape_32k_keys(rfa):
+    """The shape bench.py times: 8 sequences x 32 query / 8 kv heads, one new
+    token each, over 32768 cached keys, with the library's own split plan.
+    Every output row (all 8 x 32) against the oracle, one sequence at a time
+    so the fp64 copy of the cache stays small."""
+    B, Hq, Hkv, Sq, D, L = 8, 32, 8, 1, 128, 32768
+    q = workloads.randn16((B, Hq, Sq, D), 41)
+    kc = workloads.randn16((B, L, Hkv, D), 42)
+    vc = workloads.randn16((B, L, Hkv, D), 43)
+    q_pos = torch.full((B, Sq), L - 1, dtype=torch.int32)
+    lens = torch.full((B,), L, dtype=torch.int32)
+    out = rfa.decode_rope_attention(q.cuda(), kc.cuda(), vc.cuda(), q_pos.cuda(), lens.cuda())
+    assert rfa.get_device_status() == 0
+    got = out.float().cpu().numpy().astype(np.float64)
+    inv = oracle.inv_freq(10000.0, D)[None]
+    ref = np.concatenate([oracle.decode_attention(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], q_pos[b:b + 1].numpy(), [L],
+                                                  inv) for b in range(B)])
+    _compare(got, ref)

@@ -3,9 +3,11 @@
 Plausible mistakes are planted, one at a time, in copies of the oracle's
 sources: a flipped sign, a wrong index or partner, a dropped term, an operand
 taken from the wrong row or segment.  A C mutant is compiled with the oracle's
-own gcc flags and loaded through the oracle's RFA_ORACLE_LIB hook; a Python
-mutant (the numpy parts of the oracle) is a copy of the package module that a
-small pytest plugin installs as `oracle` before the tests import it.  The CPU
+own gcc flags; a Python mutant (the numpy parts of the oracle) is a copy of
+the package module.  A small pytest plugin, loaded only in the subprocesses
+this test starts, installs the mutant before the pins import `oracle`: it
+sets the oracle's library override (a module attribute) to the compiled C
+mutant, or installs the Python mutant as `oracle`.  The CPU
 pin suites then run against each mutant in a subprocess.  Every mutant must
 make at least one pin fail (pytest exit status 1), while unmodified copies
 pass them all, which shows that the harness itself works.  Nothing here
@@ -50,6 +52,12 @@ MUTANTS = [
     ("rms_norm_mean_dropped", "sqrt(ss / (double)D + eps)", "sqrt(ss + eps)"),
     ("rms_norm_gamma_dropped", "out[r * D + j] = gamma[j] * (x[r * D + j] * inv);",
      "out[r * D + j] = (x[r * D + j] * inv);"),
+    ("probs_scale_dropped", "p[j] = acc * d->scale;", "p[j] = acc;"),
+    ("probs_gqa_head_map", "const int32_t D = d->D, G = d->Hq / d->Hkv, kvh = h / G;",
+     "const int32_t D = d->D, G = d->Hq / d->Hkv, kvh = h % d->Hkv;"),
+    ("probs_key_at_query_position", "rotate_row(d, x, pk, inv, kr);", "rotate_row(d, x, pq, inv, kr);"),
+    ("probs_causal_diagonal_dropped", "int32_t jmax = d->causal ? i + 1 : len;",
+     "int32_t jmax = d->causal ? i : len;"),
 ]
 
 
@@ -65,10 +73,14 @@ PY_MUTANTS = [
 ]
 
 PLUGIN = """import importlib.util, os, sys
-_spec = importlib.util.spec_from_file_location("oracle", os.environ["RFA_ORACLE_PY"])
-_mod = importlib.util.module_from_spec(_spec)
-sys.modules["oracle"] = _mod
-_spec.loader.exec_module(_mod)
+if os.environ.get("RFA_MUTANT_PY"):
+    _spec = importlib.util.spec_from_file_location("oracle", os.environ["RFA_MUTANT_PY"])
+    _mod = importlib.util.module_from_spec(_spec)
+    sys.modules["oracle"] = _mod
+    _spec.loader.exec_module(_mod)
+else:
+    import oracle as _mod
+_mod._lib_override = os.environ["RFA_MUTANT_LIB"]
 """
 
 
@@ -80,14 +92,14 @@ def _compile(src: str, path: str) -> None:
 
 
 def _run_pins(lib: str, py=None, plugin_dir=None):
-    env = dict(os.environ, RFA_ORACLE_LIB=lib)
-    extra = []
+    env = dict(os.environ, RFA_MUTANT_LIB=lib)
+    env.pop("RFA_MUTANT_PY", None)
     if py is not None:
-        env["RFA_ORACLE_PY"] = py
-        env["PYTHONPATH"] = os.pathsep.join([plugin_dir] + [p for p in [os.environ.get("PYTHONPATH")] if p])
-        extra = ["-p", "rfa_oracle_mutant_plugin"]
+        env["RFA_MUTANT_PY"] = py
+    env["PYTHONPATH"] = os.pathsep.join([ROOT, plugin_dir] + [p for p in [os.environ.get("PYTHONPATH")] if p])
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "not gpu", "-p", "no:cacheprovider",
-                        *extra, *PIN_SUITES], cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+                        "-p", "rfa_oracle_mutant_plugin", *PIN_SUITES], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=900)
     return r.returncode, (r.stdout + r.stderr)[-1500:]
 
 

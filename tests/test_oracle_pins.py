@@ -276,6 +276,47 @@ def test_probability_rows_sum_to_one_and_respect_causality():
         assert abs(pn.sum() - 1.0) < 1e-14 and np.all(pn > 0)
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_probability_rows_match_complex_rope_and_torch_softmax(causal):
+    """Every row P[b, h, i, :] equals torch.softmax (a library routine) of the
+    scores of numpy's complex rotation of q and k (another route to the same
+    rotation), in fp64: the scale, the rotation, the GQA kv head h // G, the
+    causal edge and the position offsets of each batch all enter."""
+    q, k, v, pos = _small(S=29, seed=40)
+    pos = pos + np.array([[5], [-17]], np.int32)
+    inv = np.stack([oracle.inv_freq(10000.0, 64), oracle.inv_freq(300.0, 64)])
+    scale = 0.09
+
+    def crot(x, b):
+        x = x.double().numpy()
+        z = (x[..., :32] + 1j * x[..., 32:]) * np.exp(1j * pos[b][:, None] * inv[b][None, :])
+        return np.concatenate([z.real, z.imag], axis=-1)
+
+    G = q.shape[1] // k.shape[1]
+    S = q.shape[2]
+    for b in range(2):
+        qr, kr = crot(q[b], b), crot(k[b], b)
+        for h in range(q.shape[1]):
+            sc = torch.from_numpy(qr[h] @ kr[h // G].T * scale)
+            if causal:
+                sc = sc.masked_fill(torch.ones(S, S, dtype=torch.bool).triu(1), float("-inf"))
+            ref = torch.softmax(sc, dim=-1).numpy()
+            for i in (0, 11, S - 1):
+                got = oracle.attention_probs(q, k, pos, inv, b, h, i, causal=causal, scale=scale)
+                np.testing.assert_allclose(got, ref[i], atol=1e-13, rtol=0)
+
+
+def test_probability_rows_weight_the_values_into_the_output():
+    """P[b, h, i, :] @ V[b, h // G] is the pinned attention output row."""
+    q, k, v, pos = _small(S=31, seed=41)
+    inv = np.stack([oracle.inv_freq(10000.0, 64)] * 2)
+    out = oracle.attention_full(q, k, v, pos, inv)
+    vv = v.double().numpy()
+    for (b, h, i) in [(0, 0, 30), (1, 3, 12), (1, 2, 0)]:
+        p = oracle.attention_probs(q, k, pos, inv, b, h, i)
+        np.testing.assert_allclose(p @ vv[b, h // 2], out[b, h, i], atol=1e-13)
+
+
 def test_constant_values_give_constant_output():
     q, k, _, pos = _small(S=50)
     v = torch.full((2, 2, 50, 64), 0.75, dtype=torch.bfloat16)
