@@ -266,10 +266,14 @@ RFA_API size_t rfa_fused_rope_attention_workspace(const rfa_attn_params* p, int6
  *   workspace  dev   >= rfa_fused_rope_attention_workspace(p, T) bytes,
  *                    256-byte aligned; holds the cos/sin table of this call
  *                    (T*D*2 bytes: D/2 fp16 cos and D/2 fp16 sin values per
- *                    token) and per-sequence angle-recurrence seeds (9232
- *                    bytes each) -- tables, never rotated Q/K
- * Rotated Q and K exist only in shared memory.  The call enqueues two
- * kernels: the cos/sin table and the fused attention.
+ *                    token), per-sequence angle seeds (784 bytes
+ *                    each) -- tables, never rotated Q/K -- and, in its
+ *                    last 256 bytes, the attention kernel's two work counters
+ * Rotated Q and K exist only in shared memory.  The call enqueues the cos/sin
+ * table kernels (which zero the work counters) and the fused attention kernel:
+ * a persistent grid of one CTA per SM taking work items from the counters (its
+ * last CTA leaves them at zero).  Calls that share a workspace must not
+ * overlap on the GPU.
  */
 RFA_API rfa_status rfa_fused_rope_attention(const rfa_attn_params* p, const void* q, const void* k, const void* v,
                                     const int32_t* position, const int32_t* seqLens_host,
@@ -287,7 +291,9 @@ RFA_API rfa_status rfa_fused_rope_attention(const rfa_attn_params* p, const void
  *   rfa_fused_rope_attention.
  * rfa_fused_rope_attention_with_table: the attention kernel alone, reading a
  *   table that rfa_rope_attention_table wrote for the same p, positions and
- *   seqLens_host.  The workspace is only read.
+ *   seqLens_host.  The table and seeds are only read; the work counters are
+ *   used and left at zero, so the table can serve any number of calls, one
+ *   after another (calls sharing the workspace must not overlap on the GPU).
  * rfa_fused_rope_attention == rfa_rope_attention_table followed by
  * rfa_fused_rope_attention_with_table on the same stream.
  */
@@ -296,7 +302,7 @@ RFA_API rfa_status rfa_rope_attention_table(const rfa_attn_params* p, const int3
                                             size_t ws_bytes, void* stream);
 RFA_API rfa_status rfa_fused_rope_attention_with_table(const rfa_attn_params* p, const void* q, const void* k,
                                                        const void* v, const int32_t* seqLens_host, void* out,
-                                                       const void* workspace, size_t ws_bytes, void* stream);
+                                                       void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * rfa_fused_rope_attention_noalloc -- rfa_fused_rope_attention without a
@@ -308,8 +314,8 @@ RFA_API rfa_status rfa_fused_rope_attention_with_table(const rfa_attn_params* p,
  * of this library.)
  *
  * Arguments and results are those of rfa_fused_rope_attention minus
- * workspace/ws_bytes.  The scratch (cos/sin table and recurrence seeds) is a
- * fixed area of about 16.1 MB inside the library's module, held by every
+ * workspace/ws_bytes.  The scratch (cos/sin table, recurrence seeds and work
+ * counters) is a fixed area of about 16.8 MB inside the library's module, held by every
  * device that loads the library until the process exits.  Limits: at most
  * 65536 tokens (BNSD: B*S), at most 16 sequences (BNSD: batches), D <= 128;
  * larger problems return RFA_ERR_WORKSPACE before anything is enqueued.

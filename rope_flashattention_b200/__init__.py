@@ -19,6 +19,7 @@ Entry points (C name without the ``rfa_`` prefix):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -27,7 +28,7 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = [
-    "RfaError", "LIB_PATH", "EXPORTS", "load_library", "rope_sincos", "fused_rope_attention",
+    "RfaError", "LIB_PATH", "CHECKED_LIB_PATH", "EXPORTS", "load_library", "use_library", "rope_sincos", "fused_rope_attention",
     "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
     "fused_rope_attention_noalloc", "rope_apply", "kv_rms_norm_rope_cache", "KvCacheParams",
     "decode_rope_attention", "DecodeParams",
@@ -35,6 +36,8 @@ __all__ = [
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa.so")
+# the bounds-checked build of the same sources (see use_library)
+CHECKED_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa_checked.so")
 
 # Every symbol include/rfa.h declares.
 EXPORTS = (
@@ -142,9 +145,28 @@ def load_library():
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"librfa.so is not built ({LIB_PATH}); run __graft_entry__.build()")
-    lib = ctypes.CDLL(LIB_PATH)
+    _lib = _open(LIB_PATH)
+    return _lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Run this module's calls against another build of the library for the
+    duration of the block -- e.g. librfa_checked.so, the same sources compiled
+    with every device-side index bounds-checked (RFA_CHECKED)."""
+    global _lib
+    prev = load_library()
+    _lib = _open(path)
+    try:
+        yield _lib
+    finally:
+        _lib = prev
+
+
+def _open(path: str):
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} is not built ({path}); run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     lib.rfa_rope_sincos.argtypes = [P, P, P, I32, I32, I32, ctypes.c_int, P, P, P]
     lib.rfa_rope_sincos.restype = ctypes.c_int
@@ -174,7 +196,6 @@ def load_library():
     lib.rfa_status_string.restype = ctypes.c_char_p
     lib.rfa_version.argtypes = []
     lib.rfa_version.restype = I32
-    _lib = lib
     return lib
 
 

@@ -10,6 +10,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librfa.so")
+# the same sources compiled with -DRFA_CHECKED: every computed index bounds-checked
+# on the device (errors to the status word), for the checked GPU tests
+LIB_CHECKED = os.path.join(PKG, "librfa_checked.so")
 SOURCES = [os.path.join(CSRC, "rfa_api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(ROOT, "include", "rfa.h")
@@ -33,26 +36,27 @@ def flags(extra=()):
     ]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in DEPS)
 
 
-def build_library(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *flags(extra), "-shared", "-o", tmp, *SOURCES]
+def build_library(force: bool = False, verbose: bool = False, extra=(), checked: bool = False) -> str:
+    """Compile librfa.so (or, checked=True, librfa_checked.so with -DRFA_CHECKED)."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *flags(tuple(extra) + (("-DRFA_CHECKED",) if checked else ())), "-shared", "-o", tmp, *SOURCES]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build_library(force="--force" in sys.argv, verbose=True,
-                  extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ())
-    print(LIB)
+    extra = ("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ()
+    print(build_library(force="--force" in sys.argv, verbose=True, extra=extra, checked="--checked" in sys.argv))

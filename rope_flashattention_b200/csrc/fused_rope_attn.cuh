@@ -74,6 +74,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only if the 
 struct AttnArgs {
     void* out;
     const RopeSeed* seeds;  // [sequences] in the caller's order
+    const uint32_t* table;  // [tokens][D/2] cos/sin words (query rows of sequences whose positions are not consecutive)
+    int32_t* sched;         // two work counters (next item, CTAs done), zero at launch; the last CTA re-zeroes them
     int32_t layout;  // 0 BNSD, 1 TND
     int32_t B, Hq, Hkv, G;
     int32_t S;       // BNSD sequence length
@@ -99,6 +101,9 @@ struct AttnArgs {
     const int32_t* kv_lens;  // [B] keys in each sequence's cache, Sq <= len <= dec_max_len
     float* part_o;           // splits > 1: [splits][B*Hq*Sq][D] unnormalised O
     float* part_ml;          // splits > 1: [splits][B*Hq*Sq][2] (running max, row sum)
+    // extents, for the checks of the bounds-checked build (RFA_CHECKED)
+    int64_t out_elems;       // elements of out
+    int32_t ntok;            // tokens of q/k/v and rows of the table (decode: cache rows B * Smax)
 };
 
 // Work items of one sequence with nt query tiles.
@@ -122,9 +127,12 @@ struct AttnCfg {
     static constexpr int kOffT = kOffV + kStages * kTileBytes;
     static constexpr int kOffBar = kOffT + kTStages * kTabBytes;
     // barrier indices
-    static constexpr int kBarQFull = 0;  // both query tiles and their cos/sin rows landed
-    static constexpr int kBarQReady = 1; // both rotated (8 RoPE warp arrivals); their rows' V slots are free
-    static constexpr int kBarKFull = 2;
+    static constexpr int kBarQFull = 0;  // the item's query tiles landed (decode: and their cos/sin rows)
+    static constexpr int kBarQReady = 1; // both rotated (4 RoPE warp arrivals)
+    static constexpr int kBarQEmpty = 2; // the item's last QK MMAs are done: the query slots may be reloaded
+    static constexpr int kBarItemFull = 3;   // 2: item index published in the slot
+    static constexpr int kBarItemEmpty = 5;  // 2: every consumer warp has read the slot
+    static constexpr int kBarKFull = 7;
     static constexpr int kBarVFull = kBarKFull + kStages;
     static constexpr int kBarKReady = kBarVFull + kStages;
     static constexpr int kBarKEmpty = kBarKReady + kStages;
@@ -136,7 +144,8 @@ struct AttnCfg {
     static constexpr int kNumBars = kBarMmaFin + 1;
     static constexpr int kOffAbort = kOffBar + 8 * kNumBars;
     static constexpr int kOffTmemSlot = kOffAbort + 16;
-    static constexpr int kOffXchg = kOffTmemSlot + 16;  // float [2 query tiles][2 column halves][128 rows]
+    static constexpr int kOffItem = kOffTmemSlot + 16;  // int32 [2]: the item ring
+    static constexpr int kOffXchg = kOffItem + 16;      // float [2 query tiles][2 column halves][128 rows]
     // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (the
     // kernel checks it), so no alignment slack is requested.
     static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBlockM * 4;
@@ -145,7 +154,7 @@ struct AttnCfg {
     static constexpr uint32_t kColS = 0;      // S_i at 128 i
     static constexpr uint32_t kColO = 256;    // O_i at 256 + D i
     static_assert(kColO + 2 * D <= kTmemCols, "TMEM budget");
-    static_assert(kStages >= 2 && kTabBytes == kTileBytes, "query cos/sin rows are staged in V slots 0 and 1");
+    static_assert(kStages >= 2 && kTabBytes == kTileBytes, "decode stages its query rows' cos/sin in a query slot");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -245,6 +254,20 @@ __device__ __forceinline__ WorkItem decode_item(const AttnArgs& a, int32_t x) {
     }
     w.kvh = w.h[0] / a.G;
     return w;
+}
+
+// Checked build: a work item's indices lie inside the problem.
+__device__ __forceinline__ bool item_in_bounds(const AttnArgs& a, const WorkItem& w, bool decode) {
+    if (decode)
+        return in_bounds(w.seq >= 0 && w.seq < a.B && w.kvh >= 0 && w.kvh < a.Hkv && w.split >= 0 &&
+                         w.split < a.dec_splits && w.qrow0 >= 0 &&
+                         static_cast<int64_t>(w.qrow0) + a.G * a.dec_Sq <= static_cast<int64_t>(a.B) * a.Hq * a.dec_Sq &&
+                         w.tok0 >= 0 && static_cast<int64_t>(w.tok0) + w.L <= a.ntok);
+    const int32_t nseq = a.layout == 0 ? a.B : a.nseg;
+    return in_bounds(w.seq >= 0 && w.seq < nseq && w.orig >= 0 && w.orig < a.B && w.h[0] >= 0 && w.h[1] < a.Hq &&
+                     w.kvh >= 0 && w.kvh < a.Hkv && w.h[0] / a.G == w.kvh && w.h[1] / a.G == w.kvh &&
+                     w.qt[0] >= 0 && w.qt[0] * kBlockM < w.L && w.qt[1] * kBlockM < w.L && w.L >= 1 &&
+                     w.tok0 >= 0 && static_cast<int64_t>(w.tok0) + w.L <= a.ntok);
 }
 
 template <bool kFP16>
@@ -352,6 +375,11 @@ __device__ __forceinline__ void task_chunks(uint32_t tile, int32_t r, int cp, ui
     o1 = chunk_addr<D>(tile, r, kAdj ? 2 * cp : cp);
     o2 = chunk_addr<D>(tile, r, kAdj ? 2 * cp + 1 : cp + D / 16);
 }
+// Checked build: a task's row and chunk pair lie inside its 128-row tile.
+template <int D>
+__device__ __forceinline__ bool task_in_tile(int32_t r, int cp) {
+    return in_bounds(r >= 0 && r < kBlockM && cp >= 0 && cp < D / 16);
+}
 
 // Rotate the first `rows` rows of a 128-row tile in shared memory with the
 // cos/sin rows staged at `tab`.  128B swizzle: 16-byte chunk c of row r sits at
@@ -366,7 +394,7 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t r
         const int task = rt + kRopeThreads * it;
         const int r = task / kPairsPerRow;
         const int cp = task % kPairsPerRow;
-        if (r >= rows) continue;
+        if (r >= rows || !task_in_tile<D>(r, cp)) continue;
         const uint32_t sw = static_cast<uint32_t>(r & 7);
         uint32_t o1, o2;
         task_chunks<D, kAdj>(tile, r, cp, o1, o2);
@@ -406,7 +434,33 @@ __device__ __forceinline__ void rec_step(uint64_t& c, uint64_t& s, uint64_t wc, 
     c = cn;
 }
 
-// Rotate a key tile whose rows hold consecutive positions, without a table.
+// Rotate one task's two chunks with the angles of `e` (4 packed pairs of
+// frequencies 8cp .. 8cp+7).
+template <bool kFP16, bool kAdj>
+__device__ __forceinline__ void rotate8_state(uint4& x1, uint4& x2, const RecState& e) {
+    uint32_t* xa = reinterpret_cast<uint32_t*>(&x1);
+    uint32_t* xb = reinterpret_cast<uint32_t*>(&x2);
+    if constexpr (kAdj) {
+        // word k of x1 is pair 8cp + k, of x2 pair 8cp + 4 + k
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 ca = f2unpack(e.c[k >> 1]), sa = f2unpack(e.s[k >> 1]);
+            const float2 cb = f2unpack(e.c[2 + (k >> 1)]), sb = f2unpack(e.s[2 + (k >> 1)]);
+            xa[k] = rot_adj<kFP16>(xa[k], (k & 1) ? ca.y : ca.x, (k & 1) ? sa.y : sa.x);
+            xb[k] = rot_adj<kFP16>(xb[k], (k & 1) ? cb.y : cb.x, (k & 1) ? sb.y : sb.x);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint64_t X1 = IoT<kFP16>::unpack2(xa[k]);
+            const uint64_t X2 = IoT<kFP16>::unpack2(xb[k]);
+            xa[k] = pack2<kFP16>(fsub2(fmul2(X1, e.c[k]), fmul2(X2, e.s[k])));  // x1 cos - x2 sin
+            xb[k] = pack2<kFP16>(ffma2(X2, e.c[k], fmul2(X1, e.s[k])));        // x2 cos + x1 sin
+        }
+    }
+}
+
+// Rotate a tile whose rows hold consecutive positions, without a table.
 // This thread's rows are r0, r0 + step, ...; z holds the angles of row r0 and
 // (wc, ws) advance them by `step` rows.
 template <int D, bool kFP16, bool kAdj>
@@ -423,30 +477,11 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
 #pragma unroll 2
     for (int it = 0; it < kIters; ++it) {
         const int r = r0 + it * kStep;
-        if (r < rows) {
+        if (r < rows && task_in_tile<D>(r, cp)) {
             uint32_t o1, o2;
             task_chunks<D, kAdj>(tile, r, cp, o1, o2);
             uint4 x1 = lds128(o1), x2 = lds128(o2);
-            uint32_t* xa = reinterpret_cast<uint32_t*>(&x1);
-            uint32_t* xb = reinterpret_cast<uint32_t*>(&x2);
-            if constexpr (kAdj) {
-                // word k of x1 is pair 8cp + k, of x2 pair 8cp + 4 + k
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 ca = f2unpack(e.c[k >> 1]), sa = f2unpack(e.s[k >> 1]);
-                    const float2 cb = f2unpack(e.c[2 + (k >> 1)]), sb = f2unpack(e.s[2 + (k >> 1)]);
-                    xa[k] = rot_adj<kFP16>(xa[k], (k & 1) ? ca.y : ca.x, (k & 1) ? sa.y : sa.x);
-                    xb[k] = rot_adj<kFP16>(xb[k], (k & 1) ? cb.y : cb.x, (k & 1) ? sb.y : sb.x);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t X1 = IoT<kFP16>::unpack2(xa[k]);
-                    const uint64_t X2 = IoT<kFP16>::unpack2(xb[k]);
-                    xa[k] = pack2<kFP16>(fsub2(fmul2(X1, e.c[k]), fmul2(X2, e.s[k])));  // x1 cos - x2 sin
-                    xb[k] = pack2<kFP16>(ffma2(X2, e.c[k], fmul2(X1, e.s[k])));        // x2 cos + x1 sin
-                }
-            }
+            rotate8_state<kFP16, kAdj>(x1, x2, e);
             sts128(o1, x1);
             sts128(o2, x2);
         }
@@ -454,6 +489,64 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
 #pragma unroll
             for (int k = 0; k < 4; ++k) rec_step(e.c[k], e.s[k], wc[k], ws[k]);
         }
+    }
+}
+
+// Recurrence state of RoPE thread rt for row r0 = rt / (D/16) of a sequence's
+// first tile (angles (P + r0) w for its 8 frequencies), and the step (wc, ws)
+// of kStep rows, both from the sequence's seeds.
+// Angles of row `row` (relative to the sequence's first position P) for the
+// 8 frequencies w[0..7] of a RoPE thread: the angle (P + row) w is formed in
+// fp64 (exact for the fp32 w and any int32 P), reduced modulo 2 pi in fp64,
+// and its cos/sin taken on the SFU -- the seeds' method, so a query tile's
+// first rows are as accurate as the key tiles' seeds.
+__device__ __forceinline__ void angles_at(int32_t P, int32_t row, const float (&w)[8], RecState& z) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double inv_two_pi = 0.15915494309189533576888376337251;
+    const double p = static_cast<double>(P) + static_cast<double>(row);
+    float c[8], sn[8];
+#pragma unroll
+    for (int f = 0; f < 8; ++f) {
+        const double a = p * static_cast<double>(w[f]);
+        const double r = fma(-two_pi, rint(a * inv_two_pi), a);
+        __sincosf(static_cast<float>(r), &sn[f], &c[f]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        z.c[k] = f2pack(c[2 * k], c[2 * k + 1]);
+        z.s[k] = f2pack(sn[2 * k], sn[2 * k + 1]);
+    }
+}
+
+// Rotate the first `rows` rows of a tile with cos/sin rows read from the
+// global table (tab points at the tile's first row; D/2 32-bit words per row,
+// laid out as rope_table_kernel writes them).
+template <int D, bool kFP16, bool kAdj>
+__device__ __forceinline__ void rope_tile_global(uint32_t tile, const uint32_t* tab, int32_t rows, int32_t rt) {
+    constexpr int kPairsPerRow = D / 16;
+    constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
+    constexpr int kStep = kRopeThreads / kPairsPerRow;
+    const int cp = rt % kPairsPerRow;
+    const int r0 = rt / kPairsPerRow;
+    // chunk positions of frequencies 8cp..8cp+3 and 8cp+4..8cp+7 within a row
+    const int g0 = (D == 128) ? cp : 2 * cp;
+    const int g1 = (D == 128) ? 8 + cp : 2 * cp + 1;
+#pragma unroll 2
+    for (int it = 0; it < kIters; ++it) {
+        const int r = r0 + it * kStep;
+        if (r >= rows) break;
+        if (!task_in_tile<D>(r, cp) || !in_bounds(g0 < D / 8 && g1 < D / 8)) continue;
+        const uint4* row = reinterpret_cast<const uint4*>(tab + static_cast<int64_t>(r) * (D / 2));
+        const uint4 t0 = __ldg(row + g0), t1 = __ldg(row + g1);
+        uint32_t o1, o2;
+        task_chunks<D, kAdj>(tile, r, cp, o1, o2);
+        uint4 x1 = lds128(o1), x2 = lds128(o2);
+        if constexpr (kAdj)
+            rotate8_adj<kFP16>(x1, x2, t0, t1);
+        else
+            rotate8<kFP16>(x1, x2, t0, t1);
+        sts128(o1, x1);
+        sts128(o2, x2);
     }
 }
 
@@ -490,6 +583,30 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 }
 
 
+// Key-tile counts of a work item: n0 / n1 key tiles read by query tile 0 / 1
+// (0: tile absent), n_kv key tiles loaded.  Decode has one query tile and two
+// independent chains over alternate key tiles: tile j goes to S/O buffer
+// j % 2, and the two buffers' results are merged before the store.
+struct ItemShape {
+    int32_t nq, n0, n1, n_kv;
+};
+template <bool kDecode>
+__device__ __forceinline__ ItemShape item_shape(const AttnArgs& a, const WorkItem& w) {
+    ItemShape sh;
+    sh.nq = (w.qt[1] >= 0) ? 2 : 1;
+    const int32_t nkt = (w.L + kBlockN - 1) / kBlockN;
+    sh.n0 = kDecode ? (nkt + 1) / 2 : (a.causal ? (w.qt[0] + 1) : nkt);
+    sh.n1 = kDecode ? nkt / 2 : ((sh.nq == 1) ? 0 : (a.causal ? (w.qt[1] + 1) : nkt));
+    sh.n_kv = kDecode ? nkt : max(sh.n0, sh.n1);
+    return sh;
+}
+
+// Persistent: one CTA per SM takes work items one after another from a shared
+// counter (decode: one CTA per item).  The Q/K producer fetches the item
+// indices and passes them to the other roles through a two-slot ring in
+// shared memory; every barrier phase runs on across items, so the next item's
+// key tiles and query tiles load (and rotate) while the current item's last
+// tiles are still in the softmax and the tensor pipe.
 template <int D, bool kFP16, bool kAdj, bool kDecode>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     fused_rope_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -506,39 +623,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t* smem = smem_raw;
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + C::kOffAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmemSlot);
+    volatile int32_t* item_slot = reinterpret_cast<volatile int32_t*>(smem + C::kOffItem);
     auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * static_cast<uint32_t>(i); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const WorkItem w = kDecode ? decode_item_kv(a, blockIdx.x) : decode_item(a, blockIdx.x);
-    const int32_t nq = (w.qt[1] >= 0) ? 2 : 1;  // query tiles in this item
-    const int32_t nkt = (w.L + kBlockN - 1) / kBlockN;
-    // key tiles read by query tile i (0: tile absent).  Decode has one query tile and two
-    // independent chains over alternate key tiles: tile j goes to S/O buffer j % 2, and the
-    // two buffers' results are merged before the store.
-    const int32_t n0 = kDecode ? (nkt + 1) / 2 : (a.causal ? (w.qt[0] + 1) : nkt);
-    const int32_t n1 = kDecode ? nkt / 2 : ((nq == 1) ? 0 : (a.causal ? (w.qt[1] + 1) : nkt));
-    const int32_t n_kv = kDecode ? nkt : max(n0, n1);
-    // consecutive positions: K angles come from the recurrence, no cos/sin rows per K tile
-    // (decode: the cached keys are already rotated)
-    const bool rec = !kDecode && a.seeds[w.orig].consecutive != 0;
     if constexpr (kDecode) {
+        const WorkItem w = decode_item_kv(a, blockIdx.x);
         if (threadIdx.x == 0 && w.split == 0) {
             const int32_t len = a.kv_lens[w.seq];
             if (len < a.dec_Sq || len > a.dec_max_len) record_status(1 /* RFA_ERR_INVALID_ARG */);
         }
-        if (n_kv == 0) {
+        if (w.L <= 0) {
             // no keys in this split (past the sequence's length): an empty partial, or, with
             // one split, zero rows; the CTA returns before any barrier or TMEM is set up
             const int32_t rq = a.Hq * a.dec_Sq * a.B;
             for (int r = threadIdx.x; r < a.G * a.dec_Sq; r += blockDim.x) {
                 if (a.dec_splits > 1) {
                     const int64_t pr = static_cast<int64_t>(w.split) * rq + w.qrow0 + r;
+                    if (!in_bounds(pr >= 0 && pr < static_cast<int64_t>(a.dec_splits) * rq)) continue;
                     a.part_ml[2 * pr] = -INFINITY;
                     a.part_ml[2 * pr + 1] = 0.0f;
                 } else {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) +
-                                                          static_cast<int64_t>(w.qrow0 + r) * D);
+                    const int64_t o = static_cast<int64_t>(w.qrow0 + r) * D;
+                    if (!in_bounds(o >= 0 && o + D <= a.out_elems)) continue;
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + o);
                     for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
@@ -546,9 +655,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     }
 
+    // consumer warps of the item ring: 16 softmax, 4 RoPE, the MMA and the V producer warp
+    constexpr uint32_t kItemReaders = kSoftmaxWarps + kRopeWarps + 2;
     if (threadIdx.x == 0) {
         mbar_init(bar(C::kBarQFull), 1);
         mbar_init(bar(C::kBarQReady), kRopeWarps);
+        mbar_init(bar(C::kBarQEmpty), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(C::kBarItemFull + s), 1);
+            mbar_init(bar(C::kBarItemEmpty + s), kItemReaders);
+        }
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(bar(C::kBarKFull + s), 1);
             mbar_init(bar(C::kBarVFull + s), 1);
@@ -574,82 +690,154 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // The k-th item index of this CTA, -1 when none is left: decode serves
+    // blockIdx.x alone; otherwise the shared counter hands out items in order
+    // (longest first within the work order, see decode_item).
+    auto fetch = [&](int32_t k) -> int32_t {
+        if constexpr (kDecode) {
+            return k == 0 ? static_cast<int32_t>(blockIdx.x) : -1;
+        } else {
+            if (!in_bounds(a.sched != nullptr)) return -1;
+            const int32_t x = atomicAdd(a.sched, 1);
+            return x < a.n_items ? x : -1;
+        }
+    };
+    // Consumer side of the ring: the k-th index, or -2 if the wait gave up.  Called by lane 0
+    // alone (warp_wide false) or by all lanes of a warp, which then all read the slot before
+    // lane 0 releases it.
+    auto read_item = [&](int32_t k, bool warp_wide) -> int32_t {
+        const int s = k & 1;
+        const bool got = mbar_wait(bar(C::kBarItemFull + s), static_cast<uint32_t>(k >> 1) & 1u, abort_flag);
+        const int32_t x = got ? item_slot[s] : -2;
+        if (warp_wide) __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::kBarItemEmpty + s));
+        return x;
+    };
+    auto item_of = [&](int32_t x) -> WorkItem {
+        in_bounds(x >= 0 && x < a.n_items);
+        const WorkItem w = kDecode ? decode_item_kv(a, x) : decode_item(a, x);
+        item_in_bounds(a, w, kDecode);
+        return w;
+    };
+    // consecutive positions: K (and Q) angles come from the recurrence, no cos/sin rows per
+    // K tile (decode: the cached keys are already rotated)
+    auto consecutive = [&](const WorkItem& w) -> bool {
+        return !kDecode && in_bounds(w.orig >= 0 && w.orig < a.B) && a.seeds[w.orig].consecutive != 0;
+    };
+
     if (warp == kTmaWarp) {
-        // ------------------------------------------------------------ Q/K producer
+        // ------------------------------------------------------------ Q/K producer (+ item fetch)
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmT);
+            auto publish = [&](int32_t k, int32_t x) -> bool {
+                const int s = k & 1;
+                if (k >= 2 && !mbar_wait(bar(C::kBarItemEmpty + s), static_cast<uint32_t>((k >> 1) - 1) & 1u,
+                                         abort_flag))
+                    return false;
+                item_slot[s] = x;
+                mbar_arrive(bar(C::kBarItemFull + s));  // release: the slot's value is visible to the waiters
+                return true;
+            };
             const bool bnsd = (a.layout == 0);
-            const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
-            auto load_tile = [&](const CUtensorMap* m, uint32_t dst, uint32_t b, int32_t plane, int32_t row0) {
-                for (int at = 0; at < C::kAtoms; ++at) {
-                    if (bnsd)
-                        tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, row0, plane);
-                    else
-                        tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, plane, w.tok0 + row0);
+            uint32_t g = 0;        // key tiles issued so far (ring position)
+            int32_t q_items = 0;   // items whose query tiles were issued
+            int32_t cur = fetch(0);
+            bool ok = publish(0, cur);
+            for (int32_t it = 0; ok && cur >= 0; ++it) {
+                const int32_t nxt = fetch(it + 1);
+                if (!publish(it + 1, nxt)) break;
+                const WorkItem w = item_of(cur);
+                const ItemShape sh = item_shape<kDecode>(a, w);
+                const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
+                const bool ktab = !kDecode && !consecutive(w);  // cos/sin rows staged beside each K tile
+                const uint32_t kbytes = C::kTileBytes + (ktab ? C::kTabBytes : 0);
+                auto load_tile = [&](const CUtensorMap* m, uint32_t dst, uint32_t b, int32_t plane, int32_t row0) {
+                    // the copy engine clips boxes outside the tensor itself: record, then issue anyway
+                    in_bounds(row0 >= 0 && row0 < w.L && plane >= 0 &&
+                              (bnsd ? (plane < a.B * (m == &tmQ ? a.Hq : a.Hkv))
+                                    : (plane < (m == &tmQ ? a.Hq : a.Hkv))));
+                    for (int at = 0; at < C::kAtoms; ++at) {
+                        if (bnsd)
+                            tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, row0, plane);
+                        else
+                            tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, plane, w.tok0 + row0);
+                    }
+                };
+                auto load_k = [&](int32_t j) -> bool {
+                    const int s = g % C::kStages;
+                    const uint32_t u = g / C::kStages;
+                    if (u > 0 && !mbar_wait(bar(C::kBarKEmpty + s), (u - 1) & 1u, abort_flag)) return false;
+                    if (ktab && g >= static_cast<uint32_t>(C::kTStages)) {
+                        // the rows slot held the rows of key tile g - kTStages: wait until that tile is rotated
+                        const uint32_t gp = g - C::kTStages;
+                        if (!mbar_wait(bar(C::kBarKReady + gp % C::kStages), (gp / C::kStages) & 1u, abort_flag))
+                            return false;
+                    }
+                    mbar_expect_tx(bar(C::kBarKFull + s), kbytes);
+                    load_tile(&tmK, sbase + C::kOffK + s * C::kTileBytes, bar(C::kBarKFull + s), kvplane, j * kBlockN);
+                    if (ktab) {
+                        const uint32_t dst = sbase + C::kOffT + (g % C::kTStages) * C::kTabBytes;
+                        for (int bx = 0; bx < C::kTabBoxes; ++bx)
+                            tma_load_3d(dst + bx * C::kAtomBytes, &tmT, bar(C::kBarKFull + s), bx * 32,
+                                        w.tok0 + j * kBlockN, 0);
+                    }
+                    ++g;
+                    return true;
+                };
+                // key tile 0 first (its slot frees before the query slots do), then the query tiles
+                if (!load_k(0)) break;
+                if (it > 0 && !mbar_wait(bar(C::kBarQEmpty), static_cast<uint32_t>(it - 1) & 1u, abort_flag)) break;
+                mbar_expect_tx(bar(C::kBarQFull),
+                               static_cast<uint32_t>(sh.nq) * C::kTileBytes + (kDecode ? C::kTabBytes : 0));
+                for (int i = 0; i < sh.nq; ++i) {
+                    if constexpr (kDecode) {  // q viewed as [B*Hq*Sq, D]: the group's rows from qrow0,
+                                              // their cos/sin rows in the second query slot
+                        for (int at = 0; at < C::kAtoms; ++at)
+                            tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64, 0,
+                                        w.qrow0);
+                        for (int bx = 0; bx < C::kTabBoxes; ++bx)
+                            tma_load_3d(sbase + C::kOffQ + C::kTileBytes + bx * C::kAtomBytes, &tmT,
+                                        bar(C::kBarQFull), bx * 32, w.qrow0, 0);
+                    } else {
+                        const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
+                        load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane,
+                                  w.qt[i] * kBlockM);
+                    }
                 }
-            };
-            auto load_tab = [&](uint32_t dst, uint32_t b, int32_t row0) {
-                for (int bx = 0; bx < C::kTabBoxes; ++bx)
-                    tma_load_3d(dst + bx * C::kAtomBytes, &tmT, b, bx * 32, w.tok0 + row0, 0);
-            };
-            // query tiles and their cos/sin rows (staged in V slots 0 and 1 until QReady; decode:
-            // in the second query tile's slot, which it does not otherwise use, so V loads need not
-            // wait)
-            mbar_expect_tx(bar(C::kBarQFull), static_cast<uint32_t>(nq) * (C::kTileBytes + C::kTabBytes));
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (i >= nq) break;
-                if constexpr (kDecode) {  // q viewed as [B*Hq*Sq, D]: the group's rows from qrow0
-                    for (int at = 0; at < C::kAtoms; ++at)
-                        tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64, 0, w.qrow0);
-                    for (int bx = 0; bx < C::kTabBoxes; ++bx)
-                        tma_load_3d(sbase + C::kOffQ + C::kTileBytes + bx * C::kAtomBytes, &tmT, bar(C::kBarQFull),
-                                    bx * 32, w.qrow0, 0);
-                } else {
-                    const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
-                    load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane, w.qt[i] * kBlockM);
-                    load_tab(sbase + C::kOffV + i * C::kTileBytes, bar(C::kBarQFull), w.qt[i] * kBlockM);
-                }
+                q_items = it + 1;
+                bool kok = true;
+                for (int32_t j = 1; j < sh.n_kv && kok; ++j) kok = load_k(j);
+                if (!kok) break;
+                cur = nxt;
             }
-            const bool ktab = !kDecode && !rec;  // cos/sin rows staged beside each K tile
-            const uint32_t kbytes = C::kTileBytes + (ktab ? C::kTabBytes : 0);
-            int32_t issued_k = 0;
-            for (int32_t j = 0; j < n_kv; ++j) {
-                const int s = j % C::kStages;
-                const uint32_t u = static_cast<uint32_t>(j / C::kStages);
-                if (u > 0 && !mbar_wait(bar(C::kBarKEmpty + s), (u - 1) & 1u, abort_flag)) break;
-                if (ktab && j >= C::kTStages) {
-                    // the rows slot held the rows of key tile j - kTStages: wait until that tile is rotated
-                    const int32_t jp = j - C::kTStages;
-                    if (!mbar_wait(bar(C::kBarKReady + jp % C::kStages), static_cast<uint32_t>(jp / C::kStages) & 1u,
-                                   abort_flag))
-                        break;
-                }
-                mbar_expect_tx(bar(C::kBarKFull + s), kbytes);
-                load_tile(&tmK, sbase + C::kOffK + s * C::kTileBytes, bar(C::kBarKFull + s), kvplane, j * kBlockN);
-                if (ktab) load_tab(sbase + C::kOffT + (j % C::kTStages) * C::kTabBytes, bar(C::kBarKFull + s), j * kBlockN);
-                issued_k = j + 1;
-            }
-            // Drain: every issued copy must have landed before the CTA exits.
-            mbar_wait_drain(bar(C::kBarQFull), 0);
-            for (int32_t j = (issued_k > C::kStages ? issued_k - C::kStages : 0); j < issued_k; ++j)
-                mbar_wait_drain(bar(C::kBarKFull + j % C::kStages), static_cast<uint32_t>(j / C::kStages) & 1u);
+            // Drain: every issued copy must have landed before the CTA exits (earlier phases
+            // completed before their slots were reissued).
+            if (q_items > 0) mbar_wait_drain(bar(C::kBarQFull), static_cast<uint32_t>(q_items - 1) & 1u);
+            for (uint32_t t = (g > static_cast<uint32_t>(C::kStages) ? g - C::kStages : 0u); t < g; ++t)
+                mbar_wait_drain(bar(C::kBarKFull + t % C::kStages), (t / C::kStages) & 1u);
         }
     } else if (warp == kTmaVWarp) {
         // ------------------------------------------------------------ V producer
         if (lane == 0) {
             tma_prefetch_desc(&tmV);
             const bool bnsd = (a.layout == 0);
-            const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
-            int32_t issued_v = 0;
-            // V slots 0 and 1 hold the query tiles' cos/sin rows until both are rotated (not in decode)
-            if (kDecode || mbar_wait(bar(C::kBarQReady), 0, abort_flag)) {
-                for (int32_t j = 0; j < n_kv; ++j) {
-                    const int s = j % C::kStages;
-                    const uint32_t u = static_cast<uint32_t>(j / C::kStages);
-                    if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) break;
+            uint32_t g = 0;  // value tiles issued so far
+            bool ok = true;
+            for (int32_t it = 0; ok; ++it) {
+                const int32_t x = read_item(it, false);
+                if (x < 0) break;
+                const WorkItem w = item_of(x);
+                const ItemShape sh = item_shape<kDecode>(a, w);
+                const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
+                for (int32_t j = 0; j < sh.n_kv; ++j) {
+                    const int s = g % C::kStages;
+                    const uint32_t u = g / C::kStages;
+                    if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
                     const uint32_t dst = sbase + C::kOffV + s * C::kTileBytes;
                     for (int at = 0; at < C::kAtoms; ++at) {
@@ -660,23 +848,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, kvplane,
                                         w.tok0 + j * kBlockN);
                     }
-                    issued_v = j + 1;
+                    ++g;
                 }
             }
-            for (int32_t j = (issued_v > C::kStages ? issued_v - C::kStages : 0); j < issued_v; ++j)
-                mbar_wait_drain(bar(C::kBarVFull + j % C::kStages), static_cast<uint32_t>(j / C::kStages) & 1u);
+            for (uint32_t t = (g > static_cast<uint32_t>(C::kStages) ? g - C::kStages : 0u); t < g; ++t)
+                mbar_wait_drain(bar(C::kBarVFull + t % C::kStages), (t / C::kStages) & 1u);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ tcgen05 issuer
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_f16(IoT<kFP16>::kFmt, 0, 0, kBlockM, kBlockN);
             constexpr uint32_t kIdescPV = idesc_f16(IoT<kFP16>::kFmt, 0, 1, kBlockM, D);
-            // S_i = Q_i' K_j'^T into TMEM buffer i (A = Q_i' and B = K_j' from shared memory)
-            // The issuing thread must keep up with the tensor pipe (one 128x128x16 MMA per ~64
-            // cycles): a tile's descriptors are built once and each k-step adds its byte offset
-            // >> 4 to the start-address field (shared addresses < 256 KB: no carry out of it).
-            auto issue_qk = [&](int i, int32_t j) {
-                const uint64_t kd = smem_desc_sw128(sbase + C::kOffK + (j % C::kStages) * C::kTileBytes, 16, 1024);
+            // S_i = Q_i' K'^T into TMEM buffer i (A = Q_i' and B = K' from shared memory), key tile
+            // at ring position t.  The issuing thread must keep up with the tensor pipe (one
+            // 128x128x16 MMA per ~64 cycles): a tile's descriptors are built once and each k-step
+            // adds its byte offset >> 4 to the start-address field (shared addresses < 256 KB: no
+            // carry out of it).
+            auto issue_qk = [&](int i, uint32_t t) {
+                const uint64_t kd = smem_desc_sw128(sbase + C::kOffK + (t % C::kStages) * C::kTileBytes, 16, 1024);
                 const uint64_t qd = smem_desc_sw128(sbase + C::kOffQ + (kDecode ? 0 : i) * C::kTileBytes, 16, 1024);
                 const uint32_t dS = tmem + C::kColS + i * kBlockN;
 #pragma unroll
@@ -686,171 +875,210 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 tc_commit(bar(C::kBarSFull + i));
             };
-            // O_i += P_i V_j (A = P_i from TMEM buffer i: keys [64h, 64h + 64) at columns [64h, 64h + 32);
-            // B = V_j from shared memory)
-            // (acc: O_i already holds a partial sum)
-            auto issue_pv = [&](int i, int32_t j, bool acc) {
-                const uint64_t vd = smem_desc_sw128(sbase + C::kOffV + (j % C::kStages) * C::kTileBytes, C::kAtomBytes, 1024);
+            // O_i += P_i V (A = P_i from TMEM buffer i: keys [64h, 64h + 64) at columns [64h, 64h + 32);
+            // B = the value tile at ring position t) (acc: O_i already holds a partial sum)
+            auto issue_pv = [&](int i, uint32_t t, bool acc) {
+                const uint64_t vd =
+                    smem_desc_sw128(sbase + C::kOffV + (t % C::kStages) * C::kTileBytes, C::kAtomBytes, 1024);
                 const uint32_t dO = tmem + C::kColO + i * D, aP = tmem + C::kColS + i * kBlockN;
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k)
                     umma_ts(dO, aP + (k >> 2) * 64 + (k & 3) * 8, vd + ((k * 16 * 128) >> 4), kIdescPV,
                             (acc || k > 0) ? 1u : 0u);
             };
-            if constexpr (kDecode) {
-                // Two chains over alternate key tiles (tile j into buffer j % 2, its t = j / 2-th
-                // tile).  QK_i of tile j + 2 reuses S_i: it is issued after PV_i of tile j, which
-                // read P_i, and MMAs from this thread execute in order.
-                bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag);
-                for (int32_t j = 0; j < 2 && j < n_kv && ok; ++j) {
-                    ok = mbar_wait(bar(C::kBarKReady + j % C::kStages), static_cast<uint32_t>(j / C::kStages) & 1u,
-                                   abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_qk(j, j);
-                    tc_commit(bar(C::kBarKEmpty + j % C::kStages));
-                }
-                for (int32_t j = 0; j < n_kv && ok; ++j) {
-                    const int s = j % C::kStages;
-                    const int i = j & 1;
-                    const int32_t t = j >> 1;
-                    ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag) &&
-                         mbar_wait(bar(C::kBarPFull + i), static_cast<uint32_t>(t) & 1u, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(i, j, t > 0);
-                    if (j + 2 >= n_kv) tc_commit(bar(C::kBarOFull + i));  // last tile of buffer i
-                    tc_commit(bar(C::kBarVEmpty + s));
-                    const int32_t jn = j + 2;
-                    if (jn < n_kv) {
-                        ok = mbar_wait(bar(C::kBarKReady + jn % C::kStages), static_cast<uint32_t>(jn / C::kStages) & 1u,
-                                       abort_flag);
+            auto kready = [&](uint32_t t) {
+                return mbar_wait(bar(C::kBarKReady + t % C::kStages), (t / C::kStages) & 1u, abort_flag);
+            };
+            uint32_t g = 0;                  // key/value tiles consumed so far (ring position)
+            uint32_t pc[2] = {0u, 0u};       // PFull_i phases consumed so far
+            bool ok = true;
+            for (int32_t it = 0; ok; ++it) {
+                const int32_t x = read_item(it, false);
+                if (x < 0) break;
+                const ItemShape sh = item_shape<kDecode>(a, item_of(x));
+                const int32_t n0 = sh.n0, n1 = sh.n1, n_kv = sh.n_kv;
+                ok = mbar_wait(bar(C::kBarQReady), static_cast<uint32_t>(it) & 1u, abort_flag);
+                if constexpr (kDecode) {
+                    // Two chains over alternate key tiles (tile j into buffer j % 2).  QK_i of tile
+                    // j + 2 reuses S_i: it is issued after PV_i of tile j, which read P_i, and MMAs
+                    // from this thread execute in order.
+                    for (int32_t j = 0; j < 2 && j < n_kv && ok; ++j) {
+                        ok = kready(g + j);
                         if (!ok) break;
                         tc_fence_after();
-                        issue_qk(i, jn);
-                        tc_commit(bar(C::kBarKEmpty + jn % C::kStages));
+                        issue_qk(j, g + j);
+                        tc_commit(bar(C::kBarKEmpty + (g + j) % C::kStages));
+                    }
+                    for (int32_t j = 0; j < n_kv && ok; ++j) {
+                        const uint32_t t = g + j;
+                        const int i = j & 1;
+                        ok = mbar_wait(bar(C::kBarVFull + t % C::kStages), (t / C::kStages) & 1u, abort_flag) &&
+                             mbar_wait(bar(C::kBarPFull + i), pc[i] & 1u, abort_flag);
+                        if (!ok) break;
+                        ++pc[i];
+                        tc_fence_after();
+                        issue_pv(i, t, j >= 2);
+                        if (j + 2 >= n_kv) tc_commit(bar(C::kBarOFull + i));  // last tile of buffer i
+                        tc_commit(bar(C::kBarVEmpty + t % C::kStages));
+                        if (j + 2 < n_kv) {
+                            ok = kready(t + 2);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_qk(i, t + 2);
+                            tc_commit(bar(C::kBarKEmpty + (t + 2) % C::kStages));
+                        }
+                    }
+                    tc_commit(bar(C::kBarQEmpty));
+                } else {
+                    // Order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  The item's
+                    // last QK is followed by a commit to QEmpty, so the producer can load the next
+                    // item's query tiles while this item's last PVs run.
+                    if (ok) ok = kready(g);
+                    if (ok) {
+                        tc_fence_after();
+                        if (n0 > 0) issue_qk(0, g);
+                        if (n1 > 0) issue_qk(1, g);
+                        tc_commit(bar(C::kBarKEmpty + g % C::kStages));
+                        if (n_kv == 1) tc_commit(bar(C::kBarQEmpty));
+                    }
+                    for (int32_t j = 0; j < n_kv && ok; ++j) {
+                        const uint32_t t = g + j;
+                        const int32_t jn = j + 1;
+                        ok = mbar_wait(bar(C::kBarVFull + t % C::kStages), (t / C::kStages) & 1u, abort_flag);
+                        if (!ok) break;
+                        if (j < n0) {
+                            ok = mbar_wait(bar(C::kBarPFull + 0), pc[0] & 1u, abort_flag);
+                            if (!ok) break;
+                            ++pc[0];
+                            tc_fence_after();
+                            issue_pv(0, t, j > 0);
+                            if (j == n0 - 1) tc_commit(bar(C::kBarOFull + 0));
+                        }
+                        if (jn < n_kv) {
+                            ok = kready(t + 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            if (jn < n0) issue_qk(0, t + 1);
+                        }
+                        if (j < n1) {
+                            ok = mbar_wait(bar(C::kBarPFull + 1), pc[1] & 1u, abort_flag);
+                            if (!ok) break;
+                            ++pc[1];
+                            tc_fence_after();
+                            issue_pv(1, t, j > 0);
+                            if (j == n1 - 1) tc_commit(bar(C::kBarOFull + 1));
+                        }
+                        tc_commit(bar(C::kBarVEmpty + t % C::kStages));
+                        if (jn < n_kv) {
+                            if (jn < n1) issue_qk(1, t + 1);
+                            tc_commit(bar(C::kBarKEmpty + (t + 1) % C::kStages));
+                            if (jn == n_kv - 1) tc_commit(bar(C::kBarQEmpty));
+                        }
                     }
                 }
-            } else {
-                bool ok = mbar_wait(bar(C::kBarQReady), 0, abort_flag) && mbar_wait(bar(C::kBarKReady), 0, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    if (n0 > 0) issue_qk(0, 0);
-                    if (n1 > 0) issue_qk(1, 0);
-                    tc_commit(bar(C::kBarKEmpty));
-                }
-                for (int32_t j = 0; j < n_kv && ok; ++j) {
-                    const int s = j % C::kStages;
-                    const int32_t jn = j + 1;
-                    ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(j / C::kStages) & 1u, abort_flag);
-                    if (!ok) break;
-                    if (j < n0) {
-                        ok = mbar_wait(bar(C::kBarPFull + 0), static_cast<uint32_t>(j) & 1u, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(0, j, j > 0);
-                        if (j == n0 - 1) tc_commit(bar(C::kBarOFull + 0));
-                    }
-                    if (jn < n_kv) {
-                        ok = mbar_wait(bar(C::kBarKReady + jn % C::kStages), static_cast<uint32_t>(jn / C::kStages) & 1u,
-                                       abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        if (jn < n0) issue_qk(0, jn);
-                    }
-                    if (j < n1) {
-                        ok = mbar_wait(bar(C::kBarPFull + 1), static_cast<uint32_t>(j) & 1u, abort_flag);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(1, j, j > 0);
-                        if (j == n1 - 1) tc_commit(bar(C::kBarOFull + 1));
-                    }
-                    tc_commit(bar(C::kBarVEmpty + s));
-                    if (jn < n_kv) {
-                        if (jn < n1) issue_qk(1, jn);
-                        tc_commit(bar(C::kBarKEmpty + jn % C::kStages));
-                    }
-                }
+                g += static_cast<uint32_t>(n_kv);
             }
             tc_commit(bar(C::kBarMmaFin));
             mbar_wait_drain(bar(C::kBarMmaFin), 0);
         }
     } else if (warp >= kRopeWarp0 && warp < kRopeWarp0 + kRopeWarps) {
-        // ------------------------------------------------------------ RoPE warpgroups
-        const int32_t rt = threadIdx.x - kRopeWarp0 * 32;  // 0..255
+        // ------------------------------------------------------------ RoPE warpgroup
+        // Per item, one loop over the tiles to rotate: key tile 0 (it lands before the query
+        // tiles), the query tiles, then key tiles 1 .. n_kv - 1; one code path per angle
+        // source.  Consecutive positions: every tile's first-row angles are formed directly
+        // (angles_at), the thread's other rows of the tile by the in-tile step; otherwise cos/sin
+        // rows from the table (staged beside a key tile by TMA, read from global memory for the
+        // query tiles).
+        const int32_t rt = threadIdx.x - kRopeWarp0 * 32;  // 0..127
         constexpr int kPairsPerRow = D / 16;
-        constexpr int kStep = kRopeThreads / kPairsPerRow;  // rows between a thread's tasks
-        RecState z;
-        uint64_t wc[4], ws[4];
-        const RopeSeed* sd = a.seeds + w.orig;
-        if (rec) {
-            const int cp = rt % kPairsPerRow;
-            const int r0 = rt / kPairsPerRow;  // < kStep
+        const int f0 = 8 * (rt % kPairsPerRow);             // this thread's first frequency
+        const int r0 = rt / kPairsPerRow;                   // this thread's first row of a tile
+        uint32_t g = 0;  // key tiles rotated so far (ring position)
+        for (int32_t it = 0;; ++it) {
+            const int32_t x = read_item(it, true);
+            if (x < 0) break;
+            const WorkItem w = item_of(x);
+            const ItemShape sh = item_shape<kDecode>(a, w);
+            const bool rec = consecutive(w);
+            float qw[8];            // this thread's frequencies
+            uint64_t wc[4], ws[4];  // in-tile step (cos, sin) of kStep rows, packed pairs
+            int32_t p0 = 0;         // the sequence's first position
+            if (rec) {
+                const RopeSeed* sd = a.seeds + w.orig;
+                const float4 u0 = *reinterpret_cast<const float4*>(sd->inv + f0);
+                const float4 u1 = *reinterpret_cast<const float4*>(sd->inv + f0 + 4);
+                qw[0] = u0.x; qw[1] = u0.y; qw[2] = u0.z; qw[3] = u0.w;
+                qw[4] = u1.x; qw[5] = u1.y; qw[6] = u1.z; qw[7] = u1.w;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int f = 8 * cp + 2 * k;
-                const float2 z0 = sd->z0[r0 % kSeedRows][f], z1 = sd->z0[r0 % kSeedRows][f + 1];
-                const float2 w0 = sd->w16[f], w1 = sd->w16[f + 1];
-                const uint64_t w16c = f2pack(w0.x, w1.x), w16s = f2pack(w0.y, w1.y);
-                z.c[k] = f2pack(z0.x, z1.x);
-                z.s[k] = f2pack(z0.y, z1.y);
-                for (int q = 0; q < r0 / kSeedRows; ++q) rec_step(z.c[k], z.s[k], w16c, w16s);  // rows >= 16
-                // step of kStep rows: w16^(kStep/16)
-                wc[k] = w16c;
-                ws[k] = w16s;
-#pragma unroll
-                for (int q = 1; q < kStep / kSeedRows; ++q) rec_step(wc[k], ws[k], w16c, w16s);
-            }
-        }
-        if (mbar_wait(bar(C::kBarQFull), 0, abort_flag)) {
-#pragma unroll 1
-            for (int i = 0; i < nq; ++i) {
-                const int32_t q0 = (i == 0 ? w.qt[0] : w.qt[1]) * kBlockM;
-                // decode: only the group's G * Sq rows of the tile are queries of this item
-                rope_tile<D, kFP16, kAdj>(sbase + C::kOffQ + i * C::kTileBytes,
-                                          sbase + (kDecode ? C::kOffQ + C::kTileBytes : C::kOffV + i * C::kTileBytes),
-                                          kDecode ? a.G * a.dec_Sq : min(kBlockM, w.L - q0), rt);
-            }
-            fence_proxy_async_smem();  // Q' written by the generic proxy, read by the tensor cores
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarQReady));
-            for (int32_t j = 0; j < n_kv; ++j) {
-                const int s = j % C::kStages;
-                const uint32_t u = static_cast<uint32_t>(j / C::kStages);
-                if (!mbar_wait(bar(C::kBarKFull + s), u & 1u, abort_flag)) break;
-                const int32_t k0 = j * kBlockN;
-                if constexpr (kDecode) {
-                    // cached keys are already rotated: hand the tile on as it is
-                } else if (rec) {
-                    rope_tile_rec<D, kFP16, kAdj>(sbase + C::kOffK + s * C::kTileBytes, min(kBlockN, w.L - k0), rt, z, wc, ws);
-                    // advance to the next tile by 128 rows (the step is re-read from the cached seed)
-                    const int f0 = 8 * (rt % kPairsPerRow);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 v0 = sd->w128[f0 + 2 * k], v1 = sd->w128[f0 + 2 * k + 1];
-                        rec_step(z.c[k], z.s[k], f2pack(v0.x, v1.x), f2pack(v0.y, v1.y));
-                    }
-                } else {
-                    rope_tile<D, kFP16, kAdj>(sbase + C::kOffK + s * C::kTileBytes,
-                                        sbase + C::kOffT + (j % C::kTStages) * C::kTabBytes, min(kBlockN, w.L - k0), rt);
+                for (int k = 0; k < 4; ++k) {
+                    const float4 v = *reinterpret_cast<const float4*>(sd->wstep + f0 + 2 * k);  // pairs f, f + 1
+                    wc[k] = f2pack(v.x, v.z);
+                    ws[k] = f2pack(v.y, v.w);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(C::kBarKReady + s));
+                p0 = sd->pos0;
             }
+            bool ok = true;
+            const int32_t nrot = sh.n_kv + sh.nq;
+#pragma unroll 1
+            for (int32_t e = 0; e < nrot && ok; ++e) {
+                const bool isq = e >= 1 && e <= sh.nq;
+                const int qi = e - 1;                          // query tile (isq)
+                const int32_t j = (e == 0) ? 0 : e - sh.nq;    // key tile (!isq)
+                const uint32_t t = g + static_cast<uint32_t>(j);
+                const int s = t % C::kStages;
+                uint32_t tile;
+                int32_t row0;
+                if (isq) {
+                    if (qi == 0) ok = mbar_wait(bar(C::kBarQFull), static_cast<uint32_t>(it) & 1u, abort_flag);
+                    tile = sbase + C::kOffQ + qi * C::kTileBytes;
+                    row0 = w.qt[qi] * kBlockM;
+                } else {
+                    ok = mbar_wait(bar(C::kBarKFull + s), (t / C::kStages) & 1u, abort_flag);
+                    tile = sbase + C::kOffK + s * C::kTileBytes;
+                    row0 = j * kBlockN;
+                }
+                if (!ok) break;
+                const int32_t rows = min(kBlockM, w.L - row0);
+                if constexpr (kDecode) {
+                    // cached keys are already rotated; the query tile holds the group's G * Sq rows,
+                    // their cos/sin rows in the second query slot
+                    if (isq) rope_tile<D, kFP16, kAdj>(tile, sbase + C::kOffQ + C::kTileBytes, a.G * a.dec_Sq, rt);
+                } else if (rec) {
+                    RecState zz;
+                    angles_at(p0, row0 + r0, qw, zz);
+                    rope_tile_rec<D, kFP16, kAdj>(tile, rows, rt, zz, wc, ws);
+                } else if (isq) {
+                    if (in_bounds(row0 >= 0 && static_cast<int64_t>(w.tok0) + row0 + rows <= a.ntok))
+                        rope_tile_global<D, kFP16, kAdj>(tile, a.table + static_cast<int64_t>(w.tok0 + row0) * (D / 2),
+                                                         rows, rt);
+                } else {
+                    rope_tile<D, kFP16, kAdj>(tile, sbase + C::kOffT + (t % C::kTStages) * C::kTabBytes, rows, rt);
+                }
+                fence_proxy_async_smem();  // rotated tile written by the generic proxy, read by the tensor cores
+                __syncwarp();
+                if (lane == 0) {
+                    if (!isq)
+                        mbar_arrive(bar(C::kBarKReady + s));
+                    else if (qi == sh.nq - 1)
+                        mbar_arrive(bar(C::kBarQReady));
+                }
+            }
+            g += static_cast<uint32_t>(sh.n_kv);
+            if (!ok) break;
         }
     } else if (warp < kSoftmaxWarps) {
         // ------------------------------------------------------------ softmax warps
         // Query tile i has 8 warps: warp w covers TMEM lanes (rows) 32 (w % 4) .. + 31 and key
         // columns [64 hf, 64 hf + 64) of every score tile, hf = (w / 4) % 2.  The two warps of a
         // row exchange half-row maxima (then row sums) through shared memory at named barrier
-        // 1 + i (256 threads), executed exactly n_i + 2 times by every one of them: a failed
-        // (timed-out) wait only turns the remaining work into no-ops, it never skips a barrier.
-        // A slot written at tile j + 1 was read at tile j before the reader arrived on PFull_i(j),
-        // which S_i(j + 1) waits for, so one slot per row and half suffices.
+        // 1 + i (256 threads), executed exactly n_i + 2 times per item by every one of them: a
+        // failed (timed-out) wait only turns the remaining work into no-ops, it never skips a
+        // barrier.  All 16 warps decide together, at named barrier 3 (512 threads), whether to
+        // take the next item, so they always run the same items.  A slot written at tile j + 1
+        // was read at tile j before the reader arrived on PFull_i(j), which S_i(j + 1) waits
+        // for, so one slot per row and half suffices.
         const int i = warp >> 3;             // query tile
         const int hf = (warp >> 2) & 1;      // key-column half
-        const int32_t n_i = i == 0 ? n0 : n1;
         const int row = ((warp & 3) << 5) + lane;  // 0..127 == TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t sc = tmem + lane_off + C::kColS + i * kBlockN + hf * 64;  // this half of S_i; P over [0, 32)
@@ -858,27 +1086,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t oc = tmem + lane_off + C::kColO + i * D + hf * kOHalf;
         float* xch = reinterpret_cast<float*>(smem + C::kOffXchg) + i * 2 * kBlockM;  // [half][row]
         const uint32_t nb = 1u + static_cast<uint32_t>(i);
-        const int32_t qt_i = i == 0 ? w.qt[0] : w.qt[1];
-        const int32_t qi = qt_i * kBlockM + row;
-        int32_t vis = a.causal ? min(qi + 1, w.L) : w.L;  // keys [0, vis) visible to this row
-        if constexpr (kDecode) {
-            // row = g * Sq + s: new token s of the sequence's last Sq sees keys up to len - Sq + s
-            // (bottom-right causal), relative to this split's first key
-            const int32_t len = min(max(a.kv_lens[w.seq], 0), a.dec_Smax);
-            vis = a.causal ? min(w.L, len - a.dec_Sq + row % a.dec_Sq + 1 - w.split * a.dec_chunk) : w.L;
-        }
         const float sl2 = a.scale_log2;
-        float m = -INFINITY;  // running max of score * scale * log2(e) (identical in both halves)
-        float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
-        bool ok = true;       // warp-uniform; tcgen05.ld/st are warp-collective
-        for (int32_t j = 0; j < n_i; ++j) {
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + i), static_cast<uint32_t>(j) & 1u, abort_flag));
-            const int32_t kt = kDecode ? 2 * j + i : j;          // key tile of this step
-            const int32_t lim = vis - kt * kBlockN - hf * 64;  // columns [0, lim) of this half are visible
-            float mxh = -INFINITY;
-            if (ok) {
-                tc_fence_after();
-                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint32_t cs = 0;  // SFull_i phases consumed so far
+        uint32_t co = 0;  // OFull_i phases consumed so far
+        for (int32_t it = 0;; ++it) {
+            const int32_t x = read_item(it, true);
+            if (!named_bar_and(3, kSoftmaxWarps * 32, x >= 0 && *abort_flag == 0)) break;
+            const WorkItem w = item_of(x);
+            const ItemShape sh = item_shape<kDecode>(a, w);
+            const int32_t n0 = sh.n0, n1 = sh.n1;
+            const int32_t n_i = i == 0 ? n0 : n1;
+            const int32_t qt_i = i == 0 ? w.qt[0] : w.qt[1];
+            const int32_t qi = qt_i * kBlockM + row;
+            int32_t vis = a.causal ? min(qi + 1, w.L) : w.L;  // keys [0, vis) visible to this row
+            if constexpr (kDecode) {
+                // row = g * Sq + s: new token s of the sequence's last Sq sees keys up to len - Sq + s
+                // (bottom-right causal), relative to this split's first key
+                const int32_t len = in_bounds(w.seq >= 0 && w.seq < a.B) ? min(max(a.kv_lens[w.seq], 0), a.dec_Smax) : 0;
+                vis = a.causal ? min(w.L, len - a.dec_Sq + row % a.dec_Sq + 1 - w.split * a.dec_chunk) : w.L;
+            }
+            float m = -INFINITY;  // running max of score * scale * log2(e) (identical in both halves)
+            float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
+            bool ok = true;       // warp-uniform; tcgen05.ld/st are warp-collective
+            for (int32_t j = 0; j < n_i; ++j) {
+                ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + i), cs & 1u, abort_flag));
+                ++cs;
+                const int32_t kt = kDecode ? 2 * j + i : j;          // key tile of this step
+                const int32_t lim = vis - kt * kBlockN - hf * 64;  // columns [0, lim) of this half are visible
+                float mxh = -INFINITY;
+                if (ok) {
+                    tc_fence_after();
+                    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t sr[32];
+                        tmem_ld32(sc + q * 32, sr);
+                        tmem_wait_ld();
+                        mask_cols(sr, lim - q * 32);
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2)
+                            mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                    }
+                    mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+                }
+                xch[hf * kBlockM + row] = mxh;
+                named_bar_sync(nb, 256);
+                ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
+                if (!ok) continue;
+                const float m_new = fmaxf(m, fmaxf(mxh, xch[(hf ^ 1) * kBlockM + row]) * sl2);
+                if (j > 0) {
+                    // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
+                    const bool need = m_new > m + kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float alpha = need ? ex2(m - m_new) : 1.0f;
+                        const uint64_t alpha2 = f2pack(alpha, alpha);
+                        l *= alpha;
+#pragma unroll 1
+                        for (int q = 0; q < kOHalf / 32; ++q) {
+                            uint32_t o[32];
+                            tmem_ld32(oc + q * 32, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; c += 2) {
+                                const float2 v = f2unpack(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), alpha2));
+                                o[c] = __float_as_uint(v.x);
+                                o[c + 1] = __float_as_uint(v.y);
+                            }
+                            tmem_st32(oc + q * 32, o);
+                        }
+                        if (need) m = m_new;
+                    }
+                } else {
+                    m = m_new;
+                }
+                // P = exp2(S * scale_log2 - m) over this half, 32 columns at a time, written over
+                // the half's S columns already read (P columns [16q, 16q + 16) lie in [0, 32q + 32))
+                const float neg_m = (m == -INFINITY) ? 0.0f : -m;
+                const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
+                uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
 #pragma unroll 1
                 for (int q = 0; q < 2; ++q) {
                     uint32_t sr[32];
@@ -886,185 +1171,149 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     tmem_wait_ld();
                     mask_cols(sr, lim - q * 32);
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2)
-                        mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                    for (int c2 = 0; c2 < 16; ++c2) {
+                        const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
+                        const float2 xv = f2unpack(ffma2(sv, sl2x2, negm2));
+                        const uint64_t pp = f2pack(ex2(xv.x), ex2(xv.y));
+                        l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
+                        sr[c2] = pack2<kFP16>(pp);
+                    }
+                    tmem_st16(sc + q * 16, reinterpret_cast<const uint32_t(&)[16]>(sr));
                 }
-                mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+                const float2 la = f2unpack(fadd2(l2[0], l2[1]));
+                l += la.x + la.y;
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::kBarPFull + i));
             }
-            xch[hf * kBlockM + row] = mxh;
+            // epilogue: combine the two halves' row sums (the slot may still hold a maximum the
+            // other half has yet to read, hence the barrier before writing), then out = O / l
             named_bar_sync(nb, 256);
-            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
-            if (!ok) continue;
-            const float m_new = fmaxf(m, fmaxf(mxh, xch[(hf ^ 1) * kBlockM + row]) * sl2);
-            if (j > 0) {
-                // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
-                const bool need = m_new > m + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need)) {
-                    const float alpha = need ? ex2(m - m_new) : 1.0f;
-                    const uint64_t alpha2 = f2pack(alpha, alpha);
-                    l *= alpha;
+            xch[hf * kBlockM + row] = l;
+            named_bar_sync(nb, 256);
+            l += xch[(hf ^ 1) * kBlockM + row];
+            if constexpr (kDecode) {
+                // The two buffers hold alternate key tiles of this split.  With M = max(m_0, m_1) and
+                // c_b = 2^(m_b - M) (0 where l_b = 0): O = c_0 O_0 + c_1 O_1, l = c_0 l_0 + c_1 l_1.
+                // Warp (i, hf) merges column quarter 2 i + hf of its lane group's rows.  (m, l) pass
+                // through the K-tile cos/sin slot, which decode uses for nothing else: a buffer with
+                // no tiles reaches this point while the query tile may still be in flight.  A decode
+                // CTA runs one item, so both OFull phases are the first.
+                float* mlx = reinterpret_cast<float*>(smem + C::kOffT);  // [m_0, m_1, l_0, l_1][row]
+                if (hf == 0) {
+                    mlx[i * kBlockM + row] = m;
+                    mlx[(2 + i) * kBlockM + row] = l;
+                }
+                named_bar_sync(3, kSoftmaxWarps * 32);
+                const float m0 = mlx[row], m1 = mlx[kBlockM + row];
+                const float l0 = mlx[2 * kBlockM + row], l1 = mlx[3 * kBlockM + row];
+                const bool fin = __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
+                                 __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + 0), 0, abort_flag)) &&
+                                 (n1 == 0 || __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + 1), 0, abort_flag)));
+                if (fin) {
+                    tc_fence_after();
+                    const float M = fmaxf(m0, m1);
+                    const float c0 = (l0 > 0.0f) ? ex2(m0 - M) : 0.0f;
+                    const float c1 = (l1 > 0.0f) ? ex2(m1 - M) : 0.0f;
+                    const float lt = c0 * l0 + c1 * l1;
+                    // rows of q viewed as [B*Hq*Sq, D]; with several splits, unnormalised fp32 O and
+                    // (m, l) go to the partials that the combine kernel merges
+                    bool valid = row < a.G * a.dec_Sq;
+                    const bool partial = a.dec_splits > 1;
+                    int64_t o_off = static_cast<int64_t>(w.qrow0 + row) * D;
+                    if (partial) {
+                        const int64_t rq = static_cast<int64_t>(a.B) * a.Hq * a.dec_Sq;
+                        const int64_t pr = static_cast<int64_t>(w.split) * rq + w.qrow0 + row;
+                        o_off = pr * D;
+                        if (valid) valid = in_bounds(pr >= 0 && pr < a.dec_splits * rq);
+                        if (valid && i == 0 && hf == 0) {
+                            a.part_ml[2 * pr] = (lt > 0.0f) ? M : -INFINITY;
+                            a.part_ml[2 * pr + 1] = lt;
+                        }
+                    }
+                    if (valid && !partial) valid = in_bounds(o_off >= 0 && o_off + D <= a.out_elems);
+                    const float scl = partial ? 1.0f : ((lt > 0.0f) ? 1.0f / lt : 0.0f);
+                    const float w0 = c0 * scl, w1 = c1 * scl;
+                    constexpr int kOQ = D / 4;  // columns per warp
+                    const int c_lo = (2 * i + hf) * kOQ;
+                    const uint32_t o0c = tmem + lane_off + C::kColO + c_lo;  // O_1 is D columns further
+#pragma unroll 1
+                    for (int q = 0; q < kOQ / 16; ++q) {
+                        uint32_t o0[16], o1[16];
+                        tmem_ld16(o0c + q * 16, o0);
+                        if (n1 > 0) {
+                            tmem_ld16(o0c + D + q * 16, o1);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) o1[e] = 0u;
+                        }
+                        tmem_wait_ld();
+                        float v[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)  // a buffer with l = 0 contributes nothing (its O may be unset)
+                            v[e] = (c0 > 0.0f ? w0 * __uint_as_float(o0[e]) : 0.0f) +
+                                   (c1 > 0.0f ? w1 * __uint_as_float(o1[e]) : 0.0f);
+                        if (!valid) continue;
+                        if (partial) {
+                            float4* dst = reinterpret_cast<float4*>(a.part_o + o_off + c_lo + q * 16);
+#pragma unroll
+                            for (int v4 = 0; v4 < 4; ++v4)
+                                dst[v4] = make_float4(v[4 * v4], v[4 * v4 + 1], v[4 * v4 + 2], v[4 * v4 + 3]);
+                        } else {
+                            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + o_off + c_lo + q * 16);
+#pragma unroll
+                            for (int v4 = 0; v4 < 2; ++v4) {
+                                uint32_t wv[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    wv[e] = pack2<kFP16>(f2pack(v[8 * v4 + 2 * e], v[8 * v4 + 2 * e + 1]));
+                                dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                            }
+                        }
+                    }
+                }
+            } else {
+                bool fin = n_i > 0 && __all_sync(0xffffffffu, ok && *abort_flag == 0);
+                if (n_i > 0) {
+                    fin = fin && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), co & 1u, abort_flag));
+                    ++co;
+                }
+                if (fin) {
+                    tc_fence_after();
+                    const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
+                    const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+                    bool valid = qi < w.L;
+                    uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
+                    int64_t o_off;
+                    if (a.layout == 0)
+                        o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
+                    else
+                        o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
+                    o_off += hf * kOHalf;
+                    if (valid) valid = in_bounds(o_off >= 0 && o_off + kOHalf <= a.out_elems);
+                    const uint64_t il2 = f2pack(inv_l, inv_l);
 #pragma unroll 1
                     for (int q = 0; q < kOHalf / 32; ++q) {
                         uint32_t o[32];
                         tmem_ld32(oc + q * 32, o);
                         tmem_wait_ld();
+                        if (valid) {
+                            uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);
 #pragma unroll
-                        for (int c = 0; c < 32; c += 2) {
-                            const float2 v = f2unpack(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), alpha2));
-                            o[c] = __float_as_uint(v.x);
-                            o[c + 1] = __float_as_uint(v.y);
-                        }
-                        tmem_st32(oc + q * 32, o);
-                    }
-                    if (need) m = m_new;
-                }
-            } else {
-                m = m_new;
-            }
-            // P = exp2(S * scale_log2 - m) over this half, 32 columns at a time, written over
-            // the half's S columns already read (P columns [16q, 16q + 16) lie in [0, 32q + 32))
-            const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-            const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
-            uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
-#pragma unroll 1
-            for (int q = 0; q < 2; ++q) {
-                uint32_t sr[32];
-                tmem_ld32(sc + q * 32, sr);
-                tmem_wait_ld();
-                mask_cols(sr, lim - q * 32);
+                            for (int v4 = 0; v4 < 4; ++v4) {
+                                uint32_t wv[4];
 #pragma unroll
-                for (int c2 = 0; c2 < 16; ++c2) {
-                    const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
-                    const float2 x = f2unpack(ffma2(sv, sl2x2, negm2));
-                    const uint64_t pp = f2pack(ex2(x.x), ex2(x.y));
-                    l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
-                    sr[c2] = pack2<kFP16>(pp);
-                }
-                tmem_st16(sc + q * 16, reinterpret_cast<const uint32_t(&)[16]>(sr));
-            }
-            const float2 la = f2unpack(fadd2(l2[0], l2[1]));
-            l += la.x + la.y;
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarPFull + i));
-        }
-        // epilogue: combine the two halves' row sums (the slot may still hold a maximum the
-        // other half has yet to read, hence the barrier before writing), then out = O / l
-        named_bar_sync(nb, 256);
-        xch[hf * kBlockM + row] = l;
-        named_bar_sync(nb, 256);
-        l += xch[(hf ^ 1) * kBlockM + row];
-        if constexpr (kDecode) {
-            // The two buffers hold alternate key tiles of this split.  With M = max(m_0, m_1) and
-            // c_b = 2^(m_b - M) (0 where l_b = 0): O = c_0 O_0 + c_1 O_1, l = c_0 l_0 + c_1 l_1.
-            // Warp (i, hf) merges column quarter 2 i + hf of its lane group's rows.  (m, l) pass
-            // through the K-tile cos/sin slot, which decode uses for nothing else: a buffer with
-            // no tiles reaches this point while the query tile may still be in flight.
-            float* mlx = reinterpret_cast<float*>(smem + C::kOffT);  // [m_0, m_1, l_0, l_1][row]
-            if (hf == 0) {
-                mlx[i * kBlockM + row] = m;
-                mlx[(2 + i) * kBlockM + row] = l;
-            }
-            named_bar_sync(3, kSoftmaxWarps * 32);
-            const float m0 = mlx[row], m1 = mlx[kBlockM + row];
-            const float l0 = mlx[2 * kBlockM + row], l1 = mlx[3 * kBlockM + row];
-            const bool fin = __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
-                             __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + 0), 0, abort_flag)) &&
-                             (n1 == 0 || __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + 1), 0, abort_flag)));
-            if (fin) {
-                tc_fence_after();
-                const float M = fmaxf(m0, m1);
-                const float c0 = (l0 > 0.0f) ? ex2(m0 - M) : 0.0f;
-                const float c1 = (l1 > 0.0f) ? ex2(m1 - M) : 0.0f;
-                const float lt = c0 * l0 + c1 * l1;
-                // rows of q viewed as [B*Hq*Sq, D]; with several splits, unnormalised fp32 O and
-                // (m, l) go to the partials that the combine kernel merges
-                const bool valid = row < a.G * a.dec_Sq;
-                const bool partial = a.dec_splits > 1;
-                int64_t o_off = static_cast<int64_t>(w.qrow0 + row) * D;
-                if (partial) {
-                    const int64_t pr = static_cast<int64_t>(w.split) * (a.B * a.Hq * a.dec_Sq) + w.qrow0 + row;
-                    o_off = pr * D;
-                    if (valid && i == 0 && hf == 0) {
-                        a.part_ml[2 * pr] = (lt > 0.0f) ? M : -INFINITY;
-                        a.part_ml[2 * pr + 1] = lt;
-                    }
-                }
-                const float sc = partial ? 1.0f : ((lt > 0.0f) ? 1.0f / lt : 0.0f);
-                const float w0 = c0 * sc, w1 = c1 * sc;
-                constexpr int kOQ = D / 4;  // columns per warp
-                const int c_lo = (2 * i + hf) * kOQ;
-                const uint32_t o0c = tmem + lane_off + C::kColO + c_lo;  // O_1 is D columns further
-#pragma unroll 1
-                for (int q = 0; q < kOQ / 16; ++q) {
-                    uint32_t o0[16], o1[16];
-                    tmem_ld16(o0c + q * 16, o0);
-                    if (n1 > 0) {
-                        tmem_ld16(o0c + D + q * 16, o1);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) o1[e] = 0u;
-                    }
-                    tmem_wait_ld();
-                    float v[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)  // a buffer with l = 0 contributes nothing (its O may be unset)
-                        v[e] = (c0 > 0.0f ? w0 * __uint_as_float(o0[e]) : 0.0f) +
-                               (c1 > 0.0f ? w1 * __uint_as_float(o1[e]) : 0.0f);
-                    if (!valid) continue;
-                    if (partial) {
-                        float4* dst = reinterpret_cast<float4*>(a.part_o + o_off + c_lo + q * 16);
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4)
-                            dst[v4] = make_float4(v[4 * v4], v[4 * v4 + 1], v[4 * v4 + 2], v[4 * v4 + 3]);
-                    } else {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + o_off + c_lo + q * 16);
-#pragma unroll
-                        for (int v4 = 0; v4 < 2; ++v4) {
-                            uint32_t wv[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                wv[e] = pack2<kFP16>(f2pack(v[8 * v4 + 2 * e], v[8 * v4 + 2 * e + 1]));
-                            dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                        }
-                    }
-                }
-            }
-        } else {
-            const bool fin = n_i > 0 && __all_sync(0xffffffffu, ok && *abort_flag == 0) &&
-                             __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), 0, abort_flag));
-            if (fin) {
-                tc_fence_after();
-                const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
-                const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-                const bool valid = qi < w.L;
-                uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
-                int64_t o_off;
-                if (a.layout == 0)
-                    o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
-                else
-                    o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
-                o_off += hf * kOHalf;
-                const uint64_t il2 = f2pack(inv_l, inv_l);
-#pragma unroll 1
-                for (int q = 0; q < kOHalf / 32; ++q) {
-                    uint32_t o[32];
-                    tmem_ld32(oc + q * 32, o);
-                    tmem_wait_ld();
-                    if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4) {
-                            uint32_t wv[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int c = 8 * v4 + 2 * e;
-                                wv[e] = pack2<kFP16>(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), il2));
+                                for (int e = 0; e < 4; ++e) {
+                                    const int c = 8 * v4 + 2 * e;
+                                    wv[e] = pack2<kFP16>(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), il2));
+                                }
+                                dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                             }
-                            dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
                         }
                     }
+                    // the next item's PV_i(0) overwrites O_i only after this warp's PFull_i
+                    // arrival of that item, which follows these reads (tcgen05.wait::ld above)
                 }
             }
         }
@@ -1076,6 +1325,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+    if constexpr (!kDecode) {
+        // The last CTA to finish re-zeroes the work counters for the next launch on this
+        // workspace: every CTA counts itself in only after all its fetches (its producer is
+        // done before the barrier above).
+        if (threadIdx.x == 0) {
+            __threadfence();
+            if (atomicAdd(a.sched + 1, 1) == static_cast<int32_t>(gridDim.x) - 1) {
+                atomicExch(a.sched, 0);
+                atomicExch(a.sched + 1, 0);
+                __threadfence();
+            }
+        }
     }
 }
 
@@ -1114,6 +1376,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const float* __rest
             acc[6] = fmaf(wgt, v.z, acc[6]); acc[7] = fmaf(wgt, v.w, acc[7]);
         }
         const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+        if (!in_bounds(c + 8 <= D && static_cast<int64_t>(r) * D + c + 8 <= static_cast<int64_t>(rows) * D)) continue;
         uint32_t wv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) wv[e] = IoT<kFP16>::pack(acc[2 * e] * inv, acc[2 * e + 1] * inv);

@@ -158,11 +158,20 @@ int64_t total_tokens(const rfa_attn_params* p, const int32_t* lens) {
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // cos/sin table (D/2 fp16 cos and D/2 fp16 sin values per token), then one
-// recurrence seed block per sequence.
+// recurrence seed block per sequence, then the attention kernel's two work
+// counters (zeroed by the table kernel, re-zeroed by the attention kernel's
+// last CTA).
 size_t table_bytes(int64_t T, int D) { return round_up(static_cast<size_t>(T) * D * 2, 256); }
 size_t seeds_bytes(int nseg) { return round_up(static_cast<size_t>(nseg) * sizeof(rfa::RopeSeed), 256); }
-size_t workspace_bytes(int64_t T, int D, int nseg) { return table_bytes(T, D) + seeds_bytes(nseg); }
+constexpr size_t kSchedBytes = 256;
+size_t workspace_bytes(int64_t T, int D, int nseg) { return table_bytes(T, D) + seeds_bytes(nseg) + kSchedBytes; }
+int32_t* sched_of(void* workspace, int64_t T, int D, int nseg) {
+    return reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + table_bytes(T, D) + seeds_bytes(nseg));
+}
 
+// Prefill: a persistent grid, one CTA per SM (one fits: 24 warps, ~226 KB of
+// shared memory), each taking items from the work counters; decode: one CTA
+// per item.
 template <int D, bool kFP16, bool kAdj, bool kDecode = false>
 rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mt,
                        const rfa::AttnArgs& args, cudaStream_t st) {
@@ -170,7 +179,8 @@ rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     constexpr int smem = rfa::AttnCfg<D>::kSmemBytes;
     constexpr int kTag = ((D * 4 + (kFP16 ? 2 : 0) + (kAdj ? 1 : 0)) << 1) + (kDecode ? 1 : 0);
     if (ensure_smem_attr<kTag>(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
-    kern<<<args.n_items, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, mt, args);
+    const int grid = kDecode ? args.n_items : std::max(1, std::min(args.n_items, device_sms()));
+    kern<<<grid, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, mt, args);
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
@@ -431,7 +441,10 @@ rfa_status enqueue_table(const rfa_attn_params* p, int64_t T, const int32_t* pos
     ta.inv_dev = invFreq;
     ta.table = static_cast<uint32_t*>(workspace);
     ta.seeds = reinterpret_cast<rfa::RopeSeed*>(static_cast<char*>(workspace) + table_bytes(T, D));
+    ta.sched = sched_of(workspace, T, D, p->B);
     ta.ntokens = static_cast<int32_t>(T);
+    ta.npos = static_cast<int32_t>(T);
+    ta.inv_dev_rows = p->B;
     ta.half = half;
     ta.nseg = p->B;
     ta.uniform_len = tnd ? 0 : p->S;
@@ -459,13 +472,17 @@ rfa_status enqueue_table(const rfa_attn_params* p, int64_t T, const int32_t* pos
 }
 
 rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q, const void* k, const void* v,
-                             const int32_t* seqLens_host, void* out, const void* table, cudaStream_t st) {
+                             const int32_t* seqLens_host, void* out, void* table, cudaStream_t st) {
     const bool tnd = p->layout == RFA_LAYOUT_TND;
     const int D = p->D;
     rfa::AttnArgs aa;
     std::memset(&aa, 0, sizeof aa);
     aa.out = out;
     aa.seeds = reinterpret_cast<const rfa::RopeSeed*>(static_cast<const char*>(table) + table_bytes(T, D));
+    aa.table = static_cast<const uint32_t*>(table);
+    aa.sched = sched_of(table, T, D, p->B);
+    aa.out_elems = T * p->Hq * D;
+    aa.ntok = static_cast<int32_t>(T);
     aa.layout = tnd ? 1 : 0;
     aa.B = p->B;
     aa.Hq = p->Hq;
@@ -559,7 +576,7 @@ rfa_status rfa_rope_attention_table(const rfa_attn_params* p, const int32_t* pos
 }
 
 rfa_status rfa_fused_rope_attention_with_table(const rfa_attn_params* p, const void* q, const void* k, const void* v,
-                                               const int32_t* seqLens_host, void* out, const void* workspace,
+                                               const int32_t* seqLens_host, void* out, void* workspace,
                                                size_t ws_bytes, void* stream) {
     int64_t T = 0;
     rfa_status vs = check_common(p, seqLens_host, &T);
@@ -601,11 +618,11 @@ constexpr int64_t kNoAllocMaxTokens = 65536;  // T limit of the fixed scratch
 constexpr int kNoAllocMaxSeqs = 16;           // sequences (BNSD: batches) limit
 constexpr size_t kNoAllocTableBytes = static_cast<size_t>(kNoAllocMaxTokens) * 128 * 2;  // D <= 128
 constexpr size_t kNoAllocSeedBytes = (kNoAllocMaxSeqs * sizeof(rfa::RopeSeed) + 255) / 256 * 256;
-constexpr size_t kNoAllocBytes = kNoAllocTableBytes + kNoAllocSeedBytes;
+constexpr size_t kNoAllocBytes = kNoAllocTableBytes + kNoAllocSeedBytes + kSchedBytes;
 
 }  // namespace
 
-// The scratch itself: one copy per device that loads the module (~16.1 MB).
+// The scratch itself: one copy per device that loads the module (~16.8 MB).
 // Host code must not pass this symbol to a kernel (on the host it is only a
 // stand-in); its device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
@@ -650,7 +667,8 @@ rfa_status rfa_fused_rope_attention_noalloc(const rfa_attn_params* p, const void
     rfa_status r = noalloc_scratch(&scratch);
     if (r != RFA_OK) return r;
     // Nothing in the scratch needs to start at zero: the table and seed
-    // kernels write every byte the attention kernel reads.
+    // kernels write every byte the attention kernel reads, and zero its work
+    // counters.
     cudaStream_t st = as_stream(stream);
     r = enqueue_table(p, T, position, seqLens_host, invFreq, scratch, st);
     if (r != RFA_OK) return r;
@@ -766,6 +784,8 @@ rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, 
     ta.nseg = 1;
     ta.uniform_len = p->Hq * p->Sq;  // row t belongs to sequence t / (Hq * Sq)
     ta.pos_sq = p->Sq;               // and reads position q_pos[b, t % Sq]
+    ta.npos = p->B * p->Sq;
+    ta.inv_dev_rows = p->B;
     if (!invFreq) {
         ta.inv_host_rows = 1;
         inv_freq_row(p->rope_base, D, ta.inv_host);
@@ -792,6 +812,8 @@ rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, 
     aa.dec_chunk = pl.chunk;
     aa.dec_max_len = p->max_kv_len;
     aa.kv_lens = kv_lens;
+    aa.out_elems = pl.rq * D;
+    aa.ntok = p->B * p->Smax;
     aa.part_o = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.tab_bytes) : nullptr;
     aa.part_ml = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.tab_bytes + pl.po_bytes) : nullptr;
     const uint64_t esz = 2, rows_cache = static_cast<uint64_t>(p->B) * p->Smax;

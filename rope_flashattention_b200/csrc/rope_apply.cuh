@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyArgs a) 
         const int32_t hg = static_cast<int32_t>(rem % hgroups);
         const int32_t r = static_cast<int32_t>(rem / hgroups);
         const int32_t e0 = 8 * static_cast<int32_t>(c), e1 = half + e0;
+        // every row index below derives from r < R and a head < Hq + Hkv
+        if (!in_bounds(r >= 0 && r < a.R && hg * kApplyHeads < H && e1 + 8 <= a.D)) continue;
         const size_t tsz = sizeof(TabT);
         const char* srow = static_cast<const char*>(a.sin_t) + static_cast<size_t>(r) * a.D * tsz;
         const char* crow = static_cast<const char*>(a.cos_t) + static_cast<size_t>(r) * a.D * tsz;
@@ -246,11 +248,12 @@ __global__ void __launch_bounds__(256, 4) kv_norm_rope_cache_kernel(const KvCach
         const int32_t h = act ? static_cast<int32_t>(row - static_cast<uint32_t>(t) * a.Hkv) : 0;
         const int32_t e0 = 8 * static_cast<int32_t>(c), e1 = half + e0;
         const int64_t off = (static_cast<int64_t>(t) * a.Hkv + h) * a.D;
+        const bool in_range = !act || in_bounds(t < a.T && h < a.Hkv && e1 + 8 <= a.D);
         // k, v and the slot are loaded together, before any store of this iteration (the
         // caches do not overlap k and v), so their latencies overlap
         uint4 ka = make_uint4(0u, 0u, 0u, 0u), kb = ka, va = ka, vb = ka;
         int32_t slot = -1;
-        if (act) {
+        if (act && in_range) {
             const uint16_t* src = static_cast<const uint16_t*>(a.k) + off;
             const uint16_t* vs = static_cast<const uint16_t*>(a.v) + off;
             ka = *reinterpret_cast<const uint4*>(src + e0);
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(256, 4) kv_norm_rope_cache_kernel(const KvCach
 #pragma unroll
         for (int i = 0; i < 8; ++i) ss = fmaf(x0[i], x0[i], fmaf(x1[i], x1[i], ss));
         for (uint32_t o = chunks >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (!act || slot < 0) continue;
+        if (!act || !in_range || slot < 0) continue;
         if (slot >= a.cache_rows) {
             record_status(1 /* RFA_ERR_INVALID_ARG */);
             continue;

@@ -123,9 +123,12 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
 #pragma unroll
         for (int step = kMaxSeqs / 2; step > 0; step >>= 1)
             if (b + step < batch && t >= s_cum[b + step]) b += step;
+        const int64_t o = static_cast<int64_t>(t) * headSize + 8 * c;
+        if (!in_bounds(t < ntokens && b < batch && 8 * c + 8 <= half &&
+                       o + half + 8 <= static_cast<int64_t>(ntokens) * headSize))
+            continue;
         float s[8], co[8];
         sincos8(static_cast<float>(__ldg(pos + t)), inv + static_cast<int64_t>(b) * half + 8 * c, s, co);
-        const int64_t o = static_cast<int64_t>(t) * headSize + 8 * c;
         Pack8<OutT>::store(sinOut + o, s);
         Pack8<OutT>::store(sinOut + o + half, s);
         Pack8<OutT>::store(cosOut + o, co);
@@ -142,19 +145,19 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
 // lanes that share a row read distinct shared-memory banks; for other sizes
 // the order is natural.  Segments: uniform_len > 0 -> segment t / uniform_len,
 // otherwise the host-known prefix sums cum[].
-// Per-sequence seeds of the fused kernel's angle-addition recurrence, used
-// when a sequence's positions are consecutive (pos[tok0 + i] == pos[tok0] + i):
-// with w = invFreq_j, row r of key tile k has angle (P + 128k + r) w, and its
-// (cos, sin) = z0[r % 16] * w16^(r / 16) * w128^k as complex products.
-// Seeds are evaluated in fp64 and rounded once to fp32.
-constexpr int kSeedRows = 16;
+// Per-sequence seeds of the fused kernel's in-tile angle recurrence, used when
+// a sequence's positions are consecutive (pos[tok0 + i] == pos[tok0] + i): a
+// RoPE thread forms the angles (P + row) w_j of its first row of a tile
+// directly (fp64 angle reduced modulo 2 pi, then sin/cos), and reaches its
+// other rows of the tile, `step` rows apart, by complex multiplication with
+// wstep_j = (cos, sin)(step w_j), step = 1024 / (D/2) rows (the RoPE threads
+// sharing a row column).  wstep is evaluated in fp64 and rounded once to fp32.
 struct RopeSeed {
     int32_t consecutive;  // 1: the recurrence applies to this sequence
-    int32_t pos0;
+    int32_t pos0;         // P
     int32_t pad[2];
-    float2 w16[kMaxHalfHost];            // (cos, sin) of 16 w_j
-    float2 w128[kMaxHalfHost];           // (cos, sin) of 128 w_j
-    float2 z0[kSeedRows][kMaxHalfHost];  // (cos, sin) of (P + r) w_j, r < 16
+    float2 wstep[kMaxHalfHost];  // (cos, sin) of step * w_j
+    float inv[kMaxHalfHost];     // w_j
 };
 
 struct TableArgs {
@@ -162,6 +165,9 @@ struct TableArgs {
     const float* inv_dev;  // [nseg, half] or nullptr -> inv_host
     uint32_t* table;       // [ntokens][half] 32-bit words of fp16 cos/sin pairs
     RopeSeed* seeds;       // [nseg]
+    int32_t* sched;        // the fused kernel's two work counters (zeroed here), or nullptr
+    int32_t npos;          // entries of pos
+    int32_t inv_dev_rows;  // rows of inv_dev
     int32_t ntokens;
     int32_t half;
     int32_t nseg;
@@ -173,6 +179,11 @@ struct TableArgs {
 };
 
 __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__ TableArgs a) {
+    // the attention launch that follows on the stream starts from zeroed work counters
+    if (a.sched != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+        a.sched[0] = 0;
+        a.sched[1] = 0;
+    }
     const int32_t chunks = a.half >> 3;
     const int64_t work = static_cast<int64_t>(a.ntokens) * chunks;
     for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < work;
@@ -190,6 +201,12 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
                                      : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
         float s[8], co[8];
         const int32_t pt = a.pos_sq > 0 ? (t / a.uniform_len) * a.pos_sq + t % a.pos_sq : t;
+        const int g0 = (a.half == 64) ? c : 2 * c;
+        const int g1 = (a.half == 64) ? 8 + c : 2 * c + 1;
+        const bool inv_ok = a.inv_dev ? (b < a.inv_dev_rows) : (a.inv_host_rows == 1 || b < a.inv_host_rows);
+        if (!in_bounds(pt >= 0 && pt < a.npos && b >= 0 && inv_ok && 8 * c + 8 <= a.half && g0 < a.half / 4 &&
+                       g1 < a.half / 4))
+            continue;
         sincos8(static_cast<float>(__ldg(a.pos + pt)), inv + 8 * c, s, co);
         uint32_t pr[8];
 #pragma unroll
@@ -201,8 +218,6 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
         }
         uint4* row = reinterpret_cast<uint4*>(a.table + static_cast<int64_t>(t) * a.half);
         // groups 2c and 2c+1 of 4 pairs each
-        const int g0 = (a.half == 64) ? c : 2 * c;
-        const int g1 = (a.half == 64) ? 8 + c : 2 * c + 1;
         row[g0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
         row[g1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
     }
@@ -223,6 +238,9 @@ __global__ void __launch_bounds__(256) rope_seed_kernel(const __grid_constant__ 
         tok0 = a.cum[b];
         len = a.cum[b + 1] - a.cum[b];
     }
+    if (!in_bounds(b < a.nseg && tok0 >= 0 && len >= 1 && static_cast<int64_t>(tok0) + len <= a.ntokens &&
+                   static_cast<int64_t>(tok0) + len <= a.npos))
+        return;  // every thread of the block takes the same branch
     const int32_t p0 = __ldg(a.pos + tok0);
     RopeSeed* sd = a.seeds + b;
     if (blockIdx.y == 0) {
@@ -239,22 +257,15 @@ __global__ void __launch_bounds__(256) rope_seed_kernel(const __grid_constant__ 
     const float* inv = a.inv_dev ? a.inv_dev + static_cast<int64_t>(b) * a.half
                                  : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
     const double two_pi = 6.283185307179586476925286766559;
-    const int32_t nval = a.half * (kSeedRows + 2);
-    for (int32_t i = blockIdx.y * blockDim.x + threadIdx.x; i < nval; i += gridDim.y * blockDim.x) {
-        const int32_t j = i % a.half;
-        const int32_t k = i / a.half;
+    const double step = 1024.0 / static_cast<double>(a.half);  // rows between a RoPE thread's rows
+    for (int32_t j = blockIdx.y * blockDim.x + threadIdx.x; j < a.half; j += gridDim.y * blockDim.x) {
         const double w = static_cast<double>(inv[j]);
-        double ang = (k < kSeedRows) ? (static_cast<double>(p0) + k) * w : (k == kSeedRows ? 16.0 : 128.0) * w;
+        double ang = step * w;
         ang -= two_pi * rint(ang / two_pi);
         float sn, cs;
         sincosf(static_cast<float>(ang), &sn, &cs);
-        const float2 v = make_float2(cs, sn);
-        if (k < kSeedRows)
-            sd->z0[k][j] = v;
-        else if (k == kSeedRows)
-            sd->w16[j] = v;
-        else
-            sd->w128[j] = v;
+        sd->wstep[j] = make_float2(cs, sn);
+        sd->inv[j] = inv[j];
     }
 }
 

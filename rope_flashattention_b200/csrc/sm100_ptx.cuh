@@ -14,6 +14,28 @@ __device__ int32_t g_status;
 
 __device__ __forceinline__ void record_status(int32_t code) { atomicCAS(&g_status, 0, code); }
 
+// Checked build (compiled with -DRFA_CHECKED, as librfa_checked.so): every
+// computed global-memory index, shared-memory offset, TMA coordinate and
+// segment offset is tested before use.  A failed test records
+// RFA_ERR_INVALID_ARG in the status word, and the access is skipped where
+// skipping is safe (plain loads and stores; a TMA load is still issued, since
+// the copy engine clips out-of-range boxes itself and its barrier must
+// complete).  In the normal build in_bounds() is constant true and the tests
+// compile away.
+#ifdef RFA_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+__device__ __forceinline__ bool in_bounds(bool ok) {
+    if constexpr (kChecked) {
+        if (!ok) record_status(1 /* RFA_ERR_INVALID_ARG */);
+        return ok;
+    } else {
+        return true;
+    }
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -86,6 +108,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // times (no early exit between them), because it cannot time out.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also ANDs a predicate over its `count` threads: every
+// participant gets the same result.  Same rule as named_bar_sync: every
+// participating thread must reach it the same number of times.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.and.pred q, %1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(count), "r"(pred ? 1u : 0u)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------- proxies

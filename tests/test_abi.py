@@ -73,14 +73,16 @@ def _ru(x, a=256):
     return (x + a - 1) // a * a
 
 
-SEED_BYTES = 16 + 8 * 64 * 2 + 8 * 16 * 64  # per-sequence recurrence seeds
+# per-sequence seeds: flag/first position, the in-tile step (cos, sin) and the invFreq row
+SEED_BYTES = 16 + 8 * 64 + 4 * 64
+SCHED_BYTES = 256  # the attention kernel's two work counters
 
 
 def test_workspace_size(lib):
     f = lib.rfa_fused_rope_attention_workspace
-    # cos/sin table (D/2 fp16 cos + D/2 fp16 sin per token) + one seed block per sequence
-    assert f(ctypes.byref(_p()), 128) == _ru(128 * 64 * 2) + _ru(SEED_BYTES)
-    assert f(ctypes.byref(_p(D=128, B=3)), 1000) == _ru(1000 * 128 * 2) + _ru(3 * SEED_BYTES)
+    # cos/sin table (D/2 fp16 cos + D/2 fp16 sin per token) + one seed block per sequence + counters
+    assert f(ctypes.byref(_p()), 128) == _ru(128 * 64 * 2) + _ru(SEED_BYTES) + SCHED_BYTES
+    assert f(ctypes.byref(_p(D=128, B=3)), 1000) == _ru(1000 * 128 * 2) + _ru(3 * SEED_BYTES) + SCHED_BYTES
     assert f(ctypes.byref(_p(D=96)), 128) == 0          # unsupported head dim
     assert f(ctypes.byref(_p(Hq=3, Hkv=2)), 128) == 0    # Hq % Hkv != 0
     assert f(ctypes.byref(_p(io_dtype=0)), 128) == 0     # UNDEFINED dtype
