@@ -128,11 +128,11 @@ struct AttnCfg {
     static constexpr int kOffBar = kOffT + kTStages * kTabBytes;
     // barrier indices
     static constexpr int kBarQFull = 0;  // the item's query tiles landed (decode: and their cos/sin rows)
-    static constexpr int kBarQReady = 1; // both rotated (4 RoPE warp arrivals)
-    static constexpr int kBarQEmpty = 2; // the item's last QK MMAs are done: the query slots may be reloaded
-    static constexpr int kBarItemFull = 3;   // 2: item index published in the slot
-    static constexpr int kBarItemEmpty = 5;  // 2: every consumer warp has read the slot
-    static constexpr int kBarKFull = 7;
+    static constexpr int kBarQReady = 1; // 2: query tile i rotated (its 8 softmax warps; decode: the RoPE warps, tile 0)
+    static constexpr int kBarQEmpty = 3; // the item's last QK MMAs are done: the query slots may be reloaded
+    static constexpr int kBarItemFull = 4;   // 2: item index published in the slot
+    static constexpr int kBarItemEmpty = 6;  // 2: every consumer warp has read the slot
+    static constexpr int kBarKFull = 8;
     static constexpr int kBarVFull = kBarKFull + kStages;
     static constexpr int kBarKReady = kBarVFull + kStages;
     static constexpr int kBarKEmpty = kBarKReady + kStages;
@@ -144,8 +144,8 @@ struct AttnCfg {
     static constexpr int kNumBars = kBarMmaFin + 1;
     static constexpr int kOffAbort = kOffBar + 8 * kNumBars;
     static constexpr int kOffTmemSlot = kOffAbort + 16;
-    static constexpr int kOffItem = kOffTmemSlot + 16;  // int32 [2]: the item ring
-    static constexpr int kOffXchg = kOffItem + 16;      // float [2 query tiles][2 column halves][128 rows]
+    static constexpr int kOffItem = kOffTmemSlot + 16;  // ItemSlot [2]: the item ring
+    static constexpr int kOffXchg = kOffItem + 128;     // float [2 query tiles][2 column halves][128 rows]
     // The dynamic shared-memory window starts 1024-byte aligned on sm_100 (the
     // kernel checks it), so no alignment slack is requested.
     static constexpr int kSmemBytes = kOffXchg + 2 * 2 * kBlockM * 4;
@@ -462,16 +462,16 @@ __device__ __forceinline__ void rotate8_state(uint4& x1, uint4& x2, const RecSta
 
 // Rotate a tile whose rows hold consecutive positions, without a table.
 // This thread's rows are r0, r0 + step, ...; z holds the angles of row r0 and
-// (wc, ws) advance them by `step` rows.
+// (wc, ws) advance them by `step` rows.  On return z holds the angles of row
+// r0 + 128, the same thread's first row of the next tile.
 template <int D, bool kFP16, bool kAdj>
-__device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32_t rt, const RecState& z,
+__device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32_t rt, RecState& z,
                                               const uint64_t (&wc)[4], const uint64_t (&ws)[4]) {
     constexpr int kPairsPerRow = D / 16;
     constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
     constexpr int kStep = kRopeThreads / kPairsPerRow;
     const int cp = rt % kPairsPerRow;
     const int r0 = rt / kPairsPerRow;
-    RecState e = z;
     // Modest unrolling: 16 warps run five roles at once and their hot loops
     // must stay resident in the instruction cache.
 #pragma unroll 2
@@ -481,14 +481,12 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
             uint32_t o1, o2;
             task_chunks<D, kAdj>(tile, r, cp, o1, o2);
             uint4 x1 = lds128(o1), x2 = lds128(o2);
-            rotate8_state<kFP16, kAdj>(x1, x2, e);
+            rotate8_state<kFP16, kAdj>(x1, x2, z);
             sts128(o1, x1);
             sts128(o2, x2);
         }
-        if (it + 1 < kIters) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) rec_step(e.c[k], e.s[k], wc[k], ws[k]);
-        }
+        for (int k = 0; k < 4; ++k) rec_step(z.c[k], z.s[k], wc[k], ws[k]);
     }
 }
 
@@ -520,33 +518,46 @@ __device__ __forceinline__ void angles_at(int32_t P, int32_t row, const float (&
 
 // Rotate the first `rows` rows of a tile with cos/sin rows read from the
 // global table (tab points at the tile's first row; D/2 32-bit words per row,
-// laid out as rope_table_kernel writes them).
-template <int D, bool kFP16, bool kAdj>
-__device__ __forceinline__ void rope_tile_global(uint32_t tile, const uint32_t* tab, int32_t rows, int32_t rt) {
+// laid out as rope_table_kernel writes them), by kThreads threads (tid <
+// kThreads).  The table loads of kBatch rows are issued together, so one round
+// trip to L2 covers each batch.
+template <int D, bool kFP16, bool kAdj, int kThreads, int kBatch = 2>
+__device__ __forceinline__ void rope_tile_global(uint32_t tile, const uint32_t* tab, int32_t rows, int32_t tid) {
     constexpr int kPairsPerRow = D / 16;
-    constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
-    constexpr int kStep = kRopeThreads / kPairsPerRow;
-    const int cp = rt % kPairsPerRow;
-    const int r0 = rt / kPairsPerRow;
+    constexpr int kIters = kBlockM * kPairsPerRow / kThreads;
+    constexpr int kStep = kThreads / kPairsPerRow;
+    const int cp = tid % kPairsPerRow;
+    const int r0 = tid / kPairsPerRow;
     // chunk positions of frequencies 8cp..8cp+3 and 8cp+4..8cp+7 within a row
     const int g0 = (D == 128) ? cp : 2 * cp;
     const int g1 = (D == 128) ? 8 + cp : 2 * cp + 1;
-#pragma unroll 2
-    for (int it = 0; it < kIters; ++it) {
-        const int r = r0 + it * kStep;
-        if (r >= rows) break;
-        if (!task_in_tile<D>(r, cp) || !in_bounds(g0 < D / 8 && g1 < D / 8)) continue;
-        const uint4* row = reinterpret_cast<const uint4*>(tab + static_cast<int64_t>(r) * (D / 2));
-        const uint4 t0 = __ldg(row + g0), t1 = __ldg(row + g1);
-        uint32_t o1, o2;
-        task_chunks<D, kAdj>(tile, r, cp, o1, o2);
-        uint4 x1 = lds128(o1), x2 = lds128(o2);
-        if constexpr (kAdj)
-            rotate8_adj<kFP16>(x1, x2, t0, t1);
-        else
-            rotate8<kFP16>(x1, x2, t0, t1);
-        sts128(o1, x1);
-        sts128(o2, x2);
+    if (!task_in_tile<D>(r0, cp) || !in_bounds(g0 < D / 8 && g1 < D / 8)) return;
+#pragma unroll 1
+    for (int b0 = 0; b0 < kIters; b0 += kBatch) {
+        uint4 t0[kBatch], t1[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int r = r0 + (b0 + u) * kStep;
+            if (b0 + u < kIters && r < rows) {
+                const uint4* row = reinterpret_cast<const uint4*>(tab + static_cast<int64_t>(r) * (D / 2));
+                t0[u] = __ldg(row + g0);
+                t1[u] = __ldg(row + g1);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int r = r0 + (b0 + u) * kStep;
+            if (b0 + u >= kIters || r >= rows) break;
+            uint32_t o1, o2;
+            task_chunks<D, kAdj>(tile, r, cp, o1, o2);
+            uint4 x1 = lds128(o1), x2 = lds128(o2);
+            if constexpr (kAdj)
+                rotate8_adj<kFP16>(x1, x2, t0[u], t1[u]);
+            else
+                rotate8<kFP16>(x1, x2, t0[u], t1[u]);
+            sts128(o1, x1);
+            sts128(o2, x2);
+        }
     }
 }
 
@@ -590,6 +601,16 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 struct ItemShape {
     int32_t nq, n0, n1, n_kv;
 };
+// One slot of the item ring in shared memory: the index (-1: none left, -2:
+// the producer gave up) and, for an index >= 0, the item decoded once by the
+// producer for all readers.
+struct ItemSlot {
+    int32_t x;
+    WorkItem w;
+    ItemShape sh;
+};
+static_assert(2 * sizeof(ItemSlot) <= 128, "item ring slots");
+
 template <bool kDecode>
 __device__ __forceinline__ ItemShape item_shape(const AttnArgs& a, const WorkItem& w) {
     ItemShape sh;
@@ -623,7 +644,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t* smem = smem_raw;
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(smem + C::kOffAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmemSlot);
-    volatile int32_t* item_slot = reinterpret_cast<volatile int32_t*>(smem + C::kOffItem);
+    ItemSlot* item_slot = reinterpret_cast<ItemSlot*>(smem + C::kOffItem);
     auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8u * static_cast<uint32_t>(i); };
 
     const int warp = threadIdx.x >> 5;
@@ -659,7 +680,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     constexpr uint32_t kItemReaders = kSoftmaxWarps + kRopeWarps + 2;
     if (threadIdx.x == 0) {
         mbar_init(bar(C::kBarQFull), 1);
-        mbar_init(bar(C::kBarQReady), kRopeWarps);
+        mbar_init(bar(C::kBarQReady + 0), kDecode ? kRopeWarps : 8);
+        mbar_init(bar(C::kBarQReady + 1), 8);
         mbar_init(bar(C::kBarQEmpty), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(C::kBarItemFull + s), 1);
@@ -702,15 +724,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             return x < a.n_items ? x : -1;
         }
     };
-    // Consumer side of the ring: the k-th index, or -2 if the wait gave up.  Called by lane 0
-    // alone (warp_wide false) or by all lanes of a warp, which then all read the slot before
-    // lane 0 releases it.
-    auto read_item = [&](int32_t k, bool warp_wide) -> int32_t {
+    // Consumer side of the ring: wait for the k-th slot (nullptr if the wait gave up), read
+    // what the role needs from it, then release it.  Called by lane 0 alone (warp_wide false)
+    // or by all lanes of a warp, which then all read the slot before lane 0 releases it.
+    auto wait_item = [&](int32_t k) -> const ItemSlot* {
         const int s = k & 1;
-        const bool got = mbar_wait(bar(C::kBarItemFull + s), static_cast<uint32_t>(k >> 1) & 1u, abort_flag);
-        const int32_t x = got ? item_slot[s] : -2;
+        // the wait's acquire orders the slot reads after the producer's writes
+        return mbar_wait(bar(C::kBarItemFull + s), static_cast<uint32_t>(k >> 1) & 1u, abort_flag) ? item_slot + s
+                                                                                                  : nullptr;
+    };
+    auto release_item = [&](int32_t k, bool warp_wide) {
         if (warp_wide) __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::kBarItemEmpty + s));
+        if (lane == 0) mbar_arrive(bar(C::kBarItemEmpty + (k & 1)));
+    };
+    auto read_item = [&](int32_t k, bool warp_wide, WorkItem& w, ItemShape& sh) -> int32_t {
+        const ItemSlot* sl = wait_item(k);
+        int32_t x = -2;
+        if (sl != nullptr) {
+            x = sl->x;
+            w = sl->w;
+            sh = sl->sh;
+        }
+        release_item(k, warp_wide);
         return x;
     };
     auto item_of = [&](int32_t x) -> WorkItem {
@@ -736,8 +771,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (k >= 2 && !mbar_wait(bar(C::kBarItemEmpty + s), static_cast<uint32_t>((k >> 1) - 1) & 1u,
                                          abort_flag))
                     return false;
-                item_slot[s] = x;
-                mbar_arrive(bar(C::kBarItemFull + s));  // release: the slot's value is visible to the waiters
+                item_slot[s].x = x;
+                if (x >= 0) {
+                    const WorkItem w = item_of(x);
+                    item_slot[s].w = w;
+                    item_slot[s].sh = item_shape<kDecode>(a, w);
+                }
+                mbar_arrive(bar(C::kBarItemFull + s));  // release: the slot's contents are visible to the waiters
                 return true;
             };
             const bool bnsd = (a.layout == 0);
@@ -748,8 +788,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int32_t it = 0; ok && cur >= 0; ++it) {
                 const int32_t nxt = fetch(it + 1);
                 if (!publish(it + 1, nxt)) break;
-                const WorkItem w = item_of(cur);
-                const ItemShape sh = item_shape<kDecode>(a, w);
+                const WorkItem w = item_slot[it & 1].w;  // published by this thread for item it
+                const ItemShape sh = item_slot[it & 1].sh;
                 const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
                 const bool ktab = !kDecode && !consecutive(w);  // cos/sin rows staged beside each K tile
                 const uint32_t kbytes = C::kTileBytes + (ktab ? C::kTabBytes : 0);
@@ -826,10 +866,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t g = 0;  // value tiles issued so far
             bool ok = true;
             for (int32_t it = 0; ok; ++it) {
-                const int32_t x = read_item(it, false);
-                if (x < 0) break;
-                const WorkItem w = item_of(x);
-                const ItemShape sh = item_shape<kDecode>(a, w);
+                WorkItem w;
+                ItemShape sh;
+                if (read_item(it, false, w, sh) < 0) break;
                 const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
                 for (int32_t j = 0; j < sh.n_kv; ++j) {
                     const int s = g % C::kStages;
@@ -893,11 +932,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t pc[2] = {0u, 0u};       // PFull_i phases consumed so far
             bool ok = true;
             for (int32_t it = 0; ok; ++it) {
-                const int32_t x = read_item(it, false);
-                if (x < 0) break;
-                const ItemShape sh = item_shape<kDecode>(a, item_of(x));
+                WorkItem w;
+                ItemShape sh;
+                if (read_item(it, false, w, sh) < 0) break;
                 const int32_t n0 = sh.n0, n1 = sh.n1, n_kv = sh.n_kv;
-                ok = mbar_wait(bar(C::kBarQReady), static_cast<uint32_t>(it) & 1u, abort_flag);
+                const uint32_t qpar = static_cast<uint32_t>(it) & 1u;
+                ok = mbar_wait(bar(C::kBarQReady + 0), qpar, abort_flag);
                 if constexpr (kDecode) {
                     // Two chains over alternate key tiles (tile j into buffer j % 2).  QK_i of tile
                     // j + 2 reuses S_i: it is issued after PV_i of tile j, which read P_i, and MMAs
@@ -937,6 +977,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (ok) {
                         tc_fence_after();
                         if (n0 > 0) issue_qk(0, g);
+                        ok = mbar_wait(bar(C::kBarQReady + 1), qpar, abort_flag);  // both groups arrive every item
+                    }
+                    if (ok) {
+                        tc_fence_after();
                         if (n1 > 0) issue_qk(1, g);
                         tc_commit(bar(C::kBarKEmpty + g % C::kStages));
                         if (n_kv == 1) tc_commit(bar(C::kBarQEmpty));
@@ -983,47 +1027,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp >= kRopeWarp0 && warp < kRopeWarp0 + kRopeWarps) {
         // ------------------------------------------------------------ RoPE warpgroup
-        // Per item, one loop over the tiles to rotate: key tile 0 (it lands before the query
-        // tiles), the query tiles, then key tiles 1 .. n_kv - 1; one code path per angle
-        // source.  Consecutive positions: every tile's first-row angles are formed directly
-        // (angles_at), the thread's other rows of the tile by the in-tile step; otherwise cos/sin
-        // rows from the table (staged beside a key tile by TMA, read from global memory for the
-        // query tiles).
+        // Per item, one loop over the key tiles to rotate (decode: the query tile, after key tile
+        // 0; prefill query tiles are rotated by the softmax warps).  Consecutive positions: the
+        // first-row angles of key tile 0 are formed directly (angles_at); every row after that
+        // by the step of kStep rows (a thread's rows of a tile, then on into the next key tile);
+        // otherwise cos/sin rows from the table, staged beside the key tile by TMA.
         const int32_t rt = threadIdx.x - kRopeWarp0 * 32;  // 0..127
         constexpr int kPairsPerRow = D / 16;
         const int f0 = 8 * (rt % kPairsPerRow);             // this thread's first frequency
         const int r0 = rt / kPairsPerRow;                   // this thread's first row of a tile
         uint32_t g = 0;  // key tiles rotated so far (ring position)
         for (int32_t it = 0;; ++it) {
-            const int32_t x = read_item(it, true);
-            if (x < 0) break;
-            const WorkItem w = item_of(x);
-            const ItemShape sh = item_shape<kDecode>(a, w);
+            WorkItem w;
+            ItemShape sh;
+            if (read_item(it, true, w, sh) < 0) break;
             const bool rec = consecutive(w);
-            float qw[8];            // this thread's frequencies
             uint64_t wc[4], ws[4];  // in-tile step (cos, sin) of kStep rows, packed pairs
-            int32_t p0 = 0;         // the sequence's first position
+            RecState zk;            // key tiles: this thread's first row of the next tile (recurrence)
             if (rec) {
+                // key tile 0's first-row angles formed directly from the sequence's first position and
+                // this thread's frequencies; every later row by the step
                 const RopeSeed* sd = a.seeds + w.orig;
                 const float4 u0 = *reinterpret_cast<const float4*>(sd->inv + f0);
                 const float4 u1 = *reinterpret_cast<const float4*>(sd->inv + f0 + 4);
-                qw[0] = u0.x; qw[1] = u0.y; qw[2] = u0.z; qw[3] = u0.w;
-                qw[4] = u1.x; qw[5] = u1.y; qw[6] = u1.z; qw[7] = u1.w;
+                const float qw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const float4 v = *reinterpret_cast<const float4*>(sd->wstep + f0 + 2 * k);  // pairs f, f + 1
                     wc[k] = f2pack(v.x, v.z);
                     ws[k] = f2pack(v.y, v.w);
                 }
-                p0 = sd->pos0;
+                angles_at(sd->pos0, r0, qw, zk);
             }
             bool ok = true;
-            const int32_t nrot = sh.n_kv + sh.nq;
+            // decode: key tile 0, the query tile, then the other key tiles; otherwise key tiles
+            // only (the softmax warps rotate the query tiles)
+            const int32_t nqr = kDecode ? sh.nq : 0;
+            const int32_t nrot = sh.n_kv + nqr;
 #pragma unroll 1
             for (int32_t e = 0; e < nrot && ok; ++e) {
-                const bool isq = e >= 1 && e <= sh.nq;
+                const bool isq = e >= 1 && e <= nqr;
                 const int qi = e - 1;                          // query tile (isq)
-                const int32_t j = (e == 0) ? 0 : e - sh.nq;    // key tile (!isq)
+                const int32_t j = (e == 0) ? 0 : e - nqr;      // key tile (!isq)
                 const uint32_t t = g + static_cast<uint32_t>(j);
                 const int s = t % C::kStages;
                 uint32_t tile;
@@ -1044,13 +1089,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     // their cos/sin rows in the second query slot
                     if (isq) rope_tile<D, kFP16, kAdj>(tile, sbase + C::kOffQ + C::kTileBytes, a.G * a.dec_Sq, rt);
                 } else if (rec) {
-                    RecState zz;
-                    angles_at(p0, row0 + r0, qw, zz);
-                    rope_tile_rec<D, kFP16, kAdj>(tile, rows, rt, zz, wc, ws);
-                } else if (isq) {
-                    if (in_bounds(row0 >= 0 && static_cast<int64_t>(w.tok0) + row0 + rows <= a.ntok))
-                        rope_tile_global<D, kFP16, kAdj>(tile, a.table + static_cast<int64_t>(w.tok0 + row0) * (D / 2),
-                                                         rows, rt);
+                    // key tile j > 0 continues from the state key tile j - 1 left (its rows step on by 128)
+                    rope_tile_rec<D, kFP16, kAdj>(tile, rows, rt, zk, wc, ws);
                 } else {
                     rope_tile<D, kFP16, kAdj>(tile, sbase + C::kOffT + (t % C::kTStages) * C::kTabBytes, rows, rt);
                 }
@@ -1060,7 +1100,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (!isq)
                         mbar_arrive(bar(C::kBarKReady + s));
                     else if (qi == sh.nq - 1)
-                        mbar_arrive(bar(C::kBarQReady));
+                        mbar_arrive(bar(C::kBarQReady + 0));
                 }
             }
             g += static_cast<uint32_t>(sh.n_kv);
@@ -1073,8 +1113,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // row exchange half-row maxima (then row sums) through shared memory at named barrier
         // 1 + i (256 threads), executed exactly n_i + 2 times per item by every one of them: a
         // failed (timed-out) wait only turns the remaining work into no-ops, it never skips a
-        // barrier.  All 16 warps decide together, at named barrier 3 (512 threads), whether to
-        // take the next item, so they always run the same items.  A slot written at tile j + 1
+        // barrier.  The 8 warps of a group decide together, with a bar.red.and at the group's
+        // barrier (decode: all 16 at named barrier 3, which its merge also uses), whether to take
+        // the next item, so the warps that share a barrier always run the same items.  A slot
+        // written at tile j + 1
         // was read at tile j before the reader arrived on PFull_i(j), which S_i(j + 1) waits
         // for, so one slot per row and half suffices.
         const int i = warp >> 3;             // query tile
@@ -1090,20 +1132,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t cs = 0;  // SFull_i phases consumed so far
         uint32_t co = 0;  // OFull_i phases consumed so far
         for (int32_t it = 0;; ++it) {
-            const int32_t x = read_item(it, true);
-            if (!named_bar_and(3, kSoftmaxWarps * 32, x >= 0 && *abort_flag == 0)) break;
-            const WorkItem w = item_of(x);
-            const ItemShape sh = item_shape<kDecode>(a, w);
-            const int32_t n0 = sh.n0, n1 = sh.n1;
+            // only the fields this role uses are read from the slot
+            int32_t x = -2, n0 = 0, n1 = 0, nq = 0, L = 0, tok0 = 0, qt_i = 0, h_i = 0, seq = 0, split = 0, qrow0 = 0;
+            if (const ItemSlot* sl = wait_item(it)) {
+                x = sl->x;
+                n0 = sl->sh.n0;
+                n1 = sl->sh.n1;
+                nq = sl->sh.nq;
+                L = sl->w.L;
+                tok0 = sl->w.tok0;
+                qt_i = sl->w.qt[i];
+                h_i = sl->w.h[i];
+                seq = sl->w.seq;
+                if constexpr (kDecode) {
+                    split = sl->w.split;
+                    qrow0 = sl->w.qrow0;
+                }
+            }
+            release_item(it, true);
+            // Prefill: each group decides alone (the groups share no named barrier); decode: the
+            // 16 warps together, as their merge barrier (3) spans both groups.
+            if (!named_bar_and(kDecode ? 3u : nb, kDecode ? kSoftmaxWarps * 32u : 256u, x >= 0 && *abort_flag == 0))
+                break;
+            if constexpr (!kDecode) {
+                // This group rotates its own query tile (idle until its first score tile), with
+                // cos/sin rows from the global table; both groups arrive on their QReady every item.
+                bool qok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarQFull), static_cast<uint32_t>(it) & 1u, abort_flag));
+                if (qok && i < nq) {
+                    const int32_t q0 = qt_i * kBlockM;
+                    const int32_t rows = min(kBlockM, L - q0);
+                    if (in_bounds(q0 >= 0 && static_cast<int64_t>(tok0) + q0 + rows <= a.ntok))
+                        rope_tile_global<D, kFP16, kAdj, 256>(sbase + C::kOffQ + i * C::kTileBytes,
+                                                              a.table + static_cast<int64_t>(tok0 + q0) * (D / 2), rows,
+                                                              ((warp & 7) << 5) + lane);
+                    fence_proxy_async_smem();  // Q' written by the generic proxy, read by the tensor cores
+                }
+                __syncwarp();
+                if (qok && lane == 0) mbar_arrive(bar(C::kBarQReady + i));
+            }
             const int32_t n_i = i == 0 ? n0 : n1;
-            const int32_t qt_i = i == 0 ? w.qt[0] : w.qt[1];
             const int32_t qi = qt_i * kBlockM + row;
-            int32_t vis = a.causal ? min(qi + 1, w.L) : w.L;  // keys [0, vis) visible to this row
+            int32_t vis = a.causal ? min(qi + 1, L) : L;  // keys [0, vis) visible to this row
             if constexpr (kDecode) {
                 // row = g * Sq + s: new token s of the sequence's last Sq sees keys up to len - Sq + s
                 // (bottom-right causal), relative to this split's first key
-                const int32_t len = in_bounds(w.seq >= 0 && w.seq < a.B) ? min(max(a.kv_lens[w.seq], 0), a.dec_Smax) : 0;
-                vis = a.causal ? min(w.L, len - a.dec_Sq + row % a.dec_Sq + 1 - w.split * a.dec_chunk) : w.L;
+                const int32_t len = in_bounds(seq >= 0 && seq < a.B) ? min(max(a.kv_lens[seq], 0), a.dec_Smax) : 0;
+                vis = a.causal ? min(L, len - a.dec_Sq + row % a.dec_Sq + 1 - split * a.dec_chunk) : L;
+            }
+            // prefill epilogue: this thread's output half-row (computed now, so the item's other
+            // fields need not stay live through the tile loop)
+            int64_t o_off = 0;
+            bool o_valid = false;
+            if constexpr (!kDecode) {
+                o_valid = qi < L;
+                o_off = (a.layout == 0) ? ((static_cast<int64_t>(seq) * a.Hq + h_i) * a.S + qi) * D
+                                        : (static_cast<int64_t>(tok0 + qi) * a.Hq + h_i) * D;
+                o_off += hf * kOHalf;
             }
             float m = -INFINITY;  // running max of score * scale * log2(e) (identical in both halves)
             float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
@@ -1221,10 +1305,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     // (m, l) go to the partials that the combine kernel merges
                     bool valid = row < a.G * a.dec_Sq;
                     const bool partial = a.dec_splits > 1;
-                    int64_t o_off = static_cast<int64_t>(w.qrow0 + row) * D;
+                    int64_t o_off = static_cast<int64_t>(qrow0 + row) * D;
                     if (partial) {
                         const int64_t rq = static_cast<int64_t>(a.B) * a.Hq * a.dec_Sq;
-                        const int64_t pr = static_cast<int64_t>(w.split) * rq + w.qrow0 + row;
+                        const int64_t pr = static_cast<int64_t>(split) * rq + qrow0 + row;
                         o_off = pr * D;
                         if (valid) valid = in_bounds(pr >= 0 && pr < a.dec_splits * rq);
                         if (valid && i == 0 && hf == 0) {
@@ -1281,16 +1365,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 if (fin) {
                     tc_fence_after();
-                    const int32_t h_i = i == 0 ? w.h[0] : w.h[1];
                     const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-                    bool valid = qi < w.L;
+                    bool valid = o_valid;
                     uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
-                    int64_t o_off;
-                    if (a.layout == 0)
-                        o_off = ((static_cast<int64_t>(w.seq) * a.Hq + h_i) * a.S + qi) * D;
-                    else
-                        o_off = (static_cast<int64_t>(w.tok0 + qi) * a.Hq + h_i) * D;
-                    o_off += hf * kOHalf;
                     if (valid) valid = in_bounds(o_off >= 0 && o_off + kOHalf <= a.out_elems);
                     const uint64_t il2 = f2pack(inv_l, inv_l);
 #pragma unroll 1
