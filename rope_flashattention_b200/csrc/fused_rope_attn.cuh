@@ -334,31 +334,38 @@ __device__ __forceinline__ void rotate8(uint4& x1, uint4& x2, const uint4& t0, c
     }
 }
 
-// One adjacent pair (x[2i], x[2i+1]) held in a 32-bit word, turned by angle
-// (c, s):  (x0 c - x1 s, x1 c + x0 s).
+// Two adjacent pairs at once: word wa holds pair f (x0, x1), wb pair f + 1;
+// C and S are packed (cos, sin) of frequencies f and f + 1.  The even and odd
+// elements of the two words form packed operands, so one packed operation
+// serves both pairs:  x0' = x0 c - x1 s,  x1' = x1 c + x0 s.
 template <bool kFP16>
-__device__ __forceinline__ uint32_t rot_adj(uint32_t w, float c, float s) {
-    const float2 v = f2unpack(IoT<kFP16>::unpack2(w));
-    return IoT<kFP16>::pack(fmaf(v.x, c, -v.y * s), fmaf(v.y, c, v.x * s));
+__device__ __forceinline__ void rot_adj2(uint32_t& wa, uint32_t& wb, uint64_t C, uint64_t S) {
+    uint64_t X0, X1;
+    if constexpr (kFP16) {
+        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&wa));
+        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&wb));
+        X0 = f2pack(fa.x, fb.x);
+        X1 = f2pack(fa.y, fb.y);
+    } else {  // bf16 -> fp32 is a shift
+        X0 = f2pack(__uint_as_float(wa << 16), __uint_as_float(wb << 16));
+        X1 = f2pack(__uint_as_float(wa & 0xffff0000u), __uint_as_float(wb & 0xffff0000u));
+    }
+    const float2 r0 = f2unpack(fsub2(fmul2(X0, C), fmul2(X1, S)));  // x0 c - x1 s
+    const float2 r1 = f2unpack(ffma2(X1, C, fmul2(X0, S)));         // x1 c + x0 s
+    wa = IoT<kFP16>::pack(r0.x, r1.x);
+    wb = IoT<kFP16>::pack(r0.y, r1.y);
 }
 
 // Rotate 8 adjacent pairs held in two 16-byte chunks (x1: pairs i..i+3, x2:
 // pairs i+4..i+7), angles from the same table words as rotate8 (t0: pairs
-// i..i+3, t1: pairs i+4..i+7).
+// i..i+3, t1: pairs i+4..i+7): words (2m, 2m + 1) of a chunk take the table's
+// cos word 2m and sin word 2m + 1.
 template <bool kFP16>
 __device__ __forceinline__ void rotate8_adj(uint4& x1, uint4& x2, const uint4& t0, const uint4& t1) {
-    uint32_t* a = reinterpret_cast<uint32_t*>(&x1);
-    uint32_t* b = reinterpret_cast<uint32_t*>(&x2);
-    const uint32_t u0[4] = {t0.x, t0.y, t0.z, t0.w}, u1[4] = {t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float2 c0 = __half22float2(*reinterpret_cast<const __half2*>(&u0[(k >> 1) * 2]));
-        const float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&u0[(k >> 1) * 2 + 1]));
-        const float2 c1 = __half22float2(*reinterpret_cast<const __half2*>(&u1[(k >> 1) * 2]));
-        const float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&u1[(k >> 1) * 2 + 1]));
-        a[k] = rot_adj<kFP16>(a[k], (k & 1) ? c0.y : c0.x, (k & 1) ? s0.y : s0.x);
-        b[k] = rot_adj<kFP16>(b[k], (k & 1) ? c1.y : c1.x, (k & 1) ? s1.y : s1.x);
-    }
+    rot_adj2<kFP16>(x1.x, x1.y, h2f2x2(t0.x), h2f2x2(t0.y));
+    rot_adj2<kFP16>(x1.z, x1.w, h2f2x2(t0.z), h2f2x2(t0.w));
+    rot_adj2<kFP16>(x2.x, x2.y, h2f2x2(t1.x), h2f2x2(t1.y));
+    rot_adj2<kFP16>(x2.z, x2.w, h2f2x2(t1.z), h2f2x2(t1.w));
 }
 
 // Shared-memory address of logical 16-byte chunk L of row r of a 128-row
@@ -441,14 +448,12 @@ __device__ __forceinline__ void rotate8_state(uint4& x1, uint4& x2, const RecSta
     uint32_t* xa = reinterpret_cast<uint32_t*>(&x1);
     uint32_t* xb = reinterpret_cast<uint32_t*>(&x2);
     if constexpr (kAdj) {
-        // word k of x1 is pair 8cp + k, of x2 pair 8cp + 4 + k
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 ca = f2unpack(e.c[k >> 1]), sa = f2unpack(e.s[k >> 1]);
-            const float2 cb = f2unpack(e.c[2 + (k >> 1)]), sb = f2unpack(e.s[2 + (k >> 1)]);
-            xa[k] = rot_adj<kFP16>(xa[k], (k & 1) ? ca.y : ca.x, (k & 1) ? sa.y : sa.x);
-            xb[k] = rot_adj<kFP16>(xb[k], (k & 1) ? cb.y : cb.x, (k & 1) ? sb.y : sb.x);
-        }
+        // word k of x1 is pair 8cp + k, of x2 pair 8cp + 4 + k: words (2m, 2m + 1) take the
+        // packed angles of frequencies 8cp + 2m, + 1 (x2: 8cp + 4 + 2m, + 1)
+        rot_adj2<kFP16>(xa[0], xa[1], e.c[0], e.s[0]);
+        rot_adj2<kFP16>(xa[2], xa[3], e.c[1], e.s[1]);
+        rot_adj2<kFP16>(xb[0], xb[1], e.c[2], e.s[2]);
+        rot_adj2<kFP16>(xb[2], xb[3], e.c[3], e.s[3]);
     } else {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -472,18 +477,22 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
     constexpr int kStep = kRopeThreads / kPairsPerRow;
     const int cp = rt % kPairsPerRow;
     const int r0 = rt / kPairsPerRow;
+    // This thread's rows are kStep apart, a multiple of the 8-row swizzle period, so every row's
+    // chunks sit at row r0's offsets plus a multiple of kStep * 128 bytes.
+    static_assert(kStep % 8 == 0, "rows of a thread share the swizzle pattern");
+    uint32_t o1, o2;
+    task_chunks<D, kAdj>(tile, r0, cp, o1, o2);
     // Modest unrolling: 16 warps run five roles at once and their hot loops
     // must stay resident in the instruction cache.
 #pragma unroll 2
     for (int it = 0; it < kIters; ++it) {
         const int r = r0 + it * kStep;
         if (r < rows && task_in_tile<D>(r, cp)) {
-            uint32_t o1, o2;
-            task_chunks<D, kAdj>(tile, r, cp, o1, o2);
-            uint4 x1 = lds128(o1), x2 = lds128(o2);
+            const uint32_t d = static_cast<uint32_t>(it * kStep * 128);
+            uint4 x1 = lds128(o1 + d), x2 = lds128(o2 + d);
             rotate8_state<kFP16, kAdj>(x1, x2, z);
-            sts128(o1, x1);
-            sts128(o2, x2);
+            sts128(o1 + d, x1);
+            sts128(o2 + d, x2);
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) rec_step(z.c[k], z.s[k], wc[k], ws[k]);

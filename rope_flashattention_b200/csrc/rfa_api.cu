@@ -465,9 +465,10 @@ rfa_status enqueue_table(const rfa_attn_params* p, int64_t T, const int32_t* pos
             for (int b = 0; b < p->B; ++b) inv_freq_row(ntk_base(p, seqLens_host[b]), D, ta.inv_host + b * half);
         }
     }
-    rfa::rope_table_kernel<<<grid_for(T * (half / 8), 256), 256, 0, st>>>(ta);
+    // seeds first: the table kernel clears the consecutive flag the seed kernel sets
+    rfa::rope_seed_kernel<<<p->B, 64, 0, st>>>(ta);
     if (cudaGetLastError() != cudaSuccess) return RFA_ERR_CUDA;
-    rfa::rope_seed_kernel<<<dim3(p->B, rfa::kSeedSplit), 256, 0, st>>>(ta);
+    rfa::rope_table_kernel<<<grid_for(T * (half / 8), 256), 256, 0, st>>>(ta);
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 

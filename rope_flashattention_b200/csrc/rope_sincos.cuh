@@ -207,7 +207,16 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
         if (!in_bounds(pt >= 0 && pt < a.npos && b >= 0 && inv_ok && 8 * c + 8 <= a.half && g0 < a.half / 4 &&
                        g1 < a.half / 4))
             continue;
-        sincos8(static_cast<float>(__ldg(a.pos + pt)), inv + 8 * c, s, co);
+        const int32_t p = __ldg(a.pos + pt);
+        sincos8(static_cast<float>(p), inv + 8 * c, s, co);
+        if (a.seeds != nullptr && c == 0) {
+            // a position that breaks the sequence's run (compared in 64 bits, so positions wrapping
+            // past INT32_MAX do not count as consecutive) clears its consecutive flag, which
+            // rope_seed_kernel set before this kernel
+            const int32_t tok0 = a.uniform_len > 0 ? b * a.uniform_len : a.cum[b];
+            if (static_cast<int64_t>(p) != static_cast<int64_t>(__ldg(a.pos + tok0)) + (t - tok0))
+                a.seeds[b].consecutive = 0;
+        }
         uint32_t pr[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -223,42 +232,25 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
     }
 }
 
-// Consecutive-positions flag and recurrence seeds.  Grid (sequences, kSeedSplit):
-// block (b, 0) also checks the sequence's positions; every block computes a
-// share of the seed angles.  Each angle is formed and reduced modulo 2 pi in
-// fp64, then evaluated with fp32 sincos of the reduced angle (|error| ~1e-7).
-constexpr int kSeedSplit = 4;
-__global__ void __launch_bounds__(256) rope_seed_kernel(const __grid_constant__ TableArgs a) {
+// Per-sequence seeds (grid: one block per sequence; runs before
+// rope_table_kernel, which clears the consecutive flag of a sequence whose
+// positions break the run): the flag set, the first position, the invFreq row
+// and the in-tile step (cos, sin) of step * w_j, the angle formed and reduced
+// modulo 2 pi in fp64, then evaluated with fp32 sincos (|error| ~1e-7).
+__global__ void __launch_bounds__(64) rope_seed_kernel(const __grid_constant__ TableArgs a) {
     const int32_t b = blockIdx.x;
-    int32_t tok0, len;
-    if (a.uniform_len > 0) {
-        tok0 = b * a.uniform_len;
-        len = a.uniform_len;
-    } else {
-        tok0 = a.cum[b];
-        len = a.cum[b + 1] - a.cum[b];
-    }
-    if (!in_bounds(b < a.nseg && tok0 >= 0 && len >= 1 && static_cast<int64_t>(tok0) + len <= a.ntokens &&
-                   static_cast<int64_t>(tok0) + len <= a.npos))
-        return;  // every thread of the block takes the same branch
-    const int32_t p0 = __ldg(a.pos + tok0);
+    const int32_t tok0 = a.uniform_len > 0 ? b * a.uniform_len : a.cum[b];
+    if (!in_bounds(b < a.nseg && tok0 >= 0 && tok0 < a.ntokens && tok0 < a.npos)) return;
     RopeSeed* sd = a.seeds + b;
-    if (blockIdx.y == 0) {
-        int ok = 1;
-        // compared in 64 bits: positions near INT32_MAX that wrap around are not consecutive
-        for (int32_t i = threadIdx.x; i < len; i += blockDim.x)
-            if (static_cast<int64_t>(__ldg(a.pos + tok0 + i)) != static_cast<int64_t>(p0) + i) ok = 0;
-        ok = __syncthreads_and(ok);
-        if (threadIdx.x == 0) {
-            sd->consecutive = ok;
-            sd->pos0 = p0;
-        }
+    if (threadIdx.x == 0) {
+        sd->consecutive = 1;
+        sd->pos0 = __ldg(a.pos + tok0);
     }
     const float* inv = a.inv_dev ? a.inv_dev + static_cast<int64_t>(b) * a.half
                                  : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
     const double two_pi = 6.283185307179586476925286766559;
     const double step = 1024.0 / static_cast<double>(a.half);  // rows between a RoPE thread's rows
-    for (int32_t j = blockIdx.y * blockDim.x + threadIdx.x; j < a.half; j += gridDim.y * blockDim.x) {
+    for (int32_t j = threadIdx.x; j < a.half; j += blockDim.x) {
         const double w = static_cast<double>(inv[j]);
         double ang = step * w;
         ang -= two_pi * rint(ang / two_pi);
