@@ -591,14 +591,15 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
     }
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, A = P in TMEM.
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16, A = P in TMEM; only where `issue` is nonzero.
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
+                                        uint32_t accumulate, uint32_t issue) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "setp.ne.b32 e, %5, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(issue)
         : "memory");
 }
 
@@ -904,7 +905,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ tcgen05 issuer
-        if (lane == 0) {
+        // The whole warp runs the loop, converged (every wait's outcome is voted across the
+        // lanes); the elected lane issues the MMAs and commits.
+        {
+            const uint32_t leader = elect_one();
+            auto wait = [&](uint32_t b, uint32_t parity) {
+                return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag));
+            };
             constexpr uint32_t kIdescQK = idesc_f16(IoT<kFP16>::kFmt, 0, 0, kBlockM, kBlockN);
             constexpr uint32_t kIdescPV = idesc_f16(IoT<kFP16>::kFmt, 0, 1, kBlockM, D);
             // S_i = Q_i' K'^T into TMEM buffer i (A = Q_i' and B = K' from shared memory), key tile
@@ -919,9 +926,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t koff16 = ((k >> 2) * C::kAtomBytes + (k & 3) * 32) >> 4;
-                    umma_ss(dS, qd + koff16, kd + koff16, kIdescQK, k > 0 ? 1u : 0u);
+                    umma_ss(dS, qd + koff16, kd + koff16, kIdescQK, k > 0 ? 1u : 0u, leader);
                 }
-                tc_commit(bar(C::kBarSFull + i));
+                tc_commit(bar(C::kBarSFull + i), leader);
             };
             // O_i += P_i V (A = P_i from TMEM buffer i: keys [64h, 64h + 64) at columns [64h, 64h + 32);
             // B = the value tile at ring position t) (acc: O_i already holds a partial sum)
@@ -932,21 +939,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k)
                     umma_ts(dO, aP + (k >> 2) * 64 + (k & 3) * 8, vd + ((k * 16 * 128) >> 4), kIdescPV,
-                            (acc || k > 0) ? 1u : 0u);
+                            (acc || k > 0) ? 1u : 0u, leader);
             };
             auto kready = [&](uint32_t t) {
-                return mbar_wait(bar(C::kBarKReady + t % C::kStages), (t / C::kStages) & 1u, abort_flag);
+                return wait(bar(C::kBarKReady + t % C::kStages), (t / C::kStages) & 1u);
             };
             uint32_t g = 0;                  // key/value tiles consumed so far (ring position)
             uint32_t pc[2] = {0u, 0u};       // PFull_i phases consumed so far
             bool ok = true;
             for (int32_t it = 0; ok; ++it) {
-                WorkItem w;
-                ItemShape sh;
-                if (read_item(it, false, w, sh) < 0) break;
-                const int32_t n0 = sh.n0, n1 = sh.n1, n_kv = sh.n_kv;
+                // lane 0 takes the item from the ring; the warp follows its copy of the shape
+                int32_t x = -2, n0 = 0, n1 = 0, n_kv = 0;
+                if (lane == 0) {
+                    WorkItem w;
+                    ItemShape sh;
+                    x = read_item(it, false, w, sh);
+                    if (x >= 0) {
+                        n0 = sh.n0;
+                        n1 = sh.n1;
+                        n_kv = sh.n_kv;
+                    }
+                }
+                __syncwarp();
+                x = __shfl_sync(0xffffffffu, x, 0);
+                n0 = __shfl_sync(0xffffffffu, n0, 0);
+                n1 = __shfl_sync(0xffffffffu, n1, 0);
+                n_kv = __shfl_sync(0xffffffffu, n_kv, 0);
+                if (x < 0) break;
                 const uint32_t qpar = static_cast<uint32_t>(it) & 1u;
-                ok = mbar_wait(bar(C::kBarQReady + 0), qpar, abort_flag);
+                ok = wait(bar(C::kBarQReady + 0), qpar);
                 if constexpr (kDecode) {
                     // Two chains over alternate key tiles (tile j into buffer j % 2).  QK_i of tile
                     // j + 2 reuses S_i: it is issued after PV_i of tile j, which read P_i, and MMAs
@@ -956,28 +977,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         if (!ok) break;
                         tc_fence_after();
                         issue_qk(j, g + j);
-                        tc_commit(bar(C::kBarKEmpty + (g + j) % C::kStages));
+                        tc_commit(bar(C::kBarKEmpty + (g + j) % C::kStages), leader);
                     }
                     for (int32_t j = 0; j < n_kv && ok; ++j) {
                         const uint32_t t = g + j;
                         const int i = j & 1;
-                        ok = mbar_wait(bar(C::kBarVFull + t % C::kStages), (t / C::kStages) & 1u, abort_flag) &&
-                             mbar_wait(bar(C::kBarPFull + i), pc[i] & 1u, abort_flag);
+                        ok = wait(bar(C::kBarVFull + t % C::kStages), (t / C::kStages) & 1u) &&
+                             wait(bar(C::kBarPFull + i), pc[i] & 1u);
                         if (!ok) break;
                         ++pc[i];
                         tc_fence_after();
                         issue_pv(i, t, j >= 2);
-                        if (j + 2 >= n_kv) tc_commit(bar(C::kBarOFull + i));  // last tile of buffer i
-                        tc_commit(bar(C::kBarVEmpty + t % C::kStages));
+                        if (j + 2 >= n_kv) tc_commit(bar(C::kBarOFull + i), leader);  // last tile of buffer i
+                        tc_commit(bar(C::kBarVEmpty + t % C::kStages), leader);
                         if (j + 2 < n_kv) {
                             ok = kready(t + 2);
                             if (!ok) break;
                             tc_fence_after();
                             issue_qk(i, t + 2);
-                            tc_commit(bar(C::kBarKEmpty + (t + 2) % C::kStages));
+                            tc_commit(bar(C::kBarKEmpty + (t + 2) % C::kStages), leader);
                         }
                     }
-                    tc_commit(bar(C::kBarQEmpty));
+                    tc_commit(bar(C::kBarQEmpty), leader);
                 } else {
                     // Order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  The item's
                     // last QK is followed by a commit to QEmpty, so the producer can load the next
@@ -986,26 +1007,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (ok) {
                         tc_fence_after();
                         if (n0 > 0) issue_qk(0, g);
-                        ok = mbar_wait(bar(C::kBarQReady + 1), qpar, abort_flag);  // both groups arrive every item
+                        ok = wait(bar(C::kBarQReady + 1), qpar);  // both groups arrive every item
                     }
                     if (ok) {
                         tc_fence_after();
                         if (n1 > 0) issue_qk(1, g);
-                        tc_commit(bar(C::kBarKEmpty + g % C::kStages));
-                        if (n_kv == 1) tc_commit(bar(C::kBarQEmpty));
+                        tc_commit(bar(C::kBarKEmpty + g % C::kStages), leader);
+                        if (n_kv == 1) tc_commit(bar(C::kBarQEmpty), leader);
                     }
                     for (int32_t j = 0; j < n_kv && ok; ++j) {
                         const uint32_t t = g + j;
                         const int32_t jn = j + 1;
-                        ok = mbar_wait(bar(C::kBarVFull + t % C::kStages), (t / C::kStages) & 1u, abort_flag);
+                        ok = wait(bar(C::kBarVFull + t % C::kStages), (t / C::kStages) & 1u);
                         if (!ok) break;
                         if (j < n0) {
-                            ok = mbar_wait(bar(C::kBarPFull + 0), pc[0] & 1u, abort_flag);
+                            ok = wait(bar(C::kBarPFull + 0), pc[0] & 1u);
                             if (!ok) break;
                             ++pc[0];
                             tc_fence_after();
                             issue_pv(0, t, j > 0);
-                            if (j == n0 - 1) tc_commit(bar(C::kBarOFull + 0));
+                            if (j == n0 - 1) tc_commit(bar(C::kBarOFull + 0), leader);
                         }
                         if (jn < n_kv) {
                             ok = kready(t + 1);
@@ -1014,24 +1035,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             if (jn < n0) issue_qk(0, t + 1);
                         }
                         if (j < n1) {
-                            ok = mbar_wait(bar(C::kBarPFull + 1), pc[1] & 1u, abort_flag);
+                            ok = wait(bar(C::kBarPFull + 1), pc[1] & 1u);
                             if (!ok) break;
                             ++pc[1];
                             tc_fence_after();
                             issue_pv(1, t, j > 0);
-                            if (j == n1 - 1) tc_commit(bar(C::kBarOFull + 1));
+                            if (j == n1 - 1) tc_commit(bar(C::kBarOFull + 1), leader);
                         }
-                        tc_commit(bar(C::kBarVEmpty + t % C::kStages));
+                        tc_commit(bar(C::kBarVEmpty + t % C::kStages), leader);
                         if (jn < n_kv) {
                             if (jn < n1) issue_qk(1, t + 1);
-                            tc_commit(bar(C::kBarKEmpty + (t + 1) % C::kStages));
-                            if (jn == n_kv - 1) tc_commit(bar(C::kBarQEmpty));
+                            tc_commit(bar(C::kBarKEmpty + (t + 1) % C::kStages), leader);
+                            if (jn == n_kv - 1) tc_commit(bar(C::kBarQEmpty), leader);
                         }
                     }
                 }
                 g += static_cast<uint32_t>(n_kv);
             }
-            tc_commit(bar(C::kBarMmaFin));
+            tc_commit(bar(C::kBarMmaFin), leader);
             mbar_wait_drain(bar(C::kBarMmaFin), 0);
         }
     } else if (warp >= kRopeWarp0 && warp < kRopeWarp0 + kRopeWarps) {
