@@ -344,6 +344,15 @@ RFA_API rfa_status rfa_get_device_status(void* stream);
  * this library.  RFA_ERR_CUDA if the device variable cannot be written. */
 RFA_API rfa_status rfa_set_wait_limit_ns(uint64_t ns);
 
+/* Failure-detection switch on the current device, off by default.  While on
+ * (nonzero), the attention kernels (fused and decode) publish no work item:
+ * each of their roles waits on an item barrier that nothing arrives on, the
+ * wait runs out at the limit set by rfa_set_wait_limit_ns, the kernel records
+ * RFA_ERR_TIMEOUT, leaves its output unwritten and returns with the context
+ * intact.  0 turns it off.  Synchronous; must not overlap running kernels of
+ * this library.  RFA_ERR_CUDA if the device variable cannot be written. */
+RFA_API rfa_status rfa_set_hold_items(int32_t on);
+
 /* Static, human-readable name of a status code. */
 RFA_API const char* rfa_status_string(rfa_status s);
 

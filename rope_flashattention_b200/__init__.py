@@ -32,7 +32,7 @@ __all__ = [
     "fused_rope_attention_workspace", "rope_attention_table", "fused_rope_attention_with_table",
     "fused_rope_attention_noalloc", "rope_apply", "kv_rms_norm_rope_cache", "KvCacheParams",
     "decode_rope_attention", "DecodeParams",
-    "get_device_status", "set_wait_limit_ns", "status_string", "AttnParams", "RopeApplyParams",
+    "get_device_status", "set_wait_limit_ns", "set_hold_items", "status_string", "AttnParams", "RopeApplyParams",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librfa.so")
@@ -53,6 +53,7 @@ EXPORTS = (
     "rfa_fused_rope_attention_noalloc",
     "rfa_get_device_status",
     "rfa_set_wait_limit_ns",
+    "rfa_set_hold_items",
     "rfa_status_string",
     "rfa_version",
 )
@@ -190,6 +191,8 @@ def _open(path: str):
     lib.rfa_decode_rope_attention.restype = ctypes.c_int
     lib.rfa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.rfa_set_wait_limit_ns.restype = ctypes.c_int
+    lib.rfa_set_hold_items.argtypes = [I32]
+    lib.rfa_set_hold_items.restype = ctypes.c_int
     lib.rfa_get_device_status.argtypes = [P]
     lib.rfa_get_device_status.restype = ctypes.c_int
     lib.rfa_status_string.argtypes = [ctypes.c_int]
@@ -203,6 +206,12 @@ def set_wait_limit_ns(ns: int) -> None:
     """Kernel role-to-role wait limit on the current device (0: default 2 s);
     for failure-detection tests (rfa_set_wait_limit_ns)."""
     _check(load_library().rfa_set_wait_limit_ns(int(ns)), "rfa_set_wait_limit_ns")
+
+
+def set_hold_items(on: bool) -> None:
+    """Failure-detection switch on the current device (rfa_set_hold_items): while
+    on, the attention kernels publish no work item and their waits run out."""
+    _check(load_library().rfa_set_hold_items(1 if on else 0), "rfa_set_hold_items")
 
 
 def status_string(code: int) -> str:

@@ -772,31 +772,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ Q/K producer (+ item fetch)
-        if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmT);
+        // Both producer warps run converged, their waits voted across the lanes; lane 0 alone
+        // fetches, writes the item slots, arrives and issues the copies (a single-lane branch
+        // around the whole loop is starved of issue slots by the busy warps beside it).
+        {
+            const uint32_t leader = (lane == 0) ? 1u : 0u;
+            auto wait = [&](uint32_t b, uint32_t parity) {
+                return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag));
+            };
+            if (leader) {
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmT);
+            }
+            auto fetch_all = [&](int32_t k) -> int32_t {
+                int32_t x = 0;
+                if (leader) x = fetch(k);
+                return __shfl_sync(0xffffffffu, x, 0);
+            };
             auto publish = [&](int32_t k, int32_t x) -> bool {
                 const int s = k & 1;
-                if (k >= 2 && !mbar_wait(bar(C::kBarItemEmpty + s), static_cast<uint32_t>((k >> 1) - 1) & 1u,
-                                         abort_flag))
+                if (k >= 2 && !wait(bar(C::kBarItemEmpty + s), static_cast<uint32_t>((k >> 1) - 1) & 1u))
                     return false;
-                item_slot[s].x = x;
-                if (x >= 0) {
-                    const WorkItem w = item_of(x);
-                    item_slot[s].w = w;
-                    item_slot[s].sh = item_shape<kDecode>(a, w);
+                if (leader) {
+                    item_slot[s].x = x;
+                    if (x >= 0) {
+                        const WorkItem w = item_of(x);
+                        item_slot[s].w = w;
+                        item_slot[s].sh = item_shape<kDecode>(a, w);
+                    }
+                    mbar_arrive(bar(C::kBarItemFull + s));  // release: the slot's contents are visible to the waiters
                 }
-                mbar_arrive(bar(C::kBarItemFull + s));  // release: the slot's contents are visible to the waiters
+                __syncwarp();  // the other lanes read the slot back
                 return true;
             };
             const bool bnsd = (a.layout == 0);
             uint32_t g = 0;        // key tiles issued so far (ring position)
             int32_t q_items = 0;   // items whose query tiles were issued
-            int32_t cur = fetch(0);
-            bool ok = publish(0, cur);
+            int32_t cur = fetch_all(0);
+            // held: no item is published; the readers' item waits run out, this warp only drains
+            bool ok = *static_cast<volatile int32_t*>(&g_hold_items) == 0 && publish(0, cur);
             for (int32_t it = 0; ok && cur >= 0; ++it) {
-                const int32_t nxt = fetch(it + 1);
+                const int32_t nxt = fetch_all(it + 1);
                 if (!publish(it + 1, nxt)) break;
                 const WorkItem w = item_slot[it & 1].w;  // published by this thread for item it
                 const ItemShape sh = item_slot[it & 1].sh;
@@ -810,46 +827,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                     : (plane < (m == &tmQ ? a.Hq : a.Hkv))));
                     for (int at = 0; at < C::kAtoms; ++at) {
                         if (bnsd)
-                            tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, row0, plane);
+                            tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, row0, plane, leader);
                         else
-                            tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, plane, w.tok0 + row0);
+                            tma_load_3d(dst + at * C::kAtomBytes, m, b, at * 64, plane, w.tok0 + row0, leader);
                     }
                 };
                 auto load_k = [&](int32_t j) -> bool {
                     const int s = g % C::kStages;
                     const uint32_t u = g / C::kStages;
-                    if (u > 0 && !mbar_wait(bar(C::kBarKEmpty + s), (u - 1) & 1u, abort_flag)) return false;
+                    if (u > 0 && !wait(bar(C::kBarKEmpty + s), (u - 1) & 1u)) return false;
                     if (ktab && g >= static_cast<uint32_t>(C::kTStages)) {
                         // the rows slot held the rows of key tile g - kTStages: wait until that tile is rotated
                         const uint32_t gp = g - C::kTStages;
-                        if (!mbar_wait(bar(C::kBarKReady + gp % C::kStages), (gp / C::kStages) & 1u, abort_flag))
+                        if (!wait(bar(C::kBarKReady + gp % C::kStages), (gp / C::kStages) & 1u))
                             return false;
                     }
-                    mbar_expect_tx(bar(C::kBarKFull + s), kbytes);
+                    mbar_expect_tx(bar(C::kBarKFull + s), kbytes, leader);
                     load_tile(&tmK, sbase + C::kOffK + s * C::kTileBytes, bar(C::kBarKFull + s), kvplane, j * kBlockN);
                     if (ktab) {
                         const uint32_t dst = sbase + C::kOffT + (g % C::kTStages) * C::kTabBytes;
                         for (int bx = 0; bx < C::kTabBoxes; ++bx)
                             tma_load_3d(dst + bx * C::kAtomBytes, &tmT, bar(C::kBarKFull + s), bx * 32,
-                                        w.tok0 + j * kBlockN, 0);
+                                        w.tok0 + j * kBlockN, 0, leader);
                     }
                     ++g;
                     return true;
                 };
                 // key tile 0 first (its slot frees before the query slots do), then the query tiles
                 if (!load_k(0)) break;
-                if (it > 0 && !mbar_wait(bar(C::kBarQEmpty), static_cast<uint32_t>(it - 1) & 1u, abort_flag)) break;
+                if (it > 0 && !wait(bar(C::kBarQEmpty), static_cast<uint32_t>(it - 1) & 1u)) break;
                 mbar_expect_tx(bar(C::kBarQFull),
-                               static_cast<uint32_t>(sh.nq) * C::kTileBytes + (kDecode ? C::kTabBytes : 0));
+                               static_cast<uint32_t>(sh.nq) * C::kTileBytes + (kDecode ? C::kTabBytes : 0), leader);
                 for (int i = 0; i < sh.nq; ++i) {
                     if constexpr (kDecode) {  // q viewed as [B*Hq*Sq, D]: the group's rows from qrow0,
                                               // their cos/sin rows in the second query slot
                         for (int at = 0; at < C::kAtoms; ++at)
                             tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64, 0,
-                                        w.qrow0);
+                                        w.qrow0, leader);
                         for (int bx = 0; bx < C::kTabBoxes; ++bx)
                             tma_load_3d(sbase + C::kOffQ + C::kTileBytes + bx * C::kAtomBytes, &tmT,
-                                        bar(C::kBarQFull), bx * 32, w.qrow0, 0);
+                                        bar(C::kBarQFull), bx * 32, w.qrow0, 0, leader);
                     } else {
                         const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
                         load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane,
@@ -870,32 +887,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else if (warp == kTmaVWarp) {
         // ------------------------------------------------------------ V producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmV);
+        // converged like the Q/K producer: lane 0 takes the item and issues
+        {
+            const uint32_t leader = (lane == 0) ? 1u : 0u;
+            if (leader) tma_prefetch_desc(&tmV);
             const bool bnsd = (a.layout == 0);
             uint32_t g = 0;  // value tiles issued so far
             bool ok = true;
             for (int32_t it = 0; ok; ++it) {
-                WorkItem w;
-                ItemShape sh;
-                if (read_item(it, false, w, sh) < 0) break;
-                const int32_t kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
-                for (int32_t j = 0; j < sh.n_kv; ++j) {
+                int32_t x = -2, kvplane = 0, tok0 = 0, n_kv = 0;
+                if (leader) {
+                    WorkItem w;
+                    ItemShape sh;
+                    x = read_item(it, false, w, sh);
+                    if (x >= 0) {
+                        kvplane = bnsd ? (w.seq * a.Hkv + w.kvh) : w.kvh;
+                        tok0 = w.tok0;
+                        n_kv = sh.n_kv;
+                    }
+                }
+                __syncwarp();
+                x = __shfl_sync(0xffffffffu, x, 0);
+                if (x < 0) break;
+                kvplane = __shfl_sync(0xffffffffu, kvplane, 0);
+                tok0 = __shfl_sync(0xffffffffu, tok0, 0);
+                n_kv = __shfl_sync(0xffffffffu, n_kv, 0);
+                for (int32_t j = 0; j < n_kv; ++j) {
                     const int s = g % C::kStages;
                     const uint32_t u = g / C::kStages;
-                    if (u > 0 && !mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag)) {
+                    if (u > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(C::kBarVEmpty + s), (u - 1) & 1u, abort_flag))) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+                    mbar_expect_tx(bar(C::kBarVFull + s), C::kTileBytes, leader);
                     const uint32_t dst = sbase + C::kOffV + s * C::kTileBytes;
                     for (int at = 0; at < C::kAtoms; ++at) {
                         if (bnsd)
                             tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, j * kBlockN,
-                                        kvplane);
+                                        kvplane, leader);
                         else
                             tma_load_3d(dst + at * C::kAtomBytes, &tmV, bar(C::kBarVFull + s), at * 64, kvplane,
-                                        w.tok0 + j * kBlockN);
+                                        tok0 + j * kBlockN, leader);
                     }
                     ++g;
                 }
@@ -1400,22 +1432,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     uint16_t* outp = reinterpret_cast<uint16_t*>(a.out);
                     if (valid) valid = in_bounds(o_off >= 0 && o_off + kOHalf <= a.out_elems);
                     const uint64_t il2 = f2pack(inv_l, inv_l);
+                    // Each thread writes its row's kOHalf contiguous outputs: 32-byte stores (whole
+                    // sectors) when the output is 32-byte aligned, else 16-byte ones.
+                    const bool wide = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
 #pragma unroll 1
                     for (int q = 0; q < kOHalf / 32; ++q) {
                         uint32_t o[32];
                         tmem_ld32(oc + q * 32, o);
                         tmem_wait_ld();
                         if (valid) {
-                            uint4* dst = reinterpret_cast<uint4*>(outp + o_off + q * 32);
+                            uint32_t wv[16];
 #pragma unroll
-                            for (int v4 = 0; v4 < 4; ++v4) {
-                                uint32_t wv[4];
+                            for (int e = 0; e < 16; ++e)
+                                wv[e] = pack2<kFP16>(fmul2(f2pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), il2));
+                            uint16_t* dst = outp + o_off + q * 32;
+                            if (wide) {
+                                stg256(dst, reinterpret_cast<const uint32_t(&)[8]>(wv[0]));
+                                stg256(dst + 16, reinterpret_cast<const uint32_t(&)[8]>(wv[8]));
+                            } else {
+                                uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int c = 8 * v4 + 2 * e;
-                                    wv[e] = pack2<kFP16>(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), il2));
-                                }
-                                dst[v4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                                for (int v4 = 0; v4 < 4; ++v4)
+                                    d4[v4] = make_uint4(wv[4 * v4], wv[4 * v4 + 1], wv[4 * v4 + 2], wv[4 * v4 + 3]);
                             }
                         }
                     }

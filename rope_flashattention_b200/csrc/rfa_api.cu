@@ -217,6 +217,12 @@ rfa_status rfa_set_wait_limit_ns(uint64_t ns) {
     return cudaMemcpyToSymbol(rfa::g_wait_limit_ns, &v, sizeof v) == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
+rfa_status rfa_set_hold_items(int32_t on) {
+    const int32_t v = on != 0 ? 1 : 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return RFA_ERR_CUDA;
+    return cudaMemcpyToSymbol(rfa::g_hold_items, &v, sizeof v) == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+}
+
 rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, const int32_t* seqLens, int32_t batch,
                            int32_t ntokens, int32_t headSize, rfa_dtype outType, void* sinOut, void* cosOut,
                            void* stream) {

@@ -56,8 +56,14 @@ __device__ __forceinline__ void fence_mbar_init() {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+// Arrive on `bar` expecting `bytes` of copies; only where `issue` is nonzero.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes, uint32_t issue) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "setp.ne.b32 e, %2, 0;\n\t"
+        "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar),
+        "r"(bytes), "r"(issue)
+        : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -77,6 +83,10 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // kWaitLimitNs).  Host code may lower it through rfa_set_wait_limit_ns to make
 // waits run out on purpose (failure-detection tests).
 __device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+// Failure-detection switch (off unless a host call sets it): the attention
+// kernels' producers then publish no work item, so every other role waits on
+// an item barrier that nothing arrives on until its limit runs out.
+__device__ int32_t g_hold_items = 0;
 
 // Bounded wait for the phase of `bar` with parity `parity` to complete.
 // Returns false (and raises *abort) if the wait timed out or another role of
@@ -137,14 +147,17 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 // 3-D tiled load of one box into shared memory, completion counted in bytes
-// on `bar`.  c0 is the innermost (element) coordinate and must be a multiple
-// of 16 bytes; the callers only pass multiples of 64 elements.
+// on `bar`; only where `issue` is nonzero (the producer warps run converged
+// and one lane issues).  c0 is the innermost (element) coordinate and must be
+// a multiple of 16 bytes; the callers only pass multiples of 32 elements.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int32_t c0, int32_t c1,
-                                            int32_t c2) {
+                                            int32_t c2, uint32_t issue) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        "{\n\t.reg .pred e;\n\t"
+        "setp.ne.b32 e, %6, 0;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(issue)
         : "memory");
 }
 
@@ -311,6 +324,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
+}
+// 32-byte global store (one full sector); p must be 32-byte aligned.
+__device__ __forceinline__ void stg256(void* p, const uint32_t (&v)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
 }
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)

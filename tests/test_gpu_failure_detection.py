@@ -1,11 +1,17 @@
-"""Failure detection on the GPU without a GPU fault: the kernels' role-to-role
-waits are given a 1 ns limit (rfa_set_wait_limit_ns), so a wait that is not
-complete after its first few hundred polls runs out on purpose.  The kernel
-must then record RFA_ERR_TIMEOUT in the status word, stop its roles, drain
-its copies and MMAs and return; afterwards the context must still be usable:
-with the default limit restored, the same call gives the oracle's result.
-Nothing here traps, faults or hangs a GPU: every wait in the kernels is
-bounded, and the drains before a CTA exits keep their own 2 s limit.
+"""Failure detection on the GPU without a GPU fault.
+
+Two ways to make a kernel's bounded waits run out on purpose:
+- rfa_set_hold_items: the attention kernels publish no work item, so every
+  role waits on an item barrier that nothing arrives on (a flag that nothing
+  sets) until the limit from rfa_set_wait_limit_ns runs out.  Deterministic.
+- a 1 ns limit on a memory-bound call: any wait that mbarrier.try_wait could
+  not absorb in its own suspend window (about 8,000 cycles on B200) runs out
+  mid-pipeline, with copies and MMAs in flight that must be drained.
+Either way the kernel must record RFA_ERR_TIMEOUT, stop its roles, drain and
+return; afterwards the context must still be usable: with the defaults
+restored, the same call gives the oracle's result.  Nothing here traps,
+faults or hangs a GPU: every wait in the kernels is bounded, and the drains
+before a CTA exits keep their own 2 s limit.
 """
 import numpy as np
 import pytest
@@ -34,6 +40,17 @@ def _with_tiny_limit(rfa, call):
         rfa.set_wait_limit_ns(0)  # back to the default, whatever happened
 
 
+def _held(rfa, call):
+    try:
+        rfa.set_wait_limit_ns(2_000_000)  # 2 ms
+        rfa.set_hold_items(True)
+        call()
+        return rfa.get_device_status()
+    finally:
+        rfa.set_hold_items(False)
+        rfa.set_wait_limit_ns(0)
+
+
 def test_fused_kernel_wait_runs_out_and_context_survives(rfa):
     B, Hq, Hkv, S, D = 2, 4, 2, 1024, 128
     q = workloads.randn16((B, Hq, S, D), 90).cuda()
@@ -41,7 +58,7 @@ def test_fused_kernel_wait_runs_out_and_context_survives(rfa):
     v = workloads.randn16((B, Hkv, S, D), 92).cuda()
     pos = torch.arange(S, dtype=torch.int32).repeat(B, 1).contiguous().cuda()
     assert rfa.get_device_status() == 0
-    st = _with_tiny_limit(rfa, lambda: rfa.fused_rope_attention(q, k, v, pos))
+    st = _held(rfa, lambda: rfa.fused_rope_attention(q, k, v, pos))
     assert st == rfa.RFA_ERR_TIMEOUT
     out = rfa.fused_rope_attention(q, k, v, pos)
     assert rfa.get_device_status() == 0
@@ -50,6 +67,22 @@ def test_fused_kernel_wait_runs_out_and_context_survives(rfa):
     ref = oracle.attention_rows(q.cpu(), k.cpu(), v.cpu(), pos.cpu().numpy(), inv, rows)
     got = out.float().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert np.abs(got - ref).max() <= 2e-2
+
+
+def test_decode_held_items_run_out_and_context_survives(rfa):
+    B, Hq, Hkv, Sq, D, L = 2, 8, 2, 1, 128, 2048
+    q = workloads.randn16((B, Hq, Sq, D), 96).cuda()
+    kc = workloads.randn16((B, L, Hkv, D), 97).cuda()
+    vc = workloads.randn16((B, L, Hkv, D), 98).cuda()
+    q_pos = torch.full((B, Sq), L - 1, dtype=torch.int32).cuda()
+    lens = torch.full((B,), L, dtype=torch.int32).cuda()
+    st = _held(rfa, lambda: rfa.decode_rope_attention(q, kc, vc, q_pos, lens))
+    assert st == rfa.RFA_ERR_TIMEOUT
+    out = rfa.decode_rope_attention(q, kc, vc, q_pos, lens)
+    assert rfa.get_device_status() == 0
+    ref = oracle.decode_attention(q.cpu(), kc.cpu(), vc.cpu(), q_pos.cpu().numpy(), [L] * B,
+                                  np.stack([oracle.inv_freq(10000.0, D)] * B))
+    assert np.abs(out.float().cpu().numpy() - ref).max() <= 2e-2
 
 
 def test_decode_wait_runs_out_and_context_survives(rfa):
