@@ -469,12 +469,12 @@ __device__ __forceinline__ void rotate8_state(uint4& x1, uint4& x2, const RecSta
 // This thread's rows are r0, r0 + step, ...; z holds the angles of row r0 and
 // (wc, ws) advance them by `step` rows.  On return z holds the angles of row
 // r0 + 128, the same thread's first row of the next tile.
-template <int D, bool kFP16, bool kAdj>
+template <int D, bool kFP16, bool kAdj, int kThreads = kRopeThreads>
 __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32_t rt, RecState& z,
                                               const uint64_t (&wc)[4], const uint64_t (&ws)[4]) {
     constexpr int kPairsPerRow = D / 16;
-    constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
-    constexpr int kStep = kRopeThreads / kPairsPerRow;
+    constexpr int kIters = kBlockM * kPairsPerRow / kThreads;
+    constexpr int kStep = kThreads / kPairsPerRow;
     const int cp = rt % kPairsPerRow;
     const int r0 = rt / kPairsPerRow;
     // This thread's rows are kStep apart, a multiple of the 8-row swizzle period, so every row's
@@ -1196,6 +1196,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int32_t it = 0;; ++it) {
             // only the fields this role uses are read from the slot
             int32_t x = -2, n0 = 0, n1 = 0, nq = 0, L = 0, tok0 = 0, qt_i = 0, h_i = 0, seq = 0, split = 0, qrow0 = 0;
+            int32_t orig = 0;
             if (const ItemSlot* sl = wait_item(it)) {
                 x = sl->x;
                 n0 = sl->sh.n0;
@@ -1206,6 +1207,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 qt_i = sl->w.qt[i];
                 h_i = sl->w.h[i];
                 seq = sl->w.seq;
+                orig = sl->w.orig;
                 if constexpr (kDecode) {
                     split = sl->w.split;
                     qrow0 = sl->w.qrow0;
@@ -1217,16 +1219,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (!named_bar_and(kDecode ? 3u : nb, kDecode ? kSoftmaxWarps * 32u : 256u, x >= 0 && *abort_flag == 0))
                 break;
             if constexpr (!kDecode) {
-                // This group rotates its own query tile (idle until its first score tile), with
-                // cos/sin rows from the global table; both groups arrive on their QReady every item.
+                // This group rotates its own query tile (idle until its first score tile); both
+                // groups arrive on their QReady every item.  Consecutive positions: each thread's
+                // first-row angles are formed directly from the sequence's seed and its other rows
+                // follow by the recurrence (step of 32 rows, the square of the seed's 16-row step);
+                // otherwise cos/sin rows come from the global table.
                 bool qok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarQFull), static_cast<uint32_t>(it) & 1u, abort_flag));
                 if (qok && i < nq) {
                     const int32_t q0 = qt_i * kBlockM;
                     const int32_t rows = min(kBlockM, L - q0);
-                    if (in_bounds(q0 >= 0 && static_cast<int64_t>(tok0) + q0 + rows <= a.ntok))
-                        rope_tile_global<D, kFP16, kAdj, 256>(sbase + C::kOffQ + i * C::kTileBytes,
-                                                              a.table + static_cast<int64_t>(tok0 + q0) * (D / 2), rows,
-                                                              ((warp & 7) << 5) + lane);
+                    const int32_t qtid = ((warp & 7) << 5) + lane;
+                    const uint32_t qtile = sbase + C::kOffQ + i * C::kTileBytes;
+                    const bool rec = in_bounds(orig >= 0 && orig < a.B) && a.seeds[orig].consecutive != 0;
+                    if (rec) {
+                        constexpr int kPairsPerRow = D / 16;
+                        const RopeSeed* sd = a.seeds + orig;
+                        const int f0 = 8 * (qtid % kPairsPerRow);
+                        const float4 u0 = *reinterpret_cast<const float4*>(sd->inv + f0);
+                        const float4 u1 = *reinterpret_cast<const float4*>(sd->inv + f0 + 4);
+                        const float qw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                        uint64_t wc[4], ws[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float4 v = *reinterpret_cast<const float4*>(sd->wstep + f0 + 2 * k);
+                            wc[k] = f2pack(v.x, v.z);
+                            ws[k] = f2pack(v.y, v.w);
+                            uint64_t c = wc[k], sn = ws[k];
+                            rec_step(c, sn, wc[k], ws[k]);  // twice the seed's step
+                            wc[k] = c;
+                            ws[k] = sn;
+                        }
+                        RecState zq;
+                        angles_at(sd->pos0, q0 + qtid / kPairsPerRow, qw, zq);
+                        rope_tile_rec<D, kFP16, kAdj, 256>(qtile, rows, qtid, zq, wc, ws);
+                    } else if (in_bounds(q0 >= 0 && static_cast<int64_t>(tok0) + q0 + rows <= a.ntok)) {
+                        rope_tile_global<D, kFP16, kAdj, 256>(qtile, a.table + static_cast<int64_t>(tok0 + q0) * (D / 2),
+                                                              rows, qtid);
+                    }
                     fence_proxy_async_smem();  // Q' written by the generic proxy, read by the tensor cores
                 }
                 __syncwarp();
