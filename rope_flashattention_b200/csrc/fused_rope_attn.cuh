@@ -434,12 +434,14 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t r
 struct RecState {
     uint64_t c[4], s[4];     // current row's (cos f0, cos f1), (sin f0, sin f1)
 };
-// (c, s) <- (c, s) * (wc, ws) as complex numbers, two frequencies at a time
-__device__ __forceinline__ void rec_step(uint64_t& c, uint64_t& s, uint64_t wc, uint64_t ws) {
-    const uint64_t cn = fsub2(fmul2(c, wc), fmul2(s, ws));
+// (c, s) <- (c, s) * (wc, ws) as complex numbers, two frequencies at a time;
+// nws = -ws, so each part is one multiply and one fused multiply-add.
+__device__ __forceinline__ void rec_step(uint64_t& c, uint64_t& s, uint64_t wc, uint64_t ws, uint64_t nws) {
+    const uint64_t cn = ffma2(c, wc, fmul2(s, nws));
     s = ffma2(s, wc, fmul2(c, ws));
     c = cn;
 }
+__device__ __forceinline__ uint64_t fneg2(uint64_t v) { return v ^ 0x8000000080000000ull; }
 
 // Rotate one task's two chunks with the angles of `e` (4 packed pairs of
 // frequencies 8cp .. 8cp+7).
@@ -495,7 +497,7 @@ __device__ __forceinline__ void rope_tile_rec(uint32_t tile, int32_t rows, int32
             sts128(o2 + d, x2);
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) rec_step(z.c[k], z.s[k], wc[k], ws[k]);
+        for (int k = 0; k < 4; ++k) rec_step(z.c[k], z.s[k], wc[k], ws[k], fneg2(ws[k]));
     }
 }
 
@@ -1245,7 +1247,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             wc[k] = f2pack(v.x, v.z);
                             ws[k] = f2pack(v.y, v.w);
                             uint64_t c = wc[k], sn = ws[k];
-                            rec_step(c, sn, wc[k], ws[k]);  // twice the seed's step
+                            rec_step(c, sn, wc[k], ws[k], fneg2(ws[k]));  // twice the seed's step
                             wc[k] = c;
                             ws[k] = sn;
                         }
