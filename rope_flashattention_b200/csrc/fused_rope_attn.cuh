@@ -1216,11 +1216,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
             release_item(it, true);
-            // Prefill: each group decides alone (the groups share no named barrier); decode: the
-            // 16 warps together, as their merge barrier (3) spans both groups.
-            if (!named_bar_and(kDecode ? 3u : nb, kDecode ? kSoftmaxWarps * 32u : 256u, x >= 0 && *abort_flag == 0))
-                break;
-            if constexpr (!kDecode) {
+            // Decode: the 16 warps decide together whether to take the item, as their merge
+            // barrier (3) spans both groups.  Prefill: each group decides alone (the groups share
+            // no named barrier), after rotating its query tile, so that each warp starts its rows
+            // of the rotation as soon as its own epilogue is done rather than the group's slowest.
+            if constexpr (kDecode) {
+                if (!named_bar_and(3u, kSoftmaxWarps * 32u, x >= 0 && *abort_flag == 0)) break;
+            }
+            if (!kDecode && x >= 0) {
                 // This group rotates its own query tile (idle until its first score tile); both
                 // groups arrive on their QReady every item.  Consecutive positions: each thread's
                 // first-row angles are formed directly from the sequence's seed and its other rows
@@ -1262,6 +1265,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 __syncwarp();
                 if (qok && lane == 0) mbar_arrive(bar(C::kBarQReady + i));
+            }
+            if constexpr (!kDecode) {
+                if (!named_bar_and(nb, 256u, x >= 0 && *abort_flag == 0)) break;
             }
             const int32_t n_i = i == 0 ? n0 : n1;
             const int32_t qi = qt_i * kBlockM + row;
