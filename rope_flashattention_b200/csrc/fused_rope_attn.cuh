@@ -572,6 +572,22 @@ __device__ __forceinline__ void rope_tile_global(uint32_t tile, const uint32_t* 
     }
 }
 
+// 2^d for an integer-valued d <= 0 (or -inf), exactly: 0 below 2^-126.
+__device__ __forceinline__ float exp2_int(float d) {
+    return d < -126.0f ? 0.0f : __int_as_float((static_cast<int32_t>(d) + 127) << 23);
+}
+// Multiply 16 words of packed P (two bf16/fp16 values each) by f, a power of
+// two (exact but for underflow).
+template <bool kFP16>
+__device__ __forceinline__ void scale_p(uint32_t (&w)[16], float f) {
+    const uint64_t f2 = f2pack(f, f);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float2 v = IoT<kFP16>::unpack(w[e]);
+        w[e] = pack2<kFP16>(fmul2(f2pack(v.x, v.y), f2));
+    }
+}
+
 // Columns c >= lim of a 32-column slice of S are masked (-inf).
 __device__ __forceinline__ void mask_cols(uint32_t (&sr)[32], int32_t lim) {
     if (lim < 32) {
@@ -1288,7 +1304,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                         : (static_cast<int64_t>(tok0 + qi) * a.Hq + h_i) * D;
                 o_off += hf * kOHalf;
             }
-            float m = -INFINITY;  // running max of score * scale * log2(e) (identical in both halves)
+            // m: the row's reference maximum of score * scale * log2(e), identical in both halves and
+            // an integer (or -inf before the row's first visible key), so every rescale below is by
+            // an exact power of two.  It may lag the true maximum by up to 2^kRescaleThreshold.
+            float m = -INFINITY;
             float l = 0.0f;       // this half's running sum of exp2(score * scale_log2 - m)
             bool ok = true;       // warp-uniform; tcgen05.ld/st are warp-collective
             for (int32_t j = 0; j < n_i; ++j) {
@@ -1296,75 +1315,99 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 ++cs;
                 const int32_t kt = kDecode ? 2 * j + i : j;          // key tile of this step
                 const int32_t lim = vis - kt * kBlockN - hf * 64;  // columns [0, lim) of this half are visible
-                float mxh = -INFINITY;
+                // One read of this half of S, 32 columns at a time: a chunk's maximum is checked
+                // against this half's reference mt and its exponentials taken in the same pass.  A
+                // chunk more than 2^kRescaleThreshold above mt raises mt to the ceiling of its maximum,
+                // and the chunk this tile already wrote owes the factor 2^(old - new).  P is written
+                // over the half's S columns already read (P columns [16q, 16q + 16) lie in [0, 32q + 32)).
+                float mt = m;     // this half's reference for this tile
+                float lt = 0.0f;  // this half's sum of this tile's P (relative to mt)
+                float f0 = 1.0f;  // factor owed by chunk 0's P after chunk 1 raised mt
                 if (ok) {
                     tc_fence_after();
-                    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    const uint64_t sl2x2 = f2pack(sl2, sl2);
 #pragma unroll 1
                     for (int q = 0; q < 2; ++q) {
                         uint32_t sr[32];
                         tmem_ld32(sc + q * 32, sr);
                         tmem_wait_ld();
                         mask_cols(sr, lim - q * 32);
+                        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                         for (int c = 0; c < 32; c += 2)
                             mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                        const float cm = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2;
+                        if (cm > mt + kRescaleThreshold) {
+                            const float mr = ceilf(cm);
+                            const float f = exp2_int(mt - mr);
+                            lt *= f;
+                            if (q == 1) f0 = f;
+                            mt = mr;
+                        }
+                        const float neg_m = (mt == -INFINITY) ? 0.0f : -mt;
+                        const uint64_t negm2 = f2pack(neg_m, neg_m);
+                        uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
+#pragma unroll
+                        for (int c2 = 0; c2 < 16; ++c2) {
+                            const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
+                            const float2 xv = f2unpack(ffma2(sv, sl2x2, negm2));
+                            const uint64_t pp = f2pack(ex2(xv.x), ex2(xv.y));
+                            l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
+                            sr[c2] = pack2<kFP16>(pp);
+                        }
+                        tmem_st16(sc + q * 16, reinterpret_cast<const uint32_t(&)[16]>(sr));
+                        const float2 la = f2unpack(fadd2(l2[0], l2[1]));
+                        lt += la.x + la.y;
                     }
-                    mxh = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+                    if (__any_sync(0xffffffffu, f0 != 1.0f)) {
+                        uint32_t pw[16];
+                        tmem_ld16(sc, pw);
+                        tmem_wait_ld();
+                        scale_p<kFP16>(pw, f0);
+                        tmem_st16(sc, pw);
+                    }
                 }
-                xch[hf * kBlockM + row] = mxh;
+                // The two halves agree on the larger reference: a half below it rescales its P and its
+                // tile sum; when the row's reference rose, O (which holds PV_i(j-1): issued before
+                // QK_i(j), whose completion we saw) and the running sum follow.
+                xch[hf * kBlockM + row] = mt;
                 named_bar_sync(nb, 256);
                 ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
                 if (!ok) continue;
-                const float m_new = fmaxf(m, fmaxf(mxh, xch[(hf ^ 1) * kBlockM + row]) * sl2);
-                if (j > 0) {
-                    // O_i holds PV_i(j-1): it was issued before QK_i(j), whose completion we saw.
-                    const bool need = m_new > m + kRescaleThreshold;
-                    if (__any_sync(0xffffffffu, need)) {
-                        const float alpha = need ? ex2(m - m_new) : 1.0f;
-                        const uint64_t alpha2 = f2pack(alpha, alpha);
-                        l *= alpha;
+                const float mf = fmaxf(mt, xch[(hf ^ 1) * kBlockM + row]);
+                if (__any_sync(0xffffffffu, mf != mt)) {
+                    const float f = exp2_int(mt - mf);
+                    lt *= f;
+                    uint32_t pw[16];
 #pragma unroll 1
-                        for (int q = 0; q < kOHalf / 32; ++q) {
-                            uint32_t o[32];
-                            tmem_ld32(oc + q * 32, o);
-                            tmem_wait_ld();
+                    for (int q = 0; q < 2; ++q) {
+                        tmem_ld16(sc + q * 16, pw);
+                        tmem_wait_ld();
+                        scale_p<kFP16>(pw, f);
+                        tmem_st16(sc + q * 16, pw);
+                    }
+                }
+                const bool rise = mf > m;
+                if (j > 0 && __any_sync(0xffffffffu, rise)) {
+                    const float alpha = rise ? exp2_int(m - mf) : 1.0f;
+                    const uint64_t alpha2 = f2pack(alpha, alpha);
+                    l *= alpha;
+#pragma unroll 1
+                    for (int q = 0; q < kOHalf / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32(oc + q * 32, o);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int c = 0; c < 32; c += 2) {
-                                const float2 v = f2unpack(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), alpha2));
-                                o[c] = __float_as_uint(v.x);
-                                o[c + 1] = __float_as_uint(v.y);
-                            }
-                            tmem_st32(oc + q * 32, o);
+                        for (int c = 0; c < 32; c += 2) {
+                            const float2 v = f2unpack(fmul2(f2pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), alpha2));
+                            o[c] = __float_as_uint(v.x);
+                            o[c + 1] = __float_as_uint(v.y);
                         }
-                        if (need) m = m_new;
+                        tmem_st32(oc + q * 32, o);
                     }
-                } else {
-                    m = m_new;
                 }
-                // P = exp2(S * scale_log2 - m) over this half, 32 columns at a time, written over
-                // the half's S columns already read (P columns [16q, 16q + 16) lie in [0, 32q + 32))
-                const float neg_m = (m == -INFINITY) ? 0.0f : -m;
-                const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(neg_m, neg_m);
-                uint64_t l2[2] = {0ull, 0ull};  // packed (+0.0f, +0.0f)
-#pragma unroll 1
-                for (int q = 0; q < 2; ++q) {
-                    uint32_t sr[32];
-                    tmem_ld32(sc + q * 32, sr);
-                    tmem_wait_ld();
-                    mask_cols(sr, lim - q * 32);
-#pragma unroll
-                    for (int c2 = 0; c2 < 16; ++c2) {
-                        const uint64_t sv = f2pack(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1]));
-                        const float2 xv = f2unpack(ffma2(sv, sl2x2, negm2));
-                        const uint64_t pp = f2pack(ex2(xv.x), ex2(xv.y));
-                        l2[c2 & 1] = fadd2(l2[c2 & 1], pp);
-                        sr[c2] = pack2<kFP16>(pp);
-                    }
-                    tmem_st16(sc + q * 16, reinterpret_cast<const uint32_t(&)[16]>(sr));
-                }
-                const float2 la = f2unpack(fadd2(l2[0], l2[1]));
-                l += la.x + la.y;
+                if (rise) m = mf;
+                l += lt;
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
