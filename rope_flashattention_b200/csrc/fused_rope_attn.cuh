@@ -104,6 +104,7 @@ struct AttnArgs {
     // extents, for the checks of the bounds-checked build (RFA_CHECKED)
     int64_t out_elems;       // elements of out
     int32_t ntok;            // tokens of q/k/v and rows of the table (decode: cache rows B * Smax)
+    int32_t tma_out;         // 1: the output tensor map (q's geometry) describes out
 };
 
 // Work items of one sequence with nt query tiles.
@@ -660,7 +661,7 @@ template <int D, bool kFP16, bool kAdj, bool kDecode>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     fused_rope_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmT,
-                               const __grid_constant__ AttnArgs a) {
+                               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ AttnArgs a) {
     using C = AttnCfg<D>;
     static_assert(C::kTabBytes <= C::kTileBytes, "decode stages the queries' cos/sin rows in a query slot");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -739,6 +740,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Prefill, D = 128, with every sequence's positions consecutive (the flag the seed and table
+    // kernels leave in the workspace) and an output tensor map: whole output tiles are staged in the
+    // then unused cos/sin slot and written by TMA, which keeps the row-per-thread stores (32 rows
+    // 256 bytes apart per instruction) off the SM's load/store path at item boundaries.
+    const bool tstore = !kDecode && D == 128 && a.tma_out != 0 && a.sched != nullptr &&
+                        *static_cast<const volatile int32_t*>(a.sched + 2) != 0;
 
     // The k-th item index of this CTA, -1 when none is left: decode serves
     // blockIdx.x alone; otherwise the shared counter hands out items in order
@@ -1505,7 +1512,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     fin = fin && __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + i), co & 1u, abort_flag));
                     ++co;
                 }
-                if (fin) {
+                bool staged = false;  // this group's tile went out through the staging slot
+                if (tstore) {
+                    // Group i stages in its own half of the slot, one 64-column swizzle atom at a
+                    // time (the 4 warps of column half `at`, then TMA).  Whole tiles only: a tile
+                    // that runs past its sequence would overwrite the next sequence's rows.
+                    const int32_t q0 = qt_i * kBlockM;
+                    staged = named_bar_and(nb, 256u, fin && q0 + kBlockM <= L);
+                    if (staged) {
+                        tc_fence_after();
+                        const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+                        const uint64_t il2 = f2pack(inv_l, inv_l);
+                        const uint32_t buf = sbase + C::kOffT + i * (C::kTabBytes / 2);
+                        const uint32_t rbase = buf + row * 128;
+#pragma unroll 1
+                        for (int at = 0; at < 2; ++at) {
+                            if (hf == at) {
+                                // row `row`, 16-byte chunks 4q .. 4q + 3 at chunk ^ (row & 7)
+#pragma unroll 1
+                                for (int q = 0; q < kOHalf / 32; ++q) {
+                                    uint32_t o[32];
+                                    tmem_ld32(oc + q * 32, o);
+                                    tmem_wait_ld();
+                                    uint32_t wv[16];
+#pragma unroll
+                                    for (int e = 0; e < 16; ++e)
+                                        wv[e] = pack2<kFP16>(
+                                            fmul2(f2pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), il2));
+#pragma unroll
+                                    for (int c = 0; c < 4; ++c)
+                                        sts128(rbase + (static_cast<uint32_t>((4 * q + c) ^ (row & 7)) << 4),
+                                               make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]));
+                                }
+                                fence_proxy_async_smem();  // staged by the generic proxy, read by TMA
+                            }
+                            named_bar_sync(nb, 256);
+                            if ((warp & 7) == 0 && lane == 0) {
+                                if (a.layout == 0)
+                                    tma_store_3d(&tmO, buf, at * 64, q0, seq * a.Hq + h_i);
+                                else
+                                    tma_store_3d(&tmO, buf, at * 64, h_i, tok0 + q0);
+                                bulk_commit();
+                                bulk_wait_read();  // the buffer may be staged again
+                            }
+                            named_bar_sync(nb, 256);
+                        }
+                    }
+                }
+                if (fin && !staged) {
                     tc_fence_after();
                     const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
                     bool valid = o_valid;
@@ -1537,11 +1591,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             }
                         }
                     }
-                    // the next item's PV_i(0) overwrites O_i only after this warp's PFull_i
-                    // arrival of that item, which follows these reads (tcgen05.wait::ld above)
                 }
+                // the next item's PV_i(0) overwrites O_i only after this warp's PFull_i arrival of
+                // that item, which follows these reads (tcgen05.wait::ld above)
             }
         }
+        // staged tiles' stores complete before the CTA exits
+        if (tstore && (warp & 7) == 0 && lane == 0) bulk_wait();
     }
 
     __syncwarp();

@@ -174,13 +174,13 @@ int32_t* sched_of(void* workspace, int64_t T, int D, int nseg) {
 // per item.
 template <int D, bool kFP16, bool kAdj, bool kDecode = false>
 rfa_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mt,
-                       const rfa::AttnArgs& args, cudaStream_t st) {
+                       const CUtensorMap& mo, const rfa::AttnArgs& args, cudaStream_t st) {
     auto kern = rfa::fused_rope_attn_fwd_kernel<D, kFP16, kAdj, kDecode>;
     constexpr int smem = rfa::AttnCfg<D>::kSmemBytes;
     constexpr int kTag = ((D * 4 + (kFP16 ? 2 : 0) + (kAdj ? 1 : 0)) << 1) + (kDecode ? 1 : 0);
     if (ensure_smem_attr<kTag>(kern, smem) != RFA_OK) return RFA_ERR_CUDA;
     const int grid = kDecode ? args.n_items : std::max(1, std::min(args.n_items, device_sms()));
-    kern<<<grid, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, mt, args);
+    kern<<<grid, rfa::kAttnThreads, smem, st>>>(mq, mk, mv, mt, mo, args);
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
@@ -552,19 +552,29 @@ rfa_status enqueue_attention(const rfa_attn_params* p, int64_t T, const void* q,
     CUtensorMap mt;
     ok = ok && make_table_map(&mt, table, static_cast<uint64_t>(T), D);
     if (!ok) return RFA_ERR_CUDA;
+    // the output as the query's geometry, for the kernel's tiled stores of whole output tiles;
+    // when it cannot be described (e.g. not 16-byte aligned) the kernel stores rows itself
+    CUtensorMap mo = mq;
+    aa.tma_out = (tnd ? make_map(&mo, out, fp16, D, p->Hq, T, D * esz, static_cast<uint64_t>(p->Hq) * D * esz, 64,
+                                 1, rfa::kBlockM)
+                      : make_map(&mo, out, fp16, D, p->S, static_cast<uint64_t>(p->B) * p->Hq, D * esz,
+                                 p->S * D * esz, 64, rfa::kBlockM, 1))
+                     ? 1
+                     : 0;
+    if (!aa.tma_out) mo = mq;
     const bool adj = p->rope_interleaved != 0;
     if (D == 128) {
         if (adj)
-            return fp16 ? launch_attn<128, true, true>(mq, mk, mv, mt, aa, st)
-                        : launch_attn<128, false, true>(mq, mk, mv, mt, aa, st);
-        return fp16 ? launch_attn<128, true, false>(mq, mk, mv, mt, aa, st)
-                    : launch_attn<128, false, false>(mq, mk, mv, mt, aa, st);
+            return fp16 ? launch_attn<128, true, true>(mq, mk, mv, mt, mo, aa, st)
+                        : launch_attn<128, false, true>(mq, mk, mv, mt, mo, aa, st);
+        return fp16 ? launch_attn<128, true, false>(mq, mk, mv, mt, mo, aa, st)
+                    : launch_attn<128, false, false>(mq, mk, mv, mt, mo, aa, st);
     }
     if (adj)
-        return fp16 ? launch_attn<64, true, true>(mq, mk, mv, mt, aa, st)
-                    : launch_attn<64, false, true>(mq, mk, mv, mt, aa, st);
-    return fp16 ? launch_attn<64, true, false>(mq, mk, mv, mt, aa, st)
-                : launch_attn<64, false, false>(mq, mk, mv, mt, aa, st);
+        return fp16 ? launch_attn<64, true, true>(mq, mk, mv, mt, mo, aa, st)
+                    : launch_attn<64, false, true>(mq, mk, mv, mt, mo, aa, st);
+    return fp16 ? launch_attn<64, true, false>(mq, mk, mv, mt, mo, aa, st)
+                : launch_attn<64, false, false>(mq, mk, mv, mt, mo, aa, st);
 }
 
 }  // namespace
@@ -834,20 +844,21 @@ rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, 
     if (!ok) return RFA_ERR_CUDA;
     const bool adj = p->rope_interleaved != 0;
     rfa_status r;
+    const CUtensorMap& mo = mq;  // decode stores its rows itself
     if (D == 128) {
         if (adj)
-            r = fp16 ? launch_attn<128, true, true, true>(mq, mk, mv, mt, aa, st)
-                     : launch_attn<128, false, true, true>(mq, mk, mv, mt, aa, st);
+            r = fp16 ? launch_attn<128, true, true, true>(mq, mk, mv, mt, mo, aa, st)
+                     : launch_attn<128, false, true, true>(mq, mk, mv, mt, mo, aa, st);
         else
-            r = fp16 ? launch_attn<128, true, false, true>(mq, mk, mv, mt, aa, st)
-                     : launch_attn<128, false, false, true>(mq, mk, mv, mt, aa, st);
+            r = fp16 ? launch_attn<128, true, false, true>(mq, mk, mv, mt, mo, aa, st)
+                     : launch_attn<128, false, false, true>(mq, mk, mv, mt, mo, aa, st);
     } else {
         if (adj)
-            r = fp16 ? launch_attn<64, true, true, true>(mq, mk, mv, mt, aa, st)
-                     : launch_attn<64, false, true, true>(mq, mk, mv, mt, aa, st);
+            r = fp16 ? launch_attn<64, true, true, true>(mq, mk, mv, mt, mo, aa, st)
+                     : launch_attn<64, false, true, true>(mq, mk, mv, mt, mo, aa, st);
         else
-            r = fp16 ? launch_attn<64, true, false, true>(mq, mk, mv, mt, aa, st)
-                     : launch_attn<64, false, false, true>(mq, mk, mv, mt, aa, st);
+            r = fp16 ? launch_attn<64, true, false, true>(mq, mk, mv, mt, mo, aa, st)
+                     : launch_attn<64, false, false, true>(mq, mk, mv, mt, mo, aa, st);
     }
     if (r != RFA_OK || pl.splits == 1) return r;
     const int grid = grid_for(pl.rq * (D / 8), 256);

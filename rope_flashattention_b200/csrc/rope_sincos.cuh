@@ -165,7 +165,8 @@ struct TableArgs {
     const float* inv_dev;  // [nseg, half] or nullptr -> inv_host
     uint32_t* table;       // [ntokens][half] 32-bit words of fp16 cos/sin pairs
     RopeSeed* seeds;       // [nseg]
-    int32_t* sched;        // the fused kernel's two work counters (zeroed here), or nullptr
+    int32_t* sched;        // the fused kernel's work counters [0..1] (zeroed here) and, at [2], the
+                           // launch flag "every sequence's positions are consecutive", or nullptr
     int32_t npos;          // entries of pos
     int32_t inv_dev_rows;  // rows of inv_dev
     int32_t ntokens;
@@ -214,8 +215,10 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
             // past INT32_MAX do not count as consecutive) clears its consecutive flag, which
             // rope_seed_kernel set before this kernel
             const int32_t tok0 = a.uniform_len > 0 ? b * a.uniform_len : a.cum[b];
-            if (static_cast<int64_t>(p) != static_cast<int64_t>(__ldg(a.pos + tok0)) + (t - tok0))
+            if (static_cast<int64_t>(p) != static_cast<int64_t>(__ldg(a.pos + tok0)) + (t - tok0)) {
                 a.seeds[b].consecutive = 0;
+                if (a.sched != nullptr) a.sched[2] = 0;
+            }
         }
         uint32_t pr[8];
 #pragma unroll
@@ -234,7 +237,8 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const __grid_constant__
 
 // Per-sequence seeds (grid: one block per sequence; runs before
 // rope_table_kernel, which clears the consecutive flag of a sequence whose
-// positions break the run): the flag set, the first position, the invFreq row
+// positions break the run, and the launch-wide flag with it): the flags set,
+// the first position, the invFreq row
 // and the in-tile step (cos, sin) of step * w_j, the angle formed and reduced
 // modulo 2 pi in fp64, then evaluated with fp32 sincos (|error| ~1e-7).
 __global__ void __launch_bounds__(64) rope_seed_kernel(const __grid_constant__ TableArgs a) {
@@ -245,6 +249,7 @@ __global__ void __launch_bounds__(64) rope_seed_kernel(const __grid_constant__ T
     if (threadIdx.x == 0) {
         sd->consecutive = 1;
         sd->pos0 = __ldg(a.pos + tok0);
+        if (b == 0 && a.sched != nullptr) a.sched[2] = 1;  // cleared by rope_table_kernel on any break
     }
     const float* inv = a.inv_dev ? a.inv_dev + static_cast<int64_t>(b) * a.half
                                  : a.inv_host + (a.inv_host_rows == 1 ? 0 : b) * a.half;
