@@ -10,39 +10,41 @@
 // The rotated tiles exist only in shared memory; nothing rotated is written
 // back to global memory.
 //
-// One CTA = one work item: two 128-row query tiles that read the same key /
+// A persistent grid (one CTA per SM) takes work items from a counter in the
+// workspace.  A work item is two 128-row query tiles that read the same key /
 // value tiles -- two query heads of one kv group at the same rows when the
 // group size G is even, else two consecutive query tiles of one head (the
 // second may be absent at the end of a sequence).  Every key tile is loaded
-// and rotated once for both query tiles.  24 warps:
+// and rotated once for both query tiles.  24 warps, 80 registers per thread:
 //   warps 0-7  softmax of query tile 0, warps 8-15 of query tile 1.  Warp w
 //              covers TMEM lanes (rows) 32 (w % 4) .. + 31 and one 64-key half
-//              hf = (w / 4) % 2 of every score tile.  Per key tile: the half-row
-//              maximum from a first TMEM read of the half, exchanged with the
-//              other half's warp through shared memory at a named barrier; the
-//              running maximum is raised only when it grows by more than 2^8
-//              (lazy rescaling: then l and this half of O are rescaled);
-//              exponentials from a second read, P (bf16/fp16) written over the
-//              half's own S columns.  At the end: row sums combined, O / l to
-//              global memory.
-//   warps 16-19 RoPE warpgroup: rotates both query tiles once, then every key
-//              tile, in place in the 128B-swizzled shared-memory layout.
-//              Element i and its rotate-half partner i + D/2 sit at the same
-//              offset of two swizzle atoms (D = 128) or in chunks c and c ^ 4
-//              of one atom (D = 64).  Key angles come from a complex
+//              hf = (w / 4) % 2 of every score tile.  Per key tile, one read
+//              of the half in two 32-column chunks: each chunk's maximum is
+//              checked against the half's reference maximum (an integer that
+//              lags the true maximum by at most 2^8) and its exponentials are
+//              taken in the same pass; the two halves then agree on the larger
+//              reference at a named barrier, and a raised reference rescales
+//              P, l and O by exact powers of two.  P (bf16/fp16) is written
+//              over the half's own S columns.  At each item start the group
+//              rotates its own query tile; at its end, row sums combined and
+//              O / l written out (whole tiles by TMA stores when possible).
+//   warps 16-19 RoPE warpgroup: rotates every key tile once (decode: the
+//              query tile), in place in the 128B-swizzled shared-memory
+//              layout.  Element i and its rotate-half partner i + D/2 sit at
+//              the same offset of two swizzle atoms (D = 128) or in chunks c
+//              and c ^ 4 of one atom (D = 64).  Angles come from a complex
 //              recurrence in registers when the sequence's positions are
 //              consecutive, else from cos/sin rows that TMA staged beside the
-//              tile; query angles always from staged rows.
-//   warp 20    TMA producer: both query tiles (+ their cos/sin rows, staged in
-//              the first two V slots) once, then key tiles (+ rows when
-//              needed) through a kStages ring.
-//   warp 21    tcgen05 issuer (one thread) and TMEM owner.  Order per key
-//              tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), where
-//              S_i = Q_i' K_j'^T goes to TMEM buffer i and O_i += P_i V_j reads
-//              P_i from that same buffer.  MMAs issued by one thread execute
-//              in issue order, so QK_i(j+1) overwrites P_i only after PV_i(j)
-//              has read it, and S_i(j+1) being complete implies O_i holds
-//              PV_i(j).
+//              tile.
+//   warp 20    TMA producer of the query tiles and the key ring (+ cos/sin
+//              rows when needed), and the item fetcher.
+//   warp 21    tcgen05 issuer (an elected lane of the converged warp) and TMEM
+//              owner.  Order per key tile j: PV_0(j), QK_0(j+1), PV_1(j),
+//              QK_1(j+1), where S_i = Q_i' K_j'^T goes to TMEM buffer i and
+//              O_i += P_i V_j reads P_i from that same buffer.  MMAs issued by
+//              one thread execute in issue order, so QK_i(j+1) overwrites P_i
+//              only after PV_i(j) has read it, and S_i(j+1) being complete
+//              implies O_i holds PV_i(j).
 //   warp 22    TMA producer for the V ring.
 //   warp 23    idle (takes part in the block-wide barriers only).
 // Completion of every async step is tracked by mbarriers; each wait is bounded.
