@@ -116,6 +116,29 @@ int resident_grid(K kernel, int64_t work, int threads) {
     return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(blocks, static_cast<int64_t>(sms) * per_sm)));
 }
 
+// L2 size of the current device in bytes; 126 MB (a B200) when no device is visible.
+int64_t device_l2_bytes() {
+    int dev = 0, l2 = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess ||
+        l2 < 1) {
+        (void)cudaGetLastError();
+        return 126ll << 20;
+    }
+    return l2;
+}
+
+// True when a launch moving `bytes` should use the evict-first accesses of stream_mem.cuh.
+bool streams(double bytes) { return bytes > 0.5 * static_cast<double>(device_l2_bytes()); }
+
+// The public sin/cos table kernel; stream_out selects its evict-first stores.
+template <typename OutT>
+void launch_sincos(bool stream_out, int64_t work, cudaStream_t st, const int32_t* pos, const float* inv,
+                   const int32_t* lens, int32_t batch, int32_t ntokens, int32_t headSize, void* sinOut, void* cosOut) {
+    auto k = stream_out ? rfa::rope_sincos_kernel<OutT, true> : rfa::rope_sincos_kernel<OutT, false>;
+    k<<<resident_grid(k, work, 256), 256, 0, st>>>(pos, inv, lens, batch, ntokens, headSize, static_cast<OutT*>(sinOut),
+                                                   static_cast<OutT*>(cosOut));
+}
+
 // invFreq_j = base^(-2j/D) in fp64, rounded once to fp32.
 void inv_freq_row(double base, int D, float* out) {
     for (int j = 0; j < D / 2; ++j) out[j] = static_cast<float>(std::pow(base, -2.0 * j / static_cast<double>(D)));
@@ -235,22 +258,20 @@ rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, con
     if (!aligned(invFreq, 16) || !aligned(sinOut, 16) || !aligned(cosOut, 16)) return RFA_ERR_INVALID_ARG;
     const int64_t work = static_cast<int64_t>(ntokens) * (headSize / 16);
     cudaStream_t st = as_stream(stream);
+    const size_t esize = outType == RFA_DT_FP32 ? 4 : 2;
+    const bool stream_out = streams(2.0 * static_cast<double>(ntokens) * headSize * esize);  // sin + cos
     switch (outType) {
         case RFA_DT_FP16:
-            rfa::rope_sincos_kernel<__half><<<resident_grid(rfa::rope_sincos_kernel<__half>, work, 256), 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
-                                                                   headSize, static_cast<__half*>(sinOut),
-                                                                   static_cast<__half*>(cosOut));
+            launch_sincos<__half>(stream_out, work, st, positionIds, invFreq, seqLens, batch, ntokens, headSize,
+                                  sinOut, cosOut);
             break;
         case RFA_DT_BF16:
-            rfa::rope_sincos_kernel<__nv_bfloat16>
-                <<<resident_grid(rfa::rope_sincos_kernel<__nv_bfloat16>, work, 256), 256, 0, st>>>(
-                positionIds, invFreq, seqLens, batch, ntokens, headSize, static_cast<__nv_bfloat16*>(sinOut),
-                static_cast<__nv_bfloat16*>(cosOut));
+            launch_sincos<__nv_bfloat16>(stream_out, work, st, positionIds, invFreq, seqLens, batch, ntokens,
+                                         headSize, sinOut, cosOut);
             break;
         default:
-            rfa::rope_sincos_kernel<float><<<resident_grid(rfa::rope_sincos_kernel<float>, work, 256), 256, 0, st>>>(positionIds, invFreq, seqLens, batch, ntokens,
-                                                                  headSize, static_cast<float*>(sinOut),
-                                                                  static_cast<float*>(cosOut));
+            launch_sincos<float>(stream_out, work, st, positionIds, invFreq, seqLens, batch, ntokens, headSize,
+                                 sinOut, cosOut);
             break;
     }
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
@@ -261,14 +282,13 @@ rfa_status rfa_rope_sincos(const int32_t* positionIds, const float* invFreq, con
 namespace {
 
 template <bool kFP16, typename TabT>
-void launch_rope_apply(const rfa::RopeApplyArgs& a, bool interleaved, uint32_t work, cudaStream_t st) {
-    if (interleaved) {
-        auto kern = rfa::rope_apply_kernel<kFP16, TabT, true>;
-        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
-    } else {
-        auto kern = rfa::rope_apply_kernel<kFP16, TabT, false>;
-        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
-    }
+void launch_rope_apply(const rfa::RopeApplyArgs& a, bool interleaved, bool stream_mem, uint32_t work,
+                       cudaStream_t st) {
+    auto kern = interleaved ? (stream_mem ? rfa::rope_apply_kernel<kFP16, TabT, true, true>
+                                          : rfa::rope_apply_kernel<kFP16, TabT, true, false>)
+                            : (stream_mem ? rfa::rope_apply_kernel<kFP16, TabT, false, true>
+                                          : rfa::rope_apply_kernel<kFP16, TabT, false, false>);
+    kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
 }
 
 }  // namespace
@@ -327,18 +347,22 @@ rfa_status rfa_rope_apply(const rfa_rope_apply_params* p, const void* q, const v
     a.D = p->D;
     const bool fp16 = p->io_dtype == RFA_DT_FP16;
     const bool inter = p->interleaved != 0;
+    // q and k rows read, rotated rows written (k twice when it also goes to the cache)
+    const double row_bytes = static_cast<double>(p->D) * 2.0;
+    const bool sm = streams(static_cast<double>(R) * row_bytes *
+                            (2.0 * p->Hq + (1.0 + (k_out ? 1.0 : 0.0) + (k_cache ? 1.0 : 0.0)) * p->Hkv));
     const uint32_t w = static_cast<uint32_t>(work);
     cudaStream_t st = as_stream(stream);
     switch (p->table_dtype) {
         case RFA_DT_FP16:
-            fp16 ? launch_rope_apply<true, __half>(a, inter, w, st) : launch_rope_apply<false, __half>(a, inter, w, st);
+            fp16 ? launch_rope_apply<true, __half>(a, inter, sm, w, st) : launch_rope_apply<false, __half>(a, inter, sm, w, st);
             break;
         case RFA_DT_BF16:
-            fp16 ? launch_rope_apply<true, __nv_bfloat16>(a, inter, w, st)
-                 : launch_rope_apply<false, __nv_bfloat16>(a, inter, w, st);
+            fp16 ? launch_rope_apply<true, __nv_bfloat16>(a, inter, sm, w, st)
+                 : launch_rope_apply<false, __nv_bfloat16>(a, inter, sm, w, st);
             break;
         default:
-            fp16 ? launch_rope_apply<true, float>(a, inter, w, st) : launch_rope_apply<false, float>(a, inter, w, st);
+            fp16 ? launch_rope_apply<true, float>(a, inter, sm, w, st) : launch_rope_apply<false, float>(a, inter, sm, w, st);
             break;
     }
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
@@ -349,14 +373,12 @@ rfa_status rfa_rope_apply(const rfa_rope_apply_params* p, const void* q, const v
 namespace {
 
 template <bool kFP16, typename TabT>
-void launch_kv_cache(const rfa::KvCacheArgs& a, bool interleaved, uint32_t work, cudaStream_t st) {
-    if (interleaved) {
-        auto kern = rfa::kv_norm_rope_cache_kernel<kFP16, TabT, true>;
-        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
-    } else {
-        auto kern = rfa::kv_norm_rope_cache_kernel<kFP16, TabT, false>;
-        kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
-    }
+void launch_kv_cache(const rfa::KvCacheArgs& a, bool interleaved, bool stream_mem, uint32_t work, cudaStream_t st) {
+    auto kern = interleaved ? (stream_mem ? rfa::kv_norm_rope_cache_kernel<kFP16, TabT, true, true>
+                                          : rfa::kv_norm_rope_cache_kernel<kFP16, TabT, true, false>)
+                            : (stream_mem ? rfa::kv_norm_rope_cache_kernel<kFP16, TabT, false, true>
+                                          : rfa::kv_norm_rope_cache_kernel<kFP16, TabT, false, false>);
+    kern<<<resident_grid(kern, work, 256), 256, 0, st>>>(a);
 }
 
 }  // namespace
@@ -396,18 +418,20 @@ rfa_status rfa_kv_rms_norm_rope_cache(const rfa_kv_cache_params* p, const void* 
     a.D = p->D;
     a.eps = p->eps;
     const bool fp16 = p->io_dtype == RFA_DT_FP16, inter = p->interleaved != 0;
+    // k and v rows read, both caches written
+    const bool sm = streams(4.0 * static_cast<double>(p->T) * p->Hkv * p->D * 2.0);
     const uint32_t w = static_cast<uint32_t>(work);
     cudaStream_t st = as_stream(stream);
     switch (p->table_dtype) {
         case RFA_DT_FP16:
-            fp16 ? launch_kv_cache<true, __half>(a, inter, w, st) : launch_kv_cache<false, __half>(a, inter, w, st);
+            fp16 ? launch_kv_cache<true, __half>(a, inter, sm, w, st) : launch_kv_cache<false, __half>(a, inter, sm, w, st);
             break;
         case RFA_DT_BF16:
-            fp16 ? launch_kv_cache<true, __nv_bfloat16>(a, inter, w, st)
-                 : launch_kv_cache<false, __nv_bfloat16>(a, inter, w, st);
+            fp16 ? launch_kv_cache<true, __nv_bfloat16>(a, inter, sm, w, st)
+                 : launch_kv_cache<false, __nv_bfloat16>(a, inter, sm, w, st);
             break;
         default:
-            fp16 ? launch_kv_cache<true, float>(a, inter, w, st) : launch_kv_cache<false, float>(a, inter, w, st);
+            fp16 ? launch_kv_cache<true, float>(a, inter, sm, w, st) : launch_kv_cache<false, float>(a, inter, sm, w, st);
             break;
     }
     return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;

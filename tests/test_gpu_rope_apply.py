@@ -196,3 +196,48 @@ def test_kv_cache_op_slot_beyond_cache_sets_status(rfa):
     assert rfa.get_device_status() == rfa.RFA_ERR_INVALID_ARG
     assert rfa.get_device_status() == 0
     assert torch.equal(vc[1], v[0]) and torch.equal(vc[0], v[2])
+
+
+# ---------------------------------------------------------------- evict-first (streaming) launches
+# A launch that moves more than half of L2 reads and writes its rows with the
+# evict-first hint; the values must not change.  Each test runs one such launch
+# and the same rows as many small launches (ordinary accesses) and compares
+# the results bit for bit.
+
+@pytest.mark.parametrize("inter", [False, True])
+def test_rope_apply_streaming_launch_matches_small_launches(rfa, inter):
+    T, Hq, Hkv, D, rows = 8192, 32, 8, 128, 9000
+    q = workloads.randn16((T, Hq, D), 60).cuda()
+    k = workloads.randn16((T, Hkv, D), 61).cuda()
+    s, c = _tables(rfa, T, D, 62, torch.float16, inter)
+    slots = torch.randperm(rows, generator=workloads.gen(63))[:T].to(torch.int32).cuda()
+    cache = torch.zeros((rows, Hkv, D), dtype=torch.bfloat16).cuda()
+    qo, ko = rfa.rope_apply(q, k, s, c, cache_slots=slots, k_cache=cache, interleaved=inter)
+    assert rfa.get_device_status() == 0
+    cache2 = torch.zeros_like(cache)
+    for t0 in range(0, T, 512):
+        sl = slice(t0, t0 + 512)
+        qs, ks = rfa.rope_apply(q[sl].contiguous(), k[sl].contiguous(), s[sl].contiguous(), c[sl].contiguous(),
+                                cache_slots=slots[sl].contiguous(), k_cache=cache2, interleaved=inter)
+        assert torch.equal(qs, qo[sl]) and torch.equal(ks, ko[sl])
+    assert rfa.get_device_status() == 0
+    assert torch.equal(cache, cache2)
+
+
+def test_kv_cache_op_streaming_launch_matches_small_launches(rfa):
+    T, Hkv, D = 32768, 8, 128
+    k = workloads.randn16((T, Hkv, D), 64).cuda()
+    v = workloads.randn16((T, Hkv, D), 65).cuda()
+    gamma = (0.5 + torch.rand(D, generator=workloads.gen(66))).float().cuda()
+    s, c = _tables(rfa, T, D, 67, torch.float16, False)
+    slots = torch.randperm(T, generator=workloads.gen(68)).to(torch.int32).cuda()
+    kc, vc = torch.zeros_like(k), torch.zeros_like(v)
+    rfa.kv_rms_norm_rope_cache(k, v, gamma, 1e-6, s, c, slots, kc, vc)
+    assert rfa.get_device_status() == 0
+    kc2, vc2 = torch.zeros_like(k), torch.zeros_like(v)
+    for t0 in range(0, T, 1024):
+        sl = slice(t0, t0 + 1024)
+        rfa.kv_rms_norm_rope_cache(k[sl].contiguous(), v[sl].contiguous(), gamma, 1e-6, s[sl].contiguous(),
+                                   c[sl].contiguous(), slots[sl].contiguous(), kc2, vc2)
+    assert rfa.get_device_status() == 0
+    assert torch.equal(kc, kc2) and torch.equal(vc, vc2)

@@ -120,3 +120,18 @@ def test_bad_lengths_set_status_and_write_nothing(rfa):
     assert rfa.get_device_status() == rfa.RFA_ERR_INVALID_ARG
     assert torch.all(s == 7.0) and torch.all(c == 7.0)
     assert rfa.get_device_status() == 0  # cleared
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_tables_larger_than_half_of_l2(rfa, dtype):
+    """Tables larger than half of L2 are written with evict-first stores: within
+    tolerance of the oracle on sampled rows, and bit-identical to the ordinary
+    stores of a small launch over the first sequence alone."""
+    pos, inv, lens = workloads.sincos_problem(256000, 128, 16, seed=9)
+    rows = np.random.default_rng(1).choice(256000, 3000, replace=False)
+    rows = np.concatenate([rows, [0, 15999, 16000, 255999]])
+    s, c = _check(rfa, pos, inv, lens, 128, dtype, rows=rows)
+    n0 = int(lens[0])
+    s0, c0 = _run(rfa, pos[:n0], inv[:1], lens[:1], 128, dtype)
+    np.testing.assert_array_equal(s[:n0], s0.float().cpu().numpy())
+    np.testing.assert_array_equal(c[:n0], c0.float().cpu().numpy())
