@@ -445,6 +445,24 @@ def _sincos_time(rfa, pos, inv, lens, D, s, c, flush, back_to_back: bool):
     return statistics.median(times), "median of 30 single launches, each after a 256 MB read that clears L2"
 
 
+def _event_floor(flush, dev) -> float:
+    """Seconds that a single-launch measurement of _sincos_time reads for a
+    kernel that does almost nothing (a one-element torch add, timed the same
+    way after the same read flush): the floor under any single-launch figure."""
+    one = torch.zeros(1, device=dev)
+    times = []
+    for _ in range(30):
+        flush.sum()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        one.add_(1)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) * 1e-3)
+    return statistics.median(times)
+
+
 def _sincos_bytes(T: int, D: int, batch: int) -> int:
     """Algorithmic bytes: positions, invFreq rows and lengths read; sin and cos written (fp16)."""
     return T * 4 + 2 * T * D * 2 + batch * (D // 2) * 4 + batch * 4
@@ -456,7 +474,8 @@ def sincos_bench(rfa, dev):
     (U[0,1) fp32), headSize 128, fp16 out.  The 29.5 MB of outputs fit in L2
     (126 MB), so each timed launch follows a 256 MB read that leaves L2 holding
     clean lines only; the launch is short enough (a few microseconds) that
-    launch latency shows."""
+    launch latency shows.  `event_floor_us` is what the same measurement reads
+    for a one-element kernel."""
     w = workloads.PACKED
     lens_l = workloads.seq_lengths(w)
     T = sum(lens_l)
@@ -470,7 +489,8 @@ def sincos_bench(rfa, dev):
     assert rfa.get_device_status() == 0
     byts = _sincos_bytes(T, w.D, w.B)
     return {"shape": f"packed workload: T={T} over {w.B} sequences (seed {w.seed}), headSize {w.D}, fp16",
-            "bytes": byts, "us": t * 1e6, "GB/s": byts / t / 1e9, "timing": how}
+            "bytes": byts, "us": t * 1e6, "GB/s": byts / t / 1e9, "timing": how,
+            "event_floor_us": _event_floor(flush, dev) * 1e6}
 
 
 def sincos_ceiling_bench(rfa, dev):
@@ -625,9 +645,11 @@ def unfused_context(w, q, k, v, pos, dev, iters=20):
 class AttnInputs:
     """A workload's inputs resident on the device, its cos/sin table built."""
 
-    def __init__(self, rfa, w, dev):
+    def __init__(self, rfa, w, dev, adjacent_pairs: bool = False):
         self.rfa, self.w, self.dev = rfa, w, dev
         self.kw = workload_kwargs(w)
+        if adjacent_pairs:  # RoPE on pairs (2i, 2i+1) instead of (i, i + D/2)
+            self.kw = dict(self.kw, interleaved=True)
         self.q_h, self.k_h, self.v_h = workloads.make_qkv(w)
         self.pos_h = workloads.positions(w)
         inv_h = workloads.random_inv_freq(w)
@@ -661,11 +683,11 @@ def pick_peak(peaks, clk):
         "bf16_tflops_sustained" if sustained else "bf16_tflops")
 
 
-def attention_line(rfa, w, dev, peaks, peak_src, seconds: float):
+def attention_line(rfa, w, dev, peaks, peak_src, seconds: float, adjacent_pairs: bool = False):
     """The fused attention kernel alone on workload w, launched back to back
     for about `seconds` (inputs larger than L2), each launch bracketed by CUDA
     events on the launching stream, with its own clock record."""
-    a = AttnInputs(rfa, w, dev)
+    a = AttnInputs(rfa, w, dev, adjacent_pairs)
     for _ in range(3):
         a.step()
     torch.cuda.synchronize()
@@ -691,7 +713,8 @@ def attention_line(rfa, w, dev, peaks, peak_src, seconds: float):
     tf = a.flops / (ms * 1e-3) / 1e12
     del a
     torch.cuda.empty_cache()
-    return {"workload": w.name, "kernel": "fused_rope_attn_fwd_kernel", "launches": n, "kernel_ms": ms,
+    return {"workload": w.name, "rope_pairs": "adjacent (2i, 2i+1)" if adjacent_pairs else "rotate-half (i, i + D/2)",
+            "kernel": "fused_rope_attn_fwd_kernel", "launches": n, "kernel_ms": ms,
             "TFLOP/s": tf, "flops": workload_flops(w), "peak": peak, "peak_source": f"{peak_src} {which}",
             "frac": tf / peak, "tok_per_s": workloads.ntokens(w) / (ms * 1e-3), "clocks": clk}
 
@@ -844,6 +867,9 @@ def run_gpu(args, world, rank, local):
             # the other full-size workloads: the attention kernel alone, each timed for about a second
             extra["workloads"] = {key: attention_line(rfa, wl, dev, peaks, peak_src, args.workload_seconds)
                                   for key, wl in workloads.BY_KEY.items() if key not in ("tiny", args.workload)}
+            # the adjacent-pair variant of the fused kernel on the GQA 8K workload
+            extra["workloads"]["gqa8k_adjacent_pairs"] = attention_line(
+                rfa, workloads.BY_KEY["gqa8k"], dev, peaks, peak_src, args.workload_seconds, adjacent_pairs=True)
         extra["sincos"] = sincos_bench(rfa, dev)
         extra["sincos"]["frac_hbm"] = extra["sincos"]["GB/s"] / peaks["hbm_gbs"]
         extra["sincos_ceiling"] = sincos_ceiling_bench(rfa, dev)
