@@ -577,8 +577,9 @@ def kv_cache_bench(rfa, dev):
 def decode_bench(rfa, dev):
     """decode_rope_attention: 8 sequences x 32 query / 8 kv heads x D 128, one
     new token each, over 32768 cached tokens (bf16): GB/s of algorithmic bytes
-    (the K and V caches read once, plus q, out and the queries' cos/sin rows),
-    1.07 GB per launch, launches back to back."""
+    (the K and V caches read once, plus q, out and the new tokens' positions;
+    the queries' cos/sin are formed in the kernel), 1.07 GB per launch,
+    launches back to back."""
     B, Hq, Hkv, Sq, D, L = 8, 32, 8, 1, 128, 32768
     q = workloads.randn16((B, Hq, Sq, D), 41).to(dev)
     kc = workloads.randn16((B, L, Hkv, D), 42).to(dev)
@@ -600,7 +601,7 @@ def decode_bench(rfa, dev):
     torch.cuda.synchronize()
     assert rfa.get_device_status() == 0
     t = e0.elapsed_time(e1) * 1e-3 / n
-    byts = 2 * kc.numel() * 2 + 2 * q.numel() * 2 + B * Hq * Sq * D * 2
+    byts = 2 * kc.numel() * 2 + 2 * q.numel() * 2 + B * Sq * 4
     return {"shape": "B=8, Hq=32, Hkv=8, Sq=1, D=128, 32768 cached tokens, bf16", "bytes": byts, "us": t * 1e6,
             "GB/s": byts / t / 1e9, "tokens/s": B * Sq / t, "timing": f"{n} launches back to back (data > L2)"}
 

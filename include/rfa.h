@@ -205,8 +205,10 @@ typedef struct {
  *                 becomes RFA_ERR_INVALID_ARG (the length is clamped)
  *   invFreq       dev fp32 [B, D/2] or NULL (then base^(-2j/D) from rope_base)
  *   workspace     dev, 256-byte aligned, >= rfa_decode_rope_attention_workspace(p)
- *                 bytes: the queries' cos/sin rows and, when the keys are split
- *                 across CTAs, fp32 partial results merged by a second kernel
+ *                 bytes (at least 256): when the keys are split across CTAs, the
+ *                 fp32 partial results that a second kernel merges (launched as a
+ *                 programmatic dependent launch, so it starts as the first ends).
+ *                 The queries' cos/sin are formed inside the attention kernel.
  * Returns RFA_ERR_INVALID_ARG / RFA_ERR_UNSUPPORTED / RFA_ERR_WORKSPACE on
  * host-checkable errors; nothing is enqueued then.
  */

@@ -107,6 +107,10 @@ struct AttnArgs {
     int64_t out_elems;       // elements of out
     int32_t ntok;            // tokens of q/k/v and rows of the table (decode: cache rows B * Smax)
     int32_t tma_out;         // 1: the output tensor map (q's geometry) describes out
+    // decode: the RoPE warps form the query rows' cos/sin themselves (no table kernel first)
+    const int32_t* dec_qpos;           // [B, Sq] positions of the new tokens
+    const float* dec_inv;              // [B, D/2] frequencies, or nullptr: dec_inv_host for every sequence
+    float dec_inv_host[kMaxHalfHost];  // base^(-2j/D), formed on the host in fp64 and rounded once
 };
 
 // Work items of one sequence with nt query tiles.
@@ -432,6 +436,55 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t r
     }
 }
 
+// Decode: the cos/sin rows of the query tile's G * Sq rows, formed in the kernel and written
+// into the second query slot in the layout that a 128-byte-swizzled copy of the table's rows
+// would leave there (rope_tile reads them so): row r of the tile is query row qrow0 + r of q
+// viewed as [B*Hq*Sq, D], i.e. new token s of sequence b, at position dec_qpos[b][s].  The
+// angles go through the table kernels' reduction and SFU evaluation and are packed the same
+// way (fp16 (cos, cos), (sin, sin) word pairs, chunk order permuted for D = 128).  Each thread
+// takes the tasks (row, chunk pair) that its own rope_tile call reads afterwards, so the
+// rows need no barrier between the writes and the reads.
+template <int D>
+__device__ __forceinline__ void decode_query_table(uint32_t tab, const AttnArgs& a, int32_t qrow0, int32_t rt) {
+    constexpr int kPairsPerRow = D / 16;  // 8-frequency tasks per row
+    constexpr int kIters = kBlockM * kPairsPerRow / kRopeThreads;
+    constexpr int kHalf = D / 2;
+    const int32_t rows = a.G * a.dec_Sq;
+    const int32_t per_seq = a.Hq * a.dec_Sq;  // query rows of one sequence
+#pragma unroll 1
+    for (int it = 0; it < kIters; ++it) {
+        const int task = rt + kRopeThreads * it;
+        const int32_t r = task / kPairsPerRow;
+        const int c = task % kPairsPerRow;
+        if (r >= rows) continue;
+        const int32_t t = qrow0 + r;
+        const int32_t b = t / per_seq;
+        const int32_t sq = t - (t / a.dec_Sq) * a.dec_Sq;
+        if (!in_bounds(t >= 0 && b >= 0 && b < a.B && r < kBlockM && 8 * c + 8 <= kHalf)) continue;
+        const float* inv = a.dec_inv ? a.dec_inv + static_cast<int64_t>(b) * kHalf : a.dec_inv_host;
+        float sn[8], cs[8];
+        sincos8(static_cast<float>(__ldg(a.dec_qpos + static_cast<int64_t>(b) * a.dec_Sq + sq)), inv + 8 * c, sn, cs);
+        uint32_t pr[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            __half2 hc = __floats2half2_rn(cs[2 * k], cs[2 * k + 1]);
+            __half2 hs = __floats2half2_rn(sn[2 * k], sn[2 * k + 1]);
+            pr[2 * k] = *reinterpret_cast<uint32_t*>(&hc);
+            pr[2 * k + 1] = *reinterpret_cast<uint32_t*>(&hs);
+        }
+        // 16-byte chunk positions of frequencies 8c..8c+3 and 8c+4..8c+7 in a table row, each
+        // in its 128-byte box (atom), chunk index swizzled by the row
+        const int p0 = (kHalf == 64) ? c : 2 * c;
+        const int p1 = (kHalf == 64) ? 8 + c : 2 * c + 1;
+        auto at = [&](int pc) -> uint32_t {
+            return tab + static_cast<uint32_t>(pc >> 3) * AttnCfg<D>::kAtomBytes + static_cast<uint32_t>(r) * 128u +
+                   ((static_cast<uint32_t>(pc & 7) ^ static_cast<uint32_t>(r & 7)) << 4);
+        };
+        sts128(at(p0), make_uint4(pr[0], pr[1], pr[2], pr[3]));
+        sts128(at(p1), make_uint4(pr[4], pr[5], pr[6], pr[7]));
+    }
+}
+
 // Angles of one RoPE thread for a key tile whose rows hold consecutive
 // positions: 4 groups of 2 frequencies, (cos, sin) kept as packed fp32 pairs.
 struct RecState {
@@ -682,6 +735,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if constexpr (kDecode) {
+        // the combine kernel that follows may place its blocks (they wait for this grid) as soon
+        // as every decode block has started
+        griddep_launch_dependents();
         const WorkItem w = decode_item_kv(a, blockIdx.x);
         if (threadIdx.x == 0 && w.split == 0) {
             const int32_t len = a.kv_lens[w.seq];
@@ -884,17 +940,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 // key tile 0 first (its slot frees before the query slots do), then the query tiles
                 if (!load_k(0)) break;
                 if (it > 0 && !wait(bar(C::kBarQEmpty), static_cast<uint32_t>(it - 1) & 1u)) break;
-                mbar_expect_tx(bar(C::kBarQFull),
-                               static_cast<uint32_t>(sh.nq) * C::kTileBytes + (kDecode ? C::kTabBytes : 0), leader);
+                mbar_expect_tx(bar(C::kBarQFull), static_cast<uint32_t>(sh.nq) * C::kTileBytes, leader);
                 for (int i = 0; i < sh.nq; ++i) {
-                    if constexpr (kDecode) {  // q viewed as [B*Hq*Sq, D]: the group's rows from qrow0,
-                                              // their cos/sin rows in the second query slot
+                    if constexpr (kDecode) {  // q viewed as [B*Hq*Sq, D]: the group's rows from qrow0
                         for (int at = 0; at < C::kAtoms; ++at)
                             tma_load_3d(sbase + C::kOffQ + at * C::kAtomBytes, &tmQ, bar(C::kBarQFull), at * 64, 0,
                                         w.qrow0, leader);
-                        for (int bx = 0; bx < C::kTabBoxes; ++bx)
-                            tma_load_3d(sbase + C::kOffQ + C::kTileBytes + bx * C::kAtomBytes, &tmT,
-                                        bar(C::kBarQFull), bx * 32, w.qrow0, 0, leader);
                     } else {
                         const int32_t qplane = bnsd ? (w.seq * a.Hq + w.h[i]) : w.h[i];
                         load_tile(&tmQ, sbase + C::kOffQ + i * C::kTileBytes, bar(C::kBarQFull), qplane,
@@ -1131,6 +1182,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             WorkItem w;
             ItemShape sh;
             if (read_item(it, true, w, sh) < 0) break;
+            if constexpr (kDecode) decode_query_table<D>(sbase + C::kOffQ + C::kTileBytes, a, w.qrow0, rt);
             const bool rec = consecutive(w);
             uint64_t wc[4], ws[4];  // in-tile step (cos, sin) of kStep rows, packed pairs
             RecState zk;            // key tiles: this thread's first row of the next tile (recurrence)
@@ -1176,7 +1228,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int32_t rows = min(kBlockM, w.L - row0);
                 if constexpr (kDecode) {
                     // cached keys are already rotated; the query tile holds the group's G * Sq rows,
-                    // their cos/sin rows in the second query slot
+                    // their cos/sin rows in the second query slot (decode_query_table above)
                     if (isq) rope_tile<D, kFP16, kAdj>(tile, sbase + C::kOffQ + C::kTileBytes, a.G * a.dec_Sq, rt);
                 } else if (rec) {
                     // key tile j > 0 continues from the state key tile j - 1 left (its rows step on by 128)
@@ -1633,6 +1685,7 @@ template <bool kFP16>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ part_o,
                                                              const float* __restrict__ part_ml, void* out,
                                                              int32_t rows, int32_t D, int32_t splits) {
+    griddep_wait();  // the decode grid's partials complete and visible (programmatic launch)
     const int32_t per_row = D / 8;
     const int64_t work = static_cast<int64_t>(rows) * per_row;
     for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < work;

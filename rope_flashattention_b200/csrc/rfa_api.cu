@@ -724,7 +724,7 @@ namespace {
 struct DecodePlan {
     int32_t splits, chunk;
     int64_t rq;  // query rows B * Hq * Sq
-    size_t tab_bytes, po_bytes, pml_bytes, total;
+    size_t po_bytes, pml_bytes, total;
 };
 
 rfa_status decode_validate(const rfa_decode_params* p) {
@@ -782,10 +782,9 @@ DecodePlan decode_plan(const rfa_decode_params* p) {
     }
     pl.chunk = per * rfa::kBlockN;
     pl.splits = (p->max_kv_len + pl.chunk - 1) / pl.chunk;
-    pl.tab_bytes = round_up(static_cast<size_t>(pl.rq) * p->D * 2, 256);
     pl.po_bytes = pl.splits > 1 ? round_up(static_cast<size_t>(pl.splits) * pl.rq * p->D * 4, 256) : 0;
     pl.pml_bytes = pl.splits > 1 ? round_up(static_cast<size_t>(pl.splits) * pl.rq * 2 * 4, 256) : 0;
-    pl.total = pl.tab_bytes + pl.po_bytes + pl.pml_bytes;
+    pl.total = std::max<size_t>(256, pl.po_bytes + pl.pml_bytes);  // never 0: 0 reports invalid parameters
     return pl;
 }
 
@@ -810,32 +809,16 @@ rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, 
     if (invFreq && !aligned(invFreq, 16)) return RFA_ERR_INVALID_ARG;
     const DecodePlan pl = decode_plan(p);
     if (!workspace || ws_bytes < pl.total || !aligned(workspace, 256)) return RFA_ERR_WORKSPACE;
-    const int D = p->D, half = D / 2;
+    const int D = p->D;
     const bool fp16 = p->io_dtype == RFA_DT_FP16;
     cudaStream_t st = as_stream(stream);
     char* ws = static_cast<char*>(workspace);
-    // cos/sin rows of every query row (b, h, s), in the layout the attention kernel reads
-    rfa::TableArgs ta;
-    std::memset(&ta, 0, sizeof ta);
-    ta.pos = q_pos;
-    ta.inv_dev = invFreq;
-    ta.table = reinterpret_cast<uint32_t*>(ws);
-    ta.ntokens = static_cast<int32_t>(pl.rq);
-    ta.half = half;
-    ta.nseg = 1;
-    ta.uniform_len = p->Hq * p->Sq;  // row t belongs to sequence t / (Hq * Sq)
-    ta.pos_sq = p->Sq;               // and reads position q_pos[b, t % Sq]
-    ta.npos = p->B * p->Sq;
-    ta.inv_dev_rows = p->B;
-    if (!invFreq) {
-        ta.inv_host_rows = 1;
-        inv_freq_row(p->rope_base, D, ta.inv_host);
-    }
-    rfa::rope_table_kernel<<<grid_for(pl.rq * (half / 8), 256), 256, 0, st>>>(ta);
-    if (cudaGetLastError() != cudaSuccess) return RFA_ERR_CUDA;
-
     rfa::AttnArgs aa;
     std::memset(&aa, 0, sizeof aa);
+    // the query rows' cos/sin are formed in the kernel from their positions and frequencies
+    aa.dec_qpos = q_pos;
+    aa.dec_inv = invFreq;
+    if (!invFreq) inv_freq_row(p->rope_base, D, aa.dec_inv_host);
     aa.out = out;
     aa.seeds = nullptr;
     aa.layout = 1;  // cache rows token-major: [B * Smax, Hkv, D]
@@ -855,20 +838,20 @@ rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, 
     aa.kv_lens = kv_lens;
     aa.out_elems = pl.rq * D;
     aa.ntok = p->B * p->Smax;
-    aa.part_o = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.tab_bytes) : nullptr;
-    aa.part_ml = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.tab_bytes + pl.po_bytes) : nullptr;
+    aa.part_o = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
+    aa.part_ml = pl.splits > 1 ? reinterpret_cast<float*>(ws + pl.po_bytes) : nullptr;
     const uint64_t esz = 2, rows_cache = static_cast<uint64_t>(p->B) * p->Smax;
-    CUtensorMap mq, mk, mv, mt;
+    CUtensorMap mq, mk, mv;
     bool ok = make_map(&mq, q, fp16, D, 1, static_cast<uint64_t>(pl.rq), D * esz, D * esz, 64, 1, rfa::kBlockM) &&
               make_map(&mk, k_cache, fp16, D, p->Hkv, rows_cache, D * esz, static_cast<uint64_t>(p->Hkv) * D * esz, 64,
                        1, rfa::kBlockN) &&
               make_map(&mv, v_cache, fp16, D, p->Hkv, rows_cache, D * esz, static_cast<uint64_t>(p->Hkv) * D * esz, 64,
-                       1, rfa::kBlockN) &&
-              make_table_map(&mt, ws, static_cast<uint64_t>(pl.rq), D);
+                       1, rfa::kBlockN);
     if (!ok) return RFA_ERR_CUDA;
     const bool adj = p->rope_interleaved != 0;
     rfa_status r;
     const CUtensorMap& mo = mq;  // decode stores its rows itself
+    const CUtensorMap& mt = mq;  // and reads no table (the kernel forms the query rows' cos/sin)
     if (D == 128) {
         if (adj)
             r = fp16 ? launch_attn<128, true, true, true>(mq, mk, mv, mt, mo, aa, st)
@@ -885,14 +868,24 @@ rfa_status rfa_decode_rope_attention(const rfa_decode_params* p, const void* q, 
                      : launch_attn<64, false, false, true>(mq, mk, mv, mt, mo, aa, st);
     }
     if (r != RFA_OK || pl.splits == 1) return r;
-    const int grid = grid_for(pl.rq * (D / 8), 256);
-    if (fp16)
-        rfa::decode_combine_kernel<true><<<grid, 256, 0, st>>>(aa.part_o, aa.part_ml, out, static_cast<int32_t>(pl.rq),
-                                                                D, pl.splits);
-    else
-        rfa::decode_combine_kernel<false><<<grid, 256, 0, st>>>(aa.part_o, aa.part_ml, out,
-                                                                 static_cast<int32_t>(pl.rq), D, pl.splits);
-    return cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
+    // the combine kernel as a programmatic dependent launch: its blocks are placed while the
+    // decode grid finishes and wait (griddepcontrol.wait) for its partials
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid_for(pl.rq * (D / 8), 256)));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float* po = aa.part_o;
+    const float* pml = aa.part_ml;
+    const int32_t rows = static_cast<int32_t>(pl.rq), Dc = D, splits = pl.splits;
+    const cudaError_t e = fp16 ? cudaLaunchKernelEx(&cfg, rfa::decode_combine_kernel<true>, po, pml, out, rows, Dc, splits)
+                               : cudaLaunchKernelEx(&cfg, rfa::decode_combine_kernel<false>, po, pml, out, rows, Dc, splits);
+    return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? RFA_OK : RFA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -340,6 +340,14 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
 }
+// Programmatic dependent launch.  launch_dependents lets the kernel launched next on the stream
+// with programmatic stream serialization start its blocks once every block of this grid has
+// issued it (or exited); griddep_wait, in that dependent kernel, returns when this grid has
+// completed and its memory is visible.  Both are no-ops without such a launch.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // 32-byte global store (one full sector); p must be 32-byte aligned.
 __device__ __forceinline__ void stg256(void* p, const uint32_t (&v)[8]) {
     asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
