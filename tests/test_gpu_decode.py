@@ -147,3 +147,14 @@ def test_benchmarked_shape_32k_keys(rfa):
     ref = np.concatenate([oracle.decode_attention(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], q_pos[b:b + 1].numpy(), [L],
                                                   inv) for b in range(B)])
     _compare(got, ref)
+
+
+@pytest.mark.parametrize("D,dtype,inter", [(128, torch.bfloat16, False), (64, torch.float16, True)])
+def test_full_query_tile_of_new_tokens(rfa, D, dtype, inter):
+    """G * Sq = 128: the query tile is full (G = 8 heads x 16 new tokens), so the
+    cos/sin rows the kernel forms for its query rows cover every row and chunk
+    of the tile; positions end at different lengths per sequence and the keys
+    are split across CTAs."""
+    got, ref, st = _case(rfa, 2, 16, 2, 16, D, 2100, [2100, 777], seed=12, dtype=dtype, interleaved=inter)
+    assert st == 0
+    _compare(got, ref)
