@@ -382,12 +382,29 @@ __device__ __forceinline__ uint32_t chunk_addr(uint32_t tile, int32_t r, int32_t
     return tile + static_cast<uint32_t>(L >> 3) * AttnCfg<D>::kAtomBytes + static_cast<uint32_t>(r) * 128u +
            ((static_cast<uint32_t>(L & 7) ^ static_cast<uint32_t>(r & 7)) << 4);
 }
+// Adjacent pairs at D = 128: a task's chunks 2cp and 2cp + 1 lie in atom 0 for cp < 4 and in
+// atom 1 for cp >= 4, at the same bank offsets, so a quarter-warp (the 8 tasks of one row)
+// taking the even chunks first would touch every second bank twice.  Tasks with cp >= 4 take
+// their two chunks, and with them their two groups of 4 frequencies, in the other order: a
+// quarter-warp's first access then covers chunks {0,2,4,6} of atom 0 and {1,3,5,7} of atom 1,
+// each bank once.
+template <int D, bool kAdj>
+__device__ __forceinline__ constexpr bool task_swapped(int cp) {
+    return kAdj && D == 128 && cp >= 4;
+}
 // The two chunks a RoPE task rotates together hold the 8 pairs of frequencies
-// 8cp..8cp+7: chunks cp and cp + D/16 (rotate-half) or 2cp and 2cp + 1 (adjacent pairs).
+// 8cp..8cp+7: chunks cp and cp + D/16 (rotate-half) or 2cp and 2cp + 1 (adjacent pairs;
+// 2cp + 1 first for a swapped task, whose frequency groups are then 8cp+4.., 8cp..).
 template <int D, bool kAdj>
 __device__ __forceinline__ void task_chunks(uint32_t tile, int32_t r, int cp, uint32_t& o1, uint32_t& o2) {
-    o1 = chunk_addr<D>(tile, r, kAdj ? 2 * cp : cp);
-    o2 = chunk_addr<D>(tile, r, kAdj ? 2 * cp + 1 : cp + D / 16);
+    const int sw = task_swapped<D, kAdj>(cp) ? 1 : 0;
+    o1 = chunk_addr<D>(tile, r, kAdj ? 2 * cp + sw : cp);
+    o2 = chunk_addr<D>(tile, r, kAdj ? 2 * cp + 1 - sw : cp + D / 16);
+}
+// First frequency of a task's k-th group of 4 (k = 0, 1), in the order its chunks are taken.
+template <int D, bool kAdj>
+__device__ __forceinline__ int task_freq(int cp, int k) {
+    return 8 * cp + 4 * (k ^ (task_swapped<D, kAdj>(cp) ? 1 : 0));
 }
 // Checked build: a task's row and chunk pair lie inside its 128-row tile.
 template <int D>
@@ -418,8 +435,9 @@ __device__ __forceinline__ void rope_tile(uint32_t tile, uint32_t tab, int32_t r
             // chunk cp of atom 1 = pairs 8cp+4..8cp+7 (conflict-free for the 8
             // lanes of a quarter-warp, which share a row)
             const uint32_t tb = tab + r * 128 + ((cp ^ sw) << 4);
-            t0 = lds128(tb);
-            t1 = lds128(tb + AttnCfg<D>::kAtomBytes);
+            const uint32_t ta = task_swapped<D, kAdj>(cp) ? AttnCfg<D>::kAtomBytes : 0u;
+            t0 = lds128(tb + ta);
+            t1 = lds128(tb + (AttnCfg<D>::kAtomBytes - ta));
         } else {
             const uint32_t tb = tab + r * 128;
             const uint32_t tc = static_cast<uint32_t>(cp * 2);
@@ -596,9 +614,11 @@ __device__ __forceinline__ void rope_tile_global(uint32_t tile, const uint32_t* 
     constexpr int kStep = kThreads / kPairsPerRow;
     const int cp = tid % kPairsPerRow;
     const int r0 = tid / kPairsPerRow;
-    // chunk positions of frequencies 8cp..8cp+3 and 8cp+4..8cp+7 within a row
-    const int g0 = (D == 128) ? cp : 2 * cp;
-    const int g1 = (D == 128) ? 8 + cp : 2 * cp + 1;
+    // chunk positions of the task's two frequency groups within a row, in the order its chunks
+    // are taken (8cp..8cp+3 then 8cp+4..8cp+7, the other way round for a swapped task)
+    const bool swp = task_swapped<D, kAdj>(cp);
+    const int g0 = (D == 128) ? (swp ? 8 + cp : cp) : 2 * cp;
+    const int g1 = (D == 128) ? (swp ? cp : 8 + cp) : 2 * cp + 1;
     if (!task_in_tile<D>(r0, cp) || !in_bounds(g0 < D / 8 && g1 < D / 8)) return;
 #pragma unroll 1
     for (int b0 = 0; b0 < kIters; b0 += kBatch) {
@@ -1175,7 +1195,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // otherwise cos/sin rows from the table, staged beside the key tile by TMA.
         const int32_t rt = threadIdx.x - kRopeWarp0 * 32;  // 0..127
         constexpr int kPairsPerRow = D / 16;
-        const int f0 = 8 * (rt % kPairsPerRow);             // this thread's first frequency
         const int r0 = rt / kPairsPerRow;                   // this thread's first row of a tile
         uint32_t g = 0;  // key tiles rotated so far (ring position)
         for (int32_t it = 0;; ++it) {
@@ -1190,12 +1209,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 // key tile 0's first-row angles formed directly from the sequence's first position and
                 // this thread's frequencies; every later row by the step
                 const RopeSeed* sd = a.seeds + w.orig;
-                const float4 u0 = *reinterpret_cast<const float4*>(sd->inv + f0);
-                const float4 u1 = *reinterpret_cast<const float4*>(sd->inv + f0 + 4);
+                const int cpr = rt % kPairsPerRow;  // this thread's frequency groups, in task order
+                const float4 u0 = *reinterpret_cast<const float4*>(sd->inv + task_freq<D, kAdj>(cpr, 0));
+                const float4 u1 = *reinterpret_cast<const float4*>(sd->inv + task_freq<D, kAdj>(cpr, 1));
                 const float qw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const float4 v = *reinterpret_cast<const float4*>(sd->wstep + f0 + 2 * k);  // pairs f, f + 1
+                    const float4 v = *reinterpret_cast<const float4*>(sd->wstep + task_freq<D, kAdj>(cpr, k >> 1) +
+                                                                      2 * (k & 1));  // pairs f, f + 1
                     wc[k] = f2pack(v.x, v.z);
                     ws[k] = f2pack(v.y, v.w);
                 }
@@ -1317,14 +1338,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (rec) {
                         constexpr int kPairsPerRow = D / 16;
                         const RopeSeed* sd = a.seeds + orig;
-                        const int f0 = 8 * (qtid % kPairsPerRow);
-                        const float4 u0 = *reinterpret_cast<const float4*>(sd->inv + f0);
-                        const float4 u1 = *reinterpret_cast<const float4*>(sd->inv + f0 + 4);
+                        const int cpq = qtid % kPairsPerRow;  // frequency groups in task order
+                        const float4 u0 = *reinterpret_cast<const float4*>(sd->inv + task_freq<D, kAdj>(cpq, 0));
+                        const float4 u1 = *reinterpret_cast<const float4*>(sd->inv + task_freq<D, kAdj>(cpq, 1));
                         const float qw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
                         uint64_t wc[4], ws[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const float4 v = *reinterpret_cast<const float4*>(sd->wstep + f0 + 2 * k);
+                            const float4 v = *reinterpret_cast<const float4*>(
+                                sd->wstep + task_freq<D, kAdj>(cpq, k >> 1) + 2 * (k & 1));
                             wc[k] = f2pack(v.x, v.z);
                             ws[k] = f2pack(v.y, v.w);
                             uint64_t c = wc[k], sn = ws[k];
